@@ -1,0 +1,146 @@
+"""CPU oracle for the Prism Attention decode hot path (test infrastructure).
+
+The arithmetic lives in ``prism_oracle.c`` (plain sequential C, fp32 for
+everything that decides a selection, fp64 for attention outputs); this module
+compiles it with gcc and wraps it with ctypes.  ``pipeline`` drives it over
+whole layers and decode steps.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline /
+reference legs of ``bench.py`` may import this package.  The CUDA library
+never calls it, and it never calls the CUDA library.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "prism_oracle.c")
+_SO = os.path.join(_HERE, "_build", "libprism_oracle.so")
+
+# No FMA contraction and no fast-math: sums are evaluated exactly as written,
+# feature index ascending, each product and each sum rounded to fp32.
+CFLAGS = ["-O2", "-std=c99", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+          "-frounding-math"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/_build`` (idempotent)."""
+    os.makedirs(os.path.dirname(_SO), exist_ok=True)
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        tmp = _SO + f".{os.getpid()}.tmp"
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _SO)
+    return _SO
+
+
+_lib = None
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i32, i64, f64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
+        lib.oracle_quantize_rows.argtypes = [P, i64, i32, P, P]
+        lib.oracle_topk_ascending.argtypes = [P, i32, i32, P]
+        lib.oracle_topk_ascending.restype = i32
+        lib.oracle_propose_scores.argtypes = [P, i32, i32, P, P, i32, P]
+        lib.oracle_propose_row.argtypes = [P, i32, i32, P, P, i32, i32, P, P]
+        lib.oracle_propose_row.restype = i32
+        lib.oracle_refine_scores.argtypes = [P, i32, i32, P, P, i32, P]
+        lib.oracle_refine_row.argtypes = [P, i32, i32, P, P, i32, i32, P, P]
+        lib.oracle_refine_row.restype = i32
+        lib.oracle_attend.argtypes = [P, i32, P, P, P, i32, f64, P, P]
+        _lib = lib
+    return _lib
+
+
+def _p(a: np.ndarray):
+    return ctypes.c_void_p(a.ctypes.data) if a is not None else None
+
+
+def _f32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+
+
+def _i32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def quantize_rows(k):
+    """int8 symmetric per-row quantization -> (kq [rows, d] int8, scale [rows] f32)."""
+    k = _f32(k)
+    rows, d = k.shape
+    kq = np.empty((rows, d), np.int8)
+    sc = np.empty((rows,), np.float32)
+    _L().oracle_quantize_rows(_p(k), rows, d, _p(kq), _p(sc))
+    return kq, sc
+
+
+def topk_ascending(s, k: int) -> np.ndarray:
+    """Top-k indices of s (score desc, lower index wins ties), ascending."""
+    s = _f32(s)
+    out = np.empty((max(min(k, s.size), 1),), np.int32)
+    m = _L().oracle_topk_ascending(_p(s), s.size, k, _p(out))
+    return out[:m].copy()
+
+
+def propose_scores(q, kq, scale) -> np.ndarray:
+    """s_t = scale_t * max_g sum_j q[g, j] * kq[t, j] (fp32, j ascending)."""
+    q, kq, scale = _f32(q), np.ascontiguousarray(kq, dtype=np.int8), _f32(scale)
+    G, d = q.shape
+    L = kq.shape[0]
+    s = np.empty((L,), np.float32)
+    _L().oracle_propose_scores(_p(q), G, d, _p(kq), _p(scale), L, _p(s))
+    return s
+
+
+def propose_row(q, kq, scale, kappa_p: int):
+    """(pool ascending int32 [min(kappa_p, L)], proposal scores [L])."""
+    q, kq, scale = _f32(q), np.ascontiguousarray(kq, dtype=np.int8), _f32(scale)
+    G, d = q.shape
+    L = kq.shape[0]
+    s = np.empty((max(L, 1),), np.float32)
+    pool = np.empty((max(min(kappa_p, L), 1),), np.int32)
+    m = _L().oracle_propose_row(_p(q), G, d, _p(kq), _p(scale), L, kappa_p, _p(pool), _p(s))
+    return pool[:m].copy(), s[:L].copy()
+
+
+def refine_scores(q, K, pool) -> np.ndarray:
+    """r_i = max_g sum_j q[g, j] * K[pool_i, j] (fp32, j ascending)."""
+    q, K, pool = _f32(q), _f32(K), _i32(pool)
+    G, d = q.shape
+    r = np.empty((max(pool.size, 1),), np.float32)
+    _L().oracle_refine_scores(_p(q), G, d, _p(K), _p(pool), pool.size, _p(r))
+    return r[:pool.size].copy()
+
+
+def refine_row(q, K, pool, kappa: int):
+    """(refined positions ascending int32 [min(kappa, |pool|)], exact pool scores)."""
+    q, K, pool = _f32(q), _f32(K), _i32(pool)
+    G, d = q.shape
+    n = pool.size
+    r = np.empty((max(n, 1),), np.float32)
+    idx = np.empty((max(min(kappa, n), 1),), np.int32)
+    m = _L().oracle_refine_row(_p(q), G, d, _p(K), _p(pool), n, kappa, _p(idx), _p(r))
+    return idx[:m].copy(), r[:n].copy()
+
+
+def attend(q, K, V, idx, softmax_scale: float):
+    """fp64 softmax attention of one query head over rows idx (None = all rows)."""
+    q, K, V = _f32(q), _f32(K), _f32(V)
+    d = q.shape[0]
+    if idx is None:
+        n, ip = K.shape[0], None
+    else:
+        idx = _i32(idx)
+        n, ip = idx.size, _p(idx)
+    out = np.empty((d,), np.float32)
+    lse = np.empty((1,), np.float32)
+    _L().oracle_attend(_p(q), d, _p(K), _p(V), ip, n, float(softmax_scale), _p(out), _p(lse))
+    return out, float(lse[0])

@@ -1,0 +1,144 @@
+"""Layer- and step-level drivers of the CPU oracle (test infrastructure).
+
+Packed layouts, shared with the CUDA library's interface:
+  q        [B][Hq][d]
+  K, V     [Hkv][T][d]   rows of sequence b at cu_seqlens[b] .. cu_seqlens[b+1]
+  kq       [Hkv][T][d]   int8,  k_scale [Hkv][T] fp32
+  pool     [B][Hkv][kappa_p] int32 positions within the sequence, ascending,
+           -1 past pool_cnt[b][h]
+  idx      [B][Hkv][kappa]   same convention, cnt[b][h]
+  out      [B][Hq][d] fp32,  lse [B][Hq] fp32
+Query head hq reads KV head hq // G.  Each (sequence, KV head) row is
+independent, so every function loops over rows and calls the C oracle.
+
+The layer schedule (Prism Attention, sec. 5.3 "Accuracy-efficiency
+trade-off": in "g x" one layer in every x is a proposal layer) is read as
+``layer % group == 0``; the pool of the latest proposal layer serves every
+layer up to the next one.  A proposal layer also refines its own pool with
+exact scores and attends over the refined set, so every layer attends over
+kappa exactly rescored tokens (reading of sec. 6: refined layers re-select
+their own top-kappa inside the proposed region).
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, List, Optional
+
+import numpy as np
+
+from . import attend, propose_row, quantize_rows, refine_row
+
+
+def _np(x):
+    try:
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            return x.detach().to("cpu").float().numpy() if x.dtype != torch.int8 and \
+                x.dtype != torch.int32 and x.dtype != torch.int64 else x.detach().to("cpu").numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(x)
+
+
+def quantize_layer(k):
+    """kq [Hkv][T][d] int8, scale [Hkv][T] fp32 from K [Hkv][T][d]."""
+    k = _np(k).astype(np.float32)
+    Hkv, T, d = k.shape
+    kq, sc = quantize_rows(k.reshape(Hkv * T, d))
+    return kq.reshape(Hkv, T, d), sc.reshape(Hkv, T)
+
+
+def propose_layer(q, kq, scale, cu, kappa_p: int, rows=None):
+    """pool [B][Hkv][kappa_p] (-1 padded), pool_cnt [B][Hkv], scores per row."""
+    q = _np(q).astype(np.float32)
+    kq, scale = _np(kq), _np(scale).astype(np.float32)
+    B, Hq, d = q.shape
+    Hkv = kq.shape[0]
+    G = Hq // Hkv
+    pool = np.full((B, Hkv, kappa_p), -1, np.int32)
+    cnt = np.zeros((B, Hkv), np.int32)
+    scores: Dict = {}
+    for b in range(B):
+        t0, t1 = cu[b], cu[b + 1]
+        for h in range(Hkv):
+            if rows is not None and (b, h) not in rows:
+                continue
+            p, s = propose_row(q[b, h * G:(h + 1) * G], kq[h, t0:t1], scale[h, t0:t1], kappa_p)
+            pool[b, h, :p.size] = p
+            cnt[b, h] = p.size
+            scores[(b, h)] = s
+    return pool, cnt, scores
+
+
+def refine_layer(q, k, cu, pool, pool_cnt, kappa: int, rows=None):
+    """idx [B][Hkv][kappa] (-1 padded), cnt [B][Hkv], exact pool scores per row."""
+    q = _np(q).astype(np.float32)
+    k = _np(k).astype(np.float32)
+    pool, pool_cnt = _np(pool), _np(pool_cnt)
+    B, Hq, d = q.shape
+    Hkv = k.shape[0]
+    G = Hq // Hkv
+    idx = np.full((B, Hkv, kappa), -1, np.int32)
+    cnt = np.zeros((B, Hkv), np.int32)
+    scores: Dict = {}
+    for b in range(B):
+        t0, t1 = cu[b], cu[b + 1]
+        for h in range(Hkv):
+            if rows is not None and (b, h) not in rows:
+                continue
+            n = int(pool_cnt[b, h])
+            sel, r = refine_row(q[b, h * G:(h + 1) * G], k[h, t0:t1], pool[b, h, :n], kappa)
+            idx[b, h, :sel.size] = sel
+            cnt[b, h] = sel.size
+            scores[(b, h)] = r
+    return idx, cnt, scores
+
+
+def attend_layer(q, k, v, cu, idx, cnt, softmax_scale: Optional[float] = None, rows=None):
+    """Sparse attention over idx (idx None = dense over every position)."""
+    q = _np(q).astype(np.float32)
+    k = _np(k).astype(np.float32)
+    v = _np(v).astype(np.float32)
+    B, Hq, d = q.shape
+    Hkv = k.shape[0]
+    G = Hq // Hkv
+    if softmax_scale is None:
+        softmax_scale = float(np.float32(1.0 / math.sqrt(d)))
+    out = np.zeros((B, Hq, d), np.float32)
+    lse = np.full((B, Hq), -np.inf, np.float32)
+    for b in range(B):
+        t0, t1 = cu[b], cu[b + 1]
+        for h in range(Hkv):
+            if rows is not None and (b, h) not in rows:
+                continue
+            sel = None if idx is None else _np(idx)[b, h, :int(_np(cnt)[b, h])]
+            for g in range(G):
+                hq = h * G + g
+                out[b, hq], lse[b, hq] = attend(q[b, hq], k[h, t0:t1], v[h, t0:t1], sel,
+                                                softmax_scale)
+    return out, lse
+
+
+def decode_step(cfg, layers, rows=None) -> List[dict]:
+    """One decode step over the given layers (workload.Layer objects, in order).
+
+    Returns, per layer: kq/scale (proposal layers), pool/pool_cnt (from the
+    latest proposal layer), idx/cnt, out/lse.
+    """
+    cu = cfg.cu_seqlens
+    res = []
+    pool = pool_cnt = None
+    for lay in layers:
+        r = {"layer": lay.index}
+        if cfg.is_proposal(lay.index):
+            kq, sc = quantize_layer(lay.k)
+            pool, pool_cnt, _ = propose_layer(lay.q, kq, sc, cu, cfg.kappa_p, rows)
+            r["kq"], r["scale"] = kq, sc
+        assert pool is not None, "the first layer of a step must be a proposal layer"
+        r["pool"], r["pool_cnt"] = pool, pool_cnt
+        idx, cnt, _ = refine_layer(lay.q, lay.k, cu, pool, pool_cnt, cfg.kappa, rows)
+        r["idx"], r["cnt"] = idx, cnt
+        r["out"], r["lse"] = attend_layer(lay.q, lay.k, lay.v, cu, idx, cnt, rows=rows)
+        res.append(r)
+    return res
