@@ -1,0 +1,196 @@
+/*
+ * prism.h -- C ABI of libprism.so: the decode hot path of Prism Attention
+ * ("Prism Attention: Proposal-Refined Index Sharing Mechanism for Efficient
+ * LLMs Inference") on NVIDIA B200 (sm_100a).
+ *
+ * One decode step, per layer l (sec. 4 Overview, sec. 5.3 "Accuracy-efficiency
+ * trade-off": in the "g x" setting one layer in every x is a proposal layer):
+ *
+ *   proposal layer:  prism_quantize_k (new token rows) -> prism_propose
+ *   every layer:     prism_refine (on the latest pool) -> prism_sparse_decode
+ *
+ * prism_dense_decode is the dense flash-decode over the same cache, the
+ * comparison path (the pages compare against FlashAttention, sec. 5.3).
+ *
+ * Notation: B sequences, Hq query heads, Hkv KV heads, G = Hq / Hkv, head
+ * dimension d, sequence b has L_b = cu[b+1] - cu[b] tokens, T = cu[B].
+ * Query head hq reads KV head hq / G.
+ *
+ * Layouts (row-major, all device memory unless stated):
+ *   q        [B][Hq][d]          dtype of the shape (bf16 or fp32)
+ *   K, V     [Hkv][T][d]         packed over sequences: sequence b occupies
+ *                                 rows cu[b] .. cu[b+1]-1 of every head
+ *   kq       [Hkv][T][d]  int8    k_scale [Hkv][T] fp32
+ *   pool     [B][Hkv][kappa_p] int32, pool_cnt [B][Hkv] int32
+ *   idx      [B][Hkv][kappa]   int32, cnt      [B][Hkv] int32
+ *   out      [B][Hq][d] fp32,   lse [B][Hq] fp32 (natural log)
+ * Index values are positions inside their sequence (0 <= t < L_b).  Every
+ * index set is written in strictly ascending order and padded with -1 past
+ * its count.
+ *
+ * Ownership: the caller allocates and owns every buffer.  The library never
+ * allocates, frees or synchronises (prism_get_device_status excepted), keeps
+ * no mutable global state, and may be called from several streams at once
+ * with disjoint outputs and workspaces.  All work is enqueued on `stream`
+ * (a cudaStream_t; NULL is the legacy default stream).
+ *
+ * Errors: every argument that can be checked on the host (null pointers,
+ * sizes, head_dim, kappa <= kappa_p, monotone cu_seqlens_host, workspace
+ * size, supported lengths) is checked before anything is enqueued; a failed
+ * check returns PRISM_ERR_INVALID_ARG / _UNSUPPORTED / _WORKSPACE and
+ * enqueues nothing.  A launch failure returns PRISM_ERR_CUDA.  Values that
+ * live in device memory (indices, counts, token rows) are checked by the
+ * kernels: an out-of-range value is skipped and recorded in the workspace
+ * status word (read it with prism_get_device_status).  Inputs must be finite.
+ */
+#ifndef PRISM_H_
+#define PRISM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PRISM_API __attribute__((visibility("default")))
+#else
+#define PRISM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum prism_dtype { PRISM_F32 = 0, PRISM_BF16 = 1 } prism_dtype;
+
+typedef enum prism_status {
+  PRISM_OK = 0,
+  PRISM_ERR_INVALID_ARG = 1,
+  PRISM_ERR_UNSUPPORTED = 2,
+  PRISM_ERR_WORKSPACE = 3,
+  PRISM_ERR_CUDA = 4,
+  PRISM_ERR_TIMEOUT = 5
+} prism_status;
+
+typedef enum prism_op {
+  PRISM_OP_QUANTIZE = 0,
+  PRISM_OP_PROPOSE = 1,
+  PRISM_OP_REFINE = 2,
+  PRISM_OP_SPARSE_DECODE = 3,
+  PRISM_OP_DENSE_DECODE = 4
+} prism_op;
+
+/* Bits of the device status word kept in every workspace. */
+#define PRISM_DEV_BAD_INDEX 0x1   /* an index / token row outside its sequence */
+#define PRISM_DEV_TOO_LONG  0x2   /* a row longer than the selection capacity  */
+
+/* Shape of one layer's decode problem.  cu_seqlens_host mirrors
+ * cu_seqlens_dev (B+1 entries, cu[0] = 0, non-decreasing, cu[B] =
+ * total_tokens); the host copy sizes grids and is validated, the device copy
+ * is what kernels read.  head_dim is 64 or 128; num_q_heads is a multiple of
+ * num_kv_heads with G <= 16; batch <= 4096. */
+typedef struct prism_shape {
+  int32_t batch;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t dtype; /* prism_dtype of q, K and V */
+  const int32_t* cu_seqlens_dev;
+  const int32_t* cu_seqlens_host;
+  int64_t total_tokens;
+} prism_shape;
+
+/* Longest sequence (propose) and largest pool (refine) one selection row can
+ * hold: 8 cooperating thread blocks x 49152 keys. */
+#define PRISM_MAX_SELECT_ROW 393216
+
+/* Bytes of workspace an operation needs for this shape and budget
+ * (kappa_p / kappa are ignored where they do not apply).  Every workspace
+ * starts with a 256-byte header holding the device status word; zero it once
+ * (prism_clear_device_status) before first use. */
+PRISM_API prism_status prism_workspace_size(const prism_shape* shape, int32_t op, int32_t kappa_p,
+                                  int32_t kappa, size_t* bytes);
+
+/*
+ * Quantized key cache for proposal scoring (sec. 4.2 "Quantized Proposal
+ * Construction": the key cache that proposal layers read is compressed to
+ * low-bit codes; the pages' INT2 scheme is not stated, this library uses
+ * symmetric per-token int8):
+ *   scale[h][t] = max_j |K[h][t][j]| / 127            (IEEE fp32 division)
+ *   kq[h][t][j] = clamp(round_half_even(K[h][t][j] / scale), -127, 127)
+ * and scale = 0, kq = 0 for an all-zero row.
+ * tok_rows: NULL quantizes all T rows of every KV head (prefill); otherwise
+ * a device array of n_rows packed token indices in [0, T) (e.g. the newly
+ * appended token of each sequence), quantized for every KV head.
+ * ws may be NULL (no status reporting); out-of-range token rows are skipped.
+ */
+PRISM_API prism_status prism_quantize_k(const prism_shape* shape, const void* k, int8_t* kq,
+                              float* k_scale, const int32_t* tok_rows, int32_t n_rows,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Proposal layer (sec. 4.1 "Proposal-Refined Index Sharing", sec. 4.2): for
+ * every sequence b and KV head h, score every position t < L_b with the
+ * quantized keys,
+ *   s_t = k_scale[h][t] * max_{g<G} sum_j q[b][h*G+g][j] * kq[h][t][j],
+ * and keep the top min(kappa_p, L_b) positions (higher score first, lower
+ * position on ties) as the candidate pool, written ascending.
+ * kappa_p is the pool size n = rho * kappa of sec. 5.1 "Implementation
+ * Details".  L_b <= PRISM_MAX_SELECT_ROW.
+ */
+PRISM_API prism_status prism_propose(const prism_shape* shape, const void* q, const int8_t* kq,
+                           const float* k_scale, int32_t kappa_p, int32_t* pool_idx,
+                           int32_t* pool_cnt, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Refined layer (sec. 4.1; sec. 6: refined layers re-select their own top
+ * kappa inside the proposed region, at a cost independent of context
+ * length, sec. 5.3 "End-to-end latency"): exact scores of the pool members
+ *   r_i = max_g sum_j q[b][h*G+g][j] * K[h][cu[b] + pool_i][j]   (fp32)
+ * and the top min(kappa, pool_cnt) members (ties to the lower position),
+ * written as ascending positions.  kappa <= kappa_p; kappa_p is the row
+ * stride of pool_idx.  logits_opt, if not NULL, receives [B][Hq][kappa] the
+ * unscaled dot product q_hq . K[idx] of every selected position (slot order
+ * of idx); slots past cnt are left untouched.
+ */
+PRISM_API prism_status prism_refine(const prism_shape* shape, const void* q, const void* k,
+                          const int32_t* pool_idx, const int32_t* pool_cnt, int32_t kappa_p,
+                          int32_t kappa, int32_t* idx, int32_t* cnt, float* logits_opt,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Token-level sparse attention over the selected rows (sec. 1, sec. 2.1):
+ * for every query head hq of sequence b, with h = hq / G and the rows
+ * t in idx[b][h][0 .. cnt[b][h]),
+ *   l_t = softmax_scale * q[b][hq] . K[h][cu[b]+t],
+ *   out[b][hq] = sum_t softmax(l)_t V[h][cu[b]+t],   lse = log sum_t exp(l_t).
+ * Split-K over the index list with a log-sum-exp merge.  An empty set gives
+ * out = 0 and lse = -inf.  kappa is the row stride of idx.
+ */
+PRISM_API prism_status prism_sparse_decode(const prism_shape* shape, const void* q, const void* k,
+                                 const void* v, const int32_t* idx, const int32_t* cnt,
+                                 int32_t kappa, float softmax_scale, float* out, float* lse_opt,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Dense decode attention over every position t < L_b (the comparison path):
+ * the same definition as prism_sparse_decode with idx = 0 .. L_b - 1.
+ */
+PRISM_API prism_status prism_dense_decode(const prism_shape* shape, const void* q, const void* k,
+                                const void* v, float softmax_scale, float* out, float* lse_opt,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* Zero the workspace header (status word) on `stream`. */
+PRISM_API prism_status prism_clear_device_status(void* ws, size_t ws_bytes, void* stream);
+
+/* Read the status word (PRISM_DEV_* bits) after the work on `stream` ends.
+ * This call synchronises `stream`. */
+PRISM_API prism_status prism_get_device_status(const void* ws, size_t ws_bytes, void* stream,
+                                     int32_t* code);
+
+/* Static description of a status code. */
+PRISM_API const char* prism_status_str(prism_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PRISM_H_ */

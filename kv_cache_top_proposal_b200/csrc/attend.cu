@@ -1,0 +1,295 @@
+// Split-K flash-decode over a list of cache rows, with a log-sum-exp merge:
+// the token-level sparse attention over the refined set (Prism Attention,
+// sec. 1 and sec. 2.1) and, with the list "every position", the dense decode
+// the pages compare against (sec. 5.3 "End-to-end latency").
+//
+// Split s of row (b, h) covers list entries [s*per, (s+1)*per).  Every lane
+// group of d*sizeof(T)/16 lanes walks rows of K and V with 16-byte loads and
+// keeps an online softmax state per query head of the group in the log2
+// domain (logit * softmax_scale * log2 e):
+//   m = max logit so far, l = sum 2^(logit - m), o = sum 2^(logit - m) v.
+// The CTA combines its lane groups in a fixed order and writes one partial
+// (o, m, l) per query head and split; merge_kernel combines the splits:
+//   M = max_s m_s,  out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s,
+//   lse = (M + log2 sum_s 2^(m_s - M) l_s) * ln 2.
+// HBM bound: 2 * d * sizeof(T) bytes per listed row.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace prism {
+
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kWarps = kThreads / 32;
+constexpr int kUnroll = 2;
+
+struct AttendArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* cu;
+  const int32_t* idx;
+  const int32_t* cnt;
+  int idx_stride;
+  int Hkv, G, Hq;
+  int64_t T;
+  int per_split, splits;
+  float scale_log2;
+  float* part_o;
+  float* part_ml;
+  int32_t* status;
+};
+
+template <typename T, int D, int GP>
+__global__ void __launch_bounds__(kThreads) attend_kernel(const AttendArgs a) {
+  constexpr int E = Vec16<T>::E;
+  constexpr int LPR = D / E;
+  constexpr int RPW = 32 / LPR;
+  constexpr int SLOTS = kWarps * RPW;
+  extern __shared__ __align__(16) float sm[];
+  float* s_o = sm;                       // [SLOTS][GP][D]
+  float* s_m = sm + SLOTS * GP * D;      // [SLOTS][GP]
+  float* s_l = s_m + SLOTS * GP;         // [SLOTS][GP]
+
+  const int row = blockIdx.y, split = blockIdx.x;
+  const int b = row / a.Hkv, h = row - b * a.Hkv;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane / LPR, li = lane % LPR;
+  const int slot = warp * RPW + sub;
+  const int t0 = a.cu[b];
+  const int L = a.cu[b + 1] - t0;
+  int n = L;
+  if (a.idx) {
+    n = a.cnt[row];
+    if (n < 0 || n > a.idx_stride) {
+      if (threadIdx.x == 0 && split == 0) flag_status(a.status, PRISM_DEV_BAD_INDEX);
+      n = n < 0 ? 0 : a.idx_stride;
+    }
+  }
+  const int e0 = split * a.per_split;
+  const int e1 = min(n, e0 + a.per_split);
+  const int64_t off = ((int64_t)h * a.T + t0) * D + li * E;
+  const T* kbase = static_cast<const T*>(a.k) + off;
+  const T* vbase = static_cast<const T*>(a.v) + off;
+  const int32_t* idx = a.idx ? a.idx + (int64_t)row * a.idx_stride : nullptr;
+
+  float qf[GP][E];
+  {
+    const T* q = static_cast<const T*>(a.q) + ((int64_t)b * a.Hq + (int64_t)h * a.G) * D + li * E;
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      if (g < a.G) {
+        Vec16<T>::unpack(ld16(q + (int64_t)g * D), qf[g]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) qf[g][e] = 0.0f;
+      }
+    }
+  }
+  float m[GP], l[GP], o[GP][E];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    m[g] = -INFINITY;
+    l[g] = 0.0f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) o[g][e] = 0.0f;
+  }
+
+  for (int base = e0 + warp * RPW * kUnroll; base < e1; base += kWarps * RPW * kUnroll) {
+    uint4 kr[kUnroll], vr[kUnroll];
+    bool ok[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int e = base + u * RPW + sub;
+      ok[u] = e < e1;
+      int pos = e;
+      if (idx && ok[u]) pos = idx[e];
+      if (ok[u] && (pos < 0 || pos >= L)) {
+        if (li == 0) flag_status(a.status, PRISM_DEV_BAD_INDEX);
+        ok[u] = false;
+      }
+      if (!ok[u]) pos = 0;
+      if (idx) {
+        kr[u] = ok[u] ? ld16(kbase + (int64_t)pos * D) : make_uint4(0, 0, 0, 0);
+        vr[u] = ok[u] ? ld16(vbase + (int64_t)pos * D) : make_uint4(0, 0, 0, 0);
+      } else {
+        kr[u] = ok[u] ? ld16_stream(kbase + (int64_t)pos * D) : make_uint4(0, 0, 0, 0);
+        vr[u] = ok[u] ? ld16_stream(vbase + (int64_t)pos * D) : make_uint4(0, 0, 0, 0);
+      }
+    }
+    float lg[kUnroll][GP];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      float f[E];
+      Vec16<T>::unpack(kr[u], f);
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float s = 0.0f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) s = fmaf(qf[g][e], f[e], s);
+        s = group_sum<LPR>(s);
+        lg[u][g] = ok[u] ? s * a.scale_log2 : -INFINITY;
+      }
+    }
+    float vf[kUnroll][E];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) Vec16<T>::unpack(vr[u], vf[u]);
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      float mx = m[g];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) mx = fmaxf(mx, lg[u][g]);
+      if (mx == -INFINITY) continue;
+      const float alpha = exp2f(m[g] - mx);
+      float p[kUnroll];
+      float ps = 0.0f;
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        p[u] = exp2f(lg[u][g] - mx);
+        ps += p[u];
+      }
+      l[g] = l[g] * alpha + ps;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        float acc = o[g][e] * alpha;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) acc = fmaf(p[u], vf[u][e], acc);
+        o[g][e] = acc;
+      }
+      m[g] = mx;
+    }
+  }
+
+  // Combine the CTA's lane groups in slot order (deterministic).
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) s_o[(slot * GP + g) * D + li * E + e] = o[g][e];
+    if (li == 0) {
+      s_m[slot * GP + g] = m[g];
+      s_l[slot * GP + g] = l[g];
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < a.G * D; i += kThreads) {
+    const int g = i / D, j = i - g * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < SLOTS; ++s) M = fmaxf(M, s_m[s * GP + g]);
+    float Ls = 0.0f, O = 0.0f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int s = 0; s < SLOTS; ++s) {
+        const float ms = s_m[s * GP + g];
+        const float w = ms == -INFINITY ? 0.0f : exp2f(ms - M);
+        Ls = fmaf(w, s_l[s * GP + g], Ls);
+        O = fmaf(w, s_o[(s * GP + g) * D + j], O);
+      }
+    }
+    const int64_t pr = ((int64_t)b * a.Hq + (int64_t)h * a.G + g) * a.splits + split;
+    a.part_o[pr * D + j] = O;
+    if (j == 0) {
+      a.part_ml[pr * 2] = M;
+      a.part_ml[pr * 2 + 1] = Ls;
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) merge_kernel(int BHq, int splits, const float* __restrict__ part_o,
+                                                   const float* __restrict__ part_ml,
+                                                   float* __restrict__ out, float* __restrict__ lse) {
+  constexpr int PER = D / 32;
+  const int w = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (w >= BHq) return;
+  const float* ml = part_ml + (int64_t)w * splits * 2;
+  const float* po = part_o + (int64_t)w * splits * D;
+  float M = -INFINITY;
+  for (int s = lane; s < splits; s += 32) M = fmaxf(M, ml[s * 2]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float Ls = 0.0f, acc[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) acc[i] = 0.0f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < splits; ++s) {
+      const float ms = ml[s * 2];
+      if (ms == -INFINITY) continue;
+      const float wgt = exp2f(ms - M);
+      Ls = fmaf(wgt, ml[s * 2 + 1], Ls);
+#pragma unroll
+      for (int i = 0; i < PER; ++i) acc[i] = fmaf(wgt, po[(int64_t)s * D + lane + 32 * i], acc[i]);
+    }
+  }
+  const bool any = Ls > 0.0f;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) out[(int64_t)w * D + lane + 32 * i] = any ? acc[i] / Ls : 0.0f;
+  if (lse && lane == 0) lse[w] = any ? (M + log2f(Ls)) * 0.69314718055994530942f : -INFINITY;
+}
+
+template <typename T, int D, int GP>
+cudaError_t run(const Dims& d, const AttendPlan& p, const AttendArgs& a, cudaStream_t st) {
+  constexpr int RPW = 32 / (D / Vec16<T>::E);
+  constexpr int SLOTS = kWarps * RPW;
+  const int smem = (SLOTS * GP * D + 2 * SLOTS * GP) * (int)sizeof(float);
+  auto k = attend_kernel<T, D, GP>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+  }
+  k<<<dim3(p.splits, d.B * d.Hkv), kThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t by_group(const Dims& d, const AttendPlan& p, const AttendArgs& a, cudaStream_t st) {
+  switch (padded_group(d.G)) {
+    case 1: return run<T, D, 1>(d, p, a, st);
+    case 2: return run<T, D, 2>(d, p, a, st);
+    case 4: return run<T, D, 4>(d, p, a, st);
+    case 8: return run<T, D, 8>(d, p, a, st);
+    default: return run<T, D, 16>(d, p, a, st);
+  }
+}
+
+}  // namespace
+
+AttendPlan plan_attend(const Dims& d, int64_t max_rows_per_seq) {
+  constexpr int step = 16;  // rows one CTA covers per iteration (bf16, d = 128)
+  const int64_t rows = (int64_t)d.B * d.Hkv;
+  const int64_t target = 4LL * d.num_sms;
+  int64_t splits = rows > 0 ? cdiv(target, rows) : 1;
+  const int64_t max_splits = cdiv(max_rows_per_seq > 0 ? max_rows_per_seq : 1, step);
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  int64_t per = cdiv(max_rows_per_seq > 0 ? max_rows_per_seq : 1, splits);
+  per = cdiv(per, step) * step;
+  splits = cdiv(max_rows_per_seq > 0 ? max_rows_per_seq : 1, per);
+  return AttendPlan{(int)splits, (int)per};
+}
+
+cudaError_t launch_attend(const Dims& d, const AttendPlan& p, const void* q, const void* k,
+                          const void* v, const int32_t* idx, const int32_t* cnt, int idx_stride,
+                          float softmax_scale, float* part_o, float* part_ml, float* out,
+                          float* lse, int32_t* status, cudaStream_t st) {
+  if (d.B * d.Hq == 0) return cudaSuccess;
+  AttendArgs a{q, k, v, d.cu_dev, idx, cnt, idx_stride, d.Hkv, d.G, d.Hq, d.T,
+               p.per_split, p.splits, softmax_scale * 1.4426950408889634f, part_o, part_ml, status};
+  cudaError_t e;
+  if (d.bf16)
+    e = d.D == 128 ? by_group<__nv_bfloat16, 128>(d, p, a, st) : by_group<__nv_bfloat16, 64>(d, p, a, st);
+  else
+    e = d.D == 128 ? by_group<float, 128>(d, p, a, st) : by_group<float, 64>(d, p, a, st);
+  if (e != cudaSuccess) return e;
+  const int BHq = d.B * d.Hq;
+  const int blocks = (BHq + 3) / 4;
+  if (d.D == 128)
+    merge_kernel<128><<<blocks, 128, 0, st>>>(BHq, p.splits, part_o, part_ml, out, lse);
+  else
+    merge_kernel<64><<<blocks, 128, 0, st>>>(BHq, p.splits, part_o, part_ml, out, lse);
+  return cudaGetLastError();
+}
+
+}  // namespace prism

@@ -1,0 +1,76 @@
+// Internal launchers of libprism (host side).  Arguments are validated by
+// the C ABI layer (prism_api.cu) before any of these is called.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace prism {
+
+// Workspace header: the first 256 bytes of every workspace (status word).
+constexpr size_t kWsHeader = 256;
+
+struct Dims {
+  int B, Hq, Hkv, G, D;
+  int64_t T;
+  bool bf16;
+  const int32_t* cu_dev;
+  const int32_t* cu_host;
+  int max_len;  // max_b L_b (from the host mirror)
+  int num_sms;
+};
+
+// Query-group sizes a kernel is instantiated for; a group of G query heads
+// runs on the smallest instantiation >= G with the extra heads masked.
+inline int padded_group(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : G <= 8 ? 8 : 16; }
+
+cudaError_t launch_quantize(const Dims& d, const void* k, int8_t* kq, float* scale,
+                            const int32_t* tok_rows, int64_t n_rows, int32_t* status,
+                            cudaStream_t st);
+
+// Proposal scores s[h][t] (fp32, [Hkv][T]).  use_mma selects the tensor-core
+// (mma.sync, fp16 operands) scorer, valid for bf16 queries only.
+cudaError_t launch_propose_scores(const Dims& d, const void* q, const int8_t* kq,
+                                  const float* scale, float* scores, bool use_mma,
+                                  cudaStream_t st);
+
+// Cluster radix top-k.  mode 0 (propose): keys scores[h][cu[b] + i], row
+// length L_b, output position i.  mode 1 (refine): keys r[row][i], row length
+// pool_cnt[row], output position pool[row][i]; dots/logits optional.
+struct SelectArgs {
+  int mode;
+  int Hkv, G, Hq;
+  int64_t T;
+  const int32_t* cu;
+  const float* keys;
+  const int32_t* pool;
+  const int32_t* pool_cnt;
+  int pool_stride;
+  int k_req;
+  int32_t* out;
+  int32_t* out_cnt;
+  const float* dots;
+  float* logits;
+  int32_t* status;
+};
+int select_capacity_per_row();  // longest row one cluster can select from
+cudaError_t launch_select(const Dims& d, const SelectArgs& a, int max_row_len, cudaStream_t st);
+
+// Exact pool scores r[row][i] = max_g q_g . K[pool_i] (+ per-head dots).
+cudaError_t launch_refine_scores(const Dims& d, const void* q, const void* k, const int32_t* pool,
+                                 const int32_t* pool_cnt, int pool_stride, float* r, float* dots,
+                                 int32_t* status, cudaStream_t st);
+
+// Split-K attention partials over idx rows (idx == nullptr: every position).
+struct AttendPlan {
+  int splits;
+  int per_split;
+};
+AttendPlan plan_attend(const Dims& d, int64_t max_rows_per_seq);
+cudaError_t launch_attend(const Dims& d, const AttendPlan& p, const void* q, const void* k,
+                          const void* v, const int32_t* idx, const int32_t* cnt, int idx_stride,
+                          float softmax_scale, float* part_o, float* part_ml, float* out,
+                          float* lse, int32_t* status, cudaStream_t st);
+
+}  // namespace prism

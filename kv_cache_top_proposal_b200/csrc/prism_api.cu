@@ -1,0 +1,293 @@
+// C ABI of libprism.so (declared in include/prism.h): argument validation,
+// workspace layout and kernel dispatch.  Nothing here allocates device
+// memory or synchronises (prism_get_device_status excepted).
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+
+#include "../../include/prism.h"
+#include "kernels.h"
+
+namespace prism {
+namespace {
+
+// Split plans are sized for B200's 148 SMs on every device, so workspace
+// sizes (and the summation order of split-K) do not depend on the GPU.
+constexpr int kPlanSms = 148;
+constexpr int kMaxBatch = 4096;
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+prism_status check_shape(const prism_shape* s, Dims* d) {
+  if (!s || !s->cu_seqlens_dev || !s->cu_seqlens_host) return PRISM_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->batch > kMaxBatch) return PRISM_ERR_INVALID_ARG;
+  if (s->num_kv_heads < 1 || s->num_q_heads < s->num_kv_heads) return PRISM_ERR_INVALID_ARG;
+  if (s->num_q_heads % s->num_kv_heads != 0) return PRISM_ERR_INVALID_ARG;
+  if (s->num_q_heads / s->num_kv_heads > 16) return PRISM_ERR_UNSUPPORTED;
+  if (s->head_dim != 64 && s->head_dim != 128) return PRISM_ERR_UNSUPPORTED;
+  if (s->dtype != PRISM_F32 && s->dtype != PRISM_BF16) return PRISM_ERR_INVALID_ARG;
+  if (s->total_tokens < 0) return PRISM_ERR_INVALID_ARG;
+  const int32_t* cu = s->cu_seqlens_host;
+  if (cu[0] != 0) return PRISM_ERR_INVALID_ARG;
+  int max_len = 0;
+  for (int b = 0; b < s->batch; ++b) {
+    if (cu[b + 1] < cu[b]) return PRISM_ERR_INVALID_ARG;
+    const int L = cu[b + 1] - cu[b];
+    if (L > max_len) max_len = L;
+  }
+  if ((int64_t)cu[s->batch] != s->total_tokens) return PRISM_ERR_INVALID_ARG;
+  d->B = s->batch;
+  d->Hq = s->num_q_heads;
+  d->Hkv = s->num_kv_heads;
+  d->G = s->num_q_heads / s->num_kv_heads;
+  d->D = s->head_dim;
+  d->T = s->total_tokens;
+  d->bf16 = s->dtype == PRISM_BF16;
+  d->cu_dev = s->cu_seqlens_dev;
+  d->cu_host = s->cu_seqlens_host;
+  d->max_len = max_len;
+  d->num_sms = kPlanSms;
+  return PRISM_OK;
+}
+
+prism_status set_live_sms(Dims* d) {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PRISM_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return PRISM_ERR_CUDA;
+  d->num_sms = n > 0 ? n : kPlanSms;
+  return PRISM_OK;
+}
+
+prism_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PRISM_OK : PRISM_ERR_CUDA; }
+
+// Workspace layout per operation (offsets after the 256-byte header).
+struct Layout {
+  size_t a = 0, b = 0, total = 0;  // a: first array, b: second array
+};
+
+Layout layout(const Dims& d, int op, int kappa_p, int kappa) {
+  Layout L;
+  size_t off = kWsHeader;
+  const size_t rows = (size_t)d.B * d.Hkv;
+  switch (op) {
+    case PRISM_OP_QUANTIZE:
+      break;
+    case PRISM_OP_PROPOSE:  // scores [Hkv][T] fp32
+      L.a = off;
+      off = align_up(off + (size_t)d.Hkv * (size_t)d.T * sizeof(float));
+      break;
+    case PRISM_OP_REFINE:  // r [rows][kappa_p], dots [rows][G][kappa_p]
+      L.a = off;
+      off = align_up(off + rows * (size_t)kappa_p * sizeof(float));
+      L.b = off;
+      off = align_up(off + rows * (size_t)d.G * (size_t)kappa_p * sizeof(float));
+      break;
+    case PRISM_OP_SPARSE_DECODE:
+    case PRISM_OP_DENSE_DECODE: {
+      const AttendPlan p = plan_attend(d, op == PRISM_OP_SPARSE_DECODE ? kappa : d.max_len);
+      const size_t parts = (size_t)d.B * d.Hq * (size_t)p.splits;
+      L.a = off;  // partial o [B][Hq][splits][D]
+      off = align_up(off + parts * (size_t)d.D * sizeof(float));
+      L.b = off;  // partial (m, l) [B][Hq][splits][2]
+      off = align_up(off + parts * 2 * sizeof(float));
+      break;
+    }
+    default:
+      break;
+  }
+  L.total = off;
+  (void)kappa;
+  return L;
+}
+
+bool ws_ok(const void* ws, size_t ws_bytes, const Layout& L) {
+  return ws && ws_bytes >= L.total && ((uintptr_t)ws % kAlign) == 0;
+}
+
+bool use_mma_scorer() {
+  const char* e = std::getenv("PRISM_PROPOSE_SCORER");
+  return !(e && std::strcmp(e, "simt") == 0);
+}
+
+}  // namespace
+}  // namespace prism
+
+using namespace prism;
+
+extern "C" {
+
+prism_status prism_workspace_size(const prism_shape* shape, int32_t op, int32_t kappa_p,
+                                  int32_t kappa, size_t* bytes) {
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!bytes || op < PRISM_OP_QUANTIZE || op > PRISM_OP_DENSE_DECODE) return PRISM_ERR_INVALID_ARG;
+  if (op == PRISM_OP_PROPOSE && kappa_p < 1) return PRISM_ERR_INVALID_ARG;
+  if (op == PRISM_OP_REFINE && (kappa_p < 1 || kappa < 1 || kappa > kappa_p))
+    return PRISM_ERR_INVALID_ARG;
+  if (op == PRISM_OP_SPARSE_DECODE && kappa < 1) return PRISM_ERR_INVALID_ARG;
+  *bytes = layout(d, op, kappa_p, kappa).total;
+  return PRISM_OK;
+}
+
+prism_status prism_quantize_k(const prism_shape* shape, const void* k, int8_t* kq, float* k_scale,
+                              const int32_t* tok_rows, int32_t n_rows, void* ws, size_t ws_bytes,
+                              void* stream) {
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!k || !kq || !k_scale) return PRISM_ERR_INVALID_ARG;
+  if (tok_rows && n_rows < 0) return PRISM_ERR_INVALID_ARG;
+  if (ws && (ws_bytes < kWsHeader || ((uintptr_t)ws % kAlign) != 0)) return PRISM_ERR_WORKSPACE;
+  if ((s = set_live_sms(&d)) != PRISM_OK) return s;
+  const int64_t rows = tok_rows ? (int64_t)n_rows : d.T;
+  return cuda_status(launch_quantize(d, k, kq, k_scale, tok_rows, rows, static_cast<int32_t*>(ws),
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+prism_status prism_propose(const prism_shape* shape, const void* q, const int8_t* kq,
+                           const float* k_scale, int32_t kappa_p, int32_t* pool_idx,
+                           int32_t* pool_cnt, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!q || !kq || !k_scale || !pool_idx || !pool_cnt || kappa_p < 1) return PRISM_ERR_INVALID_ARG;
+  if (d.max_len > select_capacity_per_row()) return PRISM_ERR_UNSUPPORTED;
+  const Layout L = layout(d, PRISM_OP_PROPOSE, kappa_p, 0);
+  if (!ws_ok(ws, ws_bytes, L)) return PRISM_ERR_WORKSPACE;
+  if ((s = set_live_sms(&d)) != PRISM_OK) return s;
+  char* w = static_cast<char*>(ws);
+  int32_t* status = reinterpret_cast<int32_t*>(w);
+  float* scores = reinterpret_cast<float*>(w + L.a);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_propose_scores(d, q, kq, k_scale, scores, use_mma_scorer(), st);
+  if (e != cudaSuccess) return PRISM_ERR_CUDA;
+  SelectArgs a{};
+  a.mode = 0;
+  a.Hkv = d.Hkv;
+  a.G = d.G;
+  a.Hq = d.Hq;
+  a.T = d.T;
+  a.cu = d.cu_dev;
+  a.keys = scores;
+  a.k_req = kappa_p;
+  a.out = pool_idx;
+  a.out_cnt = pool_cnt;
+  a.status = status;
+  return cuda_status(launch_select(d, a, d.max_len, st));
+}
+
+prism_status prism_refine(const prism_shape* shape, const void* q, const void* k,
+                          const int32_t* pool_idx, const int32_t* pool_cnt, int32_t kappa_p,
+                          int32_t kappa, int32_t* idx, int32_t* cnt, float* logits_opt, void* ws,
+                          size_t ws_bytes, void* stream) {
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!q || !k || !pool_idx || !pool_cnt || !idx || !cnt) return PRISM_ERR_INVALID_ARG;
+  if (kappa_p < 1 || kappa < 1 || kappa > kappa_p) return PRISM_ERR_INVALID_ARG;
+  if (kappa_p > select_capacity_per_row()) return PRISM_ERR_UNSUPPORTED;
+  const Layout L = layout(d, PRISM_OP_REFINE, kappa_p, kappa);
+  if (!ws_ok(ws, ws_bytes, L)) return PRISM_ERR_WORKSPACE;
+  if ((s = set_live_sms(&d)) != PRISM_OK) return s;
+  char* w = static_cast<char*>(ws);
+  int32_t* status = reinterpret_cast<int32_t*>(w);
+  float* r = reinterpret_cast<float*>(w + L.a);
+  float* dots = logits_opt ? reinterpret_cast<float*>(w + L.b) : nullptr;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_refine_scores(d, q, k, pool_idx, pool_cnt, kappa_p, r, dots, status, st);
+  if (e != cudaSuccess) return PRISM_ERR_CUDA;
+  SelectArgs a{};
+  a.mode = 1;
+  a.Hkv = d.Hkv;
+  a.G = d.G;
+  a.Hq = d.Hq;
+  a.T = d.T;
+  a.cu = d.cu_dev;
+  a.keys = r;
+  a.pool = pool_idx;
+  a.pool_cnt = pool_cnt;
+  a.pool_stride = kappa_p;
+  a.k_req = kappa;
+  a.out = idx;
+  a.out_cnt = cnt;
+  a.dots = dots;
+  a.logits = logits_opt;
+  a.status = status;
+  return cuda_status(launch_select(d, a, kappa_p, st));
+}
+
+prism_status prism_sparse_decode(const prism_shape* shape, const void* q, const void* k,
+                                 const void* v, const int32_t* idx, const int32_t* cnt,
+                                 int32_t kappa, float softmax_scale, float* out, float* lse_opt,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!q || !k || !v || !idx || !cnt || !out || kappa < 1) return PRISM_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return PRISM_ERR_INVALID_ARG;
+  const Layout L = layout(d, PRISM_OP_SPARSE_DECODE, 0, kappa);
+  if (!ws_ok(ws, ws_bytes, L)) return PRISM_ERR_WORKSPACE;
+  const AttendPlan p = plan_attend(d, kappa);
+  if ((s = set_live_sms(&d)) != PRISM_OK) return s;
+  char* w = static_cast<char*>(ws);
+  return cuda_status(launch_attend(d, p, q, k, v, idx, cnt, kappa, softmax_scale,
+                                   reinterpret_cast<float*>(w + L.a),
+                                   reinterpret_cast<float*>(w + L.b), out, lse_opt,
+                                   reinterpret_cast<int32_t*>(w), static_cast<cudaStream_t>(stream)));
+}
+
+prism_status prism_dense_decode(const prism_shape* shape, const void* q, const void* k,
+                                const void* v, float softmax_scale, float* out, float* lse_opt,
+                                void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!q || !k || !v || !out) return PRISM_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return PRISM_ERR_INVALID_ARG;
+  const Layout L = layout(d, PRISM_OP_DENSE_DECODE, 0, 0);
+  if (!ws_ok(ws, ws_bytes, L)) return PRISM_ERR_WORKSPACE;
+  const AttendPlan p = plan_attend(d, d.max_len);
+  if ((s = set_live_sms(&d)) != PRISM_OK) return s;
+  char* w = static_cast<char*>(ws);
+  return cuda_status(launch_attend(d, p, q, k, v, nullptr, nullptr, 0, softmax_scale,
+                                   reinterpret_cast<float*>(w + L.a),
+                                   reinterpret_cast<float*>(w + L.b), out, lse_opt,
+                                   reinterpret_cast<int32_t*>(w), static_cast<cudaStream_t>(stream)));
+}
+
+prism_status prism_clear_device_status(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < kWsHeader) return PRISM_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(ws, 0, kWsHeader, static_cast<cudaStream_t>(stream)));
+}
+
+prism_status prism_get_device_status(const void* ws, size_t ws_bytes, void* stream,
+                                     int32_t* code) {
+  if (!ws || ws_bytes < kWsHeader) return PRISM_ERR_WORKSPACE;
+  if (!code) return PRISM_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return PRISM_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PRISM_ERR_CUDA;
+  *code = v;
+  return PRISM_OK;
+}
+
+const char* prism_status_str(prism_status s) {
+  switch (s) {
+    case PRISM_OK: return "ok";
+    case PRISM_ERR_INVALID_ARG: return "invalid argument";
+    case PRISM_ERR_UNSUPPORTED: return "unsupported shape or size";
+    case PRISM_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case PRISM_ERR_CUDA: return "CUDA launch or runtime error";
+    case PRISM_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

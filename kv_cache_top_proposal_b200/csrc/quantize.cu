@@ -1,0 +1,109 @@
+// Per-token symmetric int8 quantization of the key cache (Prism Attention,
+// sec. 4.2 "Quantized Proposal Construction"; int8 per-token scheme because
+// the pages do not state their INT2 one).
+//
+// One row of d elements is spread over d*sizeof(T)/16 lanes, each holding one
+// 16-byte vector: a coalesced read of the row, a shuffle max for amax, IEEE
+// divisions and round-half-even, one 8- or 4-byte store of codes per lane.
+// HBM bound: reads d*sizeof(T) and writes d + 4 bytes per row.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace prism {
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ k,
+                                                       int8_t* __restrict__ kq,
+                                                       float* __restrict__ scale, int64_t T_tok,
+                                                       int Hkv, const int32_t* __restrict__ tok_rows,
+                                                       int64_t n_rows, int32_t* status) {
+  constexpr int E = Vec16<T>::E;
+  constexpr int LPR = D / E;  // lanes per row
+  constexpr int RPW = 32 / LPR;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / LPR, li = lane % LPR;
+  const int64_t rows_total = (int64_t)Hkv * n_rows;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t base = warp0 * RPW; base < rows_total; base += nwarps * RPW) {
+    const int64_t r = base + sub;
+    bool valid = r < rows_total;
+    int64_t row = 0;
+    if (valid) {
+      const int64_t h = r / n_rows, i = r - h * n_rows;
+      const int64_t t = tok_rows ? (int64_t)tok_rows[i] : i;
+      if (t < 0 || t >= T_tok) {
+        if (li == 0) flag_status(status, PRISM_DEV_BAD_INDEX);
+        valid = false;
+      }
+      row = h * T_tok + t;
+    }
+    float f[E];
+    if (valid) {
+      Vec16<T>::unpack(ld16_stream(k + row * D + li * E), f);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) f[e] = 0.0f;
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(f[e]));
+#pragma unroll
+    for (int o = LPR / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = __fdiv_rn(amax, 127.0f);
+    uint32_t packed[E / 4];
+#pragma unroll
+    for (int w = 0; w < E / 4; ++w) {
+      uint32_t acc = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        int c = 0;
+        if (amax != 0.0f) {
+          float y = rintf(__fdiv_rn(f[w * 4 + e], s));
+          y = fminf(fmaxf(y, -127.0f), 127.0f);
+          c = (int)y;
+        }
+        acc |= ((uint32_t)(c & 0xFF)) << (8 * e);
+      }
+      packed[w] = acc;
+    }
+    if (valid) {
+      int8_t* dst = kq + row * D + li * E;
+      if constexpr (E == 8) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+      } else {
+        *reinterpret_cast<uint32_t*>(dst) = packed[0];
+      }
+      if (li == 0) scale[row] = (amax != 0.0f) ? s : 0.0f;
+    }
+  }
+}
+
+template <typename T, int D>
+static cudaError_t run(const Dims& d, const void* k, int8_t* kq, float* scale, const int32_t* tok,
+                       int64_t n_rows, int32_t* status, cudaStream_t st) {
+  constexpr int LPR = D / Vec16<T>::E;
+  const int64_t rows = (int64_t)d.Hkv * n_rows;
+  const int64_t warps = cdiv(rows, 32 / LPR);
+  int64_t blocks = cdiv(warps, 8);
+  const int64_t cap = (int64_t)d.num_sms * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  quantize_kernel<T, D><<<(unsigned)blocks, 256, 0, st>>>(
+      static_cast<const T*>(k), kq, scale, d.T, d.Hkv, tok, n_rows, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const Dims& d, const void* k, int8_t* kq, float* scale,
+                            const int32_t* tok_rows, int64_t n_rows, int32_t* status,
+                            cudaStream_t st) {
+  if (n_rows == 0 || d.Hkv == 0) return cudaSuccess;
+  if (d.bf16) {
+    return d.D == 128 ? run<__nv_bfloat16, 128>(d, k, kq, scale, tok_rows, n_rows, status, st)
+                      : run<__nv_bfloat16, 64>(d, k, kq, scale, tok_rows, n_rows, status, st);
+  }
+  return d.D == 128 ? run<float, 128>(d, k, kq, scale, tok_rows, n_rows, status, st)
+                    : run<float, 64>(d, k, kq, scale, tok_rows, n_rows, status, st);
+}
+
+}  // namespace prism

@@ -1,0 +1,152 @@
+// Exact rescoring of the candidate pool at every layer (Prism Attention,
+// sec. 4.1 "Proposal-Refined Index Sharing"; sec. 6: refined layers re-select
+// their own top-kappa inside the proposed region at a cost independent of
+// context length):
+//   r[row][i] = max_g sum_j q[b][h*G+g][j] * K[h][cu[b] + pool[row][i]][j]
+// with fp32 accumulation (bf16 x bf16 products are exact in fp32).  The
+// per-head dot products are kept as well when the caller wants logits.
+//
+// A gather of kappa_p key rows per (sequence, KV head): d*sizeof(T) bytes per
+// pool member, 256 B at bf16 d = 128.  A row is spread over d*sizeof(T)/16
+// lanes with one 16-byte load each; four rows per lane group are in flight.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace prism {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kUnroll = 4;
+
+struct RefineArgs {
+  const void* q;
+  const void* k;
+  const int32_t* cu;
+  const int32_t* pool;
+  const int32_t* pool_cnt;
+  int pool_stride;
+  int Hkv, G;
+  int64_t T;
+  int per_cta;
+  float* r;
+  float* dots;
+  int32_t* status;
+};
+
+template <typename T, int D, int GP>
+__global__ void __launch_bounds__(kThreads) refine_score_kernel(const RefineArgs a) {
+  constexpr int E = Vec16<T>::E;
+  constexpr int LPR = D / E;
+  constexpr int RPW = 32 / LPR;
+  const int row = blockIdx.y;
+  const int b = row / a.Hkv, h = row - b * a.Hkv;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane / LPR, li = lane % LPR;
+  int n = a.pool_cnt[row];
+  n = n < 0 ? 0 : (n > a.pool_stride ? a.pool_stride : n);
+  const int e0 = blockIdx.x * a.per_cta;
+  const int e1 = min(n, e0 + a.per_cta);
+  if (e0 >= e1) return;
+  const int t0 = a.cu[b];
+  const int L = a.cu[b + 1] - t0;
+  const T* kbase = static_cast<const T*>(a.k) + ((int64_t)h * a.T + t0) * D + li * E;
+  const T* q = static_cast<const T*>(a.q) + ((int64_t)b * a.Hkv * a.G + (int64_t)h * a.G) * D;
+  const int32_t* pool = a.pool + (int64_t)row * a.pool_stride;
+
+  float qf[GP][E];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    if (g < a.G) {
+      Vec16<T>::unpack(ld16(q + (int64_t)g * D + li * E), qf[g]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) qf[g][e] = 0.0f;
+    }
+  }
+
+  for (int base = e0 + warp * RPW * kUnroll; base < e1; base += kWarps * RPW * kUnroll) {
+    uint4 raw[kUnroll];
+    bool ok[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int e = base + u * RPW + sub;
+      ok[u] = e < e1;
+      int pos = ok[u] ? pool[e] : 0;
+      if (ok[u] && (pos < 0 || pos >= L)) {
+        if (li == 0) flag_status(a.status, PRISM_DEV_BAD_INDEX);
+        ok[u] = false;
+        pos = 0;
+      }
+      raw[u] = ok[u] ? ld16(kbase + (int64_t)pos * D) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      float f[E];
+      Vec16<T>::unpack(raw[u], f);
+      float acc[GP];
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float s = 0.0f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) s = fmaf(qf[g][e], f[e], s);
+        acc[g] = group_sum<LPR>(s);
+      }
+      float best = acc[0];
+#pragma unroll
+      for (int g = 1; g < GP; ++g)
+        if (g < a.G) best = fmaxf(best, acc[g]);
+      const int e = base + u * RPW + sub;
+      if (e < e1 && li == 0) {
+        a.r[(int64_t)row * a.pool_stride + e] = ok[u] ? best : -INFINITY;
+        if (a.dots) {
+#pragma unroll
+          for (int g = 0; g < GP; ++g)
+            if (g < a.G) a.dots[((int64_t)row * a.G + g) * a.pool_stride + e] = acc[g];
+        }
+      }
+    }
+  }
+}
+
+template <typename T, int D, int GP>
+cudaError_t run(const Dims& d, const RefineArgs& a0, cudaStream_t st) {
+  constexpr int RPW = 32 / (D / Vec16<T>::E);
+  constexpr int step = kWarps * RPW * kUnroll;
+  RefineArgs a = a0;
+  const int rows = d.B * d.Hkv;
+  const int64_t target = 2LL * d.num_sms;
+  int64_t per = cdiv((int64_t)a.pool_stride * rows, target);
+  per = cdiv(per, step) * step;
+  if (per < step) per = step;
+  a.per_cta = (int)per;
+  const int splits = (int)cdiv(a.pool_stride, per);
+  refine_score_kernel<T, D, GP><<<dim3(splits, rows), kThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t by_group(const Dims& d, const RefineArgs& a, cudaStream_t st) {
+  switch (padded_group(d.G)) {
+    case 1: return run<T, D, 1>(d, a, st);
+    case 2: return run<T, D, 2>(d, a, st);
+    case 4: return run<T, D, 4>(d, a, st);
+    case 8: return run<T, D, 8>(d, a, st);
+    default: return run<T, D, 16>(d, a, st);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_refine_scores(const Dims& d, const void* q, const void* k, const int32_t* pool,
+                                 const int32_t* pool_cnt, int pool_stride, float* r, float* dots,
+                                 int32_t* status, cudaStream_t st) {
+  if (d.B * d.Hkv == 0 || pool_stride == 0) return cudaSuccess;
+  RefineArgs a{q, k, d.cu_dev, pool, pool_cnt, pool_stride, d.Hkv, d.G, d.T, 0, r, dots, status};
+  if (d.bf16)
+    return d.D == 128 ? by_group<__nv_bfloat16, 128>(d, a, st) : by_group<__nv_bfloat16, 64>(d, a, st);
+  return d.D == 128 ? by_group<float, 128>(d, a, st) : by_group<float, 64>(d, a, st);
+}
+
+}  // namespace prism

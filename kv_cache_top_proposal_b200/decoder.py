@@ -1,0 +1,101 @@
+"""One decode step of Prism Attention over every layer, through the C ABI.
+
+Layer schedule (Prism Attention, sec. 5.3 "Accuracy-efficiency trade-off":
+in the "g x" setting one layer in every x is a proposal layer; the pages
+inherit the partition from an offline calibration, sec. 4 Overview, which is
+replaced here by the periodic map ``layer % group == 0``):
+
+  proposal layer l:  quantize the newly appended key row of every sequence
+                     (prism_quantize_k on the last position), then
+                     prism_propose -> candidate pool of kappa_p positions;
+  every layer l:     prism_refine on the latest pool -> kappa positions,
+                     prism_sparse_decode over them -> out[l], lse[l].
+
+A proposal layer also refines its own pool and attends over the refined set
+(every layer attends over kappa exactly rescored tokens).  All buffers are
+allocated once by torch; a step only enqueues library calls on one stream,
+so it can be captured in a CUDA graph.
+"""
+from __future__ import annotations
+
+import math
+from typing import List, Optional
+
+import torch
+
+from . import prism
+
+
+class PrismDecoder:
+    def __init__(self, seqlens, num_q_heads: int, num_kv_heads: int, head_dim: int, dtype: int,
+                 num_layers: int, group: int, kappa_p: int, kappa: int, device="cuda",
+                 softmax_scale: Optional[float] = None):
+        self.dev = torch.device(device)
+        self.p = prism.Problem(seqlens, num_q_heads, num_kv_heads, head_dim, dtype, device=self.dev)
+        self.B, self.Hq, self.Hkv, self.D = len(seqlens), num_q_heads, num_kv_heads, head_dim
+        self.num_layers, self.group = num_layers, group
+        self.kappa_p, self.kappa = kappa_p, kappa
+        self.scale = float(torch.tensor(1.0 / math.sqrt(head_dim), dtype=torch.float32)) \
+            if softmax_scale is None else float(softmax_scale)
+        B, Hkv, Hq, D = self.B, self.Hkv, self.Hq, self.D
+        i32 = dict(dtype=torch.int32, device=self.dev)
+        f32 = dict(dtype=torch.float32, device=self.dev)
+        self.proposal_layers = [l for l in range(num_layers) if l % group == 0]
+        self.pool = {l: torch.full((B, Hkv, kappa_p), -1, **i32) for l in self.proposal_layers}
+        self.pool_cnt = {l: torch.zeros((B, Hkv), **i32) for l in self.proposal_layers}
+        self.idx = [torch.full((B, Hkv, kappa), -1, **i32) for _ in range(num_layers)]
+        self.cnt = [torch.zeros((B, Hkv), **i32) for _ in range(num_layers)]
+        self.out = [torch.zeros((B, Hq, D), **f32) for _ in range(num_layers)]
+        self.lse = [torch.zeros((B, Hq), **f32) for _ in range(num_layers)]
+        # the newly appended token of every sequence (packed row index)
+        last = [c - 1 for c in self.p.cu_host[1:].tolist() if True]
+        self.new_rows = torch.tensor([r for r, L in zip(last, seqlens) if L > 0], **i32)
+
+        def ws(op, kp=0, k=0):
+            n = prism.workspace_size(self.p, op, kp, k)
+            return torch.zeros(n, dtype=torch.uint8, device=self.dev)
+
+        self.ws_q = ws(prism.OP_QUANTIZE)
+        self.ws_prop = ws(prism.OP_PROPOSE, kappa_p)
+        self.ws_ref = ws(prism.OP_REFINE, kappa_p, kappa)
+        self.ws_dec = ws(prism.OP_SPARSE_DECODE, 0, kappa)
+        self.ws_dense = None
+
+    def workspaces(self) -> List[torch.Tensor]:
+        return [w for w in (self.ws_q, self.ws_prop, self.ws_ref, self.ws_dec, self.ws_dense)
+                if w is not None]
+
+    def layer(self, l: int, q, k, v, kq=None, k_scale=None, quantize_new: bool = True,
+              stream=None):
+        """Enqueue one layer of the step (kq/k_scale required at proposal layers)."""
+        p = self.p
+        if l % self.group == 0:
+            if quantize_new and self.new_rows.numel():
+                prism.quantize_k(p, k, kq, k_scale, tok_rows=self.new_rows, ws=self.ws_q, stream=stream)
+            prism.propose(p, q, kq, k_scale, self.kappa_p, self.pool[l], self.pool_cnt[l],
+                          self.ws_prop, stream=stream)
+        src = l - l % self.group
+        prism.refine(p, q, k, self.pool[src], self.pool_cnt[src], self.kappa_p, self.kappa,
+                     self.idx[l], self.cnt[l], self.ws_ref, stream=stream)
+        prism.sparse_decode(p, q, k, v, self.idx[l], self.cnt[l], self.kappa, self.scale,
+                            self.out[l], self.ws_dec, lse=self.lse[l], stream=stream)
+
+    def step(self, qs, ks, vs, kqs, scales, quantize_new: bool = True, stream=None):
+        """One decode step over every layer.  qs/ks/vs are per-layer lists;
+        kqs/scales are dicts (or lists) indexed by proposal layer."""
+        for l in range(self.num_layers):
+            pl = l % self.group == 0
+            self.layer(l, qs[l], ks[l], vs[l], kqs[l] if pl else None, scales[l] if pl else None,
+                       quantize_new=quantize_new, stream=stream)
+
+    def dense_layer(self, l: int, q, k, v, out, lse=None, stream=None):
+        if self.ws_dense is None:
+            n = prism.workspace_size(self.p, prism.OP_DENSE_DECODE)
+            self.ws_dense = torch.zeros(n, dtype=torch.uint8, device=self.dev)
+        prism.dense_decode(self.p, q, k, v, self.scale, out, self.ws_dense, lse=lse, stream=stream)
+
+    def device_status(self) -> int:
+        s = 0
+        for w in self.workspaces():
+            s |= prism.get_device_status(w)
+        return s

@@ -1,0 +1,176 @@
+"""Thin ctypes binding of libprism.so (C ABI in include/prism.h).
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+Tensors are torch tensors on the GPU; the binding passes their data
+pointers, sizes and the current CUDA stream, and raises ``PrismError`` for a
+non-OK status.  There is no fallback: if the library is missing the import
+fails with instructions to build it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libprism.so")
+
+F32, BF16 = 0, 1
+OP_QUANTIZE, OP_PROPOSE, OP_REFINE, OP_SPARSE_DECODE, OP_DENSE_DECODE = range(5)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+DEV_BAD_INDEX, DEV_TOO_LONG = 0x1, 0x2
+MAX_SELECT_ROW = 393216
+WS_HEADER = 256
+
+EXPORTS = ("prism_workspace_size", "prism_quantize_k", "prism_propose", "prism_refine",
+           "prism_sparse_decode", "prism_dense_decode", "prism_clear_device_status",
+           "prism_get_device_status", "prism_status_str")
+
+
+class PrismError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_lib.prism_status_str(status).decode()} (status {status})")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("cu_seqlens_dev", ctypes.c_void_p),
+                ("cu_seqlens_host", ctypes.c_void_p), ("total_tokens", ctypes.c_int64)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m kv_cache_top_proposal_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, S, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32
+    sp = ctypes.POINTER(Shape)
+    sig = {
+        "prism_workspace_size": [sp, i32, i32, i32, ctypes.POINTER(ctypes.c_size_t)],
+        "prism_quantize_k": [sp, P, P, P, P, i32, P, S, P],
+        "prism_propose": [sp, P, P, P, i32, P, P, P, S, P],
+        "prism_refine": [sp, P, P, P, P, i32, i32, P, P, P, P, S, P],
+        "prism_sparse_decode": [sp, P, P, P, P, P, i32, ctypes.c_float, P, P, P, S, P],
+        "prism_dense_decode": [sp, P, P, P, ctypes.c_float, P, P, P, S, P],
+        "prism_clear_device_status": [P, S, P],
+        "prism_get_device_status": [P, S, P, ctypes.POINTER(ctypes.c_int32)],
+    }
+    for name, args in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    lib.prism_status_str.argtypes = [ctypes.c_int]
+    lib.prism_status_str.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+
+def library():
+    return _lib
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise PrismError(status, where)
+
+
+class Problem:
+    """A layer-shape descriptor (the C ``prism_shape``) plus its cu_seqlens.
+
+    ``seqlens`` are the per-sequence context lengths; the device copy of
+    cu_seqlens lives on ``device`` and the host mirror in a numpy array that
+    this object keeps alive.
+    """
+
+    def __init__(self, seqlens: Sequence[int], num_q_heads: int, num_kv_heads: int, head_dim: int,
+                 dtype: int, device="cuda", cu_dev=None):
+        import torch
+
+        cu = np.zeros(len(seqlens) + 1, np.int32)
+        cu[1:] = np.cumsum(np.asarray(seqlens, np.int64)).astype(np.int32)
+        self.cu_host = cu
+        self.cu_dev = cu_dev if cu_dev is not None else torch.tensor(cu, dtype=torch.int32, device=device)
+        self.seqlens = [int(x) for x in seqlens]
+        self.shape = Shape(len(seqlens), num_q_heads, num_kv_heads, head_dim, dtype,
+                           ctypes.c_void_p(self.cu_dev.data_ptr()),
+                           ctypes.c_void_p(cu.ctypes.data), int(cu[-1]))
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.shape)
+
+    @property
+    def total_tokens(self) -> int:
+        return int(self.cu_host[-1])
+
+
+def workspace_size(p: Problem, op: int, kappa_p: int = 0, kappa: int = 0) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.prism_workspace_size(p.ref, op, kappa_p, kappa, ctypes.byref(n)), "workspace_size")
+    return n.value
+
+
+def _nbytes(ws) -> int:
+    return 0 if ws is None else ws.numel() * ws.element_size()
+
+
+def quantize_k(p: Problem, k, kq, k_scale, tok_rows=None, ws=None, stream=None):
+    n = 0 if tok_rows is None else int(tok_rows.numel())
+    _check(_lib.prism_quantize_k(p.ref, _ptr(k), _ptr(kq), _ptr(k_scale), _ptr(tok_rows), n,
+                                 _ptr(ws), _nbytes(ws), _stream(stream)), "quantize_k")
+
+
+def propose(p: Problem, q, kq, k_scale, kappa_p: int, pool, pool_cnt, ws, stream=None):
+    _check(_lib.prism_propose(p.ref, _ptr(q), _ptr(kq), _ptr(k_scale), kappa_p, _ptr(pool),
+                              _ptr(pool_cnt), _ptr(ws), _nbytes(ws), _stream(stream)), "propose")
+
+
+def refine(p: Problem, q, k, pool, pool_cnt, kappa_p: int, kappa: int, idx, cnt, ws, logits=None,
+           stream=None):
+    _check(_lib.prism_refine(p.ref, _ptr(q), _ptr(k), _ptr(pool), _ptr(pool_cnt), kappa_p, kappa,
+                             _ptr(idx), _ptr(cnt), _ptr(logits), _ptr(ws), _nbytes(ws),
+                             _stream(stream)), "refine")
+
+
+def sparse_decode(p: Problem, q, k, v, idx, cnt, kappa: int, softmax_scale: float, out, ws,
+                  lse=None, stream=None):
+    _check(_lib.prism_sparse_decode(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt), kappa,
+                                    float(softmax_scale), _ptr(out), _ptr(lse), _ptr(ws),
+                                    _nbytes(ws), _stream(stream)), "sparse_decode")
+
+
+def dense_decode(p: Problem, q, k, v, softmax_scale: float, out, ws, lse=None, stream=None):
+    _check(_lib.prism_dense_decode(p.ref, _ptr(q), _ptr(k), _ptr(v), float(softmax_scale),
+                                   _ptr(out), _ptr(lse), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "dense_decode")
+
+
+def clear_device_status(ws, stream=None):
+    _check(_lib.prism_clear_device_status(_ptr(ws), _nbytes(ws), _stream(stream)), "clear_status")
+
+
+def get_device_status(ws, stream=None) -> int:
+    c = ctypes.c_int32(0)
+    _check(_lib.prism_get_device_status(_ptr(ws), _nbytes(ws), _stream(stream), ctypes.byref(c)),
+           "get_device_status")
+    return c.value

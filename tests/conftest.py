@@ -28,3 +28,14 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+@pytest.fixture(scope="session")
+def prism_lib():
+    """The built C-ABI library (built in-tree on first use)."""
+    from kv_cache_top_proposal_b200 import build
+
+    build.build()
+    from kv_cache_top_proposal_b200 import prism
+
+    return prism

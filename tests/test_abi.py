@@ -1,0 +1,124 @@
+"""The C-ABI library: it loads, exports every declared entry point, and
+rejects bad host-checkable arguments before touching the GPU (these tests
+run without a device: validation never dereferences device pointers)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x10000  # a non-null "device pointer" that validation never reads
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "prism.h")).read()
+    return re.findall(r"PRISM_API\s+[\w\s\*]+?\b(prism_\w+)\s*\(", src)
+
+
+def test_exports_every_declared_symbol(prism_lib):
+    names = _declared()
+    assert len(names) >= 9
+    lib = prism_lib.library()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(prism_lib.EXPORTS)
+
+
+def _shape(prism, seqlens, hq=32, hkv=8, d=128, dtype=1):
+    cu = np.zeros(len(seqlens) + 1, np.int32)
+    cu[1:] = np.cumsum(seqlens)
+    s = prism.Shape(len(seqlens), hq, hkv, d, dtype, ctypes.c_void_p(FAKE),
+                    ctypes.c_void_p(cu.ctypes.data), int(cu[-1]))
+    return s, cu
+
+
+def _ws(prism, s, op, kp=0, k=0):
+    n = ctypes.c_size_t(0)
+    st = prism.library().prism_workspace_size(ctypes.byref(s), op, kp, k, ctypes.byref(n))
+    return st, n.value
+
+
+def test_workspace_sizes(prism_lib):
+    P = prism_lib
+    s, cu = _shape(P, [1000, 3000])
+    st, n = _ws(P, s, P.OP_PROPOSE, 256)
+    assert st == P.OK and n >= 256 + 8 * 4000 * 4 and n % 256 == 0
+    st, n = _ws(P, s, P.OP_REFINE, 256, 64)
+    assert st == P.OK and n >= 256 + 2 * 8 * 256 * 4 * (1 + 4)
+    st, n0 = _ws(P, s, P.OP_QUANTIZE)
+    assert st == P.OK and n0 == 256
+    st, n = _ws(P, s, P.OP_SPARSE_DECODE, 0, 64)
+    assert st == P.OK and n > 256
+    st, n = _ws(P, s, P.OP_DENSE_DECODE)
+    assert st == P.OK and n > 256
+
+
+@pytest.mark.parametrize("bad", [
+    dict(hq=30, hkv=8), dict(hq=4, hkv=8), dict(d=96), dict(dtype=7), dict(hq=8 * 17, hkv=8),
+])
+def test_bad_shapes_rejected(prism_lib, bad):
+    P = prism_lib
+    kw = dict(hq=32, hkv=8, d=128, dtype=1)
+    kw.update(bad)
+    s, cu = _shape(P, [100], **kw)
+    st, _ = _ws(P, s, P.OP_PROPOSE, 16)
+    assert st in (P.ERR_INVALID_ARG, P.ERR_UNSUPPORTED)
+
+
+def test_bad_cu_seqlens_rejected(prism_lib):
+    P = prism_lib
+    s, cu = _shape(P, [100, 50])
+    cu[1] = 200  # not monotone
+    assert _ws(P, s, P.OP_PROPOSE, 16)[0] == P.ERR_INVALID_ARG
+    s, cu = _shape(P, [100, 50])
+    s.total_tokens = 151  # disagrees with cu[B]
+    assert _ws(P, s, P.OP_PROPOSE, 16)[0] == P.ERR_INVALID_ARG
+    s, cu = _shape(P, [100])
+    cu[0] = 1
+    assert _ws(P, s, P.OP_PROPOSE, 16)[0] == P.ERR_INVALID_ARG
+
+
+def test_calls_validate_before_launch(prism_lib):
+    P = prism_lib
+    lib = P.library()
+    s, cu = _shape(P, [4096])
+    ref = ctypes.byref(s)
+    f = ctypes.c_void_p(FAKE)
+    _, nprop = _ws(P, s, P.OP_PROPOSE, 1024)
+    ws = ctypes.c_void_p(FAKE)  # 256-aligned fake workspace
+    # null pointers
+    assert lib.prism_propose(ref, None, f, f, 1024, f, f, ws, nprop, None) == P.ERR_INVALID_ARG
+    # kappa_p < 1
+    assert lib.prism_propose(ref, f, f, f, 0, f, f, ws, nprop, None) == P.ERR_INVALID_ARG
+    # workspace too small / misaligned
+    assert lib.prism_propose(ref, f, f, f, 1024, f, f, ws, nprop - 1, None) == P.ERR_WORKSPACE
+    assert lib.prism_propose(ref, f, f, f, 1024, f, f, ctypes.c_void_p(FAKE + 4), nprop,
+                             None) == P.ERR_WORKSPACE
+    # kappa > kappa_p
+    _, nref = _ws(P, s, P.OP_REFINE, 256, 64)
+    assert lib.prism_refine(ref, f, f, f, f, 256, 512, f, f, None, ws, nref, None) == P.ERR_INVALID_ARG
+    assert lib.prism_refine(ref, f, f, f, f, 256, 0, f, f, None, ws, nref, None) == P.ERR_INVALID_ARG
+    # non-finite softmax scale
+    _, ndec = _ws(P, s, P.OP_SPARSE_DECODE, 0, 64)
+    assert lib.prism_sparse_decode(ref, f, f, f, f, f, 64, float("nan"), f, None, ws, ndec,
+                                   None) == P.ERR_INVALID_ARG
+    assert lib.prism_dense_decode(ref, f, f, None, 0.1, f, None, ws, 1 << 30, None) == P.ERR_INVALID_ARG
+    assert lib.prism_quantize_k(ref, f, None, f, None, 0, None, 0, None) == P.ERR_INVALID_ARG
+    assert lib.prism_get_device_status(None, 0, None, None) == P.ERR_WORKSPACE
+
+
+def test_too_long_rows_unsupported(prism_lib):
+    P = prism_lib
+    s, cu = _shape(P, [P.MAX_SELECT_ROW + 1])
+    _, n = _ws(P, s, P.OP_PROPOSE, 1024)
+    f = ctypes.c_void_p(FAKE)
+    assert P.library().prism_propose(ctypes.byref(s), f, f, f, 1024, f, f, f, n, None) == P.ERR_UNSUPPORTED
+
+
+def test_status_strings(prism_lib):
+    lib = prism_lib.library()
+    for code in range(6):
+        assert lib.prism_status_str(code)
+    assert b"workspace" in lib.prism_status_str(prism_lib.ERR_WORKSPACE)

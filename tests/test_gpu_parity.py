@@ -1,0 +1,313 @@
+"""CUDA path vs the CPU oracle, stage by stage, on identical inputs.
+
+Every stage gets the same inputs on both sides (the GPU's own upstream index
+set is handed to the oracle for the downstream stage, so a permitted
+near-tie swap upstream cannot cascade).  Quantized keys and scales must be
+bit-exact; index sets may differ only by near-ties (parity_util); attention
+outputs must agree within 2e-3 max-abs for bf16 caches and 1e-5 for fp32.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import pipeline
+from parity_util import atol_for, check_index_set
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def P(prism_lib):
+    return prism_lib
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy() if t.dtype not in (torch.int32, torch.int8, torch.int64) \
+        else t.detach().cpu().numpy()
+
+
+def make_case(seqlens, hq, hkv, d, dtype, seed=0, scale_rows=False):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    T = int(sum(seqlens))
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    q = torch.randn((len(seqlens), hq, d), generator=g)
+    k = torch.randn((hkv, T, d), generator=g)
+    v = torch.randn((hkv, T, d), generator=g)
+    if scale_rows:
+        k = k * torch.exp(torch.randn((hkv, T, 1), generator=g) * 3)
+    return q.to(tdt).to(DEV), k.to(tdt).to(DEV), v.to(tdt).to(DEV)
+
+
+def problem(P, seqlens, hq, hkv, d, dtype):
+    return P.Problem(seqlens, hq, hkv, d, P.BF16 if dtype == "bf16" else P.F32, device=DEV)
+
+
+def ws_for(P, prob, op, kp=0, k=0):
+    w = torch.zeros(P.workspace_size(prob, op, kp, k), dtype=torch.uint8, device=DEV)
+    return w
+
+
+# ------------------------------------------------------------------ quantize
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("d", [64, 128])
+def test_quantize_bit_exact(P, dtype, d):
+    seqlens = [1000, 37, 0, 2049]
+    prob = problem(P, seqlens, 8, 4, d, dtype)
+    _, k, _ = make_case(seqlens, 8, 4, d, dtype, seed=1, scale_rows=True)
+    k[0, 5] = 0  # an all-zero row
+    k[1, 7, :] = 0
+    k[1, 7, 3] = -2.5e-3
+    T = prob.total_tokens
+    kq = torch.zeros((4, T, d), dtype=torch.int8, device=DEV)
+    sc = torch.zeros((4, T), dtype=torch.float32, device=DEV)
+    ws = ws_for(P, prob, P.OP_QUANTIZE)
+    P.quantize_k(prob, k, kq, sc, ws=ws)
+    okq, osc = oracle.quantize_rows(_np(k).reshape(-1, d))
+    assert np.array_equal(_np(kq).reshape(-1, d), okq)
+    assert np.array_equal(_np(sc).reshape(-1).view(np.uint32), osc.view(np.uint32))
+    # token-row path: only the listed rows change
+    rows = torch.tensor([0, 999, 1037, T - 1], dtype=torch.int32, device=DEV)
+    kq2 = torch.full_like(kq, 55)
+    sc2 = torch.full_like(sc, -1.0)
+    P.quantize_k(prob, k, kq2, sc2, tok_rows=rows, ws=ws)
+    r = rows.cpu().numpy()
+    assert np.array_equal(_np(kq2)[:, r], _np(kq)[:, r])
+    assert np.array_equal(_np(sc2)[:, r], _np(sc)[:, r])
+    mask = np.ones(T, bool)
+    mask[r] = False
+    assert np.all(_np(kq2)[:, mask] == 55) and np.all(_np(sc2)[:, mask] == -1.0)
+    assert P.get_device_status(ws) == 0
+
+
+# ------------------------------------------------------------------ propose
+
+PROPOSE_CASES = [
+    # seqlens, hq, hkv, d, dtype, kappa_p
+    ([1024], 4, 1, 64, "f32", 256),
+    ([5000, 1031, 0, 300], 8, 2, 128, "bf16", 1024),
+    ([3000, 777], 8, 8, 64, "bf16", 200),       # G = 1
+    ([2500], 64, 8, 128, "bf16", 333),          # G = 8
+    ([1800], 32, 2, 64, "bf16", 500),           # G = 16
+    ([1024, 1025, 1023], 16, 4, 128, "bf16", 1024),  # L == kappa_p, +-1
+    ([40000], 8, 2, 128, "bf16", 4096),         # many tiles and chunks
+    ([9000], 12, 3, 128, "f32", 700),           # G = 4, fp32
+]
+
+
+@pytest.mark.parametrize("case", PROPOSE_CASES, ids=lambda c: f"{c[0]}-{c[1]}/{c[2]}-d{c[3]}-{c[4]}-kp{c[5]}")
+@pytest.mark.parametrize("scorer", ["mma", "simt"])
+def test_propose_vs_oracle(P, case, scorer, monkeypatch):
+    seqlens, hq, hkv, d, dtype, kp = case
+    if scorer == "simt":
+        monkeypatch.setenv("PRISM_PROPOSE_SCORER", "simt")
+    elif dtype != "bf16":
+        pytest.skip("the tensor-core scorer takes bf16 queries")
+    prob = problem(P, seqlens, hq, hkv, d, dtype)
+    q, k, _ = make_case(seqlens, hq, hkv, d, dtype, seed=2)
+    T = prob.total_tokens
+    kq = torch.zeros((hkv, T, d), dtype=torch.int8, device=DEV)
+    sc = torch.zeros((hkv, T), dtype=torch.float32, device=DEV)
+    P.quantize_k(prob, k, kq, sc)
+    pool = torch.full((len(seqlens), hkv, kp), -7, dtype=torch.int32, device=DEV)
+    cnt = torch.full((len(seqlens), hkv), -7, dtype=torch.int32, device=DEV)
+    ws = ws_for(P, prob, P.OP_PROPOSE, kp)
+    P.propose(prob, q, kq, sc, kp, pool, cnt, ws)
+    torch.cuda.synchronize()
+    assert P.get_device_status(ws) == 0
+    gscores = _np(ws[256:256 + hkv * T * 4].view(torch.float32)).reshape(hkv, T)
+    opool, ocnt, oscores = pipeline.propose_layer(q, kq, sc, prob.cu_host.tolist(), kp)
+    gp, gc = _np(pool), _np(cnt)
+    assert np.array_equal(gc, ocnt)
+    cu = prob.cu_host
+    for b in range(len(seqlens)):
+        for h in range(hkv):
+            s = oscores[(b, h)]
+            n = int(ocnt[b, h])
+            if n:
+                gs = gscores[h, cu[b]:cu[b + 1]]
+                assert np.allclose(gs, s, rtol=2e-6, atol=2e-6 * np.abs(s).max()), (b, h)
+            check_index_set(gp[b, h, :n], opool[b, h, :n], lambda t: s[t], f"pool b{b} h{h}")
+            assert np.all(gp[b, h, n:] == -1)
+
+
+def test_propose_all_ties_lower_index_wins(P):
+    seqlens, hq, hkv, d, kp = [3000, 500], 8, 2, 128, 1000
+    prob = problem(P, seqlens, hq, hkv, d, "bf16")
+    q, k, _ = make_case(seqlens, hq, hkv, d, "bf16", seed=3)
+    k[:] = k[:, :1]  # every key row identical -> every score equal
+    T = prob.total_tokens
+    kq = torch.zeros((hkv, T, d), dtype=torch.int8, device=DEV)
+    sc = torch.zeros((hkv, T), dtype=torch.float32, device=DEV)
+    P.quantize_k(prob, k, kq, sc)
+    pool = torch.zeros((2, hkv, kp), dtype=torch.int32, device=DEV)
+    cnt = torch.zeros((2, hkv), dtype=torch.int32, device=DEV)
+    P.propose(prob, q, kq, sc, kp, pool, cnt, ws_for(P, prob, P.OP_PROPOSE, kp))
+    gp = _np(pool)
+    for h in range(hkv):
+        assert np.array_equal(gp[0, h], np.arange(kp))
+        assert np.array_equal(gp[1, h, :500], np.arange(500)) and np.all(gp[1, h, 500:] == -1)
+    assert _np(cnt).tolist() == [[kp, kp], [500, 500]]
+
+
+# ------------------------------------------------------------------ refine
+
+REFINE_CASES = [
+    ([1024], 4, 1, 64, "f32", 256, 64),
+    ([5000, 1031, 0, 300], 8, 2, 128, "bf16", 1024, 256),
+    ([3000, 777], 8, 8, 64, "bf16", 200, 200),   # rho = 1: idx == pool
+    ([2500], 64, 8, 128, "bf16", 333, 100),
+    ([1800], 32, 2, 64, "bf16", 500, 17),
+    ([40000], 8, 2, 128, "bf16", 8192, 2048),
+]
+
+
+@pytest.mark.parametrize("case", REFINE_CASES, ids=lambda c: f"{c[0]}-{c[1]}/{c[2]}-d{c[3]}-{c[4]}-{c[5]}-{c[6]}")
+def test_refine_vs_oracle(P, case):
+    seqlens, hq, hkv, d, dtype, kp, kap = case
+    B = len(seqlens)
+    prob = problem(P, seqlens, hq, hkv, d, dtype)
+    q, k, _ = make_case(seqlens, hq, hkv, d, dtype, seed=4)
+    cu = prob.cu_host
+    # an arbitrary ascending pool per row (what a proposal layer hands over)
+    rng = np.random.default_rng(5)
+    pool = np.full((B, hkv, kp), -1, np.int32)
+    pcnt = np.zeros((B, hkv), np.int32)
+    for b, L in enumerate(seqlens):
+        for h in range(hkv):
+            n = min(kp, L)
+            pool[b, h, :n] = np.sort(rng.choice(L, n, replace=False))
+            pcnt[b, h] = n
+    dpool = torch.tensor(pool, device=DEV)
+    dcnt = torch.tensor(pcnt, device=DEV)
+    idx = torch.full((B, hkv, kap), -7, dtype=torch.int32, device=DEV)
+    cnt = torch.zeros((B, hkv), dtype=torch.int32, device=DEV)
+    logits = torch.full((B, hq, kap), 12345.0, device=DEV)
+    ws = ws_for(P, prob, P.OP_REFINE, kp, kap)
+    P.refine(prob, q, k, dpool, dcnt, kp, kap, idx, cnt, ws, logits=logits)
+    torch.cuda.synchronize()
+    assert P.get_device_status(ws) == 0
+    oidx, ocnt, oscores = pipeline.refine_layer(q, k, cu.tolist(), pool, pcnt, kap)
+    gi, gc, gl = _np(idx), _np(cnt), _np(logits)
+    assert np.array_equal(gc, ocnt)
+    qn, kn = _np(q).astype(np.float64), _np(k).astype(np.float64)
+    G = hq // hkv
+    for b in range(B):
+        for h in range(hkv):
+            n = int(pcnt[b, h])
+            r = dict(zip(pool[b, h, :n].tolist(), oscores[(b, h)].tolist()))
+            c = int(ocnt[b, h])
+            check_index_set(gi[b, h, :c], oidx[b, h, :c], lambda t: r[t], f"idx b{b} h{h}")
+            assert set(gi[b, h, :c].tolist()) <= set(pool[b, h, :n].tolist())
+            assert np.all(gi[b, h, c:] == -1)
+            if c:
+                rows = kn[h, cu[b] + gi[b, h, :c]]
+                want = qn[b, h * G:(h + 1) * G] @ rows.T
+                got = gl[b, h * G:(h + 1) * G, :c]
+                assert np.allclose(got, want, rtol=1e-5, atol=1e-4), (b, h)
+            assert np.all(gl[b, h * G:(h + 1) * G, c:] == 12345.0)
+
+
+# ------------------------------------------------------------------ attention
+
+ATTEND_CASES = [
+    ([1024], 4, 1, 64, "f32", 64),
+    ([5000, 1031, 0, 300], 8, 2, 128, "bf16", 256),
+    ([3000, 777], 8, 8, 64, "bf16", 200),
+    ([2500], 64, 8, 128, "bf16", 100),
+    ([1800], 32, 2, 64, "bf16", 17),
+    ([40000], 8, 2, 128, "bf16", 2048),
+    ([700, 2], 16, 1, 128, "f32", 1000),
+]
+
+
+@pytest.mark.parametrize("case", ATTEND_CASES, ids=lambda c: f"{c[0]}-{c[1]}/{c[2]}-d{c[3]}-{c[4]}-{c[5]}")
+def test_sparse_decode_vs_oracle(P, case):
+    seqlens, hq, hkv, d, dtype, kap = case
+    B = len(seqlens)
+    prob = problem(P, seqlens, hq, hkv, d, dtype)
+    q, k, v = make_case(seqlens, hq, hkv, d, dtype, seed=6)
+    rng = np.random.default_rng(7)
+    idx = np.full((B, hkv, kap), -1, np.int32)
+    cnt = np.zeros((B, hkv), np.int32)
+    for b, L in enumerate(seqlens):
+        for h in range(hkv):
+            n = min(kap, L) if (b + h) % 3 else min(kap, L) // 2
+            idx[b, h, :n] = np.sort(rng.choice(L, n, replace=False))
+            cnt[b, h] = n
+    out = torch.full((B, hq, d), 77.0, device=DEV)
+    lse = torch.full((B, hq), 77.0, device=DEV)
+    ws = ws_for(P, prob, P.OP_SPARSE_DECODE, 0, kap)
+    scale = float(np.float32(1 / math.sqrt(d)))
+    P.sparse_decode(prob, q, k, v, torch.tensor(idx, device=DEV), torch.tensor(cnt, device=DEV),
+                    kap, scale, out, ws, lse=lse)
+    torch.cuda.synchronize()
+    assert P.get_device_status(ws) == 0
+    oout, olse = pipeline.attend_layer(q, k, v, prob.cu_host.tolist(), idx, cnt, scale)
+    tol = atol_for(dtype)
+    assert np.abs(_np(out) - oout).max() <= tol
+    gl = _np(lse)
+    fin = np.isfinite(olse)
+    assert np.array_equal(np.isfinite(gl), fin)
+    assert np.abs(gl[fin] - olse[fin]).max() <= tol * 10
+    assert np.all(_np(out)[~fin] == 0)
+
+
+@pytest.mark.parametrize("case", [([1024], 4, 1, 64, "f32"), ([5000, 1031, 0, 300], 8, 2, 128, "bf16"),
+                                  ([20000], 32, 8, 128, "bf16"), ([999], 16, 1, 64, "bf16")],
+                         ids=lambda c: f"{c[0]}-{c[1]}/{c[2]}-d{c[3]}-{c[4]}")
+def test_dense_decode_vs_oracle(P, case):
+    seqlens, hq, hkv, d, dtype = case
+    prob = problem(P, seqlens, hq, hkv, d, dtype)
+    q, k, v = make_case(seqlens, hq, hkv, d, dtype, seed=8)
+    out = torch.zeros((len(seqlens), hq, d), device=DEV)
+    lse = torch.zeros((len(seqlens), hq), device=DEV)
+    scale = float(np.float32(1 / math.sqrt(d)))
+    ws = ws_for(P, prob, P.OP_DENSE_DECODE)
+    P.dense_decode(prob, q, k, v, scale, out, ws, lse=lse)
+    torch.cuda.synchronize()
+    oout, olse = pipeline.attend_layer(q, k, v, prob.cu_host.tolist(), None, None, scale)
+    tol = atol_for(dtype)
+    assert np.abs(_np(out) - oout).max() <= tol
+    fin = np.isfinite(olse)
+    assert np.abs(_np(lse)[fin] - olse[fin]).max() <= tol * 10
+
+
+def test_full_budget_sparse_equals_dense(P):
+    seqlens, hq, hkv, d = [600, 257], 8, 2, 128
+    prob = problem(P, seqlens, hq, hkv, d, "bf16")
+    q, k, v = make_case(seqlens, hq, hkv, d, "bf16", seed=9)
+    kap = 600
+    idx = torch.full((2, hkv, kap), -1, dtype=torch.int32, device=DEV)
+    cnt = torch.zeros((2, hkv), dtype=torch.int32, device=DEV)
+    for b, L in enumerate(seqlens):
+        idx[b, :, :L] = torch.arange(L, device=DEV, dtype=torch.int32)
+        cnt[b] = L
+    scale = 0.1
+    o1 = torch.zeros((2, hq, d), device=DEV)
+    o2 = torch.zeros((2, hq, d), device=DEV)
+    P.sparse_decode(prob, q, k, v, idx, cnt, kap, scale, o1, ws_for(P, prob, P.OP_SPARSE_DECODE, 0, kap))
+    P.dense_decode(prob, q, k, v, scale, o2, ws_for(P, prob, P.OP_DENSE_DECODE))
+    assert (o1 - o2).abs().max().item() <= 1e-5
+
+
+def test_bad_indices_flagged_not_read(P):
+    seqlens, hq, hkv, d, kap = [300], 4, 1, 128, 8
+    prob = problem(P, seqlens, hq, hkv, d, "bf16")
+    q, k, v = make_case(seqlens, hq, hkv, d, "bf16", seed=10)
+    idx = torch.tensor([[[0, 5, 299, 300, -3, 1 << 30, 7, 8]]], dtype=torch.int32, device=DEV)
+    cnt = torch.tensor([[8]], dtype=torch.int32, device=DEV)
+    ws = ws_for(P, prob, P.OP_SPARSE_DECODE, 0, kap)
+    out = torch.zeros((1, hq, d), device=DEV)
+    P.sparse_decode(prob, q, k, v, idx, cnt, kap, 0.1, out, ws)
+    assert P.get_device_status(ws) & P.DEV_BAD_INDEX
+    good = np.array([0, 5, 299, 7, 8], np.int32)
+    oout, _ = pipeline.attend_layer(q, k, v, [0, 300], good[None, None], np.array([[5]]), 0.1)
+    assert np.abs(_np(out) - oout).max() <= 2e-3
+    P.clear_device_status(ws)
+    assert P.get_device_status(ws) == 0

@@ -1,0 +1,132 @@
+"""Whole decode steps through the layer driver vs the oracle.
+
+Small configurations are checked on every (sequence, KV head) row of every
+layer.  The full-size configurations run in the launch configuration the
+benchmark times (same kernels, same split plans) and are checked on sampled
+rows the oracle computes one by one, plus invariants on every row.  Each
+stage is checked on the GPU's own upstream set (cascade control).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from kv_cache_top_proposal_b200 import workload
+from kv_cache_top_proposal_b200.decoder import PrismDecoder
+from oracle import pipeline
+from parity_util import atol_for, check_index_set
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy() if t.dtype not in (torch.int32, torch.int8) \
+        else t.detach().cpu().numpy()
+
+
+def _decoder(P, cfg):
+    return PrismDecoder(cfg.seqlens, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim,
+                        P.F32 if cfg.dtype == "f32" else P.BF16, cfg.num_layers, cfg.group,
+                        cfg.kappa_p, cfg.kappa, device=DEV)
+
+
+def _prefill_kq(P, dec, cfg, lay):
+    kq = torch.zeros(lay.k.shape, dtype=torch.int8, device=DEV)
+    sc = torch.zeros(lay.k.shape[:2], dtype=torch.float32, device=DEV)
+    P.quantize_k(dec.p, lay.k, kq, sc)
+    return kq, sc
+
+
+def _check_layer(dec, cfg, l, lay, kq, sc, rows):
+    cu = cfg.cu_seqlens
+    src = l - l % cfg.group
+    gpool, gpc = _np(dec.pool[src]), _np(dec.pool_cnt[src])
+    if l == src:
+        opool, ocnt, osc = pipeline.propose_layer(lay.q, kq, sc, cu, cfg.kappa_p, rows=rows)
+        for (b, h) in rows:
+            n = int(ocnt[b, h])
+            assert int(gpc[b, h]) == n
+            check_index_set(gpool[b, h, :n], opool[b, h, :n], lambda t: osc[(b, h)][t],
+                            f"L{l} pool {b},{h}")
+            assert np.all(gpool[b, h, n:] == -1)
+    gidx, gcnt = _np(dec.idx[l]), _np(dec.cnt[l])
+    oidx, ocnt, orr = pipeline.refine_layer(lay.q, lay.k, cu, gpool, gpc, cfg.kappa, rows=rows)
+    for (b, h) in rows:
+        n = int(gpc[b, h])
+        r = dict(zip(gpool[b, h, :n].tolist(), orr[(b, h)].tolist()))
+        c = int(ocnt[b, h])
+        assert int(gcnt[b, h]) == c
+        check_index_set(gidx[b, h, :c], oidx[b, h, :c], lambda t: r[t], f"L{l} idx {b},{h}")
+        assert set(gidx[b, h, :c].tolist()) <= set(gpool[b, h, :n].tolist())
+    oout, olse = pipeline.attend_layer(lay.q, lay.k, lay.v, cu, gidx, gcnt, dec.scale, rows=rows)
+    gout, glse = _np(dec.out[l]), _np(dec.lse[l])
+    G = cfg.G
+    tol = atol_for(cfg.dtype)
+    for (b, h) in rows:
+        sl = slice(h * G, (h + 1) * G)
+        assert np.abs(gout[b, sl] - oout[b, sl]).max() <= tol, (l, b, h)
+        assert np.abs(glse[b, sl] - olse[b, sl]).max() <= 10 * tol, (l, b, h)
+
+
+def _all_rows(cfg):
+    return [(b, h) for b in range(cfg.batch) for h in range(cfg.num_kv_heads)]
+
+
+def _invariants(dec, cfg, l):
+    src = l - l % cfg.group
+    gp, gpc = _np(dec.pool[src]), _np(dec.pool_cnt[src])
+    gi, gc = _np(dec.idx[l]), _np(dec.cnt[l])
+    for b, L in enumerate(cfg.seqlens):
+        for h in range(cfg.num_kv_heads):
+            n, c = int(gpc[b, h]), int(gc[b, h])
+            assert n == min(cfg.kappa_p, L) and c == min(cfg.kappa, n)
+            p, i = gp[b, h, :n], gi[b, h, :c]
+            assert np.all(np.diff(p) > 0) and (n == 0 or (p[0] >= 0 and p[-1] < L))
+            assert np.all(np.diff(i) > 0) and np.all(np.isin(i, p))
+    assert np.all(np.isfinite(_np(dec.out[l])))
+
+
+@pytest.mark.parametrize("name", ["tiny", "c8k"])
+def test_step_small_configs_every_row(prism_lib, name):
+    P = prism_lib
+    cfg = workload.config(name)
+    layers = list(workload.generate(cfg, DEV))
+    dec = _decoder(P, cfg)
+    kqs, scs = {}, {}
+    for lay in layers:
+        if cfg.is_proposal(lay.index):
+            kqs[lay.index], scs[lay.index] = _prefill_kq(P, dec, cfg, lay)
+    dec.step([x.q for x in layers], [x.k for x in layers], [x.v for x in layers], kqs, scs)
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    for lay in layers:
+        l = lay.index
+        src = l - l % cfg.group
+        _invariants(dec, cfg, l)
+        _check_layer(dec, cfg, l, lay, kqs[src], scs[src], _all_rows(cfg))
+
+
+@pytest.mark.parametrize("name", ["c8k", "c32k_b4", "c128k", "ragged16"])
+def test_step_full_size_sampled(prism_lib, name):
+    """First proposal group's first two layers at the full sizes."""
+    P = prism_lib
+    cfg = workload.config(name)
+    want = [0, 1]
+    layers = list(workload.generate(cfg, DEV, layers=want))
+    cfg2 = cfg.replace(num_layers=2)
+    dec = _decoder(P, cfg2)
+    kqs, scs = {}, {}
+    kqs[0], scs[0] = _prefill_kq(P, dec, cfg, layers[0])
+    dec.step([x.q for x in layers], [x.k for x in layers], [x.v for x in layers], kqs, scs)
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    rng = np.random.default_rng(11)
+    rows = sorted({(int(rng.integers(cfg.batch)), int(rng.integers(cfg.num_kv_heads))) for _ in range(3)}
+                  | {(cfg.batch - 1, cfg.num_kv_heads - 1)})
+    for lay in layers:
+        _invariants(dec, cfg2, lay.index)
+        _check_layer(dec, cfg2, lay.index, lay, kqs[0], scs[0], rows)
+    del layers, dec
+    torch.cuda.empty_cache()
