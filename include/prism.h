@@ -127,6 +127,18 @@ PRISM_API prism_status prism_quantize_k(const prism_shape* shape, const void* k,
                               void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Decode-time cache update (the step either side of the method: the new
+ * token's key and value join the cache before attention; the decode query
+ * sits at position L_b - 1).  k_new, v_new are [B][Hkv][d] in the shape's
+ * dtype; row b is written to position L_b - 1 of sequence b (packed row
+ * cu[b+1] - 1) of every KV head in k_cache / v_cache.  Sequences with
+ * L_b = 0 are skipped.
+ */
+PRISM_API prism_status prism_append_kv(const prism_shape* shape, const void* k_new,
+                                       const void* v_new, void* k_cache, void* v_cache,
+                                       void* stream);
+
+/*
  * Proposal layer (sec. 4.1 "Proposal-Refined Index Sharing", sec. 4.2): for
  * every sequence b and KV head h, score every position t < L_b with the
  * quantized keys,

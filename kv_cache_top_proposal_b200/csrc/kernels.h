@@ -25,6 +25,9 @@ struct Dims {
 // runs on the smallest instantiation >= G with the extra heads masked.
 inline int padded_group(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : G <= 8 ? 8 : 16; }
 
+cudaError_t launch_append(const Dims& d, const void* k_new, const void* v_new, void* k_cache,
+                          void* v_cache, cudaStream_t st);
+
 cudaError_t launch_quantize(const Dims& d, const void* k, int8_t* kq, float* scale,
                             const int32_t* tok_rows, int64_t n_rows, int32_t* status,
                             cudaStream_t st);

@@ -134,6 +134,17 @@ prism_status prism_workspace_size(const prism_shape* shape, int32_t op, int32_t 
   return PRISM_OK;
 }
 
+prism_status prism_append_kv(const prism_shape* shape, const void* k_new, const void* v_new,
+                             void* k_cache, void* v_cache, void* stream) {
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!k_new || !v_new || !k_cache || !v_cache) return PRISM_ERR_INVALID_ARG;
+  const uintptr_t all = (uintptr_t)k_new | (uintptr_t)v_new | (uintptr_t)k_cache | (uintptr_t)v_cache;
+  if (all % 16 != 0) return PRISM_ERR_INVALID_ARG;
+  return cuda_status(launch_append(d, k_new, v_new, k_cache, v_cache, static_cast<cudaStream_t>(stream)));
+}
+
 prism_status prism_quantize_k(const prism_shape* shape, const void* k, int8_t* kq, float* k_scale,
                               const int32_t* tok_rows, int32_t n_rows, void* ws, size_t ws_bytes,
                               void* stream) {

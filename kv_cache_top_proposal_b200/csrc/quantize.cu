@@ -1,4 +1,4 @@
-// Per-token symmetric int8 quantization of the key cache (Prism Attention,
+// Cache update and per-token symmetric int8 quantization of the key cache (Prism Attention,
 // sec. 4.2 "Quantized Proposal Construction"; int8 per-token scheme because
 // the pages do not state their INT2 one).
 //
@@ -77,6 +77,46 @@ __global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ k,
       if (li == 0) scale[row] = (amax != 0.0f) ? s : 0.0f;
     }
   }
+}
+
+// Write the new token row of every (sequence, KV head): one 16-byte vector
+// per thread, rows of k_new / v_new to packed row cu[b+1] - 1.
+template <int VEC_PER_ROW>
+__global__ void __launch_bounds__(256) append_kernel(const uint4* __restrict__ k_new,
+                                                     const uint4* __restrict__ v_new,
+                                                     uint4* __restrict__ k_cache,
+                                                     uint4* __restrict__ v_cache,
+                                                     const int32_t* __restrict__ cu, int B, int Hkv,
+                                                     int64_t T_tok) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t per_seq = (int64_t)Hkv * VEC_PER_ROW;
+  if (i >= (int64_t)B * per_seq) return;
+  const int b = (int)(i / per_seq);
+  const int64_t r = i - (int64_t)b * per_seq;
+  const int h = (int)(r / VEC_PER_ROW), c = (int)(r % VEC_PER_ROW);
+  const int end = cu[b + 1];
+  if (end <= cu[b]) return;
+  const int64_t dst = ((int64_t)h * T_tok + end - 1) * VEC_PER_ROW + c;
+  k_cache[dst] = k_new[i];
+  v_cache[dst] = v_new[i];
+}
+
+cudaError_t launch_append(const Dims& d, const void* k_new, const void* v_new, void* k_cache,
+                          void* v_cache, cudaStream_t st) {
+  const int vec = d.D * (d.bf16 ? 2 : 4) / 16;
+  const int64_t n = (int64_t)d.B * d.Hkv * vec;
+  if (n == 0) return cudaSuccess;
+  const unsigned blocks = (unsigned)cdiv(n, 256);
+  auto* kn = static_cast<const uint4*>(k_new);
+  auto* vn = static_cast<const uint4*>(v_new);
+  auto* kc = static_cast<uint4*>(k_cache);
+  auto* vc = static_cast<uint4*>(v_cache);
+  switch (vec) {
+    case 8: append_kernel<8><<<blocks, 256, 0, st>>>(kn, vn, kc, vc, d.cu_dev, d.B, d.Hkv, d.T); break;
+    case 16: append_kernel<16><<<blocks, 256, 0, st>>>(kn, vn, kc, vc, d.cu_dev, d.B, d.Hkv, d.T); break;
+    default: append_kernel<32><<<blocks, 256, 0, st>>>(kn, vn, kc, vc, d.cu_dev, d.B, d.Hkv, d.T); break;
+  }
+  return cudaGetLastError();
 }
 
 template <typename T, int D>

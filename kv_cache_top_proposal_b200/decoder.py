@@ -45,8 +45,11 @@ class PrismDecoder:
         self.pool_cnt = {l: torch.zeros((B, Hkv), **i32) for l in self.proposal_layers}
         self.idx = [torch.full((B, Hkv, kappa), -1, **i32) for _ in range(num_layers)]
         self.cnt = [torch.zeros((B, Hkv), **i32) for _ in range(num_layers)]
-        self.out = [torch.zeros((B, Hq, D), **f32) for _ in range(num_layers)]
-        self.lse = [torch.zeros((B, Hq), **f32) for _ in range(num_layers)]
+        # per-layer outputs are views of one buffer (one device-to-host copy)
+        self.out_all = torch.zeros((num_layers, B, Hq, D), **f32)
+        self.lse_all = torch.zeros((num_layers, B, Hq), **f32)
+        self.out = [self.out_all[l] for l in range(num_layers)]
+        self.lse = [self.lse_all[l] for l in range(num_layers)]
         # the newly appended token of every sequence (packed row index)
         last = [c - 1 for c in self.p.cu_host[1:].tolist() if True]
         self.new_rows = torch.tensor([r for r, L in zip(last, seqlens) if L > 0], **i32)
@@ -66,9 +69,14 @@ class PrismDecoder:
                 if w is not None]
 
     def layer(self, l: int, q, k, v, kq=None, k_scale=None, quantize_new: bool = True,
-              stream=None):
-        """Enqueue one layer of the step (kq/k_scale required at proposal layers)."""
+              k_new=None, v_new=None, stream=None):
+        """Enqueue one layer of the step (kq/k_scale required at proposal layers).
+
+        k_new / v_new ([B][Hkv][d]), when given, are first written to the last
+        position of every sequence (the token being decoded)."""
         p = self.p
+        if k_new is not None:
+            prism.append_kv(p, k_new, v_new, k, v, stream=stream)
         if l % self.group == 0:
             if quantize_new and self.new_rows.numel():
                 prism.quantize_k(p, k, kq, k_scale, tok_rows=self.new_rows, ws=self.ws_q, stream=stream)
@@ -80,13 +88,27 @@ class PrismDecoder:
         prism.sparse_decode(p, q, k, v, self.idx[l], self.cnt[l], self.kappa, self.scale,
                             self.out[l], self.ws_dec, lse=self.lse[l], stream=stream)
 
-    def step(self, qs, ks, vs, kqs, scales, quantize_new: bool = True, stream=None):
-        """One decode step over every layer.  qs/ks/vs are per-layer lists;
-        kqs/scales are dicts (or lists) indexed by proposal layer."""
+    def step(self, qs, ks, vs, kqs, scales, quantize_new: bool = True, k_new=None, v_new=None,
+             stream=None):
+        """One decode step over every layer.  qs/ks/vs (and k_new/v_new) are
+        per-layer sequences; kqs/scales are indexed by proposal layer."""
         for l in range(self.num_layers):
             pl = l % self.group == 0
             self.layer(l, qs[l], ks[l], vs[l], kqs[l] if pl else None, scales[l] if pl else None,
-                       quantize_new=quantize_new, stream=stream)
+                       quantize_new=quantize_new,
+                       k_new=None if k_new is None else k_new[l],
+                       v_new=None if v_new is None else v_new[l], stream=stream)
+
+    def launches_per_step(self, append: bool) -> int:
+        """Kernels one step enqueues (append, quantize, score, select, refine
+        score, select, attend, merge)."""
+        n = 0
+        for l in range(self.num_layers):
+            n += 1 if append else 0
+            if l % self.group == 0:
+                n += (1 if self.new_rows.numel() else 0) + 2
+            n += 2 + 2
+        return n
 
     def dense_layer(self, l: int, q, k, v, out, lse=None, stream=None):
         if self.ws_dense is None:

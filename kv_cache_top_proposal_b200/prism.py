@@ -24,7 +24,7 @@ DEV_BAD_INDEX, DEV_TOO_LONG = 0x1, 0x2
 MAX_SELECT_ROW = 393216
 WS_HEADER = 256
 
-EXPORTS = ("prism_workspace_size", "prism_quantize_k", "prism_propose", "prism_refine",
+EXPORTS = ("prism_workspace_size", "prism_append_kv", "prism_quantize_k", "prism_propose", "prism_refine",
            "prism_sparse_decode", "prism_dense_decode", "prism_clear_device_status",
            "prism_get_device_status", "prism_status_str")
 
@@ -51,6 +51,7 @@ def _load():
     sp = ctypes.POINTER(Shape)
     sig = {
         "prism_workspace_size": [sp, i32, i32, i32, ctypes.POINTER(ctypes.c_size_t)],
+        "prism_append_kv": [sp, P, P, P, P, P],
         "prism_quantize_k": [sp, P, P, P, P, i32, P, S, P],
         "prism_propose": [sp, P, P, P, i32, P, P, P, S, P],
         "prism_refine": [sp, P, P, P, P, i32, i32, P, P, P, P, S, P],
@@ -132,6 +133,11 @@ def workspace_size(p: Problem, op: int, kappa_p: int = 0, kappa: int = 0) -> int
 
 def _nbytes(ws) -> int:
     return 0 if ws is None else ws.numel() * ws.element_size()
+
+
+def append_kv(p: Problem, k_new, v_new, k_cache, v_cache, stream=None):
+    _check(_lib.prism_append_kv(p.ref, _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                _stream(stream)), "append_kv")
 
 
 def quantize_k(p: Problem, k, kq, k_scale, tok_rows=None, ws=None, stream=None):
