@@ -74,9 +74,13 @@ def step_bytes(cfg) -> dict:
     refine = sum(min(cfg.kappa_p, L) for L in cfg.seqlens) * Hkv * D * el
     sparse = sum(min(cfg.kappa, cfg.kappa_p, L) for L in cfg.seqlens) * Hkv * D * el * 2
     dense = Hkv * T * D * el * 2
+    # fused refined layer: the pool's key rows once, the selected value rows once
+    refine_decode = refine + sparse // 2
     n_prop = len(cfg.proposal_layers)
     return {"propose": propose, "refine": refine, "sparse_decode": sparse, "dense_decode": dense,
-            "step": n_prop * propose + cfg.num_layers * (refine + sparse),
+            "refine_decode": refine_decode,
+            "step": n_prop * propose + cfg.num_layers * refine_decode,
+            "step_unfused": n_prop * propose + cfg.num_layers * (refine + sparse),
             "dense_step": cfg.num_layers * dense}
 
 
@@ -385,19 +389,15 @@ def run_prism(args, dist: Dist):
             prism.propose(dec.p, q_layers[l], kqs[l], scs[l], cfg.kappa_p, dec.pool[l],
                           dec.pool_cnt[l], dec.ws_prop)
 
-        def f_ref(l=l):
+        def f_rd(l=l):
             src = l - l % cfg.group
-            prism.refine(dec.p, q_layers[l], ks[l], dec.pool[src], dec.pool_cnt[src], cfg.kappa_p,
-                         cfg.kappa, dec.idx[l], dec.cnt[l], dec.ws_ref)
-
-        def f_dec(l=l):
-            prism.sparse_decode(dec.p, q_layers[l], ks[l], vs[l], dec.idx[l], dec.cnt[l], cfg.kappa,
-                                dec.scale, dec.out[l], dec.ws_dec, lse=dec.lse[l])
+            prism.refine_decode(dec.p, q_layers[l], ks[l], vs[l], dec.pool[src], dec.pool_cnt[src],
+                                cfg.kappa_p, cfg.kappa, dec.scale, dec.idx[l], dec.cnt[l],
+                                dec.out[l], dec.ws_rd, lse=dec.lse[l])
 
         if pl:
             ops.append(("propose", graph_of(f_prop, stream)))
-        ops.append(("refine", graph_of(f_ref, stream)))
-        ops.append(("sparse_decode", graph_of(f_dec, stream)))
+        ops.append(("refine_decode", graph_of(f_rd, stream)))
     gate = torch.empty(6 << 30, dtype=torch.uint8, device=dev)
     per_op = {}
     for _ in range(args.profile_steps):
@@ -470,11 +470,14 @@ def run_prism(args, dist: Dist):
             "data": "synthetic (seeded drifting-Gaussian RoPE keys, planted salient tokens)",
             "config": dict(workload_config(cfg), l2="inputs larger than L2: a step touches "
                            f"{nbytes['step'] / 1e9:.2f} GB of distinct cache rows (L2 126 MB)",
+                           refined_layers="fused refine+select+sparse-decode (prism_refine_decode)",
                            graph="one CUDA graph per step"),
             "roofline": roofline,
             "step_roofline": {"achieved": round(step_achieved, 1), "peak": peak, "unit": "GB/s",
                               "frac": round(step_achieved / peak, 4),
                               "algorithmic_bytes_per_step": nbytes["step"],
+                              "frac_with_unfused_byte_model": round(
+                                  nbytes["step_unfused"] / (ms_per_step * 1e-3) / 1e9 / peak, 4),
                               "frac_of_8TBps_nominal": round(step_achieved / 8000.0, 4)},
             "ops": ops_summary,
             "cpu_baseline": cpu,

@@ -75,7 +75,8 @@ typedef enum prism_op {
   PRISM_OP_PROPOSE = 1,
   PRISM_OP_REFINE = 2,
   PRISM_OP_SPARSE_DECODE = 3,
-  PRISM_OP_DENSE_DECODE = 4
+  PRISM_OP_DENSE_DECODE = 4,
+  PRISM_OP_REFINE_DECODE = 5
 } prism_op;
 
 /* Bits of the device status word kept in every workspace. */
@@ -181,6 +182,23 @@ PRISM_API prism_status prism_sparse_decode(const prism_shape* shape, const void*
                                  const void* v, const int32_t* idx, const int32_t* cnt,
                                  int32_t kappa, float softmax_scale, float* out, float* lse_opt,
                                  void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * A refined layer in one call: prism_refine followed by prism_sparse_decode
+ * on its result, with the same outputs (idx, cnt, out, lse_opt) and the same
+ * definitions.  The exact scores, the selection and the attention partials
+ * stay on chip (one thread-block cluster per sequence and KV head), so the
+ * workspace is only the 256-byte status header (PRISM_OP_REFINE_DECODE), and
+ * the key rows of the pool are read once.  Returns PRISM_ERR_UNSUPPORTED when
+ * a pool of kappa_p members does not fit on chip (kappa_p > 16 x the slice
+ * capacity: 6144 members per CTA at G <= 4, d = 128); use the two calls then.
+ */
+PRISM_API prism_status prism_refine_decode(const prism_shape* shape, const void* q, const void* k,
+                                           const void* v, const int32_t* pool_idx,
+                                           const int32_t* pool_cnt, int32_t kappa_p,
+                                           int32_t kappa, float softmax_scale, int32_t* idx,
+                                           int32_t* cnt, float* out, float* lse_opt, void* ws,
+                                           size_t ws_bytes, void* stream);
 
 /*
  * Dense decode attention over every position t < L_b (the comparison path):

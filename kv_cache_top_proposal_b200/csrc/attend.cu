@@ -196,37 +196,58 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendArgs a) {
   }
 }
 
+// One CTA of D threads per (sequence, query head): the split weights
+// 2^(m_s - M) are computed in parallel into shared memory, then thread j sums
+// its feature over the splits with independent (pipelined) loads.
 template <int D>
-__global__ void __launch_bounds__(128) merge_kernel(int BHq, int splits, const float* __restrict__ part_o,
-                                                   const float* __restrict__ part_ml,
-                                                   float* __restrict__ out, float* __restrict__ lse) {
-  constexpr int PER = D / 32;
-  const int w = blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (w >= BHq) return;
+__global__ void __launch_bounds__(D) merge_kernel(int splits, const float* __restrict__ part_o,
+                                                 const float* __restrict__ part_ml,
+                                                 float* __restrict__ out, float* __restrict__ lse) {
+  extern __shared__ float s_w[];  // [splits]
+  __shared__ float s_red[D / 32];
+  __shared__ float s_M, s_L;
+  const int w = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* ml = part_ml + (int64_t)w * splits * 2;
   const float* po = part_o + (int64_t)w * splits * D;
   float M = -INFINITY;
-  for (int s = lane; s < splits; s += 32) M = fmaxf(M, ml[s * 2]);
+  for (int s = tid; s < splits; s += D) M = fmaxf(M, ml[s * 2]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float Ls = 0.0f, acc[PER];
-#pragma unroll
-  for (int i = 0; i < PER; ++i) acc[i] = 0.0f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < splits; ++s) {
-      const float ms = ml[s * 2];
-      if (ms == -INFINITY) continue;
-      const float wgt = exp2f(ms - M);
-      Ls = fmaf(wgt, ml[s * 2 + 1], Ls);
-#pragma unroll
-      for (int i = 0; i < PER; ++i) acc[i] = fmaf(wgt, po[(int64_t)s * D + lane + 32 * i], acc[i]);
-    }
+  if (lane == 0) s_red[warp] = M;
+  __syncthreads();
+  if (tid == 0) {
+    float v = s_red[0];
+    for (int i = 1; i < D / 32; ++i) v = fmaxf(v, s_red[i]);
+    s_M = v;
   }
-  const bool any = Ls > 0.0f;
+  __syncthreads();
+  M = s_M;
+  float Ls = 0.0f;
+  for (int s = tid; s < splits; s += D) {
+    const float ms = ml[s * 2];
+    const float wt = (M == -INFINITY || ms == -INFINITY) ? 0.0f : exp2f(ms - M);
+    s_w[s] = wt;
+    Ls = fmaf(wt, ml[s * 2 + 1], Ls);
+  }
 #pragma unroll
-  for (int i = 0; i < PER; ++i) out[(int64_t)w * D + lane + 32 * i] = any ? acc[i] / Ls : 0.0f;
-  if (lse && lane == 0) lse[w] = any ? (M + log2f(Ls)) * 0.69314718055994530942f : -INFINITY;
+  for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+  __syncthreads();
+  if (lane == 0) s_red[warp] = Ls;
+  __syncthreads();
+  if (tid == 0) {
+    float v = 0.0f;
+    for (int i = 0; i < D / 32; ++i) v += s_red[i];
+    s_L = v;
+  }
+  __syncthreads();
+  Ls = s_L;
+  float acc = 0.0f;
+#pragma unroll 8
+  for (int s = 0; s < splits; ++s) acc = fmaf(s_w[s], po[(int64_t)s * D + tid], acc);
+  const bool any = Ls > 0.0f;
+  out[(int64_t)w * D + tid] = any ? acc / Ls : 0.0f;
+  if (lse && tid == 0) lse[w] = any ? (M + log2f(Ls)) * 0.69314718055994530942f : -INFINITY;
 }
 
 template <typename T, int D, int GP>
@@ -284,11 +305,11 @@ cudaError_t launch_attend(const Dims& d, const AttendPlan& p, const void* q, con
     e = d.D == 128 ? by_group<float, 128>(d, p, a, st) : by_group<float, 64>(d, p, a, st);
   if (e != cudaSuccess) return e;
   const int BHq = d.B * d.Hq;
-  const int blocks = (BHq + 3) / 4;
+  const size_t smem = (size_t)p.splits * sizeof(float);
   if (d.D == 128)
-    merge_kernel<128><<<blocks, 128, 0, st>>>(BHq, p.splits, part_o, part_ml, out, lse);
+    merge_kernel<128><<<BHq, 128, smem, st>>>(p.splits, part_o, part_ml, out, lse);
   else
-    merge_kernel<64><<<blocks, 128, 0, st>>>(BHq, p.splits, part_o, part_ml, out, lse);
+    merge_kernel<64><<<BHq, 64, smem, st>>>(p.splits, part_o, part_ml, out, lse);
   return cudaGetLastError();
 }
 

@@ -65,6 +65,21 @@ cudaError_t launch_refine_scores(const Dims& d, const void* q, const void* k, co
                                  const int32_t* pool_cnt, int pool_stride, float* r, float* dots,
                                  int32_t* status, cudaStream_t st);
 
+// Fused refine -> top-kappa -> sparse decode, one cluster of `cluster` CTAs
+// per (sequence, KV head); mc = pool members per CTA.  ok = false when the
+// pool does not fit on chip.
+struct RefineDecodePlan {
+  int cluster;
+  int mc;
+  bool ok;
+};
+RefineDecodePlan plan_refine_decode(const Dims& d, int kappa_p);
+cudaError_t launch_refine_decode(const Dims& d, const RefineDecodePlan& p, const void* q,
+                                 const void* k, const void* v, const int32_t* pool,
+                                 const int32_t* pool_cnt, int kappa_p, int kappa,
+                                 float softmax_scale, int32_t* idx, int32_t* cnt, float* out,
+                                 float* lse, int32_t* status, cudaStream_t st);
+
 // Split-K attention partials over idx rows (idx == nullptr: every position).
 struct AttendPlan {
   int splits;

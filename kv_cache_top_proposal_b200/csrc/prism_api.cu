@@ -125,9 +125,10 @@ prism_status prism_workspace_size(const prism_shape* shape, int32_t op, int32_t 
   Dims d;
   prism_status s = check_shape(shape, &d);
   if (s != PRISM_OK) return s;
-  if (!bytes || op < PRISM_OP_QUANTIZE || op > PRISM_OP_DENSE_DECODE) return PRISM_ERR_INVALID_ARG;
+  if (!bytes || op < PRISM_OP_QUANTIZE || op > PRISM_OP_REFINE_DECODE) return PRISM_ERR_INVALID_ARG;
   if (op == PRISM_OP_PROPOSE && kappa_p < 1) return PRISM_ERR_INVALID_ARG;
-  if (op == PRISM_OP_REFINE && (kappa_p < 1 || kappa < 1 || kappa > kappa_p))
+  if ((op == PRISM_OP_REFINE || op == PRISM_OP_REFINE_DECODE) &&
+      (kappa_p < 1 || kappa < 1 || kappa > kappa_p))
     return PRISM_ERR_INVALID_ARG;
   if (op == PRISM_OP_SPARSE_DECODE && kappa < 1) return PRISM_ERR_INVALID_ARG;
   *bytes = layout(d, op, kappa_p, kappa).total;
@@ -250,6 +251,26 @@ prism_status prism_sparse_decode(const prism_shape* shape, const void* q, const 
                                    reinterpret_cast<float*>(w + L.a),
                                    reinterpret_cast<float*>(w + L.b), out, lse_opt,
                                    reinterpret_cast<int32_t*>(w), static_cast<cudaStream_t>(stream)));
+}
+
+prism_status prism_refine_decode(const prism_shape* shape, const void* q, const void* k,
+                                 const void* v, const int32_t* pool_idx, const int32_t* pool_cnt,
+                                 int32_t kappa_p, int32_t kappa, float softmax_scale, int32_t* idx,
+                                 int32_t* cnt, float* out, float* lse_opt, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!q || !k || !v || !pool_idx || !pool_cnt || !idx || !cnt || !out) return PRISM_ERR_INVALID_ARG;
+  if (kappa_p < 1 || kappa < 1 || kappa > kappa_p) return PRISM_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return PRISM_ERR_INVALID_ARG;
+  const Layout L = layout(d, PRISM_OP_REFINE_DECODE, kappa_p, kappa);
+  if (!ws_ok(ws, ws_bytes, L)) return PRISM_ERR_WORKSPACE;
+  const RefineDecodePlan p = plan_refine_decode(d, kappa_p);
+  if (!p.ok) return PRISM_ERR_UNSUPPORTED;
+  return cuda_status(launch_refine_decode(d, p, q, k, v, pool_idx, pool_cnt, kappa_p, kappa,
+                                          softmax_scale, idx, cnt, out, lse_opt,
+                                          static_cast<int32_t*>(ws), static_cast<cudaStream_t>(stream)));
 }
 
 prism_status prism_dense_decode(const prism_shape* shape, const void* q, const void* k,

@@ -29,7 +29,7 @@ from . import prism
 class PrismDecoder:
     def __init__(self, seqlens, num_q_heads: int, num_kv_heads: int, head_dim: int, dtype: int,
                  num_layers: int, group: int, kappa_p: int, kappa: int, device="cuda",
-                 softmax_scale: Optional[float] = None):
+                 softmax_scale: Optional[float] = None, fused: bool = True):
         self.dev = torch.device(device)
         self.p = prism.Problem(seqlens, num_q_heads, num_kv_heads, head_dim, dtype, device=self.dev)
         self.B, self.Hq, self.Hkv, self.D = len(seqlens), num_q_heads, num_kv_heads, head_dim
@@ -62,11 +62,14 @@ class PrismDecoder:
         self.ws_prop = ws(prism.OP_PROPOSE, kappa_p)
         self.ws_ref = ws(prism.OP_REFINE, kappa_p, kappa)
         self.ws_dec = ws(prism.OP_SPARSE_DECODE, 0, kappa)
+        self.ws_rd = ws(prism.OP_REFINE_DECODE, kappa_p, kappa)
         self.ws_dense = None
+        # refined layers in one fused call (refine -> select -> sparse decode)
+        self.fused = fused
 
     def workspaces(self) -> List[torch.Tensor]:
-        return [w for w in (self.ws_q, self.ws_prop, self.ws_ref, self.ws_dec, self.ws_dense)
-                if w is not None]
+        return [w for w in (self.ws_q, self.ws_prop, self.ws_ref, self.ws_dec, self.ws_rd,
+                            self.ws_dense) if w is not None]
 
     def layer(self, l: int, q, k, v, kq=None, k_scale=None, quantize_new: bool = True,
               k_new=None, v_new=None, stream=None):
@@ -83,6 +86,11 @@ class PrismDecoder:
             prism.propose(p, q, kq, k_scale, self.kappa_p, self.pool[l], self.pool_cnt[l],
                           self.ws_prop, stream=stream)
         src = l - l % self.group
+        if self.fused:
+            prism.refine_decode(p, q, k, v, self.pool[src], self.pool_cnt[src], self.kappa_p,
+                                self.kappa, self.scale, self.idx[l], self.cnt[l], self.out[l],
+                                self.ws_rd, lse=self.lse[l], stream=stream)
+            return
         prism.refine(p, q, k, self.pool[src], self.pool_cnt[src], self.kappa_p, self.kappa,
                      self.idx[l], self.cnt[l], self.ws_ref, stream=stream)
         prism.sparse_decode(p, q, k, v, self.idx[l], self.cnt[l], self.kappa, self.scale,
@@ -107,7 +115,7 @@ class PrismDecoder:
             n += 1 if append else 0
             if l % self.group == 0:
                 n += (1 if self.new_rows.numel() else 0) + 2
-            n += 2 + 2
+            n += 1 if self.fused else 2 + 2
         return n
 
     def dense_layer(self, l: int, q, k, v, out, lse=None, stream=None):

@@ -18,14 +18,15 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "_lib", "libprism.so")
 
 F32, BF16 = 0, 1
-OP_QUANTIZE, OP_PROPOSE, OP_REFINE, OP_SPARSE_DECODE, OP_DENSE_DECODE = range(5)
+OP_QUANTIZE, OP_PROPOSE, OP_REFINE, OP_SPARSE_DECODE, OP_DENSE_DECODE, OP_REFINE_DECODE = range(6)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
 DEV_BAD_INDEX, DEV_TOO_LONG = 0x1, 0x2
 MAX_SELECT_ROW = 393216
 WS_HEADER = 256
 
 EXPORTS = ("prism_workspace_size", "prism_append_kv", "prism_quantize_k", "prism_propose", "prism_refine",
-           "prism_sparse_decode", "prism_dense_decode", "prism_clear_device_status",
+           "prism_sparse_decode", "prism_refine_decode", "prism_dense_decode",
+           "prism_clear_device_status",
            "prism_get_device_status", "prism_status_str")
 
 
@@ -56,6 +57,7 @@ def _load():
         "prism_propose": [sp, P, P, P, i32, P, P, P, S, P],
         "prism_refine": [sp, P, P, P, P, i32, i32, P, P, P, P, S, P],
         "prism_sparse_decode": [sp, P, P, P, P, P, i32, ctypes.c_float, P, P, P, S, P],
+        "prism_refine_decode": [sp, P, P, P, P, P, i32, i32, ctypes.c_float, P, P, P, P, P, S, P],
         "prism_dense_decode": [sp, P, P, P, ctypes.c_float, P, P, P, S, P],
         "prism_clear_device_status": [P, S, P],
         "prism_get_device_status": [P, S, P, ctypes.POINTER(ctypes.c_int32)],
@@ -163,6 +165,14 @@ def sparse_decode(p: Problem, q, k, v, idx, cnt, kappa: int, softmax_scale: floa
     _check(_lib.prism_sparse_decode(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt), kappa,
                                     float(softmax_scale), _ptr(out), _ptr(lse), _ptr(ws),
                                     _nbytes(ws), _stream(stream)), "sparse_decode")
+
+
+def refine_decode(p: Problem, q, k, v, pool, pool_cnt, kappa_p: int, kappa: int,
+                  softmax_scale: float, idx, cnt, out, ws, lse=None, stream=None):
+    _check(_lib.prism_refine_decode(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(pool), _ptr(pool_cnt),
+                                    kappa_p, kappa, float(softmax_scale), _ptr(idx), _ptr(cnt),
+                                    _ptr(out), _ptr(lse), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "refine_decode")
 
 
 def dense_decode(p: Problem, q, k, v, softmax_scale: float, out, ws, lse=None, stream=None):

@@ -311,3 +311,77 @@ def test_bad_indices_flagged_not_read(P):
     assert np.abs(_np(out) - oout).max() <= 2e-3
     P.clear_device_status(ws)
     assert P.get_device_status(ws) == 0
+
+
+# ------------------------------------------------------------------ fused refine + decode
+
+@pytest.mark.parametrize("case", REFINE_CASES + [([8192], 32, 8, 128, "bf16", 8192, 2048),
+                                                  ([70000, 3], 8, 2, 64, "bf16", 6000, 1500)],
+                         ids=lambda c: f"{c[0]}-{c[1]}/{c[2]}-d{c[3]}-{c[4]}-{c[5]}-{c[6]}")
+def test_refine_decode_vs_oracle(P, case):
+    seqlens, hq, hkv, d, dtype, kp, kap = case
+    B = len(seqlens)
+    prob = problem(P, seqlens, hq, hkv, d, dtype)
+    q, k, v = make_case(seqlens, hq, hkv, d, dtype, seed=12)
+    cu = prob.cu_host
+    rng = np.random.default_rng(13)
+    pool = np.full((B, hkv, kp), -1, np.int32)
+    pcnt = np.zeros((B, hkv), np.int32)
+    for b, L in enumerate(seqlens):
+        for h in range(hkv):
+            n = min(kp, L)
+            pool[b, h, :n] = np.sort(rng.choice(L, n, replace=False))
+            pcnt[b, h] = n
+    idx = torch.full((B, hkv, kap), -7, dtype=torch.int32, device=DEV)
+    cnt = torch.zeros((B, hkv), dtype=torch.int32, device=DEV)
+    out = torch.full((B, hq, d), 77.0, device=DEV)
+    lse = torch.full((B, hq), 77.0, device=DEV)
+    ws = ws_for(P, prob, P.OP_REFINE_DECODE, kp, kap)
+    assert ws.numel() == 256
+    scale = float(np.float32(1 / math.sqrt(d)))
+    P.refine_decode(prob, q, k, v, torch.tensor(pool, device=DEV), torch.tensor(pcnt, device=DEV),
+                    kp, kap, scale, idx, cnt, out, ws, lse=lse)
+    torch.cuda.synchronize()
+    assert P.get_device_status(ws) == 0
+    oidx, ocnt, oscores = pipeline.refine_layer(q, k, cu.tolist(), pool, pcnt, kap)
+    gi, gc = _np(idx), _np(cnt)
+    assert np.array_equal(gc, ocnt)
+    for b in range(B):
+        for h in range(hkv):
+            n = int(pcnt[b, h])
+            r = dict(zip(pool[b, h, :n].tolist(), oscores[(b, h)].tolist()))
+            c = int(ocnt[b, h])
+            check_index_set(gi[b, h, :c], oidx[b, h, :c], lambda t: r[t], f"idx b{b} h{h}")
+            assert np.all(gi[b, h, c:] == -1)
+    # attention over the GPU's own set (cascade control)
+    oout, olse = pipeline.attend_layer(q, k, v, cu.tolist(), gi, gc, scale)
+    tol = atol_for(dtype)
+    assert np.abs(_np(out) - oout).max() <= tol
+    gl = _np(lse)
+    fin = np.isfinite(olse)
+    assert np.array_equal(np.isfinite(gl), fin)
+    assert np.abs(gl[fin] - olse[fin]).max() <= tol * 10
+    assert np.all(_np(out)[~fin] == 0)
+
+
+def test_refine_decode_ties_and_bad_positions(P):
+    seqlens, hq, hkv, d, kp, kap = [4000], 8, 2, 128, 1000, 300
+    prob = problem(P, seqlens, hq, hkv, d, "bf16")
+    q, k, v = make_case(seqlens, hq, hkv, d, "bf16", seed=14)
+    k[:, :] = k[:, :1]  # all scores equal: the lowest pool slots win
+    pool = torch.arange(0, 4 * kp, 4, dtype=torch.int32, device=DEV).repeat(1, hkv, 1)
+    cnt_p = torch.full((1, hkv), kp, dtype=torch.int32, device=DEV)
+    idx = torch.zeros((1, hkv, kap), dtype=torch.int32, device=DEV)
+    cnt = torch.zeros((1, hkv), dtype=torch.int32, device=DEV)
+    out = torch.zeros((1, hq, d), device=DEV)
+    ws = ws_for(P, prob, P.OP_REFINE_DECODE, kp, kap)
+    P.refine_decode(prob, q, k, v, pool, cnt_p, kp, kap, 0.1, idx, cnt, out, ws)
+    for h in range(hkv):
+        assert np.array_equal(_np(idx)[0, h], np.arange(0, 4 * kap, 4))
+    oout, _ = pipeline.attend_layer(q, k, v, [0, 4000], _np(idx), _np(cnt), 0.1)
+    assert np.abs(_np(out) - oout).max() <= 2e-3
+    assert P.get_device_status(ws) == 0
+    # a pool position past the sequence is flagged, ranks last, carries no weight
+    pool[0, 0, 5] = 4000
+    P.refine_decode(prob, q, k, v, pool, cnt_p, kp, kap, 0.1, idx, cnt, out, ws)
+    assert P.get_device_status(ws) & P.DEV_BAD_INDEX

@@ -26,10 +26,10 @@ def _np(t):
         else t.detach().cpu().numpy()
 
 
-def _decoder(P, cfg):
+def _decoder(P, cfg, fused=True):
     return PrismDecoder(cfg.seqlens, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim,
                         P.F32 if cfg.dtype == "f32" else P.BF16, cfg.num_layers, cfg.group,
-                        cfg.kappa_p, cfg.kappa, device=DEV)
+                        cfg.kappa_p, cfg.kappa, device=DEV, fused=fused)
 
 
 def _prefill_kq(P, dec, cfg, lay):
@@ -88,12 +88,13 @@ def _invariants(dec, cfg, l):
     assert np.all(np.isfinite(_np(dec.out[l])))
 
 
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "two-call"])
 @pytest.mark.parametrize("name", ["tiny", "c8k"])
-def test_step_small_configs_every_row(prism_lib, name):
+def test_step_small_configs_every_row(prism_lib, name, fused):
     P = prism_lib
     cfg = workload.config(name)
     layers = list(workload.generate(cfg, DEV))
-    dec = _decoder(P, cfg)
+    dec = _decoder(P, cfg, fused)
     kqs, scs = {}, {}
     for lay in layers:
         if cfg.is_proposal(lay.index):
