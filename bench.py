@@ -398,7 +398,10 @@ def run_prism(args, dist: Dist):
         if pl:
             ops.append(("propose", graph_of(f_prop, stream)))
         ops.append(("refine_decode", graph_of(f_rd, stream)))
-    gate = torch.empty(6 << 30, dtype=torch.uint8, device=dev)
+    # ~30 MB of memset per queued graph launch keeps the device busy while the
+    # host enqueues the profiled sequence
+    gate = torch.empty(min(6 << 30, max(256 << 20, len(ops) * (30 << 20))), dtype=torch.uint8,
+                       device=dev)
     per_op = {}
     for _ in range(args.profile_steps):
         gate.zero_()

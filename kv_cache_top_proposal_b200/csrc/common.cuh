@@ -113,6 +113,76 @@ __device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) 
   return res;
 }
 
+
+// ---- cp.async (16-byte global -> shared copies, L2 only), no mbarrier waits
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+// Copies 16 bytes, or writes 16 zero bytes without reading when !valid.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// Sums each of the GP values v[] over the LPR lanes of an aligned lane group
+// with a transposed butterfly: at each of the first log2(min(GP, LPR)) levels
+// a lane keeps half of the values it carries (the lower half if its level bit
+// is clear) and adds the partner's copy of that half, so GP totals cost about
+// GP + log2(LPR) shuffles instead of GP * log2(LPR).  On return v[0..NH) hold
+// the totals of heads head0(li) .. head0(li) + NH - 1, NH = GP / min(GP, LPR);
+// lanes that differ only in the remaining bits hold identical values.
+template <int GP, int LPR>
+struct GroupSumT {
+  static constexpr int SPLIT = GP < LPR ? GP : LPR;
+  static constexpr int NH = GP / SPLIT;
+
+  __device__ __forceinline__ static void run(float (&v)[GP], int li) {
+    int nh = GP;
+#pragma unroll
+    for (int o = LPR / 2; o > 0; o >>= 1) {
+      if (nh > NH) {
+        const bool up = (li & o) != 0;
+        const int half = nh / 2;
+#pragma unroll
+        for (int j = 0; j < GP / 2; ++j) {
+          if (j < half) {
+            const float mine = up ? v[half + j] : v[j];
+            const float other = up ? v[j] : v[half + j];
+            v[j] = mine + __shfl_xor_sync(0xffffffffu, other, o);
+          }
+        }
+        nh = half;
+      } else {
+#pragma unroll
+        for (int j = 0; j < NH; ++j) v[j] += __shfl_xor_sync(0xffffffffu, v[j], o);
+      }
+    }
+  }
+
+  __device__ __forceinline__ static int head0(int li) {
+    int nh = GP, h = 0;
+#pragma unroll
+    for (int o = LPR / 2; o > 0; o >>= 1) {
+      if (nh > NH) {
+        nh /= 2;
+        if (li & o) h += nh;
+      }
+    }
+    return h;
+  }
+
+  // true on one lane per distinct head set (the lowest such lane)
+  __device__ __forceinline__ static bool writer(int li) { return (li % (LPR / SPLIT)) == 0; }
+};
+
 __host__ __device__ __forceinline__ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 }  // namespace prism

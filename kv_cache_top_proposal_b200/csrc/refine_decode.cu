@@ -5,25 +5,26 @@
 // sec. 1 / 2.1: token-level sparse attention over the selected tokens).
 //
 // One thread-block cluster of CL CTAs owns one (sequence, KV head) row.  CTA
-// c takes a contiguous slice of the row's pool:
-//   1. gathers the key rows of its slice (16-byte loads, lane groups), and
-//      keeps per query head the exact dot products q_g . k (the logits) and
-//      the selection key ord(max_g q_g . k) in shared memory;
+// c takes a contiguous slice of the row's pool (mc members at most):
+//   1. the slice's key rows stream into a ring of shared-memory stages with
+//      cp.async (all stages in flight at once); lane groups compute the exact
+//      dot product with every query head of the group (a transposed butterfly
+//      reduction), keeping the logits and the selection key
+//      ord(max_g q_g . k) in shared memory;
 //   2. the cluster finds the exact kappa-th largest key by an MSD radix
 //      select (11/11/10-bit digits): CTAs push their non-zero histogram bins
 //      into rank 0's shared memory (distributed shared memory atomics), rank 0
 //      locates the digit, every CTA reads it back;
 //   3. every CTA marks its selected members (keys above the threshold, plus
-//      the lowest-position members equal to it), writes their positions to
-//      idx in ascending order (counts exchanged over DSMEM);
-//   4. softmax partial over its selected members: the logits are already in
-//      shared memory, so only the value rows are gathered; the CTA's maximum
-//      is known before the value pass, so no online rescaling is needed;
+//      the lowest-position members equal to it) and writes their positions to
+//      idx in ascending order (per-CTA counts exchanged over DSMEM);
+//   4. softmax partial over the selected members: the logits are already on
+//      chip, so the CTA maximum and the weights 2^(l - m) are computed first
+//      and only the value rows are streamed (same cp.async ring);
 //   5. the CL partials (m, l, o) are merged through DSMEM, each CTA merging a
-//      slice of the G*d outputs: out and lse are written directly.
-// Nothing goes to global scratch; the key rows are read once, the value rows
-// of the selected members once.  Bytes per row: kappa_p key rows + kappa
-// value rows (d * sizeof(T) each).
+//      slice of the G*d outputs, and out / lse are written directly.
+// Nothing goes to global scratch.  Bytes per row: kappa_p key rows and kappa
+// value rows, d * sizeof(T) each.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -37,7 +38,13 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kUnroll = 4;
+constexpr int kStages = 4;
+
+// bytes of one pipeline stage (kStages are in flight)
+template <int GP>
+struct Stage {
+  static constexpr int BYTES = GP <= 4 ? 32768 : 16384;
+};
 
 struct RDArgs {
   const void* q;
@@ -50,7 +57,7 @@ struct RDArgs {
   int kappa;  // selection budget and idx row stride
   int Hkv, G, Hq;
   int64_t T;
-  int mc;     // slice capacity (keys per CTA)
+  int mc;     // slice capacity (members per CTA)
   float scale_log2;
   int32_t* idx;
   int32_t* cnt;
@@ -59,18 +66,60 @@ struct RDArgs {
   int32_t* status;
 };
 
+// Streams `rows` cache rows (row j at position spos[list ? list[j] : j] of
+// base; negative positions are zero-filled without reading) through the
+// stage ring and calls body(first_row, stage, rows_in_chunk) once per chunk
+// of SR rows, with kStages chunks in flight.
+template <typename T, int D, int GP, typename Body>
+__device__ __forceinline__ void stream_rows(const T* base, const int* spos, const int* list,
+                                            int rows, unsigned char* stage, Body body) {
+  constexpr int RB = D * (int)sizeof(T);  // row bytes
+  constexpr int VPR = RB / 16;            // 16-byte vectors per row
+  constexpr int SR = Stage<GP>::BYTES / RB;
+  const int tid = threadIdx.x;
+  const int nchunk = (rows + SR - 1) / SR;
+  auto issue = [&](int c) {
+    if (c < nchunk) {
+      const int r0 = c * SR, n = min(SR, rows - r0);
+      unsigned char* buf = stage + (c % kStages) * Stage<GP>::BYTES;
+      for (int x = tid; x < n * VPR; x += kThreads) {
+        const int r = x / VPR, vv = x - r * VPR;
+        const int pos = spos[list ? list[r0 + r] : r0 + r];
+        const T* src = base + (int64_t)(pos >= 0 ? pos : 0) * D + vv * (16 / (int)sizeof(T));
+        cp_async16(smem_u32(buf + r * RB + vv * 16), src, pos >= 0);
+      }
+    }
+    cp_async_commit();  // one group per call (possibly empty): constant wait depth
+  };
+#pragma unroll
+  for (int c = 0; c < kStages; ++c) issue(c);
+  for (int c = 0; c < nchunk; ++c) {
+    cp_async_wait<kStages - 1>();
+    __syncthreads();
+    body(c * SR, stage + (c % kStages) * Stage<GP>::BYTES, min(SR, rows - c * SR));
+    __syncthreads();
+    issue(c + kStages);
+  }
+  cp_async_wait<0>();
+}
+
 template <typename T, int D, int GP>
-__global__ void __launch_bounds__(kThreads) refine_decode_kernel(const RDArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) refine_decode_kernel(const RDArgs a) {
   constexpr int E = Vec16<T>::E;
   constexpr int LPR = D / E;     // lanes per cache row
   constexpr int RPW = 32 / LPR;  // rows per warp
   constexpr int NG = kThreads / LPR;  // lane groups per CTA
+  constexpr int RB = D * (int)sizeof(T);
+  using GS = GroupSumT<GP, LPR>;
 
   extern __shared__ __align__(16) unsigned char dsm[];
-  uint32_t* keys = reinterpret_cast<uint32_t*>(dsm);              // [mc]
-  float* dots = reinterpret_cast<float*>(keys + a.mc);             // [GP][mc]
-  int* sel = reinterpret_cast<int*>(dots + GP * a.mc);             // [mc]
-  float* comb = reinterpret_cast<float*>(sel + a.mc);              // [kWarps][GP][D]
+  unsigned char* stage = dsm;                                              // kStages stages
+  int* spos = reinterpret_cast<int*>(dsm + kStages * Stage<GP>::BYTES);    // [mc]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(spos + a.mc);               // [mc]
+  float* dots = reinterpret_cast<float*>(keys + a.mc);                     // [GP][mc]
+  float* pw = dots + GP * a.mc;                                            // [mc][GP] weights
+  int* sel = reinterpret_cast<int*>(pw + GP * a.mc);                       // [mc]
+  float* comb = reinterpret_cast<float*>(stage);  // [kWarps][GP][D], after the value pass
 
   __shared__ uint32_t ghist[2][2048];  // cluster histogram (used in rank 0)
   __shared__ uint32_t lh[2048];        // this CTA's histogram
@@ -78,7 +127,7 @@ __global__ void __launch_bounds__(kThreads) refine_decode_kernel(const RDArgs a)
   __shared__ int s_res[2];             // rank 0: digit, count above it
   __shared__ int s_cnt[2];             // published: #equal, #greater
   __shared__ int s_before[2];
-  __shared__ float s_max[kWarps][GP];
+  __shared__ float s_red[kWarps][GP];
   __shared__ float part_o[GP * D];     // published partial
   __shared__ float part_m[GP], part_l[GP];
 
@@ -102,9 +151,20 @@ __global__ void __launch_bounds__(kThreads) refine_decode_kernel(const RDArgs a)
   const int lo = min(n, rank * chunk), hi = min(n, lo + chunk);
   const int m = hi - lo;
   const int32_t* pool = a.pool + (int64_t)row * a.kp + lo;
-  const int64_t off = ((int64_t)h * a.T + t0) * D + li * E;
-  const T* kbase = static_cast<const T*>(a.k) + off;
-  const T* vbase = static_cast<const T*>(a.v) + off;
+  const int64_t rowbase = ((int64_t)h * a.T + t0) * D;
+  const T* kb = static_cast<const T*>(a.k) + rowbase;
+  const T* vb = static_cast<const T*>(a.v) + rowbase;
+
+  // ---- 0. the slice's positions (an out-of-range one is flagged, skipped)
+  for (int i = tid; i < m; i += kThreads) {
+    const int p = pool[i];
+    const bool ok = p >= 0 && p < L;
+    if (!ok) flag_status(a.status, PRISM_DEV_BAD_INDEX);
+    spos[i] = ok ? p : -1;
+  }
+  if (rank == 0)
+    for (int i = tid; i < 2048; i += kThreads) ghist[0][i] = 0;
+  __syncthreads();
 
   // ---- 1. exact scores of the slice
   {
@@ -119,49 +179,44 @@ __global__ void __launch_bounds__(kThreads) refine_decode_kernel(const RDArgs a)
         for (int e = 0; e < E; ++e) qf[g][e] = 0.0f;
       }
     }
-    // warp-uniform trip count (group_sum shuffles over the whole warp);
-    // lane group grp takes members grp, grp + NG, grp + 2*NG, ...
-    for (int wb = warp * RPW; wb < m; wb += NG * kUnroll) {
-      const int base = wb + sub;
-      uint4 raw[kUnroll];
-      bool ok[kUnroll];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int e = base + u * NG;
-        const bool in = e < m;
-        const int pos = in ? pool[e] : 0;
-        ok[u] = in && pos >= 0 && pos < L;
-        if (in && !ok[u] && li == 0) flag_status(a.status, PRISM_DEV_BAD_INDEX);
-        raw[u] = ok[u] ? ld16(kbase + (int64_t)pos * D) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+    const int h0 = GS::head0(li);
+    stream_rows<T, D, GP>(kb, spos, nullptr, m, stage,
+                          [&](int r0, const unsigned char* buf, int nrows) {
+      // warp-uniform trip count: the reduction shuffles over the whole warp
+      for (int wb = warp * RPW; wb < nrows; wb += NG) {
+        const int r = wb + sub;
+        const bool in = r < nrows;
         float f[E];
-        Vec16<T>::unpack(raw[u], f);
+        Vec16<T>::unpack(in ? *reinterpret_cast<const uint4*>(buf + r * RB + li * 16)
+                            : make_uint4(0, 0, 0, 0), f);
         float acc[GP];
 #pragma unroll
         for (int g = 0; g < GP; ++g) {
           float s = 0.0f;
 #pragma unroll
           for (int e = 0; e < E; ++e) s = fmaf(qf[g][e], f[e], s);
-          acc[g] = group_sum<LPR>(s);
+          acc[g] = s;
         }
-        float best = acc[0];
+        GS::run(acc, li);
+        float best = -INFINITY;
 #pragma unroll
-        for (int g = 1; g < GP; ++g)
-          if (g < a.G) best = fmaxf(best, acc[g]);
-        const int e = base + u * NG;
-        if (e < m && li == 0) {
-          // a position outside its sequence ranks last and carries no weight
-          keys[e] = ord_key(ok[u] ? best : -INFINITY);
+        for (int j = 0; j < GS::NH; ++j)
+          if (h0 + j < a.G) best = fmaxf(best, acc[j]);
 #pragma unroll
-          for (int g = 0; g < GP; ++g) dots[g * a.mc + e] = ok[u] ? acc[g] : -INFINITY;
+        for (int o = LPR / 2; o >= LPR / GS::SPLIT && o > 0; o >>= 1)
+          best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
+        if (in) {
+          const int i = r0 + r;
+          const bool ok = spos[i] >= 0;  // an out-of-range position ranks last, weighs 0
+          if (GS::writer(li)) {
+#pragma unroll
+            for (int j = 0; j < GS::NH; ++j) dots[(h0 + j) * a.mc + i] = ok ? acc[j] : -INFINITY;
+          }
+          if (li == 0) keys[i] = ord_key(ok ? best : -INFINITY);
         }
       }
-    }
+    });
   }
-  if (rank == 0)
-    for (int i = tid; i < 2048; i += kThreads) ghist[0][i] = 0;
   cluster.sync();  // scores of every slice ready; rank 0's histogram cleared
 
   // ---- 2. cluster radix select of the kappa-th largest key
@@ -297,68 +352,70 @@ __global__ void __launch_bounds__(kThreads) refine_decode_kernel(const RDArgs a)
   for (int g = 0; g < GP; ++g) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], o));
-    if (lane == 0) s_max[warp][g] = mx[g];
+    if (lane == 0) s_red[warp][g] = mx[g];
   }
   __syncthreads();
 #pragma unroll
   for (int g = 0; g < GP; ++g) {
-    float v = s_max[0][g];
+    float v = s_red[0][g];
 #pragma unroll
-    for (int w = 1; w < kWarps; ++w) v = fmaxf(v, s_max[w][g]);
+    for (int w = 1; w < kWarps; ++w) v = fmaxf(v, s_red[w][g]);
     mx[g] = v * a.scale_log2;  // CTA maximum logit (log2 domain); -inf if nothing selected
   }
-  float lsum[GP], o[GP][E];
+  __syncthreads();
+  float lsum[GP];
 #pragma unroll
-  for (int g = 0; g < GP; ++g) {
-    lsum[g] = 0.0f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) o[g][e] = 0.0f;
-  }
-  for (int wb = warp * RPW; wb < nsel; wb += NG * kUnroll) {
-    const int base = wb + sub;
-    uint4 raw[kUnroll];
-    int il[kUnroll];
-    bool ok[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int j = base + u * NG;
-      ok[u] = j < nsel;
-      il[u] = ok[u] ? sel[j] : 0;
-      const int pos = ok[u] ? pool[il[u]] : 0;
-      ok[u] = ok[u] && pos >= 0 && pos < L;
-      raw[u] = ok[u] ? ld16(vbase + (int64_t)pos * D) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (!ok[u]) continue;
-      float f[E];
-      Vec16<T>::unpack(raw[u], f);
-#pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        const float p = exp2f(dots[g * a.mc + il[u]] * a.scale_log2 - mx[g]);
-        lsum[g] += p;
-#pragma unroll
-        for (int e = 0; e < E; ++e) o[g][e] = fmaf(p, f[e], o[g][e]);
-      }
-    }
-  }
-  // lane groups of a warp hold the same feature slice: add them, then warps
-#pragma unroll
-  for (int g = 0; g < GP; ++g) {
-#pragma unroll
-    for (int s = LPR; s < 32; s <<= 1) {
-      lsum[g] += __shfl_xor_sync(0xffffffffu, lsum[g], s);
-#pragma unroll
-      for (int e = 0; e < E; ++e) o[g][e] += __shfl_xor_sync(0xffffffffu, o[g][e], s);
-    }
-  }
-  if (sub == 0) {
+  for (int g = 0; g < GP; ++g) lsum[g] = 0.0f;
+  for (int j = tid; j < nsel; j += kThreads) {
+    const int i = sel[j];
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
+      const float l = dots[g * a.mc + i];
+      const float p = l == -INFINITY ? 0.0f : exp2f(l * a.scale_log2 - mx[g]);
+      pw[j * GP + g] = p;
+      lsum[g] += p;
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lsum[g] += __shfl_xor_sync(0xffffffffu, lsum[g], o);
+    if (lane == 0) s_red[warp][g] = lsum[g];
+  }
+  float o[GP][E];
+#pragma unroll
+  for (int g = 0; g < GP; ++g)
+#pragma unroll
+    for (int e = 0; e < E; ++e) o[g][e] = 0.0f;
+  // stream the selected value rows (the weights are read after the first
+  // stage barrier inside stream_rows)
+  stream_rows<T, D, GP>(vb, spos, sel, nsel, stage,
+                        [&](int j0, const unsigned char* buf, int nrows) {
+    for (int r = warp * RPW + sub; r < nrows; r += NG) {
+      float f[E];
+      Vec16<T>::unpack(*reinterpret_cast<const uint4*>(buf + r * RB + li * 16), f);
+      const float* p = pw + (j0 + r) * GP;
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        const float pg = p[g];
+#pragma unroll
+        for (int e = 0; e < E; ++e) o[g][e] = fmaf(pg, f[e], o[g][e]);
+      }
+    }
+  });
+  // lane groups of a warp hold the same feature slice: add them, then warps
+#pragma unroll
+  for (int g = 0; g < GP; ++g)
+#pragma unroll
+    for (int s = LPR; s < 32; s <<= 1)
+#pragma unroll
+      for (int e = 0; e < E; ++e) o[g][e] += __shfl_xor_sync(0xffffffffu, o[g][e], s);
+  __syncthreads();  // the stage ring is free: reuse it for the warp partials
+  if (sub == 0) {
+#pragma unroll
+    for (int g = 0; g < GP; ++g)
 #pragma unroll
       for (int e = 0; e < E; ++e) comb[(warp * GP + g) * D + li * E + e] = o[g][e];
-      if (li == 0) s_max[warp][g] = lsum[g];
-    }
   }
   __syncthreads();
   for (int i = tid; i < GP * D; i += kThreads) {
@@ -370,7 +427,7 @@ __global__ void __launch_bounds__(kThreads) refine_decode_kernel(const RDArgs a)
   if (tid < GP) {
     float s = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) s += s_max[w][tid];
+    for (int w = 0; w < kWarps; ++w) s += s_red[w][tid];
     part_l[tid] = s;
     part_m[tid] = mx[tid];
   }
@@ -411,18 +468,23 @@ __global__ void __launch_bounds__(kThreads) refine_decode_kernel(const RDArgs a)
   cluster.sync();  // keep shared memory alive until every remote read is done
 }
 
-template <typename T, int D, int GP>
-int smem_bytes(int mc) {
-  return mc * (int)(sizeof(uint32_t) + GP * sizeof(float) + sizeof(int)) +
-         kWarps * GP * D * (int)sizeof(float);
+template <int GP>
+constexpr int per_member_bytes() {
+  return (int)(2 * sizeof(int) + sizeof(uint32_t) + 2 * GP * sizeof(float));
 }
 
-constexpr int kMaxDynSmem = 160 * 1024;
+template <int GP>
+int smem_bytes(int mc) {
+  return kStages * Stage<GP>::BYTES + mc * per_member_bytes<GP>();
+}
+
+// dynamic shared memory available next to the kernel's static arrays
+constexpr int kDynBudget = 227 * 1024 - 40 * 1024;
 
 template <typename T, int D, int GP>
 cudaError_t run(const Dims& d, RDArgs a, int cl, cudaStream_t st) {
   auto kern = refine_decode_kernel<T, D, GP>;
-  const int smem = smem_bytes<T, D, GP>(a.mc);
+  const int smem = smem_bytes<GP>(a.mc);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   if (cl > 8) {
@@ -455,10 +517,10 @@ cudaError_t by_group(const Dims& d, const RDArgs& a, int cl, cudaStream_t st) {
   }
 }
 
-int slice_capacity(int D, int GP) {
-  const int fixed = kWarps * GP * D * (int)sizeof(float);
-  const int per = (int)(sizeof(uint32_t) + GP * sizeof(float) + sizeof(int));
-  return (kMaxDynSmem - fixed) / per;
+int slice_capacity(int GP) {
+  const int stages = kStages * (GP <= 4 ? 32768 : 16384);
+  const int per = (int)(2 * sizeof(int) + sizeof(uint32_t) + 2 * GP * sizeof(float));
+  return (kDynBudget - stages) / per;
 }
 
 }  // namespace
@@ -468,7 +530,7 @@ RefineDecodePlan plan_refine_decode(const Dims& d, int kappa_p) {
   const int GP = padded_group(d.G);
   int cl = 1;
   while (cl < 16 && (int64_t)rows * cl < d.num_sms) cl *= 2;
-  const int cap = slice_capacity(d.D, GP);
+  const int cap = slice_capacity(GP);
   while (cl < 16 && (kappa_p + cl - 1) / cl > cap) cl *= 2;
   const int mc = (kappa_p + cl - 1) / cl;
   return RefineDecodePlan{cl, mc, mc <= cap};
