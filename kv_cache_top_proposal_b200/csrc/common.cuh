@@ -183,6 +183,18 @@ struct GroupSumT {
   __device__ __forceinline__ static bool writer(int li) { return (li % (LPR / SPLIT)) == 0; }
 };
 
+// Histogram increment aggregated over the warp: lanes with valid = true add
+// one to hist[bin]; lanes that share a bin issue a single atomic (scores
+// concentrate in few bins, where per-lane atomics would serialise).  Call
+// with the whole warp (warp-uniform control flow).
+__device__ __forceinline__ void warp_hist_add(uint32_t* hist, uint32_t bin, bool valid) {
+  const unsigned act = __ballot_sync(0xffffffffu, valid);
+  if (!act) return;
+  const unsigned peers = __match_any_sync(0xffffffffu, valid ? bin : 0xffffffffu) & act;
+  const int lane = threadIdx.x & 31;
+  if (valid && (peers & ((1u << lane) - 1u)) == 0) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+}
+
 __host__ __device__ __forceinline__ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 }  // namespace prism

@@ -110,9 +110,10 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelectArgs a)
     const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
     const int nb = pass == 2 ? 1024 : 2048;
     uint32_t* hh = hist[pass & 1];
-    for (int i = tid; i < m; i += kThreads) {
-      const uint32_t key = skeys[i];
-      if ((key & pmask) == prefix) atomicAdd(&hh[(key >> shift) & (nb - 1)], 1u);
+    for (int i0 = tid & ~31; i0 < m; i0 += kThreads) {  // warp-uniform trip count
+      const int i = i0 + (tid & 31);
+      const uint32_t key = i < m ? skeys[i] : 0u;
+      warp_hist_add(hh, (key >> shift) & (nb - 1), i < m && (key & pmask) == prefix);
     }
     cluster.sync();  // every CTA's histogram of this pass is complete
     // All CTAs have finished reading the other buffer (previous pass) before
