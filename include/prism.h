@@ -192,13 +192,18 @@ PRISM_API prism_status prism_sparse_decode(const prism_shape* shape, const void*
  * the key rows of the pool are read once.  Returns PRISM_ERR_UNSUPPORTED when
  * a pool of kappa_p members does not fit on chip (kappa_p > 16 x the slice
  * capacity: 6144 members per CTA at G <= 4, d = 128); use the two calls then.
+ * k_prefetch, if not NULL, is the key cache ([Hkv][T][d], same shape) of the
+ * next layer that will be refined on the same pool: once this layer's key
+ * rows are consumed, the same pool rows of k_prefetch are prefetched into L2
+ * (a hint; results do not depend on it).
  */
 PRISM_API prism_status prism_refine_decode(const prism_shape* shape, const void* q, const void* k,
                                            const void* v, const int32_t* pool_idx,
                                            const int32_t* pool_cnt, int32_t kappa_p,
                                            int32_t kappa, float softmax_scale, int32_t* idx,
-                                           int32_t* cnt, float* out, float* lse_opt, void* ws,
-                                           size_t ws_bytes, void* stream);
+                                           int32_t* cnt, float* out, float* lse_opt,
+                                           const void* k_prefetch, void* ws, size_t ws_bytes,
+                                           void* stream);
 
 /*
  * Dense decode attention over every position t < L_b (the comparison path):

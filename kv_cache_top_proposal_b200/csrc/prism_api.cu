@@ -66,7 +66,7 @@ prism_status cuda_status(cudaError_t e) { return e == cudaSuccess ? PRISM_OK : P
 
 // Workspace layout per operation (offsets after the 256-byte header).
 struct Layout {
-  size_t a = 0, b = 0, total = 0;  // a: first array, b: second array
+  size_t a = 0, b = 0, c = 0, d = 0, e = 0, total = 0;  // array offsets
 };
 
 Layout layout(const Dims& d, int op, int kappa_p, int kappa) {
@@ -76,10 +76,21 @@ Layout layout(const Dims& d, int op, int kappa_p, int kappa) {
   switch (op) {
     case PRISM_OP_QUANTIZE:
       break;
-    case PRISM_OP_PROPOSE:  // scores [Hkv][T] fp32
+    case PRISM_OP_PROPOSE: {  // scores [Hkv][T] fp32, then the selection scratch
       L.a = off;
       off = align_up(off + (size_t)d.Hkv * (size_t)d.T * sizeof(float));
+      const size_t cl = (size_t)propose_select_cluster();
+      const size_t cap = (size_t)propose_select_cap(d.max_len);
+      L.b = off;  // hist [rows][4096] u32
+      off = align_up(off + rows * 4096 * 4);
+      L.c = off;  // candidate keys [rows][cl][cap]
+      off = align_up(off + rows * cl * cap * 4);
+      L.d = off;  // candidate positions [rows][cl][cap]
+      off = align_up(off + rows * cl * cap * 4);
+      L.e = off;  // per-CTA counts [rows][cl][2], results [rows][2 + cl]
+      off = align_up(off + rows * cl * 2 * 4 + rows * (2 + cl) * 4);
       break;
+    }
     case PRISM_OP_REFINE:  // r [rows][kappa_p], dots [rows][G][kappa_p]
       L.a = off;
       off = align_up(off + rows * (size_t)kappa_p * sizeof(float));
@@ -176,7 +187,21 @@ prism_status prism_propose(const prism_shape* shape, const void* q, const int8_t
   int32_t* status = reinterpret_cast<int32_t*>(w);
   float* scores = reinterpret_cast<float*>(w + L.a);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_propose_scores(d, q, kq, k_scale, scores, use_mma_scorer(), st);
+  const bool mma = use_mma_scorer() && d.bf16;
+  if (mma && d.max_len <= propose_select_max_row()) {
+    // scorer builds the first-digit histogram; selection resolves from it
+    uint32_t* hist = reinterpret_cast<uint32_t*>(w + L.b);
+    const size_t rows = (size_t)d.B * d.Hkv;
+    if (cudaMemsetAsync(hist, 0, rows * 4096 * 4, st) != cudaSuccess) return PRISM_ERR_CUDA;
+    cudaError_t e = launch_propose_scores(d, q, kq, k_scale, scores, hist, true, st);
+    if (e != cudaSuccess) return PRISM_ERR_CUDA;
+    int32_t* meta = reinterpret_cast<int32_t*>(w + L.e);
+    return cuda_status(launch_propose_select(
+        d, scores, hist, kappa_p, propose_select_cap(d.max_len), reinterpret_cast<uint32_t*>(w + L.c),
+        reinterpret_cast<int32_t*>(w + L.d), meta, meta + rows * propose_select_cluster() * 2,
+        pool_idx, pool_cnt, status, st));
+  }
+  cudaError_t e = launch_propose_scores(d, q, kq, k_scale, scores, nullptr, mma, st);
   if (e != cudaSuccess) return PRISM_ERR_CUDA;
   SelectArgs a{};
   a.mode = 0;
@@ -256,8 +281,8 @@ prism_status prism_sparse_decode(const prism_shape* shape, const void* q, const 
 prism_status prism_refine_decode(const prism_shape* shape, const void* q, const void* k,
                                  const void* v, const int32_t* pool_idx, const int32_t* pool_cnt,
                                  int32_t kappa_p, int32_t kappa, float softmax_scale, int32_t* idx,
-                                 int32_t* cnt, float* out, float* lse_opt, void* ws,
-                                 size_t ws_bytes, void* stream) {
+                                 int32_t* cnt, float* out, float* lse_opt, const void* k_prefetch,
+                                 void* ws, size_t ws_bytes, void* stream) {
   Dims d;
   prism_status s = check_shape(shape, &d);
   if (s != PRISM_OK) return s;
@@ -268,8 +293,8 @@ prism_status prism_refine_decode(const prism_shape* shape, const void* q, const 
   if (!ws_ok(ws, ws_bytes, L)) return PRISM_ERR_WORKSPACE;
   const RefineDecodePlan p = plan_refine_decode(d, kappa_p);
   if (!p.ok) return PRISM_ERR_UNSUPPORTED;
-  return cuda_status(launch_refine_decode(d, p, q, k, v, pool_idx, pool_cnt, kappa_p, kappa,
-                                          softmax_scale, idx, cnt, out, lse_opt,
+  return cuda_status(launch_refine_decode(d, p, q, k, v, k_prefetch, pool_idx, pool_cnt, kappa_p,
+                                          kappa, softmax_scale, idx, cnt, out, lse_opt,
                                           static_cast<int32_t*>(ws), static_cast<cudaStream_t>(stream)));
 }
 

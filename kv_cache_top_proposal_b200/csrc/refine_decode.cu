@@ -55,6 +55,7 @@ struct RDArgs {
   const void* q;
   const void* k;
   const void* v;
+  const void* k_next;  // next layer's keys: pool rows prefetched into L2, or null
   const int32_t* cu;
   const int32_t* pool;
   const int32_t* pool_cnt;
@@ -579,6 +580,18 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
                       },
                       [] {});
   }
+  // the next layer's key rows at the same pool positions into L2, while
+  // this layer selects and attends (the DRAM is otherwise idle meanwhile)
+  if (a.k_next && wid >= 0) {
+    const T* kn = static_cast<const T*>(a.k_next) + rowbase;
+    for (int i = tid; i < m; i += kThreads) {
+      const int pos = spos[i];
+      if (pos >= 0)
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(kn + (int64_t)pos * D),
+                     "r"(RB)
+                     : "memory");
+    }
+  }
   cluster_wait();
   __syncthreads();
   // the local first-digit histogram into rank 0's (a lone CTA: into its ring)
@@ -887,12 +900,13 @@ RefineDecodePlan plan_refine_decode(const Dims& d, int kappa_p) {
 }
 
 cudaError_t launch_refine_decode(const Dims& d, const RefineDecodePlan& p, const void* q,
-                                 const void* k, const void* v, const int32_t* pool,
+                                 const void* k, const void* v, const void* k_next,
+                                 const int32_t* pool,
                                  const int32_t* pool_cnt, int kappa_p, int kappa,
                                  float softmax_scale, int32_t* idx, int32_t* cnt, float* out,
                                  float* lse, int32_t* status, cudaStream_t st) {
   if (d.B * d.Hkv == 0) return cudaSuccess;
-  RDArgs a{q, k, v, d.cu_dev, pool, pool_cnt, kappa_p, kappa, d.Hkv, d.G, d.Hq, d.T, p.mc,
+  RDArgs a{q, k, v, k_next, d.cu_dev, pool, pool_cnt, kappa_p, kappa, d.Hkv, d.G, d.Hq, d.T, p.mc,
            ring_bytes(kappa_p, padded_group(d.G), d.D, p.cluster),
            softmax_scale * 1.4426950408889634f, idx, cnt, out, lse, status};
   if (d.bf16)

@@ -17,9 +17,10 @@
 //    to fp16, exact for every element down to 2^-31 of the largest; products
 //    are exact and accumulate in fp32.  The feature axis is permuted so that
 //    each thread's A-fragment elements are two contiguous 16-byte pieces of
-//    its rows (the same permutation is applied to the query), so rows load
-//    straight from global memory with fully used 32-byte sectors, double
-//    buffered in registers.
+//    its rows (the same permutation is applied to the query).  Rows stream
+//    through a ring of shared-memory stages filled by cp.async (six 16 KB
+//    stages in flight per CTA, two CTAs per SM), so the kernel keeps enough
+//    bytes in flight to run at HBM speed.
 //  * score_simt_kernel: plain fp32 FMAs on CUDA cores (fp32 queries, and the
 //    comparison kernel for bf16).
 #include "common.cuh"
@@ -30,7 +31,6 @@ namespace prism {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
 constexpr int kChunkRows = 1024;  // key rows of one (sequence, KV head) per work item
 
 struct ScoreArgs {
@@ -38,20 +38,21 @@ struct ScoreArgs {
   const int8_t* kq;
   const float* scale;
   float* scores;
+  uint32_t* hist;  // [B*Hkv][kHist] first-digit histogram of ord(score), or null
   const int32_t* cu;
   int64_t T;
   int B, Hkv, G;
 };
 
 // s_pref[b] = number of work items of sequences before b (per KV head).
-__device__ void chunk_prefix(const int32_t* __restrict__ cu, int B, int* s_pref) {
+__device__ void chunk_prefix(const int32_t* __restrict__ cu, int B, int rows_per_item, int* s_pref) {
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
     int carry = 0;
     for (int b0 = 0; b0 < B; b0 += 32) {
       const int b = b0 + lane;
       int n = 0;
-      if (b < B) n = (cu[b + 1] - cu[b] + kChunkRows - 1) / kChunkRows;
+      if (b < B) n = (cu[b + 1] - cu[b] + rows_per_item - 1) / rows_per_item;
       const int inc = warp_incl_scan(n);
       if (b < B) s_pref[b + 1] = carry + inc;
       carry += __shfl_sync(0xffffffffu, inc, 31);
@@ -100,97 +101,195 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
 }
 
 // Tensor-core scorer.  NT = number of 8-wide query-head tiles (G <= 8*NT).
+// Persistent CTAs walk a flat list of 128-row stages (stage s of KV head h,
+// sequence b), kScoreStages of them in flight per CTA through a cp.async ring
+// (codes + scales); warp w takes 16-row tile w of each stage.
+constexpr int kStageRows = 128;
+constexpr int kScoreStages = 5;
+constexpr int kHist = 4096;  // first radix digit of the selection keys (12 bits)
+
+template <int D>
+struct StageLayout {
+  static constexpr int ROWB = D;                         // int8 codes per row
+  static constexpr int CODES = kStageRows * ROWB;        // code bytes per stage
+  static constexpr int BYTES = CODES + kStageRows * 4;   // + fp32 scales
+  // 16-byte chunk c of row r: rows g and g+1 of a quarter-warp read chunks
+  // tig (and 4 + tig); flipping bit 2 on odd rows puts them in different
+  // bank halves at d = 128
+  __device__ __forceinline__ static int off(int r, int c) {
+    return r * ROWB + ((D == 128 ? (c ^ ((r & 1) << 2)) : c) << 4);
+  }
+};
+
+// 2^e as an exact float for e in [-126, 127]
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
+
+// Walks stages (KV head h, sequence b, first row r0) in order, skipping empty
+// sequences; cu is the shared-memory copy of cu_seqlens.  No divisions.
+struct StageIter {
+  int h, b, r0;
+  __device__ __forceinline__ void advance(const int* cu, int B) {
+    r0 += kStageRows;
+    while (h >= 0 && r0 >= cu[b + 1] - cu[b]) {
+      r0 = 0;
+      if (++b == B) {
+        b = 0;
+        ++h;
+      }
+    }
+  }
+};
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src) : "memory");
+}
+
 template <int D, int NT>
-__global__ void __launch_bounds__(kThreads) score_mma_kernel(ScoreArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) score_mma_kernel(ScoreArgs a) {
   constexpr int KS = D / 16;   // k-steps of 16 features
   constexpr int NCH = D / 64;  // 16-byte pieces per thread per row
-  extern __shared__ int s_pref[];
-  chunk_prefix(a.cu, a.B, s_pref);
+  constexpr int VPR = D / 16;  // 16-byte chunks per row
+  using SL = StageLayout<D>;
+  extern __shared__ __align__(16) unsigned char ring[];  // stages, hist, s_pref[B+1], cu[B+1]
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(ring + kScoreStages * SL::BYTES);
+  int* s_pref = reinterpret_cast<int*>(s_hist + kHist);
+  int* s_cu = s_pref + a.B + 1;
+  for (int i = threadIdx.x; i <= a.B; i += kThreads) s_cu[i] = a.cu[i];
+  for (int i = threadIdx.x; i < kHist; i += kThreads) s_hist[i] = 0u;
+  chunk_prefix(a.cu, a.B, kStageRows, s_pref);
   const int per_head = s_pref[a.B];
   const int64_t total = (int64_t)a.Hkv * per_head;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tig = lane & 3;
   const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
-
-  for (int64_t c = blockIdx.x; c < total; c += gridDim.x) {
-    const int h = (int)(c / per_head);
-    const int cc = (int)(c - (int64_t)h * per_head);
+  // this CTA's contiguous range of stages
+  const int64_t s_begin = total * blockIdx.x / gridDim.x;
+  const int64_t s_end = total * (blockIdx.x + 1) / gridDim.x;
+  const int nk = (int)(s_end - s_begin);
+  StageIter it_issue, it_comp;
+  {
+    const int h = (int)(s_begin / per_head);
+    const int cc = (int)(s_begin - (int64_t)h * per_head);
     const int b = find_seq(s_pref, a.B, cc);
-    const int t0 = a.cu[b];
-    const int r0 = (cc - s_pref[b]) * kChunkRows;
-    const int rows = min(kChunkRows, a.cu[b + 1] - t0 - r0);
-    const int64_t rowbase = (int64_t)h * a.T + t0 + r0;
+    it_issue = StageIter{h, b, (cc - s_pref[b]) * kStageRows};
+    it_comp = it_issue;
+  }
 
-    // Query fragments (B operand, "col" layout): thread (g, tig) holds
-    // column n = g of each head tile; k-step s covers features
-    // base(s) .. base(s)+3 with base(s) = 64*(s/4) + 16*tig + 4*(s%4).
-    uint32_t bq[NT][KS][2];
-    int qexp;
-    {
+  auto issue = [&](int kk) {
+    if (kk < nk) {
+      const int L = s_cu[it_issue.b + 1] - s_cu[it_issue.b];
+      const int rows = min(kStageRows, L - it_issue.r0);
+      const int64_t rowbase = (int64_t)it_issue.h * a.T + s_cu[it_issue.b] + it_issue.r0;
+      unsigned char* buf = ring + (kk % kScoreStages) * SL::BYTES;
+      const int8_t* src = a.kq + rowbase * D;
+      for (int x = tid; x < rows * VPR; x += kThreads) {
+        const int r = x / VPR, c = x - r * VPR;
+        cp_async16(smem_u32(buf + SL::off(r, c)), src + r * D + c * 16, true);
+      }
+      if (tid < rows) cp_async4(smem_u32(buf + SL::CODES + tid * 4), a.scale + rowbase + tid);
+      it_issue.advance(s_cu, a.B);
+    }
+    cp_async_commit();
+  };
+
+  uint32_t bq[NT][KS][2];
+  float unscale = 1.0f;
+  int cur_b = -1, cur_h = -1;
+  int hist_row = -1;  // (sequence, KV head) row the shared histogram holds
+  auto flush = [&]() {  // shared histogram -> global (non-zero bins), then clear
+    if (a.hist && hist_row >= 0) {
+      uint32_t* gh = a.hist + (int64_t)hist_row * kHist;
+      for (int i = tid; i < kHist; i += kThreads) {
+        const uint32_t c = s_hist[i];
+        if (c) {
+          atomicAdd(gh + i, c);
+          s_hist[i] = 0u;
+        }
+      }
+    }
+    __syncthreads();
+  };
+#pragma unroll 1
+  for (int kk = 0; kk < kScoreStages; ++kk) issue(kk);
+#pragma unroll 1
+  for (int kk = 0; kk < nk; ++kk) {
+    const int L = s_cu[it_comp.b + 1] - s_cu[it_comp.b];
+    const int rows = min(kStageRows, L - it_comp.r0);
+    const int64_t rowbase = (int64_t)it_comp.h * a.T + s_cu[it_comp.b] + it_comp.r0;
+    if (it_comp.b != cur_b || it_comp.h != cur_h) {
+      // query fragments of (b, h), scaled by a power of two into fp16 range;
+      // thread (g, tig) holds column n = g; k-step s covers features
+      // base(s) .. base(s)+3, base(s) = 64*(s/4) + 16*tig + 4*(s%4)
+      cur_b = it_comp.b;
+      cur_h = it_comp.h;
       float qv[NT][KS][4];
       float mx = 0.0f;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int n = nt * 8 + g;
 #pragma unroll
-        for (int s = 0; s < KS; ++s) {
-          const int base = 64 * (s / 4) + 16 * tig + 4 * (s % 4);
+        for (int s2 = 0; s2 < KS; ++s2) {
+          const int base = 64 * (s2 / 4) + 16 * tig + 4 * (s2 % 4);
           if (n < a.G) {
             const uint2 w = *reinterpret_cast<const uint2*>(
-                q + ((int64_t)b * a.Hkv * a.G + (int64_t)h * a.G + n) * D + base);
-            qv[nt][s][0] = bf16lo(w.x); qv[nt][s][1] = bf16hi(w.x);
-            qv[nt][s][2] = bf16lo(w.y); qv[nt][s][3] = bf16hi(w.y);
+                q + ((int64_t)cur_b * a.Hkv * a.G + (int64_t)cur_h * a.G + n) * D + base);
+            qv[nt][s2][0] = bf16lo(w.x); qv[nt][s2][1] = bf16hi(w.x);
+            qv[nt][s2][2] = bf16lo(w.y); qv[nt][s2][3] = bf16hi(w.y);
           } else {
-            qv[nt][s][0] = qv[nt][s][1] = qv[nt][s][2] = qv[nt][s][3] = 0.0f;
+            qv[nt][s2][0] = qv[nt][s2][1] = qv[nt][s2][2] = qv[nt][s2][3] = 0.0f;
           }
 #pragma unroll
-          for (int e = 0; e < 4; ++e) mx = fmaxf(mx, fabsf(qv[nt][s][e]));
+          for (int e = 0; e < 4; ++e) mx = fmaxf(mx, fabsf(qv[nt][s2][e]));
         }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      int e2 = 0;
-      frexpf(mx, &e2);  // mx < 2^e2
-      qexp = (mx > 0.0f) ? 15 - e2 : 0;
+      // largest |q| scaled into [2^14, 2^15): exponent of mx from its bits
+      // (mx is a normal fp32 or 0); kept inside the normal range of 2^e
+      int qexp = 0;
+      if (mx > 0.0f) {
+        const int e2 = ((__float_as_int(mx) >> 23) & 0xFF) - 126;  // mx < 2^e2
+        qexp = min(126, max(-126, 15 - e2));
+      }
+      const float up = pow2f(qexp);
+      unscale = pow2f(-qexp);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int s = 0; s < KS; ++s) {
-          bq[nt][s][0] = pack_f16(ldexpf(qv[nt][s][0], qexp), ldexpf(qv[nt][s][1], qexp));
-          bq[nt][s][1] = pack_f16(ldexpf(qv[nt][s][2], qexp), ldexpf(qv[nt][s][3], qexp));
+        for (int s2 = 0; s2 < KS; ++s2) {
+          bq[nt][s2][0] = pack_f16(qv[nt][s2][0] * up, qv[nt][s2][1] * up);
+          bq[nt][s2][1] = pack_f16(qv[nt][s2][2] * up, qv[nt][s2][3] * up);
         }
     }
-
-    const int ntiles = (rows + 15) / 16;
-    uint4 cur[2][NCH], nxt[2][NCH];
-    float csc = 0.0f, nsc = 0.0f;
-    auto load = [&](int t, uint4 (&buf)[2][NCH], float& sc) {
+    const int row_id = it_comp.b * a.Hkv + it_comp.h;  // CTA-uniform
+    if (row_id != hist_row) {
+      flush();
+      hist_row = row_id;
+    }
+    it_comp.advance(s_cu, a.B);
+    cp_async_wait<kScoreStages - 1>();
+    __syncthreads();
+    const unsigned char* buf = ring + (kk % kScoreStages) * SL::BYTES;
+    const int t = warp;  // one 16-row tile per warp
+    if (t * 16 < rows) {
+      uint4 cur[2][NCH];
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const int r = t * 16 + g + 8 * half;
 #pragma unroll
         for (int ch = 0; ch < NCH; ++ch)
-          buf[half][ch] = (r < rows) ? ld16_stream(a.kq + (rowbase + r) * D + ch * 64 + tig * 16)
-                                     : make_uint4(0, 0, 0, 0);
+          cur[half][ch] = *reinterpret_cast<const uint4*>(buf + SL::off(r, ch * 4 + tig));
       }
-      const int rs = t * 16 + g + 8 * tig;  // tig 0: row g, tig 1: row g + 8
-      sc = (tig < 2 && rs < rows) ? __ldg(a.scale + rowbase + rs) : 0.0f;
-    };
-    int t = warp;
-    if (t < ntiles) load(t, cur, csc);
-    for (; t < ntiles; t += kWarps) {
-      const int tn = t + kWarps;
-      if (tn < ntiles) load(tn, nxt, nsc);
       float acc[NT][4];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
 #pragma unroll
-      for (int s = 0; s < KS; ++s) {
+      for (int s2 = 0; s2 < KS; ++s2) {
         uint32_t a0, a1, a2, a3;
-        i8x4_to_f16(word_of(cur[0][s / 4], s % 4), a0, a2);  // row g
-        i8x4_to_f16(word_of(cur[1][s / 4], s % 4), a1, a3);  // row g + 8
+        i8x4_to_f16(word_of(cur[0][s2 / 4], s2 % 4), a0, a2);  // row g
+        i8x4_to_f16(word_of(cur[1][s2 / 4], s2 % 4), a1, a3);  // row g + 8
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma16816(acc[nt], a0, a1, a2, a3, bq[nt][s][0], bq[nt][s][1]);
+        for (int nt = 0; nt < NT; ++nt) mma16816(acc[nt], a0, a1, a2, a3, bq[nt][s2][0], bq[nt][s2][1]);
       }
       float mA = -INFINITY, mB = -INFINITY;
 #pragma unroll
@@ -203,15 +302,21 @@ __global__ void __launch_bounds__(kThreads) score_mma_kernel(ScoreArgs a) {
       mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
       mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
       mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
-      const int rs = t * 16 + g + 8 * tig;
-      if (tig < 2 && rs < rows) a.scores[rowbase + rs] = csc * ldexpf(tig == 0 ? mA : mB, -qexp);
-#pragma unroll
-      for (int half = 0; half < 2; ++half)
-#pragma unroll
-        for (int ch = 0; ch < NCH; ++ch) cur[half][ch] = nxt[half][ch];
-      csc = nsc;
+      const int rs = t * 16 + g + 8 * tig;  // tig 0: row g, tig 1: row g + 8
+      const bool mine = tig < 2 && rs < rows;
+      float score = 0.0f;
+      if (mine) {
+        const float sc = reinterpret_cast<const float*>(buf + SL::CODES)[rs];
+        score = sc * ((tig == 0 ? mA : mB) * unscale);
+        a.scores[rowbase + rs] = score;
+      }
+      if (a.hist) warp_hist_add(s_hist, ord_key(score) >> 20, mine);
     }
+    __syncthreads();
+    issue(kk + kScoreStages);
   }
+  cp_async_wait<0>();
+  flush();
 }
 
 // CUDA-core scorer: one thread per key row, query in shared memory (fp32).
@@ -220,7 +325,7 @@ __global__ void __launch_bounds__(kThreads) score_simt_kernel(ScoreArgs a) {
   extern __shared__ int smem[];
   int* s_pref = smem;
   float* sq = reinterpret_cast<float*>(smem + ((a.B + 1 + 3) & ~3));
-  chunk_prefix(a.cu, a.B, s_pref);
+  chunk_prefix(a.cu, a.B, kChunkRows, s_pref);
   const int per_head = s_pref[a.B];
   const int64_t total = (int64_t)a.Hkv * per_head;
   const T* q = static_cast<const T*>(a.q);
@@ -279,9 +384,15 @@ int grid_for(K kernel, int smem, int num_sms, int64_t total) {
 }
 
 template <int D, int NT>
-cudaError_t run_mma(const Dims& d, const ScoreArgs& a, int64_t total, cudaStream_t st) {
-  const int smem = (d.B + 1) * (int)sizeof(int);
+cudaError_t run_mma(const Dims& d, const ScoreArgs& a, cudaStream_t st) {
+  int64_t per_head = 0;
+  for (int b = 0; b < d.B; ++b) per_head += cdiv(d.cu_host[b + 1] - d.cu_host[b], kStageRows);
+  const int64_t total = per_head * d.Hkv;
+  if (total == 0) return cudaSuccess;
+  const int smem = kScoreStages * StageLayout<D>::BYTES + kHist * 4 + 2 * (d.B + 1) * (int)sizeof(int);
   auto k = score_mma_kernel<D, NT>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
   const int grid = grid_for(k, smem, d.num_sms, total);
   k<<<grid, kThreads, smem, st>>>(a);
   return cudaGetLastError();
@@ -314,16 +425,16 @@ cudaError_t simt_by_group(const Dims& d, const ScoreArgs& a, int64_t total, cuda
 }  // namespace
 
 cudaError_t launch_propose_scores(const Dims& d, const void* q, const int8_t* kq,
-                                  const float* scale, float* scores, bool use_mma,
+                                  const float* scale, float* scores, uint32_t* hist, bool use_mma,
                                   cudaStream_t st) {
   int64_t per_head = 0;
   for (int b = 0; b < d.B; ++b) per_head += cdiv(d.cu_host[b + 1] - d.cu_host[b], kChunkRows);
   const int64_t total = per_head * d.Hkv;
   if (total == 0) return cudaSuccess;
-  ScoreArgs a{q, kq, scale, scores, d.cu_dev, d.T, d.B, d.Hkv, d.G};
+  ScoreArgs a{q, kq, scale, scores, hist, d.cu_dev, d.T, d.B, d.Hkv, d.G};
   if (use_mma && d.bf16) {
-    if (d.D == 128) return d.G <= 8 ? run_mma<128, 1>(d, a, total, st) : run_mma<128, 2>(d, a, total, st);
-    return d.G <= 8 ? run_mma<64, 1>(d, a, total, st) : run_mma<64, 2>(d, a, total, st);
+    if (d.D == 128) return d.G <= 8 ? run_mma<128, 1>(d, a, st) : run_mma<128, 2>(d, a, st);
+    return d.G <= 8 ? run_mma<64, 1>(d, a, st) : run_mma<64, 2>(d, a, st);
   }
   if (d.bf16) {
     return d.D == 128 ? simt_by_group<__nv_bfloat16, 128>(d, a, total, st)

@@ -72,7 +72,7 @@ class PrismDecoder:
                             self.ws_dense) if w is not None]
 
     def layer(self, l: int, q, k, v, kq=None, k_scale=None, quantize_new: bool = True,
-              k_new=None, v_new=None, stream=None):
+              k_new=None, v_new=None, k_next=None, stream=None):
         """Enqueue one layer of the step (kq/k_scale required at proposal layers).
 
         k_new / v_new ([B][Hkv][d]), when given, are first written to the last
@@ -89,7 +89,7 @@ class PrismDecoder:
         if self.fused:
             prism.refine_decode(p, q, k, v, self.pool[src], self.pool_cnt[src], self.kappa_p,
                                 self.kappa, self.scale, self.idx[l], self.cnt[l], self.out[l],
-                                self.ws_rd, lse=self.lse[l], stream=stream)
+                                self.ws_rd, lse=self.lse[l], k_prefetch=k_next, stream=stream)
             return
         prism.refine(p, q, k, self.pool[src], self.pool_cnt[src], self.kappa_p, self.kappa,
                      self.idx[l], self.cnt[l], self.ws_ref, stream=stream)
@@ -102,10 +102,12 @@ class PrismDecoder:
         per-layer sequences; kqs/scales are indexed by proposal layer."""
         for l in range(self.num_layers):
             pl = l % self.group == 0
+            # the next layer refines on the same pool unless it is a proposal layer
+            nxt = ks[l + 1] if l + 1 < self.num_layers and (l + 1) % self.group else None
             self.layer(l, qs[l], ks[l], vs[l], kqs[l] if pl else None, scales[l] if pl else None,
                        quantize_new=quantize_new,
                        k_new=None if k_new is None else k_new[l],
-                       v_new=None if v_new is None else v_new[l], stream=stream)
+                       v_new=None if v_new is None else v_new[l], k_next=nxt, stream=stream)
 
     def launches_per_step(self, append: bool) -> int:
         """Kernels one step enqueues (append, quantize, score, select, refine

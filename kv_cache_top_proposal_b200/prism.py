@@ -57,7 +57,7 @@ def _load():
         "prism_propose": [sp, P, P, P, i32, P, P, P, S, P],
         "prism_refine": [sp, P, P, P, P, i32, i32, P, P, P, P, S, P],
         "prism_sparse_decode": [sp, P, P, P, P, P, i32, ctypes.c_float, P, P, P, S, P],
-        "prism_refine_decode": [sp, P, P, P, P, P, i32, i32, ctypes.c_float, P, P, P, P, P, S, P],
+        "prism_refine_decode": [sp, P, P, P, P, P, i32, i32, ctypes.c_float, P, P, P, P, P, P, S, P],
         "prism_dense_decode": [sp, P, P, P, ctypes.c_float, P, P, P, S, P],
         "prism_clear_device_status": [P, S, P],
         "prism_get_device_status": [P, S, P, ctypes.POINTER(ctypes.c_int32)],
@@ -168,10 +168,11 @@ def sparse_decode(p: Problem, q, k, v, idx, cnt, kappa: int, softmax_scale: floa
 
 
 def refine_decode(p: Problem, q, k, v, pool, pool_cnt, kappa_p: int, kappa: int,
-                  softmax_scale: float, idx, cnt, out, ws, lse=None, stream=None):
+                  softmax_scale: float, idx, cnt, out, ws, lse=None, k_prefetch=None, stream=None):
     _check(_lib.prism_refine_decode(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(pool), _ptr(pool_cnt),
                                     kappa_p, kappa, float(softmax_scale), _ptr(idx), _ptr(cnt),
-                                    _ptr(out), _ptr(lse), _ptr(ws), _nbytes(ws), _stream(stream)),
+                                    _ptr(out), _ptr(lse), _ptr(k_prefetch), _ptr(ws), _nbytes(ws),
+                                    _stream(stream)),
            "refine_decode")
 
 

@@ -385,3 +385,27 @@ def test_refine_decode_ties_and_bad_positions(P):
     pool[0, 0, 5] = 4000
     P.refine_decode(prob, q, k, v, pool, cnt_p, kp, kap, 0.1, idx, cnt, out, ws)
     assert P.get_device_status(ws) & P.DEV_BAD_INDEX
+
+
+def test_refine_decode_prefetch_changes_nothing(P):
+    seqlens, hq, hkv, d, kp, kap = [20000], 8, 2, 128, 4096, 1024
+    prob = problem(P, seqlens, hq, hkv, d, "bf16")
+    q, k, v = make_case(seqlens, hq, hkv, d, "bf16", seed=15)
+    k2 = torch.randn_like(k)
+    rng = np.random.default_rng(16)
+    pool = torch.tensor(np.sort(rng.choice(20000, (hkv, kp), replace=True), axis=1)[None], device=DEV)
+    pool = torch.tensor(np.stack([np.sort(rng.choice(20000, kp, replace=False)) for _ in range(hkv)])[None],
+                        dtype=torch.int32, device=DEV)
+    cnt_p = torch.full((1, hkv), kp, dtype=torch.int32, device=DEV)
+    ws = ws_for(P, prob, P.OP_REFINE_DECODE, kp, kap)
+    res = []
+    for kpf in (None, k2):
+        idx = torch.zeros((1, hkv, kap), dtype=torch.int32, device=DEV)
+        cnt = torch.zeros((1, hkv), dtype=torch.int32, device=DEV)
+        out = torch.zeros((1, hq, d), device=DEV)
+        P.refine_decode(prob, q, k, v, pool, cnt_p, kp, kap, 0.1, idx, cnt, out, ws, k_prefetch=kpf)
+        res.append((idx, cnt, out))
+    torch.cuda.synchronize()
+    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
+    assert torch.equal(res[0][2], res[1][2])
+    assert P.get_device_status(ws) == 0
