@@ -145,24 +145,30 @@ class ClockSampler:
 
 
 class Dist:
-    def __init__(self):
+    """One process per GPU.  The ranks share no data: the only collectives
+    are the barriers around the timed region and the max over ranks of its
+    duration.  `backend` is "nccl" on GPUs; "gloo" serves the CPU tests of
+    this host logic."""
+
+    def __init__(self, backend: str = "nccl"):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
         self.pg = None
 
     def init(self):
+        cuda = self.backend == "nccl"
+        if cuda:
+            torch.cuda.set_device(self.local)
         if self.world > 1:
             import datetime
 
             import torch.distributed as dist
 
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            kw = {"device_id": torch.device("cuda", self.local)} if cuda else {}
+            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=120), **kw)
             self.pg = dist
-        else:
-            torch.cuda.set_device(self.local)
 
     def barrier(self):
         if self.pg:
@@ -171,7 +177,8 @@ class Dist:
     def max(self, x: float) -> float:
         if not self.pg:
             return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dev = "cuda" if self.backend == "nccl" else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
