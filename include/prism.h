@@ -31,7 +31,9 @@
  * Ownership: the caller allocates and owns every buffer.  The library never
  * allocates, frees or synchronises (prism_get_device_status excepted), keeps
  * no mutable global state, and may be called from several streams at once
- * with disjoint outputs and workspaces.  All work is enqueued on `stream`
+ * with disjoint outputs and workspaces.  The one exception is
+ * prism_sparse_decode_noalloc (end of this file), which works in a fixed
+ * scratch array that the library itself holds on every device.  All work is enqueued on `stream`
  * (a cudaStream_t; NULL is the legacy default stream).
  *
  * Errors: every argument that can be checked on the host (null pointers,
@@ -67,7 +69,8 @@ typedef enum prism_status {
   PRISM_ERR_UNSUPPORTED = 2,
   PRISM_ERR_WORKSPACE = 3,
   PRISM_ERR_CUDA = 4,
-  PRISM_ERR_TIMEOUT = 5
+  PRISM_ERR_TIMEOUT = 5,
+  PRISM_ERR_SCRATCH_LIMIT = 6
 } prism_status;
 
 typedef enum prism_op {
@@ -223,6 +226,45 @@ PRISM_API prism_status prism_get_device_status(const void* ws, size_t ws_bytes, 
 
 /* Static description of a status code. */
 PRISM_API const char* prism_status_str(prism_status s);
+
+/*
+ * No-allocation variant of prism_sparse_decode.  The paper has no
+ * counterpart to this entry point: it exists for callers that cannot hand
+ * the library a workspace, because they may not allocate device memory at
+ * the point of the call -- code that runs inside a memory pool it does not
+ * own, an allocator callback, or an engine whose device memory is fixed
+ * once at start-up.  It computes exactly what prism_sparse_decode computes
+ * (same kernels, same split plan, same summation order), but keeps the
+ * split-K partial results in a scratch array that the library declares at
+ * file scope: PRISM_NOALLOC_SCRATCH_BYTES (4 MiB) of device memory, held by
+ * every GPU that loads the library until the process exits.
+ *
+ * Arguments are those of prism_sparse_decode, except that the workspace is
+ * replaced by status_dev: a caller-owned device int32 into which the
+ * kernels OR the PRISM_DEV_* bits of any bad index or count they meet (the
+ * caller zeroes it and reads it back).  It must not be NULL.
+ *
+ * The call allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ * library routine.  Its first call on a device, with that device current,
+ * looks up the device address of the scratch array (cudaGetSymbolAddress),
+ * which may load the library's device code onto that device; make that
+ * first call before any stream capture begins.
+ *
+ * A request whose partial results need more than the scratch holds
+ * (B * Hq * splits * (d + 2) * 4 bytes, rounded up) returns
+ * PRISM_ERR_SCRATCH_LIMIT and enqueues nothing.  Every call on a device
+ * shares the one array, and the array keeps the last call's contents (every
+ * partial a call reads is first written by that call).  Calls whose work
+ * overlaps on the GPU -- on different streams, or from different host
+ * threads -- race on the array and give wrong results: serialise them.
+ */
+#define PRISM_NOALLOC_SCRATCH_BYTES (4u << 20)
+PRISM_API prism_status prism_sparse_decode_noalloc(const prism_shape* shape, const void* q,
+                                                   const void* k, const void* v,
+                                                   const int32_t* idx, const int32_t* cnt,
+                                                   int32_t kappa, float softmax_scale, float* out,
+                                                   float* lse_opt, int32_t* status_dev,
+                                                   void* stream);
 
 #ifdef __cplusplus
 }

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/prism.h"
 #include "kernels.h"
@@ -343,8 +344,71 @@ const char* prism_status_str(prism_status s) {
     case PRISM_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case PRISM_ERR_CUDA: return "CUDA launch or runtime error";
     case PRISM_ERR_TIMEOUT: return "device-side wait timed out";
+    case PRISM_ERR_SCRATCH_LIMIT:
+      return "request needs more than the fixed scratch of the no-allocation entry point";
   }
   return "unknown status";
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// No-allocation sparse decode.  Callers that may not allocate device memory
+// when they call (a memory pool they do not own, an allocator callback, an
+// engine whose memory is fixed at start-up) get the split-K partials kept in
+// this file-scope array instead of a caller workspace.  In host code the name
+// is only a stand-in for the device symbol; its device address is looked up
+// once per device with that device current, and the lookup's result is
+// checked before any kernel sees it.
+namespace prism {
+namespace {
+
+static __device__ __align__(256) unsigned char noalloc_scratch[PRISM_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex noalloc_mu;
+void* noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch on the current device (looked up on the
+// first call on that device).
+prism_status noalloc_scratch_ptr(char** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PRISM_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return PRISM_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(noalloc_mu);
+  if (!noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, noalloc_scratch) != cudaSuccess || !p) return PRISM_ERR_CUDA;
+    noalloc_ptr[dev] = p;
+  }
+  *out = static_cast<char*>(noalloc_ptr[dev]);
+  return PRISM_OK;
+}
+
+}  // namespace
+}  // namespace prism
+
+extern "C" prism_status prism_sparse_decode_noalloc(const prism_shape* shape, const void* q,
+                                                    const void* k, const void* v,
+                                                    const int32_t* idx, const int32_t* cnt,
+                                                    int32_t kappa, float softmax_scale, float* out,
+                                                    float* lse_opt, int32_t* status_dev,
+                                                    void* stream) {
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!q || !k || !v || !idx || !cnt || !out || !status_dev || kappa < 1) return PRISM_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return PRISM_ERR_INVALID_ARG;
+  // The same partial layout as the workspace of prism_sparse_decode; the
+  // header bytes at its start stay unused (the status goes to status_dev).
+  const Layout L = layout(d, PRISM_OP_SPARSE_DECODE, 0, kappa);
+  if (L.total > (size_t)PRISM_NOALLOC_SCRATCH_BYTES) return PRISM_ERR_SCRATCH_LIMIT;
+  const AttendPlan p = plan_attend(d, kappa);
+  if ((s = set_live_sms(&d)) != PRISM_OK) return s;
+  char* w = nullptr;
+  if ((s = noalloc_scratch_ptr(&w)) != PRISM_OK) return s;
+  return cuda_status(launch_attend(d, p, q, k, v, idx, cnt, kappa, softmax_scale,
+                                   reinterpret_cast<float*>(w + L.a),
+                                   reinterpret_cast<float*>(w + L.b), out, lse_opt, status_dev,
+                                   static_cast<cudaStream_t>(stream)));
+}

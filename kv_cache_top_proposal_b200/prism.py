@@ -19,7 +19,8 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libprism.so")
 
 F32, BF16 = 0, 1
 OP_QUANTIZE, OP_PROPOSE, OP_REFINE, OP_SPARSE_DECODE, OP_DENSE_DECODE, OP_REFINE_DECODE = range(6)
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_SCRATCH_LIMIT = range(7)
+NOALLOC_SCRATCH_BYTES = 4 << 20
 DEV_BAD_INDEX, DEV_TOO_LONG = 0x1, 0x2
 MAX_SELECT_ROW = 393216
 WS_HEADER = 256
@@ -27,7 +28,7 @@ WS_HEADER = 256
 EXPORTS = ("prism_workspace_size", "prism_append_kv", "prism_quantize_k", "prism_propose", "prism_refine",
            "prism_sparse_decode", "prism_refine_decode", "prism_dense_decode",
            "prism_clear_device_status",
-           "prism_get_device_status", "prism_status_str")
+           "prism_get_device_status", "prism_status_str", "prism_sparse_decode_noalloc")
 
 
 class PrismError(RuntimeError):
@@ -61,6 +62,7 @@ def _load():
         "prism_dense_decode": [sp, P, P, P, ctypes.c_float, P, P, P, S, P],
         "prism_clear_device_status": [P, S, P],
         "prism_get_device_status": [P, S, P, ctypes.POINTER(ctypes.c_int32)],
+        "prism_sparse_decode_noalloc": [sp, P, P, P, P, P, i32, ctypes.c_float, P, P, P, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -180,6 +182,20 @@ def dense_decode(p: Problem, q, k, v, softmax_scale: float, out, ws, lse=None, s
     _check(_lib.prism_dense_decode(p.ref, _ptr(q), _ptr(k), _ptr(v), float(softmax_scale),
                                    _ptr(out), _ptr(lse), _ptr(ws), _nbytes(ws), _stream(stream)),
            "dense_decode")
+
+
+def sparse_decode_noalloc(p: Problem, q, k, v, idx, cnt, kappa: int, softmax_scale: float, out,
+                          status, lse=None, stream=None):
+    """prism_sparse_decode without a workspace, for callers that may not
+    allocate device memory at the call: the partials live in the library's
+    fixed 4 MiB per-device scratch.  `status` is a device int32 tensor the
+    kernels OR bad-index bits into.  Calls that overlap on the GPU race on
+    the shared scratch; the first call on a device must precede any stream
+    capture."""
+    _check(_lib.prism_sparse_decode_noalloc(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt),
+                                            kappa, float(softmax_scale), _ptr(out), _ptr(lse),
+                                            _ptr(status), _stream(stream)),
+           "sparse_decode_noalloc")
 
 
 def clear_device_status(ws, stream=None):
