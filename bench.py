@@ -398,10 +398,11 @@ def run_prism(args, dist: Dist):
 
         def f_rd(l=l):
             src = l - l % cfg.group
-            nxt = ks[l + 1] if l + 1 < L and not cfg.is_proposal(l + 1) else None
+            fa = not cfg.is_proposal(l)  # refined layers append their new rows themselves
             prism.refine_decode(dec.p, q_layers[l], ks[l], vs[l], dec.pool[src], dec.pool_cnt[src],
                                 cfg.kappa_p, cfg.kappa, dec.scale, dec.idx[l], dec.cnt[l],
-                                dec.out[l], dec.ws_rd, lse=dec.lse[l], k_prefetch=nxt)
+                                dec.out[l], dec.ws_rd, lse=dec.lse[l],
+                                k_new=k_new[l] if fa else None, v_new=v_new[l] if fa else None)
 
         if pl:
             ops.append(("propose", graph_of(f_prop, stream)))

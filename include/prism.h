@@ -85,6 +85,7 @@ typedef enum prism_op {
 /* Bits of the device status word kept in every workspace. */
 #define PRISM_DEV_BAD_INDEX 0x1   /* an index / token row outside its sequence */
 #define PRISM_DEV_TOO_LONG  0x2   /* a row longer than the selection capacity  */
+#define PRISM_DEV_TIMEOUT   0x4   /* a bounded device-side wait gave up        */
 
 /* Shape of one layer's decode problem.  cu_seqlens_host mirrors
  * cu_seqlens_dev (B+1 entries, cu[0] = 0, non-decreasing, cu[B] =
@@ -190,23 +191,41 @@ PRISM_API prism_status prism_sparse_decode(const prism_shape* shape, const void*
  * A refined layer in one call: prism_refine followed by prism_sparse_decode
  * on its result, with the same outputs (idx, cnt, out, lse_opt) and the same
  * definitions.  The exact scores, the selection and the attention partials
- * stay on chip (one thread-block cluster per sequence and KV head), so the
- * workspace is only the 256-byte status header (PRISM_OP_REFINE_DECODE), and
- * the key rows of the pool are read once.  Returns PRISM_ERR_UNSUPPORTED when
- * a pool of kappa_p members does not fit on chip (kappa_p > 16 x the slice
- * capacity: 6144 members per CTA at G <= 4, d = 128); use the two calls then.
+ * stay on chip (one thread-block cluster of up to 16 CTAs per sequence and
+ * KV head), so the workspace is only the 256-byte status header
+ * (PRISM_OP_REFINE_DECODE), and the key rows of the pool are read once.
+ * Returns PRISM_ERR_UNSUPPORTED when a pool of kappa_p members does not fit
+ * on chip (kappa_p > 65535, or more than 16 x 3328 members at G <= 4,
+ * d = 128); use the two calls then.
+ *
+ * k_new_opt / v_new_opt, if not NULL, are this token's key and value rows,
+ * [B][Hkv][d] in the cache dtype: the call first appends them at position
+ * L_b - 1 of every sequence (as prism_append_kv would; k and v are written
+ * there) and every read of that position uses them.  NULL: the caches
+ * already hold the rows, and k and v are only read.
+ *
  * k_prefetch, if not NULL, is the key cache ([Hkv][T][d], same shape) of the
  * next layer that will be refined on the same pool: once this layer's key
  * rows are consumed, the same pool rows of k_prefetch are prefetched into L2
  * (a hint; results do not depend on it).
+ *
+ * flags: PRISM_RD_OVERLAP lets the launch begin while the previous kernel on
+ * `stream` is still running (programmatic dependent launch).  Until that
+ * kernel ends the call reads only cu_seqlens_dev, pool_idx, pool_cnt and the
+ * key rows at pool positions other than L_b - 1, and writes nothing but the
+ * status word; it touches q, v, k_new_opt, v_new_opt and its outputs only
+ * afterwards.  Set it only when the previous kernel writes none of the
+ * former (e.g. the refined layer before this one, on the same pool).
  */
-PRISM_API prism_status prism_refine_decode(const prism_shape* shape, const void* q, const void* k,
-                                           const void* v, const int32_t* pool_idx,
+#define PRISM_RD_OVERLAP 0x1u
+PRISM_API prism_status prism_refine_decode(const prism_shape* shape, const void* q, void* k,
+                                           void* v, const int32_t* pool_idx,
                                            const int32_t* pool_cnt, int32_t kappa_p,
                                            int32_t kappa, float softmax_scale, int32_t* idx,
                                            int32_t* cnt, float* out, float* lse_opt,
-                                           const void* k_prefetch, void* ws, size_t ws_bytes,
-                                           void* stream);
+                                           const void* k_new_opt, const void* v_new_opt,
+                                           const void* k_prefetch, uint32_t flags, void* ws,
+                                           size_t ws_bytes, void* stream);
 
 /*
  * Dense decode attention over every position t < L_b (the comparison path):

@@ -38,7 +38,7 @@ cudaError_t launch_quantize(const Dims& d, const void* k, int8_t* kq, float* sca
 // ord(score), added to (the caller clears it).
 cudaError_t launch_propose_scores(const Dims& d, const void* q, const int8_t* kq,
                                   const float* scale, float* scores, uint32_t* hist, bool use_mma,
-                                  cudaStream_t st);
+                                  int32_t* status, cudaStream_t st);
 
 // Cluster radix top-k.  mode 0 (propose): keys scores[h][cu[b] + i], row
 // length L_b, output position i.  mode 1 (refine): keys r[row][i], row length
@@ -62,14 +62,12 @@ struct SelectArgs {
 int select_capacity_per_row();  // longest row one cluster can select from
 
 // Proposal-layer selection from the scorer's first-digit histogram (see
-// propose_select.cu); cap = ceil(max L_b / cluster) candidate slots per CTA.
-int propose_select_cap(int max_len);
+// propose_select.cu); rows up to propose_select_max_row() positions.
 int propose_select_cluster();
 int propose_select_max_row();
 cudaError_t launch_propose_select(const Dims& d, const float* scores, const uint32_t* hist,
-                                  int kappa_p, int cap, uint32_t* ckey, int32_t* cpos,
-                                  int32_t* cmeta, int32_t* res, int32_t* pool, int32_t* pool_cnt,
-                                  int32_t* status, cudaStream_t st);
+                                  int kappa_p, int32_t* pool, int32_t* pool_cnt, int32_t* status,
+                                  cudaStream_t st);
 cudaError_t launch_select(const Dims& d, const SelectArgs& a, int max_row_len, cudaStream_t st);
 
 // Exact pool scores r[row][i] = max_g q_g . K[pool_i] (+ per-head dots).
@@ -87,11 +85,11 @@ struct RefineDecodePlan {
 };
 RefineDecodePlan plan_refine_decode(const Dims& d, int kappa_p);
 cudaError_t launch_refine_decode(const Dims& d, const RefineDecodePlan& p, const void* q,
-                                 const void* k, const void* v, const void* k_next,
-                                 const int32_t* pool,
+                                 const void* k, const void* v, const void* k_new,
+                                 const void* v_new, const void* k_next, const int32_t* pool,
                                  const int32_t* pool_cnt, int kappa_p, int kappa,
                                  float softmax_scale, int32_t* idx, int32_t* cnt, float* out,
-                                 float* lse, int32_t* status, cudaStream_t st);
+                                 float* lse, int32_t* status, bool overlap, cudaStream_t st);
 
 // Split-K attention partials over idx rows (idx == nullptr: every position).
 struct AttendPlan {

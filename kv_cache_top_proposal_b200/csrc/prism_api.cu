@@ -77,21 +77,12 @@ Layout layout(const Dims& d, int op, int kappa_p, int kappa) {
   switch (op) {
     case PRISM_OP_QUANTIZE:
       break;
-    case PRISM_OP_PROPOSE: {  // scores [Hkv][T] fp32, then the selection scratch
+    case PRISM_OP_PROPOSE:  // scores [Hkv][T] fp32, first-digit histogram [rows][4096] u32
       L.a = off;
       off = align_up(off + (size_t)d.Hkv * (size_t)d.T * sizeof(float));
-      const size_t cl = (size_t)propose_select_cluster();
-      const size_t cap = (size_t)propose_select_cap(d.max_len);
-      L.b = off;  // hist [rows][4096] u32
+      L.b = off;
       off = align_up(off + rows * 4096 * 4);
-      L.c = off;  // candidate keys [rows][cl][cap]
-      off = align_up(off + rows * cl * cap * 4);
-      L.d = off;  // candidate positions [rows][cl][cap]
-      off = align_up(off + rows * cl * cap * 4);
-      L.e = off;  // per-CTA counts [rows][cl][2], results [rows][2 + cl]
-      off = align_up(off + rows * cl * 2 * 4 + rows * (2 + cl) * 4);
       break;
-    }
     case PRISM_OP_REFINE:  // r [rows][kappa_p], dots [rows][G][kappa_p]
       L.a = off;
       off = align_up(off + rows * (size_t)kappa_p * sizeof(float));
@@ -194,15 +185,11 @@ prism_status prism_propose(const prism_shape* shape, const void* q, const int8_t
     uint32_t* hist = reinterpret_cast<uint32_t*>(w + L.b);
     const size_t rows = (size_t)d.B * d.Hkv;
     if (cudaMemsetAsync(hist, 0, rows * 4096 * 4, st) != cudaSuccess) return PRISM_ERR_CUDA;
-    cudaError_t e = launch_propose_scores(d, q, kq, k_scale, scores, hist, true, st);
+    cudaError_t e = launch_propose_scores(d, q, kq, k_scale, scores, hist, true, status, st);
     if (e != cudaSuccess) return PRISM_ERR_CUDA;
-    int32_t* meta = reinterpret_cast<int32_t*>(w + L.e);
-    return cuda_status(launch_propose_select(
-        d, scores, hist, kappa_p, propose_select_cap(d.max_len), reinterpret_cast<uint32_t*>(w + L.c),
-        reinterpret_cast<int32_t*>(w + L.d), meta, meta + rows * propose_select_cluster() * 2,
-        pool_idx, pool_cnt, status, st));
+    return cuda_status(launch_propose_select(d, scores, hist, kappa_p, pool_idx, pool_cnt, status, st));
   }
-  cudaError_t e = launch_propose_scores(d, q, kq, k_scale, scores, nullptr, mma, st);
+  cudaError_t e = launch_propose_scores(d, q, kq, k_scale, scores, nullptr, mma, status, st);
   if (e != cudaSuccess) return PRISM_ERR_CUDA;
   SelectArgs a{};
   a.mode = 0;
@@ -279,10 +266,11 @@ prism_status prism_sparse_decode(const prism_shape* shape, const void* q, const 
                                    reinterpret_cast<int32_t*>(w), static_cast<cudaStream_t>(stream)));
 }
 
-prism_status prism_refine_decode(const prism_shape* shape, const void* q, const void* k,
-                                 const void* v, const int32_t* pool_idx, const int32_t* pool_cnt,
+prism_status prism_refine_decode(const prism_shape* shape, const void* q, void* k, void* v,
+                                 const int32_t* pool_idx, const int32_t* pool_cnt,
                                  int32_t kappa_p, int32_t kappa, float softmax_scale, int32_t* idx,
-                                 int32_t* cnt, float* out, float* lse_opt, const void* k_prefetch,
+                                 int32_t* cnt, float* out, float* lse_opt, const void* k_new_opt,
+                                 const void* v_new_opt, const void* k_prefetch, uint32_t flags,
                                  void* ws, size_t ws_bytes, void* stream) {
   Dims d;
   prism_status s = check_shape(shape, &d);
@@ -290,13 +278,20 @@ prism_status prism_refine_decode(const prism_shape* shape, const void* q, const 
   if (!q || !k || !v || !pool_idx || !pool_cnt || !idx || !cnt || !out) return PRISM_ERR_INVALID_ARG;
   if (kappa_p < 1 || kappa < 1 || kappa > kappa_p) return PRISM_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale)) return PRISM_ERR_INVALID_ARG;
+  if (flags & ~PRISM_RD_OVERLAP) return PRISM_ERR_INVALID_ARG;
+  if ((k_new_opt == nullptr) != (v_new_opt == nullptr)) return PRISM_ERR_INVALID_ARG;
+  if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v) % 16) return PRISM_ERR_INVALID_ARG;
+  if (k_new_opt && (((uintptr_t)k_new_opt | (uintptr_t)v_new_opt | (uintptr_t)k | (uintptr_t)v) % 16))
+    return PRISM_ERR_INVALID_ARG;
   const Layout L = layout(d, PRISM_OP_REFINE_DECODE, kappa_p, kappa);
   if (!ws_ok(ws, ws_bytes, L)) return PRISM_ERR_WORKSPACE;
   const RefineDecodePlan p = plan_refine_decode(d, kappa_p);
   if (!p.ok) return PRISM_ERR_UNSUPPORTED;
-  return cuda_status(launch_refine_decode(d, p, q, k, v, k_prefetch, pool_idx, pool_cnt, kappa_p,
-                                          kappa, softmax_scale, idx, cnt, out, lse_opt,
-                                          static_cast<int32_t*>(ws), static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_refine_decode(d, p, q, k, v, k_new_opt, v_new_opt, k_prefetch, pool_idx,
+                                          pool_cnt, kappa_p, kappa, softmax_scale, idx, cnt, out,
+                                          lse_opt, static_cast<int32_t*>(ws),
+                                          (flags & PRISM_RD_OVERLAP) != 0,
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 prism_status prism_dense_decode(const prism_shape* shape, const void* q, const void* k,

@@ -5,20 +5,19 @@
 // "Implementation Details").
 //
 // The scorer has already built, per row, the histogram of the first 12 bits
-// of ord(score).  One cluster of kCL CTAs per row, each owning a contiguous
-// slice of positions:
-//   1. every CTA reads the row's histogram and locates the bin b1 that holds
-//      the kappa_p-th largest key (same answer in every CTA), loads its slice
-//      of keys into shared memory, counts its keys above b1 and lists its
-//      keys in b1 -- in position order -- into a global candidate region;
-//   2. rank 0 resolves the exact threshold T (the two remaining digits) and
-//      the last taken position I* among keys equal to T (lower positions
-//      first) over the concatenated candidate lists, and every slice's
-//      output offset;
-//   3. every CTA writes its kept positions (key > T, or key == T and position
-//      <= I*) in ascending order from its offset.
-// Hand-offs go through global memory (L2) ordered by the cluster barrier;
-// two barriers in all, no distributed shared memory.
+// of ord(score).  One cluster of kCL CTAs per row; CTA r owns the contiguous
+// slice r of positions and keeps its keys in registers (KPT per thread,
+// coalesced: key u of thread t is slice position u * kThreads + t):
+//   1. every CTA reads the row's histogram and locates the bin holding the
+//      kappa_p-th largest key (same answer in every CTA).  Unless the whole
+//      bin is taken, the keys in it build the histogram of the next 10 bits
+//      in rank 0's shared memory (remote atomics), every CTA reads it, and
+//      so on for the last 10 bits: this gives the threshold prefix P and how
+//      many keys at P are taken (in position order);
+//   2. the CTAs exchange their counts above and at P, which gives each one
+//      its share of the keys at P and its output offset;
+//   3. every CTA writes its kept positions in ascending order (ballot counts
+//      per (key block, warp), one block scan, placement).
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -33,114 +32,86 @@ namespace {
 constexpr int kCL = 8;
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
-constexpr int kHist = 4096;
-constexpr int kMaxSlice = 16384;  // keys per CTA (+ the candidate copy: 192 KB of shared memory)
+constexpr int kKPT = 16;                      // keys per thread
+constexpr int kMaxSlice = kKPT * kThreads;    // keys per CTA
+constexpr int kHist = 4096;                   // first digit (from the scorer)
+constexpr int kBins = 1024;                   // second and third digits
 
 struct PSArgs {
-  const float* scores;  // [Hkv][T]
+  const float* scores;   // [Hkv][T]
   const uint32_t* hist;  // [rows][kHist]
   const int32_t* cu;
   int Hkv;
   int64_t T;
   int kp;
-  int cap;               // candidate capacity per CTA (slice length bound)
-  uint32_t* ckey;        // [rows][kCL][cap]
-  int32_t* cpos;         // [rows][kCL][cap]
-  int32_t* cmeta;        // [rows][kCL][2]: listed count, count above b1
-  int32_t* res;          // [rows][2 + kCL]: T, I*, offsets
   int32_t* out;          // [rows][kp]
   int32_t* out_cnt;      // [rows]
   int32_t* status;
 };
 
-// bin of `nb` (padded-free) holding the r-th largest among keys matching
-// prefix/pmask, over n keys read by get(j); whole CTA; returns in s3[0..2]
-// (bin, count above, count in bin).
-template <typename Get>
-__device__ void find_bin_any(Get get, int n, uint32_t prefix, uint32_t pmask, int shift, int nb,
-                             int r, uint32_t* hist, int* scratch, int* s3) {
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+
+// Bin of an NB-bin histogram (PER consecutive bins per thread, read through
+// load(bin)) holding the r-th largest counted key, bins ranked in descending
+// order: res = (bin, keys above it, keys in it).  Whole CTA.
+template <int PER, typename Load>
+__device__ void find_digit(Load load, int r, int* scratch, int* res) {
   const int tid = threadIdx.x;
-  for (int i = tid; i < nb; i += kThreads) hist[i] = 0u;
-  __syncthreads();
-  for (int j0 = tid & ~31; j0 < n; j0 += kThreads) {  // warp-uniform trip count
-    const int j = j0 + (tid & 31);
-    const uint32_t key = j < n ? get(j) : 0u;
-    warp_hist_add(hist, (key >> shift) & (uint32_t)(nb - 1), j < n && (key & pmask) == prefix);
+  uint32_t c[PER];
+  int v = 0;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    c[j] = load(tid * PER + j);
+    v += (int)c[j];
   }
-  __syncthreads();
-  const int v = tid < nb ? (int)hist[tid] : 0;  // nb <= kThreads
+  if (tid == 0) res[0] = res[1] = res[2] = 0;
   int total;
   const int excl = block_excl_scan(v, scratch, &total);
-  const int above = total - excl - v;
-  if (tid < nb && above < r && r <= above + v) {
-    s3[0] = tid;
-    s3[1] = above;
-    s3[2] = v;
+  int above = total - excl - v;
+#pragma unroll
+  for (int j = PER - 1; j >= 0; --j) {
+    if (above < r && r <= above + (int)c[j]) {
+      res[0] = tid * PER + j;
+      res[1] = above;
+      res[2] = (int)c[j];
+    }
+    above += (int)c[j];
   }
   __syncthreads();
 }
 
-
-// Ordered compaction of the CTA's m items: pred(i) selects, emit(i, slot)
-// receives slot = base + rank of i among the selected, in index order.
-// Two passes over blocks of kThreads items: ballot counts per (block, warp)
-// into tab, one block-wide scan, then placement.  tab holds >= ceil(m /
-// kThreads) * kWarps ints.  Returns the selected count.  Whole CTA.
-template <typename Pred, typename Emit>
-__device__ int ordered_compact(int m, int base, Pred pred, Emit emit, int* tab, int* scratch) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nblk = (m + kThreads - 1) / kThreads;
-#pragma unroll 4
-  for (int u = 0; u < nblk; ++u) {
-    const int i = u * kThreads + tid;
-    const unsigned bal = __ballot_sync(0xffffffffu, i < m && pred(i));
-    if (lane == 0) tab[u * kWarps + warp] = __popc(bal);
-  }
-  __syncthreads();
-  const int ne = nblk * kWarps;
-  const int per = (ne + kThreads - 1) / kThreads;
-  int v = 0;
-  for (int j = 0; j < per; ++j) {
-    const int e = tid * per + j;
-    if (e < ne) v += tab[e];
-  }
+// Exclusive scan, in place, of the kKPT * kWarps per-(block, warp) counts
+// (one entry per thread for the first kKPT * kWarps threads), plus `base`.
+__device__ __forceinline__ void scan_table(int* tab, int base, int* scratch) {
+  const int tid = threadIdx.x;
+  const int v = tid < kKPT * kWarps ? tab[tid] : 0;
   int total;
-  int acc = block_excl_scan(v, scratch, &total) + base;
-  for (int j = 0; j < per; ++j) {
-    const int e = tid * per + j;
-    if (e < ne) {
-      const int c = tab[e];
-      tab[e] = acc;
-      acc += c;
-    }
-  }
+  const int excl = block_excl_scan(v, scratch, &total);
+  if (tid < kKPT * kWarps) tab[tid] = excl + base;
   __syncthreads();
-#pragma unroll 4
-  for (int u = 0; u < nblk; ++u) {
-    const int i = u * kThreads + tid;
-    const bool s = i < m && pred(i);
-    const unsigned bal = __ballot_sync(0xffffffffu, s);
-    if (s) emit(i, tab[u * kWarps + warp] + __popc(bal & ((1u << lane) - 1u)));
-  }
-  __syncthreads();
-  return total;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) propose_select_kernel(const PSArgs a) {
-  extern __shared__ __align__(16) uint32_t skeys[];  // [slice], then the candidate copy
-  __shared__ uint32_t hist[kThreads];
-  __shared__ int tab[(kMaxSlice / kThreads) * kWarps];
+  __shared__ __align__(16) uint32_t hist2[kBins];  // rank 0: digit-2 counts of the cluster
+  __shared__ __align__(16) uint32_t hist3[kBins];  // rank 0: digit-3 counts
+  __shared__ int tabE[kKPT * kWarps];  // per (key block, warp): keys at P, then their prefix
+  __shared__ int tabK[kKPT * kWarps];  // per (key block, warp): kept keys, then output slots
   __shared__ int scratch[33];
-  __shared__ int s3[3];
-  __shared__ int s_wc[kWarps];
-  __shared__ int s_meta[kCL][2];
-  __shared__ int s_res[2 + kCL];
+  __shared__ int s_dig[3];
+  __shared__ int s_cnt[2];   // this CTA's keys above / at the prefix
+  __shared__ int s_mine[2];  // output offset, keys at the prefix taken
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
   const int row = blockIdx.x / kCL;
   const int b = row / a.Hkv, h = row - b * a.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned lt = (1u << lane) - 1u;
   const int t0 = a.cu[b];
   const int n = a.cu[b + 1] - t0;
   const int chunk = (n + kCL - 1) / kCL;
@@ -149,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1) propose_select_kernel(const PSArg
   int32_t* out = a.out + (int64_t)row * a.kp;
 
   // every branch depends on cluster-wide values only
-  if (n <= a.kp || chunk > a.cap) {
+  if (n <= a.kp || chunk > kMaxSlice) {
     const bool all = n <= a.kp;
     if (all) {
       for (int i = lo + tid; i < hi; i += kThreads) out[i] = i;
@@ -162,206 +133,164 @@ __global__ void __launch_bounds__(kThreads, 1) propose_select_kernel(const PSArg
     return;
   }
   const int k = a.kp;
+  uint32_t* h2 = cluster.map_shared_rank(hist2, 0);
+  uint32_t* h3 = cluster.map_shared_rank(hist3, 0);
+  if (rank == 0) {
+    hist2[tid] = 0u;  // kBins == kThreads
+    hist3[tid] = 0u;
+  }
+  __syncthreads();
+  cluster_arrive();  // rank 0's histograms are cleared once every CTA has arrived
 
-  // ---- 1. first digit from the histogram; the slice's keys
-  const uint32_t* gh = a.hist + (int64_t)row * kHist;
+  // ---- the slice's keys, kKPT loads in flight per thread
+  uint32_t key[kKPT];
   {
-    // 4 bins per thread, consecutive: bins 4t .. 4t+3
-    const uint4 v4 = reinterpret_cast<const uint4*>(gh)[tid];
-    const int v = (int)(v4.x + v4.y + v4.z + v4.w);
-    int total;
-    const int excl = block_excl_scan(v, scratch, &total);
-    int above = total - excl - v;
-    const uint32_t c4[4] = {v4.x, v4.y, v4.z, v4.w};
+    const float* kb = a.scores + (int64_t)h * a.T + t0 + lo;
+    float v[kKPT];
 #pragma unroll
-    for (int j = 3; j >= 0; --j) {
-      const int c = (int)c4[j];
-      if (above < k && k <= above + c) {
-        s3[0] = 4 * tid + j;
-        s3[1] = above;
-        s3[2] = c;
-      }
-      above += c;
+    for (int u = 0; u < kKPT; ++u) {
+      const int i = u * kThreads + tid;
+      v[u] = i < m ? __ldcg(kb + i) : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < kKPT; ++u) key[u] = ord_key(v[u]);
+  }
+  auto in = [&](int u) { return u * kThreads + tid < m; };
+
+  // ---- 1. threshold prefix P: keys with (key >> shift) > P are taken, and
+  // the first rtie keys with (key >> shift) == P in position order
+  const uint32_t* gh = a.hist + (int64_t)row * kHist;
+  find_digit<kHist / kThreads>([&](int bin) { return __ldcg(gh + bin); }, k, scratch, s_dig);
+  uint32_t P = (uint32_t)s_dig[0];
+  int shift = 20;
+  int r = k - s_dig[1];
+  cluster_wait();
+  if (r < s_dig[2]) {  // part of the bin: the second digit of its keys
+#pragma unroll
+    for (int u = 0; u < kKPT; ++u)
+      if (in(u) && (key[u] >> 20) == P) atomicAdd(h2 + ((key[u] >> 10) & (kBins - 1)), 1u);
+    cluster.sync();  // S1
+    find_digit<kBins / kThreads>([&](int bin) { return h2[bin]; }, r, scratch, s_dig);
+    P = (P << 10) | (uint32_t)s_dig[0];
+    shift = 10;
+    r -= s_dig[1];
+    if (r < s_dig[2]) {  // the last digit
+#pragma unroll
+      for (int u = 0; u < kKPT; ++u)
+        if (in(u) && (key[u] >> 10) == P) atomicAdd(h3 + (key[u] & (kBins - 1)), 1u);
+      cluster.sync();  // S2
+      find_digit<kBins / kThreads>([&](int bin) { return h3[bin]; }, r, scratch, s_dig);
+      P = (P << 10) | (uint32_t)s_dig[0];
+      shift = 0;
+      r -= s_dig[1];
     }
   }
-  const float* kbase = a.scores + (int64_t)h * a.T + t0 + lo;
-  for (int i0 = 0; i0 < m; i0 += 8 * kThreads) {  // eight independent loads in flight
-    float v[8];
+  const int rtie = r;
+
+  // ---- 2. counts above / at P, then every CTA's, in rank order
+  {
+    int gt = 0, eq = 0;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * kThreads + tid;
-      v[u] = i < m ? __ldcg(kbase + i) : 0.0f;
+    for (int u = 0; u < kKPT; ++u) {
+      if (in(u)) {
+        const uint32_t pre = key[u] >> shift;
+        gt += pre > P;
+        eq += pre == P;
+      }
     }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * kThreads + tid;
-      if (i < m) skeys[i] = ord_key(v[u]);
+    int tot;
+    block_excl_scan((gt << 16) | eq, scratch, &tot);  // both counts <= kMaxSlice < 65536
+    if (tid == 0) {
+      s_cnt[0] = tot >> 16;
+      s_cnt[1] = tot & 0xFFFF;
+    }
+  }
+  cluster.sync();  // S3: every CTA's counts are published
+  if (warp == 0) {
+    int g_s = 0, e_s = 0;
+    if (lane < kCL) {
+      const int* rc = cluster.map_shared_rank(s_cnt, lane);
+      g_s = rc[0];
+      e_s = rc[1];
+    }
+    const int ebefore = warp_incl_scan(e_s) - e_s;
+    const int take = min(max(rtie - ebefore, 0), e_s);
+    const int nsel = g_s + take;
+    const int before = warp_incl_scan(nsel) - nsel;
+    if (lane == rank) {
+      s_mine[0] = before;
+      s_mine[1] = take;
     }
   }
   __syncthreads();
-  const uint32_t b1 = (uint32_t)s3[0];
-  const int r1 = k - s3[1];
-  // keys above b1 (count) and in b1 (listed in position order)
-  {
-    uint32_t* ck = a.ckey + ((int64_t)row * kCL + rank) * a.cap;
-    int32_t* cp = a.cpos + ((int64_t)row * kCL + rank) * a.cap;
-    int gt = 0;
-    for (int i = tid; i < m; i += kThreads) gt += (skeys[i] >> 20) > b1;
-    const int nc = ordered_compact(
-        m, 0, [&](int i) { return (skeys[i] >> 20) == b1; },
-        [&](int i, int at) {
-          ck[at] = skeys[i];
-          cp[at] = lo + i;
-        },
-        tab, scratch);
-    int gtot;
-    block_excl_scan(gt, scratch, &gtot);
-    if (tid == 0) {
-      a.cmeta[((int64_t)row * kCL + rank) * 2] = nc;
-      a.cmeta[((int64_t)row * kCL + rank) * 2 + 1] = gtot;
-    }
-  }
-  cluster.sync();  // S1: every candidate list is in global memory
-
-  // ---- 2. rank 0: exact threshold over the concatenated lists, offsets
-  if (rank == 0) {
-    if (tid < kCL * 2) s_meta[tid / 2][tid % 2] = __ldcg(a.cmeta + (int64_t)row * kCL * 2 + tid);
-    __syncthreads();
-    int pre[kCL + 1];
-    pre[0] = 0;
-#pragma unroll
-    for (int c = 0; c < kCL; ++c) pre[c + 1] = pre[c] + s_meta[c][0];
-    const int nc = pre[kCL];
-    const uint32_t* ckr = a.ckey + (int64_t)row * kCL * a.cap;
-    const int32_t* cpr = a.cpos + (int64_t)row * kCL * a.cap;
-    // list index j -> (CTA c, entry) by the prefix of the counts
-    auto where = [&](int j) {
-      int c = 0;
-#pragma unroll
-      for (int x = 1; x < kCL; ++x) c += j >= pre[x];
-      return (int64_t)c * a.cap + (j - pre[c]);
-    };
-    // the concatenated list into shared memory when it fits (else read from L2)
-    uint32_t* lk = skeys + ((a.cap + 3) & ~3);
-    int32_t* lp = reinterpret_cast<int32_t*>(lk + a.cap);
-    const bool local = nc <= a.cap;
-    if (local) {
-      for (int c = 0; c < kCL; ++c) {
-        const int cnt = s_meta[c][0];
-        for (int j = tid; j < cnt; j += kThreads) {
-          lk[pre[c] + j] = __ldcg(ckr + (int64_t)c * a.cap + j);
-          lp[pre[c] + j] = __ldcg(cpr + (int64_t)c * a.cap + j);
-        }
-      }
-      __syncthreads();
-    }
-    auto getk = [&](int j) { return local ? lk[j] : __ldcg(ckr + where(j)); };
-    auto getp = [&](int j) { return local ? lp[j] : __ldcg(cpr + where(j)); };
-    uint32_t prefix = b1 << 20, pmask = 0xFFF00000u;
-    int r = r1;
-    find_bin_any(getk, nc, prefix, pmask, 10, 1024, r, hist, scratch, s3);
-    prefix |= (uint32_t)s3[0] << 10;
-    pmask |= 0x000FFC00u;
-    r -= s3[1];
-    find_bin_any(getk, nc, prefix, pmask, 0, 1024, r, hist, scratch, s3);
-    prefix |= (uint32_t)s3[0];
-    r -= s3[1];
-    const uint32_t T = prefix;
-    // the r-th listed key equal to T, in list (= position) order
-    __shared__ int s_I;
-    int before = 0;
-    for (int j0 = 0; j0 < nc && before < r; j0 += kThreads) {  // CTA-uniform
-      const int j = j0 + tid;
-      const unsigned eqm = __ballot_sync(0xffffffffu, j < nc && getk(j) == T);
-      if (lane == 0) s_wc[warp] = __popc(eqm);
-      __syncthreads();
-      int mine = before, tot = before;
-      for (int w = 0; w < kWarps; ++w) {
-        if (w < warp) mine += s_wc[w];
-        tot += s_wc[w];
-      }
-      if (lane == 0 && mine < r && r <= mine + __popc(eqm)) {
-        unsigned msk = eqm;
-        for (int t = 1; t < r - mine; ++t) msk &= msk - 1;
-        s_I = getp(j - lane + __ffs(msk) - 1);
-      }
-      before = tot;
-      __syncthreads();
-    }
-    const int I = s_I;
-    // selected listed keys per CTA region -> offsets
-    __shared__ int s_sel[kCL];
-    if (tid < kCL) s_sel[tid] = 0;
-    __syncthreads();
-    for (int j0 = warp * 32; j0 < nc; j0 += kThreads) {  // warp-uniform trip count
-      const int j = j0 + lane;
-      bool sel = false;
-      int c = 0;
-      if (j < nc) {
-        const uint32_t key = getk(j);
-        sel = key > T || (key == T && getp(j) <= I);
-#pragma unroll
-        for (int x = 1; x < kCL; ++x) c += j >= pre[x];
-      }
-      const int cf = __shfl_sync(0xffffffffu, c, 0);
-      const int cl = __shfl_sync(0xffffffffu, c, min(31, nc - 1 - j0));
-      for (int cc = cf; cc <= cl; ++cc) {  // the regions this block of 32 spans
-        const unsigned m2 = __ballot_sync(0xffffffffu, sel && c == cc);
-        if (lane == 0 && m2) atomicAdd(&s_sel[cc], __popc(m2));
-      }
-    }
-    __syncthreads();
-    if (tid == 0) {
-      int32_t* rr = a.res + (int64_t)row * (2 + kCL);
-      rr[0] = (int32_t)T;
-      rr[1] = I;
-      int acc = 0;
-      for (int c = 0; c < kCL; ++c) {
-        rr[2 + c] = acc;
-        acc += s_meta[c][1] + s_sel[c];
-      }
-      a.out_cnt[row] = k;
-    }
-  }
-  cluster.sync();  // S2: threshold and offsets are in global memory
+  const int off = s_mine[0], take = s_mine[1];
+  const bool part = take < s_cnt[1];  // the slice keeps only some of its keys at P
 
   // ---- 3. kept positions of the slice, ascending, from the offset
-  if (tid < 3) s_res[tid] = __ldcg(a.res + (int64_t)row * (2 + kCL) + (tid < 2 ? tid : 2 + rank));
+  if (part) {  // rank of each key at P among the slice's keys at P
+#pragma unroll
+    for (int u = 0; u < kKPT; ++u) {
+      const unsigned bal = __ballot_sync(0xffffffffu, in(u) && (key[u] >> shift) == P);
+      if (lane == 0) tabE[u * kWarps + warp] = __popc(bal);
+    }
+    __syncthreads();
+    scan_table(tabE, 0, scratch);
+  }
+#pragma unroll
+  for (int u = 0; u < kKPT; ++u) {
+    const uint32_t pre = key[u] >> shift;
+    const bool at = in(u) && pre == P;
+    bool keep = in(u) && pre > P;
+    if (part) {
+      const unsigned eb = __ballot_sync(0xffffffffu, at);
+      keep = keep || (at && tabE[u * kWarps + warp] + __popc(eb & lt) < take);
+    } else {
+      keep = keep || at;
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) tabK[u * kWarps + warp] = __popc(bal);
+  }
   __syncthreads();
-  const uint32_t T = (uint32_t)s_res[0];
-  const int I = s_res[1];
-  ordered_compact(
-      m, s_res[2], [&](int i) { return skeys[i] > T || (skeys[i] == T && lo + i <= I); },
-      [&](int i, int slot) {
-        if (slot < k) out[slot] = lo + i;
-        else flag_status(a.status, PRISM_DEV_TOO_LONG);  // unreachable if counts are right
-      },
-      tab, scratch);
+  scan_table(tabK, off, scratch);
+#pragma unroll
+  for (int u = 0; u < kKPT; ++u) {
+    const uint32_t pre = key[u] >> shift;
+    const bool at = in(u) && pre == P;
+    bool keep = in(u) && pre > P;
+    if (part) {
+      const unsigned eb = __ballot_sync(0xffffffffu, at);
+      keep = keep || (at && tabE[u * kWarps + warp] + __popc(eb & lt) < take);
+    } else {
+      keep = keep || at;
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (keep) {
+      const int slot = tabK[u * kWarps + warp] + __popc(bal & lt);
+      if (slot < k) out[slot] = lo + u * kThreads + tid;
+      else flag_status(a.status, PRISM_DEV_TOO_LONG);  // unreachable if counts are right
+    }
+  }
+  if (rank == 0 && tid == 0) a.out_cnt[row] = k;
+  // no CTA exits while rank 0's histograms or its counts may still be read
+  cluster_arrive();
+  cluster_wait();
 }
 
 }  // namespace
 
-int propose_select_cap(int max_len) { return (max_len + kCL - 1) / kCL; }
 int propose_select_cluster() { return kCL; }
 int propose_select_max_row() { return kCL * kMaxSlice; }
 
 cudaError_t launch_propose_select(const Dims& d, const float* scores, const uint32_t* hist,
-                                  int kappa_p, int cap, uint32_t* ckey, int32_t* cpos,
-                                  int32_t* cmeta, int32_t* res, int32_t* pool, int32_t* pool_cnt,
-                                  int32_t* status, cudaStream_t st) {
+                                  int kappa_p, int32_t* pool, int32_t* pool_cnt, int32_t* status,
+                                  cudaStream_t st) {
   const int rows = d.B * d.Hkv;
   if (rows == 0) return cudaSuccess;
-  PSArgs a{scores, hist, d.cu_dev, d.Hkv, d.T, kappa_p, cap, ckey, cpos, cmeta, res, pool, pool_cnt,
-           status};
-  const int slice = cap > 0 ? cap : 1;
-  const size_t smem = (size_t)(((slice + 3) & ~3) + 2 * slice) * sizeof(uint32_t);
-  cudaError_t e = cudaFuncSetAttribute(propose_select_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  PSArgs a{scores, hist, d.cu_dev, d.Hkv, d.T, kappa_p, pool, pool_cnt, status};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(rows * kCL));
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;

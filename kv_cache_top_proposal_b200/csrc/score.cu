@@ -23,6 +23,12 @@
 //    bytes in flight to run at HBM speed.
 //  * score_simt_kernel: plain fp32 FMAs on CUDA cores (fp32 queries, and the
 //    comparison kernel for bf16).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstdlib>
+#include <cstring>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -42,6 +48,7 @@ struct ScoreArgs {
   const int32_t* cu;
   int64_t T;
   int B, Hkv, G;
+  int32_t* status;
 };
 
 // s_pref[b] = number of work items of sequences before b (per KV head).
@@ -80,6 +87,17 @@ __device__ __forceinline__ void i8x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& 
   hi = __byte_perm(x, 0x64646464u, 0x4342);
   asm("sub.rn.f16x2 %0, %0, %1;" : "+r"(lo) : "r"(0x64806480u));
   asm("sub.rn.f16x2 %0, %0, %1;" : "+r"(hi) : "r"(0x64806480u));
+}
+
+// Shared first-digit histogram with two 16-bit counts per word (bin b in
+// word b / 2, high half when b is odd); lanes sharing a bin issue one atomic.
+__device__ __forceinline__ void warp_hist_add_packed(uint32_t* hw, uint32_t bin, bool valid) {
+  const unsigned act = __ballot_sync(0xffffffffu, valid);
+  if (!act) return;
+  const unsigned peers = __match_any_sync(0xffffffffu, valid ? bin : 0xffffffffu) & act;
+  const int lane = threadIdx.x & 31;
+  if (valid && (peers & ((1u << lane) - 1u)) == 0)
+    atomicAdd(&hw[bin >> 1], (uint32_t)__popc(peers) << ((bin & 1u) * 16));
 }
 
 __device__ __forceinline__ uint32_t pack_f16(float a, float b) {
@@ -319,6 +337,232 @@ __global__ void __launch_bounds__(kThreads, 2) score_mma_kernel(ScoreArgs a) {
   flush();
 }
 
+// TMA scorer (d = 128).  The same arithmetic as score_mma_kernel, with each
+// 128-row stage of codes moved by one 2D tensor copy (cp.async.bulk.tensor,
+// 128-byte swizzle: 16-byte chunk c of row r lands at chunk c ^ (r & 7))
+// that completes on the stage's mbarrier, so one thread issues a whole stage.
+// Thread (g, tig) reads chunks 2 tig and 2 tig + 1 of its two rows -- under
+// the swizzle, the 8 lanes of each quarter-warp hit 8 different chunks -- so
+// k-step s covers features 32 tig + 4 s .. + 3 of the permuted feature axis.
+// Scales come straight from global memory, one per row.  The first-digit
+// histogram keeps two 16-bit counts per word (flushed before they could
+// overflow), so three CTAs fit on an SM.
+constexpr int kTmaStages = 4;
+constexpr int kTmaStageBytes = kStageRows * 128;
+constexpr int kTmaFlushStages = 256;  // stages between histogram flushes (< 65536 keys)
+constexpr uint32_t kWaitLimit = 1u << 24;  // polls of a stage barrier before giving up
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// rows [y, y + 128) of the code tensor into a swizzled stage; completes on bar
+__device__ __forceinline__ void tma_rows(void* dst, const CUtensorMap* tm, int y, uint64_t* bar) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
+               "r"(kTmaStageBytes)
+               : "memory");
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(0), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 3) score_tma_kernel(const __grid_constant__ CUtensorMap tm,
+                                                                ScoreArgs a) {
+  constexpr int D = 128;
+  constexpr int KS = D / 16;
+  extern __shared__ unsigned char dsm_raw[];
+  // the swizzle pattern repeats every 1024 bytes: stages start on that boundary
+  unsigned char* ring =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(ring + kTmaStages * kTmaStageBytes);  // [kHist / 2]
+  int* s_pref = reinterpret_cast<int*>(s_hist + kHist / 2);
+  int* s_cu = s_pref + a.B + 1;
+  __shared__ __align__(8) uint64_t full[kTmaStages];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, tig = lane & 3;
+  for (int i = tid; i <= a.B; i += kThreads) s_cu[i] = a.cu[i];
+  for (int i = tid; i < kHist / 2; i += kThreads) s_hist[i] = 0u;
+  if (tid == 0) {
+    for (int i = 0; i < kTmaStages; ++i) mbar_init(&full[i], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  chunk_prefix(a.cu, a.B, kStageRows, s_pref);  // ends with __syncthreads
+  const int per_head = s_pref[a.B];
+  const int64_t total = (int64_t)a.Hkv * per_head;
+  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
+  const int64_t s_begin = total * blockIdx.x / gridDim.x;
+  const int64_t s_end = total * (blockIdx.x + 1) / gridDim.x;
+  const int nk = (int)(s_end - s_begin);
+  StageIter it_issue, it_comp;
+  {
+    const int h = (int)(s_begin / per_head);
+    const int cc = (int)(s_begin - (int64_t)h * per_head);
+    const int b = find_seq(s_pref, a.B, cc);
+    it_issue = StageIter{h, b, (cc - s_pref[b]) * kStageRows};
+    it_comp = it_issue;
+  }
+  auto issue = [&](int kk) {  // thread 0
+    if (kk < nk) {
+      const int64_t y = (int64_t)it_issue.h * a.T + s_cu[it_issue.b] + it_issue.r0;
+      tma_rows(ring + (kk % kTmaStages) * kTmaStageBytes, &tm, (int)y, &full[kk % kTmaStages]);
+      it_issue.advance(s_cu, a.B);
+    }
+  };
+  if (tid == 0) {
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tm)) : "memory");
+    for (int kk = 0; kk < kTmaStages; ++kk) issue(kk);
+  }
+
+  uint32_t bq[NT][KS][2];
+  float unscale = 1.0f;
+  int cur_b = -1, cur_h = -1;
+  int hist_row = -1, since_flush = 0;
+  auto flush = [&]() {  // packed shared histogram -> global (non-zero bins), then clear
+    if (a.hist && hist_row >= 0) {
+      uint32_t* gh = a.hist + (int64_t)hist_row * kHist;
+      for (int i = tid; i < kHist / 2; i += kThreads) {
+        const uint32_t c = s_hist[i];
+        if (c) {
+          if (c & 0xFFFFu) atomicAdd(gh + 2 * i, c & 0xFFFFu);
+          if (c >> 16) atomicAdd(gh + 2 * i + 1, c >> 16);
+          s_hist[i] = 0u;
+        }
+      }
+    }
+    since_flush = 0;
+    __syncthreads();
+  };
+#pragma unroll 1
+  for (int kk = 0; kk < nk; ++kk) {
+    const int L = s_cu[it_comp.b + 1] - s_cu[it_comp.b];
+    const int rows = min(kStageRows, L - it_comp.r0);
+    const int64_t rowbase = (int64_t)it_comp.h * a.T + s_cu[it_comp.b] + it_comp.r0;
+    if (it_comp.b != cur_b || it_comp.h != cur_h) {
+      // query fragments of (b, h), scaled by a power of two into fp16 range;
+      // thread (g, tig) holds column n = g; k-step s covers features
+      // 32 tig + 4 s .. + 3
+      cur_b = it_comp.b;
+      cur_h = it_comp.h;
+      float qv[NT][KS][4];
+      float mx = 0.0f;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int n = nt * 8 + g;
+#pragma unroll
+        for (int s2 = 0; s2 < KS; ++s2) {
+          const int base = 32 * tig + 4 * s2;
+          if (n < a.G) {
+            const uint2 w = *reinterpret_cast<const uint2*>(
+                q + ((int64_t)cur_b * a.Hkv * a.G + (int64_t)cur_h * a.G + n) * D + base);
+            qv[nt][s2][0] = bf16lo(w.x); qv[nt][s2][1] = bf16hi(w.x);
+            qv[nt][s2][2] = bf16lo(w.y); qv[nt][s2][3] = bf16hi(w.y);
+          } else {
+            qv[nt][s2][0] = qv[nt][s2][1] = qv[nt][s2][2] = qv[nt][s2][3] = 0.0f;
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) mx = fmaxf(mx, fabsf(qv[nt][s2][e]));
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      int qexp = 0;
+      if (mx > 0.0f) {
+        const int e2 = ((__float_as_int(mx) >> 23) & 0xFF) - 126;  // mx < 2^e2
+        qexp = min(126, max(-126, 15 - e2));
+      }
+      const float up = pow2f(qexp);
+      unscale = pow2f(-qexp);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int s2 = 0; s2 < KS; ++s2) {
+          bq[nt][s2][0] = pack_f16(qv[nt][s2][0] * up, qv[nt][s2][1] * up);
+          bq[nt][s2][1] = pack_f16(qv[nt][s2][2] * up, qv[nt][s2][3] * up);
+        }
+    }
+    const int row_id = it_comp.b * a.Hkv + it_comp.h;  // CTA-uniform
+    if (row_id != hist_row || since_flush == kTmaFlushStages) {
+      flush();
+      hist_row = row_id;
+    }
+    ++since_flush;
+    it_comp.advance(s_cu, a.B);
+    const int slot = kk % kTmaStages;
+    {
+      uint32_t it = 0;
+      while (!mbar_try_wait(&full[slot], (uint32_t)(kk / kTmaStages) & 1u)) {
+        if (++it == kWaitLimit) {
+          if (tid == 0) flag_status(a.status, PRISM_DEV_TIMEOUT);
+          break;
+        }
+      }
+    }
+    const unsigned char* buf = ring + slot * kTmaStageBytes;
+    const int t = warp;  // one 16-row tile per warp
+    if (t * 16 < rows) {
+      const int rs = t * 16 + g + 8 * tig;  // tig 0: row g, tig 1: row g + 8
+      const bool mine = tig < 2 && rs < rows;
+      const float sc = mine ? __ldg(a.scale + rowbase + rs) : 0.0f;
+      uint4 cur[2][2];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int r = t * 16 + g + 8 * half;  // r & 7 == g
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch)
+          cur[half][ch] = *reinterpret_cast<const uint4*>(buf + r * 128 + (((2 * tig + ch) ^ g) << 4));
+      }
+      float acc[2][NT][4];
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) acc[u][nt][0] = acc[u][nt][1] = acc[u][nt][2] = acc[u][nt][3] = 0.0f;
+#pragma unroll
+      for (int s2 = 0; s2 < KS; ++s2) {
+        uint32_t a0, a1, a2, a3;
+        i8x4_to_f16(word_of(cur[0][s2 / 4], s2 % 4), a0, a2);  // row g
+        i8x4_to_f16(word_of(cur[1][s2 / 4], s2 % 4), a1, a3);  // row g + 8
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          mma16816(acc[s2 & 1][nt], a0, a1, a2, a3, bq[nt][s2][0], bq[nt][s2][1]);
+      }
+      float mA = -INFINITY, mB = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int col = nt * 8 + 2 * tig;
+        const float c0 = acc[0][nt][0] + acc[1][nt][0], c1 = acc[0][nt][1] + acc[1][nt][1];
+        const float c2 = acc[0][nt][2] + acc[1][nt][2], c3 = acc[0][nt][3] + acc[1][nt][3];
+        if (col < a.G) { mA = fmaxf(mA, c0); mB = fmaxf(mB, c2); }
+        if (col + 1 < a.G) { mA = fmaxf(mA, c1); mB = fmaxf(mB, c3); }
+      }
+      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
+      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
+      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
+      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
+      float score = 0.0f;
+      if (mine) {
+        score = sc * ((tig == 0 ? mA : mB) * unscale);
+        a.scores[rowbase + rs] = score;
+      }
+      if (a.hist) warp_hist_add_packed(s_hist, ord_key(score) >> 20, mine);
+    }
+    __syncthreads();  // every warp is done with the stage
+    if (tid == 0) issue(kk + kTmaStages);
+  }
+  flush();
+}
+
 // CUDA-core scorer: one thread per key row, query in shared memory (fp32).
 template <typename T, int D, int GP>
 __global__ void __launch_bounds__(kThreads) score_simt_kernel(ScoreArgs a) {
@@ -398,6 +642,54 @@ cudaError_t run_mma(const Dims& d, const ScoreArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// PRISM_PROPOSE_SCORER=tma selects the tensor-copy scorer
+bool use_tma_scorer() {
+  const char* e = std::getenv("PRISM_PROPOSE_SCORER");
+  return e && std::strcmp(e, "tma") == 0;
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult res;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &res) != cudaSuccess ||
+        res != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// Launches the TMA scorer when the code tensor can be described by a tensor
+// map (d = 128, 16-byte aligned base); returns false to fall back.
+template <int NT>
+bool run_tma(const Dims& d, const ScoreArgs& a, int64_t total, cudaError_t* err, cudaStream_t st) {
+  const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode || d.D != 128 || (reinterpret_cast<uintptr_t>(a.kq) & 15) != 0) return false;
+  const uint64_t nrows = (uint64_t)d.Hkv * (uint64_t)d.T;
+  if (nrows == 0 || nrows > 0x7fffffffull) return false;
+  CUtensorMap tm;
+  const cuuint64_t dims[2] = {128, (cuuint64_t)nrows};
+  const cuuint64_t strides[1] = {128};
+  const cuuint32_t box[2] = {128, (cuuint32_t)kStageRows};
+  const cuuint32_t estr[2] = {1, 1};
+  if (encode(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(a.kq), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  const int smem = 1024 + kTmaStages * kTmaStageBytes + kHist / 2 * 4 + 2 * (d.B + 1) * (int)sizeof(int);
+  auto k = score_tma_kernel<NT>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) {
+    const int grid = grid_for(k, smem, d.num_sms, total);
+    k<<<grid, kThreads, smem, st>>>(tm, a);
+    e = cudaGetLastError();
+  }
+  *err = e;
+  return true;
+}
+
 template <typename T, int D, int GP>
 cudaError_t run_simt(const Dims& d, const ScoreArgs& a, int64_t total, cudaStream_t st) {
   const int smem = (((d.B + 1 + 3) & ~3) + GP * D) * (int)sizeof(int);
@@ -426,12 +718,20 @@ cudaError_t simt_by_group(const Dims& d, const ScoreArgs& a, int64_t total, cuda
 
 cudaError_t launch_propose_scores(const Dims& d, const void* q, const int8_t* kq,
                                   const float* scale, float* scores, uint32_t* hist, bool use_mma,
-                                  cudaStream_t st) {
+                                  int32_t* status, cudaStream_t st) {
   int64_t per_head = 0;
   for (int b = 0; b < d.B; ++b) per_head += cdiv(d.cu_host[b + 1] - d.cu_host[b], kChunkRows);
   const int64_t total = per_head * d.Hkv;
   if (total == 0) return cudaSuccess;
-  ScoreArgs a{q, kq, scale, scores, hist, d.cu_dev, d.T, d.B, d.Hkv, d.G};
+  ScoreArgs a{q, kq, scale, scores, hist, d.cu_dev, d.T, d.B, d.Hkv, d.G, status};
+  if (use_mma && d.bf16 && d.D == 128 && use_tma_scorer()) {
+    int64_t stages = 0;
+    for (int b = 0; b < d.B; ++b) stages += cdiv(d.cu_host[b + 1] - d.cu_host[b], kStageRows);
+    cudaError_t e = cudaSuccess;
+    const bool ran = d.G <= 8 ? run_tma<1>(d, a, stages * d.Hkv, &e, st)
+                              : run_tma<2>(d, a, stages * d.Hkv, &e, st);
+    if (ran) return e;
+  }
   if (use_mma && d.bf16) {
     if (d.D == 128) return d.G <= 8 ? run_mma<128, 1>(d, a, st) : run_mma<128, 2>(d, a, st);
     return d.G <= 8 ? run_mma<64, 1>(d, a, st) : run_mma<64, 2>(d, a, st);

@@ -72,15 +72,20 @@ class PrismDecoder:
                             self.ws_dense) if w is not None]
 
     def layer(self, l: int, q, k, v, kq=None, k_scale=None, quantize_new: bool = True,
-              k_new=None, v_new=None, k_next=None, stream=None):
+              k_new=None, v_new=None, k_next=None, overlap: bool = False, stream=None):
         """Enqueue one layer of the step (kq/k_scale required at proposal layers).
 
         k_new / v_new ([B][Hkv][d]), when given, are first written to the last
-        position of every sequence (the token being decoded)."""
+        position of every sequence (the token being decoded).  overlap: the
+        previous kernel on the stream is the fused refined layer before this
+        one, so this layer's launch may begin before it ends."""
         p = self.p
-        if k_new is not None:
+        proposal = l % self.group == 0
+        # a fused refined layer appends the new rows itself
+        fused_append = self.fused and not proposal and k_new is not None
+        if k_new is not None and not fused_append:
             prism.append_kv(p, k_new, v_new, k, v, stream=stream)
-        if l % self.group == 0:
+        if proposal:
             if quantize_new and self.new_rows.numel():
                 prism.quantize_k(p, k, kq, k_scale, tok_rows=self.new_rows, ws=self.ws_q, stream=stream)
             prism.propose(p, q, kq, k_scale, self.kappa_p, self.pool[l], self.pool_cnt[l],
@@ -89,7 +94,10 @@ class PrismDecoder:
         if self.fused:
             prism.refine_decode(p, q, k, v, self.pool[src], self.pool_cnt[src], self.kappa_p,
                                 self.kappa, self.scale, self.idx[l], self.cnt[l], self.out[l],
-                                self.ws_rd, lse=self.lse[l], k_prefetch=k_next, stream=stream)
+                                self.ws_rd, lse=self.lse[l],
+                                k_new=k_new if fused_append else None,
+                                v_new=v_new if fused_append else None, k_prefetch=k_next,
+                                overlap=overlap, stream=stream)
             return
         prism.refine(p, q, k, self.pool[src], self.pool_cnt[src], self.kappa_p, self.kappa,
                      self.idx[l], self.cnt[l], self.ws_ref, stream=stream)
@@ -102,19 +110,18 @@ class PrismDecoder:
         per-layer sequences; kqs/scales are indexed by proposal layer."""
         for l in range(self.num_layers):
             pl = l % self.group == 0
-            # the next layer refines on the same pool unless it is a proposal layer
-            nxt = ks[l + 1] if l + 1 < self.num_layers and (l + 1) % self.group else None
             self.layer(l, qs[l], ks[l], vs[l], kqs[l] if pl else None, scales[l] if pl else None,
                        quantize_new=quantize_new,
                        k_new=None if k_new is None else k_new[l],
-                       v_new=None if v_new is None else v_new[l], k_next=nxt, stream=stream)
+                       v_new=None if v_new is None else v_new[l],
+                       overlap=self.fused and not pl and l > 0, stream=stream)
 
     def launches_per_step(self, append: bool) -> int:
         """Kernels one step enqueues (append, quantize, score, select, refine
         score, select, attend, merge)."""
         n = 0
         for l in range(self.num_layers):
-            n += 1 if append else 0
+            n += 1 if append and (l % self.group == 0 or not self.fused) else 0
             if l % self.group == 0:
                 n += (1 if self.new_rows.numel() else 0) + 2
             n += 1 if self.fused else 2 + 2

@@ -21,8 +21,9 @@ F32, BF16 = 0, 1
 OP_QUANTIZE, OP_PROPOSE, OP_REFINE, OP_SPARSE_DECODE, OP_DENSE_DECODE, OP_REFINE_DECODE = range(6)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_SCRATCH_LIMIT = range(7)
 NOALLOC_SCRATCH_BYTES = 4 << 20
-DEV_BAD_INDEX, DEV_TOO_LONG = 0x1, 0x2
+DEV_BAD_INDEX, DEV_TOO_LONG, DEV_TIMEOUT = 0x1, 0x2, 0x4
 MAX_SELECT_ROW = 393216
+RD_OVERLAP = 0x1
 WS_HEADER = 256
 
 EXPORTS = ("prism_workspace_size", "prism_append_kv", "prism_quantize_k", "prism_propose", "prism_refine",
@@ -58,7 +59,8 @@ def _load():
         "prism_propose": [sp, P, P, P, i32, P, P, P, S, P],
         "prism_refine": [sp, P, P, P, P, i32, i32, P, P, P, P, S, P],
         "prism_sparse_decode": [sp, P, P, P, P, P, i32, ctypes.c_float, P, P, P, S, P],
-        "prism_refine_decode": [sp, P, P, P, P, P, i32, i32, ctypes.c_float, P, P, P, P, P, P, S, P],
+        "prism_refine_decode": [sp, P, P, P, P, P, i32, i32, ctypes.c_float, P, P, P, P, P, P, P,
+                                ctypes.c_uint32, P, S, P],
         "prism_dense_decode": [sp, P, P, P, ctypes.c_float, P, P, P, S, P],
         "prism_clear_device_status": [P, S, P],
         "prism_get_device_status": [P, S, P, ctypes.POINTER(ctypes.c_int32)],
@@ -170,11 +172,16 @@ def sparse_decode(p: Problem, q, k, v, idx, cnt, kappa: int, softmax_scale: floa
 
 
 def refine_decode(p: Problem, q, k, v, pool, pool_cnt, kappa_p: int, kappa: int,
-                  softmax_scale: float, idx, cnt, out, ws, lse=None, k_prefetch=None, stream=None):
+                  softmax_scale: float, idx, cnt, out, ws, lse=None, k_new=None, v_new=None,
+                  k_prefetch=None, overlap: bool = False, stream=None):
+    """Refined layer in one call; k_new / v_new ([B][Hkv][d]) are appended
+    at the last position of every sequence first.  overlap: the launch may
+    begin before the previous kernel on the stream ends (see PRISM_RD_OVERLAP)."""
     _check(_lib.prism_refine_decode(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(pool), _ptr(pool_cnt),
                                     kappa_p, kappa, float(softmax_scale), _ptr(idx), _ptr(cnt),
-                                    _ptr(out), _ptr(lse), _ptr(k_prefetch), _ptr(ws), _nbytes(ws),
-                                    _stream(stream)),
+                                    _ptr(out), _ptr(lse), _ptr(k_new), _ptr(v_new),
+                                    _ptr(k_prefetch), RD_OVERLAP if overlap else 0, _ptr(ws),
+                                    _nbytes(ws), _stream(stream)),
            "refine_decode")
 
 

@@ -107,6 +107,18 @@ def test_calls_validate_before_launch(prism_lib):
     assert lib.prism_dense_decode(ref, f, f, None, 0.1, f, None, ws, 1 << 30, None) == P.ERR_INVALID_ARG
     assert lib.prism_quantize_k(ref, f, None, f, None, 0, None, 0, None) == P.ERR_INVALID_ARG
     assert lib.prism_get_device_status(None, 0, None, None) == P.ERR_WORKSPACE
+    # fused refined layer: unknown flags, a lone new row, misaligned rows
+    _, nrd = _ws(P, s, P.OP_REFINE_DECODE, 1024, 256)
+    rd = lib.prism_refine_decode
+    assert rd(ref, f, f, f, f, f, 1024, 256, 0.1, f, f, f, None, None, None, None, 2, ws, nrd,
+              None) == P.ERR_INVALID_ARG
+    assert rd(ref, f, f, f, f, f, 1024, 256, 0.1, f, f, f, None, f, None, None, 0, ws, nrd,
+              None) == P.ERR_INVALID_ARG
+    bad = ctypes.c_void_p(FAKE + 8)
+    assert rd(ref, bad, f, f, f, f, 1024, 256, 0.1, f, f, f, None, None, None, None, 0, ws, nrd,
+              None) == P.ERR_INVALID_ARG
+    assert rd(ref, f, f, f, f, f, 1024, 2048, 0.1, f, f, f, None, None, None, None, 0, ws, nrd,
+              None) == P.ERR_INVALID_ARG
 
 
 def test_too_long_rows_unsupported(prism_lib):

@@ -101,13 +101,17 @@ PROPOSE_CASES = [
 
 
 @pytest.mark.parametrize("case", PROPOSE_CASES, ids=lambda c: f"{c[0]}-{c[1]}/{c[2]}-d{c[3]}-{c[4]}-kp{c[5]}")
-@pytest.mark.parametrize("scorer", ["mma", "simt"])
+@pytest.mark.parametrize("scorer", ["tma", "mma", "simt"])
 def test_propose_vs_oracle(P, case, scorer, monkeypatch):
+    """mma: the default tensor-core scorer (cp.async stages); tma: the
+    tensor-core scorer fed by tensor copies (d = 128); simt: CUDA cores."""
     seqlens, hq, hkv, d, dtype, kp = case
     if scorer == "simt":
         monkeypatch.setenv("PRISM_PROPOSE_SCORER", "simt")
     elif dtype != "bf16":
-        pytest.skip("the tensor-core scorer takes bf16 queries")
+        pytest.skip("the tensor-core scorers take bf16 queries")
+    elif scorer == "tma":
+        monkeypatch.setenv("PRISM_PROPOSE_SCORER", "tma")
     prob = problem(P, seqlens, hq, hkv, d, dtype)
     q, k, _ = make_case(seqlens, hq, hkv, d, dtype, seed=2)
     T = prob.total_tokens
@@ -409,3 +413,100 @@ def test_refine_decode_prefetch_changes_nothing(P):
     assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
     assert torch.equal(res[0][2], res[1][2])
     assert P.get_device_status(ws) == 0
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_refine_decode_appends_new_rows(P, dtype):
+    """Rows passed as k_new / v_new are written at position L_b - 1 and used
+    there: the result equals prism_append_kv followed by the plain call, and
+    the last position is in every pool (it must be read from the new rows)."""
+    seqlens, hq, hkv, d, kp, kap = [5000, 2100, 1], 8, 2, 128, 1024, 256
+    B = len(seqlens)
+    prob = problem(P, seqlens, hq, hkv, d, dtype)
+    q, k, v = make_case(seqlens, hq, hkv, d, dtype, seed=17)
+    g = torch.Generator(device="cpu").manual_seed(18)
+    k_new = (torch.randn((B, hkv, d), generator=g) * 3).to(k.dtype).to(DEV)
+    v_new = torch.randn((B, hkv, d), generator=g).to(v.dtype).to(DEV)
+    rng = np.random.default_rng(19)
+    pool = np.full((B, hkv, kp), -1, np.int32)
+    pcnt = np.zeros((B, hkv), np.int32)
+    for b, L in enumerate(seqlens):
+        for h in range(hkv):
+            n = min(kp, L)
+            sel = set(rng.choice(L, n, replace=False).tolist())
+            if L - 1 not in sel:
+                sel.discard(min(sel))
+                sel.add(L - 1)
+            pool[b, h, :n] = np.sort(np.array(sorted(sel)))
+            pcnt[b, h] = n
+    pool_t, pcnt_t = torch.tensor(pool, device=DEV), torch.tensor(pcnt, device=DEV)
+    scale = float(np.float32(1 / math.sqrt(d)))
+    ws = ws_for(P, prob, P.OP_REFINE_DECODE, kp, kap)
+    res = []
+    for fused in (False, True):
+        kc, vc = k.clone(), v.clone()
+        idx = torch.full((B, hkv, kap), -7, dtype=torch.int32, device=DEV)
+        cnt = torch.zeros((B, hkv), dtype=torch.int32, device=DEV)
+        out = torch.full((B, hq, d), 77.0, device=DEV)
+        lse = torch.full((B, hq), 77.0, device=DEV)
+        if fused:
+            P.refine_decode(prob, q, kc, vc, pool_t, pcnt_t, kp, kap, scale, idx, cnt, out, ws,
+                            lse=lse, k_new=k_new, v_new=v_new)
+        else:
+            P.append_kv(prob, k_new, v_new, kc, vc)
+            P.refine_decode(prob, q, kc, vc, pool_t, pcnt_t, kp, kap, scale, idx, cnt, out, ws,
+                            lse=lse)
+        torch.cuda.synchronize()
+        res.append((kc, vc, idx, cnt, out, lse))
+    assert P.get_device_status(ws) == 0
+    (k0, v0, i0, c0, o0, l0), (k1, v1, i1, c1, o1, l1) = res
+    assert torch.equal(k0, k1) and torch.equal(v0, v1)
+    assert torch.equal(i0, i1) and torch.equal(c0, c1)
+    assert torch.equal(o0, o1) and torch.equal(l0, l1)
+    # the new rows took part: the last position is selected somewhere, and the
+    # result matches the oracle on the appended cache
+    gi, gc = _np(i1), _np(c1)
+    assert any((gi[b, h, :gc[b, h]] == seqlens[b] - 1).any() for b in range(B) for h in range(hkv))
+    oout, _ = pipeline.attend_layer(q, k1, v1, prob.cu_host.tolist(), gi, gc, scale)
+    assert np.abs(_np(o1) - oout).max() <= atol_for(dtype)
+
+
+def test_refine_decode_overlapped_launches_match(P):
+    """Consecutive refined layers launched with PRISM_RD_OVERLAP (each may
+    start before the previous one ends) give the results of plain launches."""
+    seqlens, hq, hkv, d, kp, kap = [30000, 7000], 32, 8, 128, 4096, 1024
+    B = len(seqlens)
+    prob = problem(P, seqlens, hq, hkv, d, "bf16")
+    rng = np.random.default_rng(21)
+    pool = np.full((B, hkv, kp), -1, np.int32)
+    pcnt = np.zeros((B, hkv), np.int32)
+    for b, L in enumerate(seqlens):
+        for h in range(hkv):
+            pool[b, h] = np.sort(rng.choice(L, kp, replace=False))
+            pcnt[b, h] = kp
+    pool_t, pcnt_t = torch.tensor(pool, device=DEV), torch.tensor(pcnt, device=DEV)
+    layers = [make_case(seqlens, hq, hkv, d, "bf16", seed=30 + l) for l in range(4)]
+    g = torch.Generator(device="cpu").manual_seed(22)
+    news = [(torch.randn((B, hkv, d), generator=g).to(torch.bfloat16).to(DEV),
+             torch.randn((B, hkv, d), generator=g).to(torch.bfloat16).to(DEV)) for _ in range(4)]
+    ws = ws_for(P, prob, P.OP_REFINE_DECODE, kp, kap)
+    res = []
+    for overlap in (False, True):
+        outs = []
+        for l, (q, k, v) in enumerate(layers):
+            kc, vc = k.clone(), v.clone()
+            idx = torch.zeros((B, hkv, kap), dtype=torch.int32, device=DEV)
+            cnt = torch.zeros((B, hkv), dtype=torch.int32, device=DEV)
+            out = torch.zeros((B, hq, d), device=DEV)
+            outs.append((kc, vc, idx, cnt, out))
+        torch.cuda.synchronize()
+        for l, (q, k, v) in enumerate(layers):
+            kc, vc, idx, cnt, out = outs[l]
+            P.refine_decode(prob, q, kc, vc, pool_t, pcnt_t, kp, kap, 0.0883883, idx, cnt, out, ws,
+                            k_new=news[l][0], v_new=news[l][1], overlap=overlap and l > 0)
+        torch.cuda.synchronize()
+        res.append(outs)
+    assert P.get_device_status(ws) == 0
+    for a, b in zip(res[0], res[1]):
+        for x, y in zip(a, b):
+            assert torch.equal(x, y)
