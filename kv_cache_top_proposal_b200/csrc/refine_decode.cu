@@ -59,6 +59,7 @@ constexpr int kH3 = kH2 + kBins2 / 2;
 constexpr int kHistWords = kH3 + kBins2 / 2;
 constexpr int kMaxCount = 65535;  // largest pool a 16-bit bin count can hold
 constexpr int kMaxCluster = 16;
+constexpr int kCandCap = 256;     // first-digit candidates per CTA ranked by rank 0 (8 B each)
 
 struct RDArgs {
   const void* q;
@@ -224,12 +225,18 @@ struct ScoreMma {
     }
   }
 
+  // Warp w takes 16-row tiles w % 4, w % 4 + 4, ... and k-steps of half
+  // w / 4 (all eight warps busy on a 64-row stage); the two halves' sums go to
+  // dots and dots2, added by the key pass.
+  static constexpr bool kSplit = true;
   __device__ __forceinline__ void run(const unsigned char* buf, int r0, int nrows, const int* spos,
-                                      int G, int mc, float* dots) const {
+                                      int G, int mc, float* dots, float* dots2) const {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, tig = lane & 3;
+    const int kh = warp >> 2;
+    float* out = kh ? dots2 : dots;
     const int ntile = (nrows + 15) >> 4;
-    for (int t = warp; t < ntile; t += kWarps) {
+    for (int t = warp & 3; t < ntile; t += kWarps / 2) {
       float acc[2][NT][4];
 #pragma unroll
       for (int u = 0; u < 2; ++u)
@@ -237,12 +244,16 @@ struct ScoreMma {
         for (int nt = 0; nt < NT; ++nt) acc[u][nt][0] = acc[u][nt][1] = acc[u][nt][2] = acc[u][nt][3] = 0.0f;
       const int lrow = t * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-      for (int s = 0; s < KS; ++s) {
+      for (int s2 = 0; s2 < KS / 2; ++s2) {
+        const int s = kh * (KS / 2) + s2;
         uint32_t a0, a1, a2, a3;
         ldmatrix_x4(smem_u32(buf + swz<D * 2>(lrow, 2 * s + (lane >> 4))), a0, a1, a2, a3);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-          mma_bf16(acc[s & 1][nt], a0, a1, a2, a3, bq[nt][s][0], bq[nt][s][1]);
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint32_t b0 = kh ? bq[nt][KS / 2 + s2][0] : bq[nt][s2][0];
+          const uint32_t b1 = kh ? bq[nt][KS / 2 + s2][1] : bq[nt][s2][1];
+          mma_bf16(acc[s2 & 1][nt], a0, a1, a2, a3, b0, b1);
+        }
       }
       // c0,c1: row t*16+g, heads col, col+1; c2,c3: row t*16+g+8
 #pragma unroll
@@ -256,8 +267,8 @@ struct ScoreMma {
             const int col = nt * 8 + 2 * tig;
             const float v0 = acc[0][nt][2 * half] + acc[1][nt][2 * half];
             const float v1 = acc[0][nt][2 * half + 1] + acc[1][nt][2 * half + 1];
-            if (col < G) dots[col * mc + i] = ok ? v0 : -INFINITY;
-            if (col + 1 < G) dots[(col + 1) * mc + i] = ok ? v1 : -INFINITY;
+            if (col < G) out[col * mc + i] = ok ? v0 : -INFINITY;
+            if (col + 1 < G) out[(col + 1) * mc + i] = ok ? v1 : -INFINITY;
           }
         }
       }
@@ -289,8 +300,9 @@ struct ScoreSimt {
     }
   }
 
+  static constexpr bool kSplit = false;
   __device__ __forceinline__ void run(const unsigned char* buf, int r0, int nrows, const int* spos,
-                                      int G, int mc, float* dots) const {
+                                      int G, int mc, float* dots, float*) const {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int sub = lane / LPR, li = lane % LPR;
     const int h0 = GS::head0(li);
@@ -370,9 +382,86 @@ __device__ void find_digit(const uint32_t* hw, int r, int* scratch, int* res) {
   __syncthreads();
 }
 
-// count one key into a packed histogram word of rank 0
+// count one key into a packed histogram word (local or rank 0's)
 __device__ __forceinline__ void hist_push(uint32_t* hw, uint32_t bin) {
   atomicAdd(hw + (bin >> 1), 1u << ((bin & 1u) << 4));
+}
+
+// Rank 0: the candidates are every CTA's keys of first-digit bin b1, CTA w's
+// in cand[w * kCandCap ..] in slot order, cnt[2w] of them, with cnt[2w + 1]
+// of its keys above the bin.  Finds the r-th largest candidate T (two
+// 10-bit digits over local histograms) and writes fin = {0, T, then per CTA
+// (output offset, keys equal to T it takes)}: keys equal to T are taken in
+// CTA order, then slot order ("lower index wins").  fin[0] = 1 (nothing else
+// written) when a CTA had more than kCandCap candidates.  Whole CTA.
+__device__ void rank_candidates(const uint2* cand, int CL, uint32_t b1, int r, uint32_t* hist,
+                                int* scratch, int* dig, const int* cnt, int* fin) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ int s_over;
+  __shared__ int s_ge[kMaxCluster][2];
+  if (tid == 0) s_over = 0;
+  __syncthreads();
+  if (tid < CL && cnt[2 * tid] > kCandCap) s_over = 1;
+  __syncthreads();
+  if (s_over) {
+    if (tid == 0) fin[0] = 1;
+    __syncthreads();
+    return;
+  }
+  uint32_t* h2 = hist + kH2;
+  uint32_t* h3 = hist + kH3;
+  for (int i = tid; i < kBins2; i += kThreads) h2[i] = 0u;  // both packed halves (h2, h3)
+  __syncthreads();
+  for (int w = warp; w < CL; w += kWarps)
+    for (int j = lane; j < cnt[2 * w]; j += 32) hist_push(h2, (cand[w * kCandCap + j].x >> 10) & 1023u);
+  __syncthreads();
+  find_digit<kBins2>(h2, r, scratch, dig);
+  const uint32_t p2 = (b1 << 10) | (uint32_t)dig[0];
+  r -= dig[1];
+  for (int w = warp; w < CL; w += kWarps)
+    for (int j = lane; j < cnt[2 * w]; j += 32) {
+      const uint32_t key = cand[w * kCandCap + j].x;
+      if ((key >> 10) == p2) hist_push(h3, key & 1023u);
+    }
+  __syncthreads();
+  find_digit<kBins2>(h3, r, scratch, dig);
+  const uint32_t T = (p2 << 10) | (uint32_t)dig[0];
+  r -= dig[1];  // keys equal to T to take, in order
+  for (int w = warp; w < CL; w += kWarps) {
+    int gt = 0, eq = 0;
+    for (int j = lane; j < cnt[2 * w]; j += 32) {
+      const uint32_t key = cand[w * kCandCap + j].x;
+      gt += key > T;
+      eq += key == T;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      gt += __shfl_xor_sync(0xffffffffu, gt, o);
+      eq += __shfl_xor_sync(0xffffffffu, eq, o);
+    }
+    if (lane == 0) {
+      s_ge[w][0] = gt;
+      s_ge[w][1] = eq;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int gt = lane < CL ? cnt[2 * lane + 1] + s_ge[lane][0] : 0;
+    const int eq = lane < CL ? s_ge[lane][1] : 0;
+    const int ebefore = warp_incl_scan(eq) - eq;
+    const int take = min(max(r - ebefore, 0), eq);
+    const int nsel = gt + take;
+    const int before = warp_incl_scan(nsel) - nsel;
+    if (lane < CL) {
+      fin[2 + 2 * lane] = before;
+      fin[3 + 2 * lane] = take;
+    }
+    if (lane == 0) {
+      fin[0] = 0;
+      fin[1] = (int)T;
+    }
+  }
+  __syncthreads();
 }
 
 // the stage ring, which also holds the warps' value partials at the end
@@ -397,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
   int* spos = reinterpret_cast<int*>(hist + kHistWords);              // [mc]
   uint32_t* keys = reinterpret_cast<uint32_t*>(spos + a.mc);          // [mc]
   float* dots = reinterpret_cast<float*>(keys + a.mc);                // [GP][mc]
-  float* pw = dots + GP * a.mc;                                       // [mc][GP] weights
+  float* pw = dots + GP * a.mc;  // [GP][mc] second half-sums of the logits, then [mc][GP] weights
   int* sel = reinterpret_cast<int*>(pw + GP * a.mc);                  // [mc]
   // partials of this CTA's outputs from every CTA: o [CL][per], (m, l) [CL][2 GP]
   float* recv = reinterpret_cast<float*>(sel + a.mc);
@@ -405,7 +494,9 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
   __shared__ int scratch[33];
   __shared__ int s_dig[3];
   __shared__ int s_cnt[2];        // this CTA's keys above / at the threshold prefix
-  __shared__ int s_mine[2];       // output offset, keys at the prefix taken
+  __shared__ int s_mine[4];       // output offset, keys at the prefix taken (+ scratch)
+  __shared__ int s_cand[2 * kMaxCluster];      // rank 0: per CTA, candidates and keys above
+  __shared__ int s_fin[2 + 2 * kMaxCluster];   // rank 0: mode, T, per CTA (offset, share)
   __shared__ int s_wa[kWarps], s_wb[kWarps];
   __shared__ float s_red[kWarps][GP];
   __shared__ __align__(16) float part[PART];  // this CTA's partial o, m, l
@@ -477,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
     typename ScorePick<T, D, GP>::type sc;
     sc.init(qrow, a.G);
     kst.run([&](int r0, const unsigned char* buf, int nrows) {
-      sc.run(buf, r0, nrows, spos, a.G, a.mc, dots);
+      sc.run(buf, r0, nrows, spos, a.G, a.mc, dots, pw);
     });
   }
   // the next layer's key rows at the same pool positions into L2, while
@@ -496,19 +587,30 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
   cluster_wait();
 
   // ---- 2. selection keys; their first digit into the cluster histogram
+  constexpr bool kSplit = ScorePick<T, D, GP>::type::kSplit;  // second half-sums in pw
   for (int i = tid; i < m; i += kThreads) {
     float best = -INFINITY;
 #pragma unroll
-    for (int g = 0; g < GP; ++g)
-      if (g < a.G) best = fmaxf(best, dots[g * a.mc + i]);
+    for (int g = 0; g < GP; ++g) {
+      if (g < a.G) {
+        float v = dots[g * a.mc + i];
+        if (kSplit) dots[g * a.mc + i] = v = v + pw[g * a.mc + i];
+        best = fmaxf(best, v);
+      }
+    }
     const uint32_t key = ord_key(best);
     keys[i] = key;
     if (!all) hist_push(h0 + kH1, key >> 20);
   }
 
-  // ---- 3. threshold prefix P: keys with (key >> shift) > P are taken, and
-  // the first rtie keys with (key >> shift) == P in pool-slot order.  Rank 0
-  // resolves each digit from its own histograms; the others read the answer.
+  // ---- 3. threshold: keys with (key >> shift) > P are taken, and the first
+  // rtie keys with (key >> shift) == P in pool-slot order.  Rank 0 finds the
+  // first digit's bin from the cluster histogram.  Each CTA then hands rank 0
+  // its keys in that bin (in slot order) and its count above the bin; rank 0
+  // ranks those candidates exactly and returns every CTA's output offset and
+  // share of the keys equal to the threshold T (then P = T, shift = 0).  When
+  // a CTA has more than kCandCap candidates, the digits are resolved over the
+  // whole cluster instead (remote histograms, one digit per round).
   uint32_t P = 0u;
   int shift = 0, rtie = 0;
   if (!all) {
@@ -525,61 +627,117 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
     };
     int r = k;
     resolve(hist + kH1, kBins1, r);
-    P = (uint32_t)s_dig[0];
-    shift = 20;
+    const uint32_t b1 = (uint32_t)s_dig[0];
+    const int c1 = s_dig[2];
     r -= s_dig[1];
-    if (r < s_dig[2]) {  // part of the bin: the second digit of its keys
-      for (int i = tid; i < m; i += kThreads) {
-        const uint32_t key = keys[i];
-        if ((key >> 20) == P) hist_push(h0 + kH2, (key >> 10) & 1023u);
-      }
-      resolve(hist + kH2, kBins2, r);
-      P = (P << 10) | (uint32_t)s_dig[0];
-      shift = 10;
-      r -= s_dig[1];
-      if (r < s_dig[2]) {  // the last digit
-        for (int i = tid; i < m; i += kThreads) {
-          const uint32_t key = keys[i];
-          if ((key >> 10) == P) hist_push(h0 + kH3, key & 1023u);
+    {
+      uint2* region = reinterpret_cast<uint2*>(cluster.map_shared_rank(ring, 0)) + rank * kCandCap;
+      int base = 0, gt1 = 0;
+      for (int i0 = 0; i0 < m; i0 += kThreads) {  // CTA-uniform trip count
+        const int i = i0 + tid;
+        const uint32_t key = i < m ? keys[i] : 0u;
+        const bool cand = i < m && (key >> 20) == b1;
+        gt1 += i < m && (key >> 20) > b1;
+        const unsigned bal = __ballot_sync(0xffffffffu, cand);
+        if (lane == 0) s_wa[warp] = __popc(bal);
+        __syncthreads();
+        int before = base, tot = base;
+        for (int w = 0; w < kWarps; ++w) {
+          if (w < warp) before += s_wa[w];
+          tot += s_wa[w];
         }
-        resolve(hist + kH3, kBins2, r);
-        P = (P << 10) | (uint32_t)s_dig[0];
-        shift = 0;
-        r -= s_dig[1];
+        if (cand) {
+          const int o = before + __popc(bal & lt);
+          if (o < kCandCap) region[o] = make_uint2(key, (uint32_t)i);
+        }
+        base = tot;
+        __syncthreads();
+      }
+      int gtot;
+      block_excl_scan(gt1, scratch, &gtot);
+      if (tid == 0) {
+        int* cm = cluster.map_shared_rank(s_cand, 0);
+        cm[2 * rank] = base;
+        cm[2 * rank + 1] = gtot;
       }
     }
-    rtie = r;
-    // this CTA's counts above and at P, then every CTA's, in rank order
-    int gt = 0, eq = 0;
-    for (int i = tid; i < m; i += kThreads) {
-      const uint32_t pre = keys[i] >> shift;
-      gt += pre > P;
-      eq += pre == P;
-    }
-    int tot;
-    block_excl_scan((gt << 16) | eq, scratch, &tot);  // both counts <= 65535
-    if (tid == 0) {
-      s_cnt[0] = tot >> 16;
-      s_cnt[1] = tot & 0xFFFF;
-    }
-    cluster.sync();  // S4: every CTA's counts are published
-    if (warp == 0) {
-      int g_s = 0, e_s = 0;
-      if (lane < CL) {
-        const int* rc = cluster.map_shared_rank(s_cnt, lane);
-        g_s = rc[0];
-        e_s = rc[1];
-      }
-      const int ebefore = warp_incl_scan(e_s) - e_s;
-      const int take = min(max(rtie - ebefore, 0), e_s);
-      const int nsel_s = g_s + take;
-      const int before = warp_incl_scan(nsel_s) - nsel_s;
-      if (lane == rank) {
-        s_mine[0] = before;
-        s_mine[1] = take;
-      }
+    cluster.sync();  // S2: every slice's candidates and count are with rank 0
+    if (rank == 0) rank_candidates(reinterpret_cast<const uint2*>(ring), CL, b1, r, hist, scratch, s_dig, s_cand, s_fin);
+    cluster.sync();  // S2b: rank 0's answer is ready
+    if (tid < 3) {
+      const int* f = cluster.map_shared_rank(s_fin, 0);
+      s_mine[tid] = tid == 0 ? f[0] : tid == 1 ? f[1] : f[2 + 2 * rank];
+      if (tid == 2) s_mine[3] = f[3 + 2 * rank];
     }
     __syncthreads();
+    const int ranked = s_mine[0] == 0;
+    const uint32_t T = (uint32_t)s_mine[1];
+    const int off_T = s_mine[2], take_T = s_mine[3];
+    __syncthreads();
+    if (ranked) {  // threshold T with this CTA's offset and share of keys equal to T
+      P = T;
+      shift = 0;
+      if (tid == 0) {
+        s_mine[0] = off_T;
+        s_mine[1] = take_T;
+      }
+      __syncthreads();
+    } else {
+      P = b1;
+      shift = 20;
+      if (r < c1) {  // part of the bin: the second digit of its keys
+        for (int i = tid; i < m; i += kThreads) {
+          const uint32_t key = keys[i];
+          if ((key >> 20) == P) hist_push(h0 + kH2, (key >> 10) & 1023u);
+        }
+        resolve(hist + kH2, kBins2, r);
+        P = (P << 10) | (uint32_t)s_dig[0];
+        shift = 10;
+        r -= s_dig[1];
+        if (r < s_dig[2]) {  // the last digit
+          for (int i = tid; i < m; i += kThreads) {
+            const uint32_t key = keys[i];
+            if ((key >> 10) == P) hist_push(h0 + kH3, key & 1023u);
+          }
+          resolve(hist + kH3, kBins2, r);
+          P = (P << 10) | (uint32_t)s_dig[0];
+          shift = 0;
+          r -= s_dig[1];
+        }
+      }
+      rtie = r;
+      // this CTA's counts above and at P, then every CTA's, in rank order
+      int gt = 0, eq = 0;
+      for (int i = tid; i < m; i += kThreads) {
+        const uint32_t pre = keys[i] >> shift;
+        gt += pre > P;
+        eq += pre == P;
+      }
+      int tot;
+      block_excl_scan((gt << 16) | eq, scratch, &tot);  // both counts <= 65535
+      if (tid == 0) {
+        s_cnt[0] = tot >> 16;
+        s_cnt[1] = tot & 0xFFFF;
+      }
+      cluster.sync();  // S4: every CTA's counts are published
+      if (warp == 0) {
+        int g_s = 0, e_s = 0;
+        if (lane < CL) {
+          const int* rc = cluster.map_shared_rank(s_cnt, lane);
+          g_s = rc[0];
+          e_s = rc[1];
+        }
+        const int ebefore = warp_incl_scan(e_s) - e_s;
+        const int take = min(max(rtie - ebefore, 0), e_s);
+        const int nsel_s = g_s + take;
+        const int before = warp_incl_scan(nsel_s) - nsel_s;
+        if (lane == rank) {
+          s_mine[0] = before;
+          s_mine[1] = take;
+        }
+      }
+      __syncthreads();
+    }
   }
 
   // ---- 4. selected members of the slice, positions to idx (ascending)

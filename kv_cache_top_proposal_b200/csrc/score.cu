@@ -429,6 +429,16 @@ __global__ void __launch_bounds__(kThreads, 3) score_tma_kernel(const __grid_con
   float unscale = 1.0f;
   int cur_b = -1, cur_h = -1;
   int hist_row = -1, since_flush = 0;
+  // this thread's key-row scale, loaded one stage ahead (row g of tile warp
+  // for tig 0, row g + 8 for tig 1)
+  const int rs = warp * 16 + g + 8 * tig;
+  auto load_scale = [&](const StageIter& it) {
+    if (tig >= 2 || it.h >= a.Hkv) return 0.0f;
+    const int L = s_cu[it.b + 1] - s_cu[it.b];
+    if (rs >= min(kStageRows, L - it.r0)) return 0.0f;
+    return __ldg(a.scale + (int64_t)it.h * a.T + s_cu[it.b] + it.r0 + rs);
+  };
+  float sc_next = nk > 0 ? load_scale(it_comp) : 0.0f;
   auto flush = [&]() {  // packed shared histogram -> global (non-zero bins), then clear
     if (a.hist && hist_row >= 0) {
       uint32_t* gh = a.hist + (int64_t)hist_row * kHist;
@@ -499,6 +509,8 @@ __global__ void __launch_bounds__(kThreads, 3) score_tma_kernel(const __grid_con
     }
     ++since_flush;
     it_comp.advance(s_cu, a.B);
+    const float sc = sc_next;
+    if (kk + 1 < nk) sc_next = load_scale(it_comp);
     const int slot = kk % kTmaStages;
     {
       uint32_t it = 0;
@@ -512,9 +524,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_tma_kernel(const __grid_con
     const unsigned char* buf = ring + slot * kTmaStageBytes;
     const int t = warp;  // one 16-row tile per warp
     if (t * 16 < rows) {
-      const int rs = t * 16 + g + 8 * tig;  // tig 0: row g, tig 1: row g + 8
-      const bool mine = tig < 2 && rs < rows;
-      const float sc = mine ? __ldg(a.scale + rowbase + rs) : 0.0f;
+      const bool mine = tig < 2 && rs < rows;  // tig 0: row g, tig 1: row g + 8
       uint4 cur[2][2];
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -642,10 +652,10 @@ cudaError_t run_mma(const Dims& d, const ScoreArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// PRISM_PROPOSE_SCORER=tma selects the tensor-copy scorer
+// PRISM_PROPOSE_SCORER=mma selects the cp.async tensor-core scorer instead
 bool use_tma_scorer() {
   const char* e = std::getenv("PRISM_PROPOSE_SCORER");
-  return e && std::strcmp(e, "tma") == 0;
+  return !(e && std::strcmp(e, "mma") == 0);
 }
 
 // cuTensorMapEncodeTiled from the driver, looked up once

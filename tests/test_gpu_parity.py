@@ -103,15 +103,16 @@ PROPOSE_CASES = [
 @pytest.mark.parametrize("case", PROPOSE_CASES, ids=lambda c: f"{c[0]}-{c[1]}/{c[2]}-d{c[3]}-{c[4]}-kp{c[5]}")
 @pytest.mark.parametrize("scorer", ["tma", "mma", "simt"])
 def test_propose_vs_oracle(P, case, scorer, monkeypatch):
-    """mma: the default tensor-core scorer (cp.async stages); tma: the
-    tensor-core scorer fed by tensor copies (d = 128); simt: CUDA cores."""
+    """tma: the default tensor-core scorer, fed by tensor copies (d = 128;
+    d = 64 takes the cp.async one); mma: the cp.async tensor-core scorer;
+    simt: CUDA cores."""
     seqlens, hq, hkv, d, dtype, kp = case
     if scorer == "simt":
         monkeypatch.setenv("PRISM_PROPOSE_SCORER", "simt")
     elif dtype != "bf16":
         pytest.skip("the tensor-core scorers take bf16 queries")
-    elif scorer == "tma":
-        monkeypatch.setenv("PRISM_PROPOSE_SCORER", "tma")
+    elif scorer == "mma":
+        monkeypatch.setenv("PRISM_PROPOSE_SCORER", "mma")
     prob = problem(P, seqlens, hq, hkv, d, dtype)
     q, k, _ = make_case(seqlens, hq, hkv, d, dtype, seed=2)
     T = prob.total_tokens
@@ -140,8 +141,12 @@ def test_propose_vs_oracle(P, case, scorer, monkeypatch):
             assert np.all(gp[b, h, n:] == -1)
 
 
-def test_propose_all_ties_lower_index_wins(P):
-    seqlens, hq, hkv, d, kp = [3000, 500], 8, 2, 128, 1000
+@pytest.mark.parametrize("L0,kp", [(3000, 1000), (60000, 8192)], ids=["small", "many-candidates"])
+def test_propose_all_ties_lower_index_wins(P, L0, kp):
+    """Equal scores: the lowest positions win.  At 60000 positions every CTA of
+    the selection holds more first-digit candidates than rank 0 ranks, so the
+    cluster-wide digit rounds run."""
+    seqlens, hq, hkv, d = [L0, 500], 8, 2, 128
     prob = problem(P, seqlens, hq, hkv, d, "bf16")
     q, k, _ = make_case(seqlens, hq, hkv, d, "bf16", seed=3)
     k[:] = k[:, :1]  # every key row identical -> every score equal
@@ -510,3 +515,28 @@ def test_refine_decode_overlapped_launches_match(P):
     for a, b in zip(res[0], res[1]):
         for x, y in zip(a, b):
             assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("kp,kap", [(8192, 2048), (8192, 8191), (3000, 1)])
+def test_refine_decode_large_ties(P, kp, kap):
+    """All scores equal over pools big enough that every CTA holds more
+    first-digit candidates than the ranking buffer: the lowest pool slots win
+    on every path, and the attention matches the oracle on that set."""
+    seqlens, hq, hkv, d = [40000], 8, 2, 128
+    prob = problem(P, seqlens, hq, hkv, d, "bf16")
+    q, k, v = make_case(seqlens, hq, hkv, d, "bf16", seed=23)
+    k[:, :] = k[:, :1]
+    pool = torch.arange(0, 4 * kp, 4, dtype=torch.int32, device=DEV).repeat(1, hkv, 1)
+    cnt_p = torch.full((1, hkv), kp, dtype=torch.int32, device=DEV)
+    idx = torch.zeros((1, hkv, kap), dtype=torch.int32, device=DEV)
+    cnt = torch.zeros((1, hkv), dtype=torch.int32, device=DEV)
+    out = torch.zeros((1, hq, d), device=DEV)
+    ws = ws_for(P, prob, P.OP_REFINE_DECODE, kp, kap)
+    P.refine_decode(prob, q, k, v, pool, cnt_p, kp, kap, 0.1, idx, cnt, out, ws)
+    torch.cuda.synchronize()
+    assert P.get_device_status(ws) == 0
+    for h in range(hkv):
+        assert int(_np(cnt)[0, h]) == kap
+        assert np.array_equal(_np(idx)[0, h], np.arange(0, 4 * kap, 4))
+    oout, _ = pipeline.attend_layer(q, k, v, [0, 40000], _np(idx), _np(cnt), 0.1)
+    assert np.abs(_np(out) - oout).max() <= 2e-3
