@@ -29,14 +29,14 @@ namespace prism {
 
 namespace {
 
-constexpr int kCL = 8;
-constexpr int kThreads = 1024;
+constexpr int kCL = 16;                       // CTAs per row (a non-portable cluster size)
+constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kKPT = 16;                      // keys per thread
 constexpr int kMaxSlice = kKPT * kThreads;    // keys per CTA
 constexpr int kHist = 4096;                   // first digit (from the scorer)
 constexpr int kBins = 1024;                   // second and third digits
-constexpr int kCandCap = 2048;                // first-digit candidates per CTA ranked by rank 0
+constexpr int kCandCap = 512;                 // first-digit candidates per CTA ranked by rank 0
 
 struct PSArgs {
   const float* scores;   // [Hkv][T]
@@ -176,7 +176,7 @@ __device__ void rank_candidates(const uint2* cand, uint32_t b1, int r, uint32_t*
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kThreads, 1) propose_select_kernel(const PSArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArgs a) {
   extern __shared__ __align__(16) uint2 cand[];      // rank 0: [kCL][kCandCap] (key, position)
   __shared__ __align__(16) uint32_t hist2[kBins];  // rank 0: digit-2 counts
   __shared__ __align__(16) uint32_t hist3[kBins];  // rank 0: digit-3 counts
@@ -218,8 +218,10 @@ __global__ void __launch_bounds__(kThreads, 1) propose_select_kernel(const PSArg
   uint32_t* h2 = cluster.map_shared_rank(hist2, 0);
   uint32_t* h3 = cluster.map_shared_rank(hist3, 0);
   if (rank == 0) {
-    hist2[tid] = 0u;  // kBins == kThreads
-    hist3[tid] = 0u;
+    for (int i = tid; i < kBins; i += kThreads) {
+      hist2[i] = 0u;
+      hist3[i] = 0u;
+    }
   }
   __syncthreads();
   cluster_arrive();  // rank 0's histograms are cleared once every CTA has arrived
@@ -435,6 +437,8 @@ cudaError_t launch_propose_select(const Dims& d, const float* scores, const uint
   const int smem = kCL * kCandCap * (int)sizeof(uint2);
   cudaError_t e = cudaFuncSetAttribute(propose_select_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(propose_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e != cudaSuccess) return e;
   cfg.dynamicSmemBytes = (size_t)smem;
   cfg.stream = st;

@@ -19,10 +19,10 @@
 //      (remote shared-memory atomics, two 16-bit counts per word);
 //   3. rank 0 finds the bin of that histogram holding the kappa-th largest
 //      key and every CTA reads the answer.  Unless the whole bin is taken,
-//      the keys in it build a histogram of the next 10 bits, and then of the
-//      last 10: this gives the threshold prefix P (12, 22 or 32 bits) and how
-//      many keys at P are taken.  Keys at P are taken in pool-slot order
-//      ("lower index wins");
+//      the keys in it build a histogram of the next 10 bits in rank 0, and
+//      then of the last 10: this gives the threshold prefix P (12, 22 or 32
+//      bits) and how many keys at P are taken.  Keys at P are taken in
+//      pool-slot order ("lower index wins");
 //   4. the CTAs exchange their counts above and at P, which gives each one
 //      its share of the keys at P and its output offset; it writes its
 //      selected positions to idx in ascending order;
@@ -35,6 +35,8 @@
 // Nothing goes to global scratch.  Bytes per row: kappa_p key rows and kappa
 // value rows, d * sizeof(T) each.
 #include <cooperative_groups.h>
+
+#include <cstdlib>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -59,7 +61,6 @@ constexpr int kH3 = kH2 + kBins2 / 2;
 constexpr int kHistWords = kH3 + kBins2 / 2;
 constexpr int kMaxCount = 65535;  // largest pool a 16-bit bin count can hold
 constexpr int kMaxCluster = 16;
-constexpr int kCandCap = 256;     // first-digit candidates per CTA ranked by rank 0 (8 B each)
 
 struct RDArgs {
   const void* q;
@@ -382,87 +383,11 @@ __device__ void find_digit(const uint32_t* hw, int r, int* scratch, int* res) {
   __syncthreads();
 }
 
-// count one key into a packed histogram word (local or rank 0's)
+// count one key into a packed histogram word of rank 0
 __device__ __forceinline__ void hist_push(uint32_t* hw, uint32_t bin) {
   atomicAdd(hw + (bin >> 1), 1u << ((bin & 1u) << 4));
 }
 
-// Rank 0: the candidates are every CTA's keys of first-digit bin b1, CTA w's
-// in cand[w * kCandCap ..] in slot order, cnt[2w] of them, with cnt[2w + 1]
-// of its keys above the bin.  Finds the r-th largest candidate T (two
-// 10-bit digits over local histograms) and writes fin = {0, T, then per CTA
-// (output offset, keys equal to T it takes)}: keys equal to T are taken in
-// CTA order, then slot order ("lower index wins").  fin[0] = 1 (nothing else
-// written) when a CTA had more than kCandCap candidates.  Whole CTA.
-__device__ void rank_candidates(const uint2* cand, int CL, uint32_t b1, int r, uint32_t* hist,
-                                int* scratch, int* dig, const int* cnt, int* fin) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  __shared__ int s_over;
-  __shared__ int s_ge[kMaxCluster][2];
-  if (tid == 0) s_over = 0;
-  __syncthreads();
-  if (tid < CL && cnt[2 * tid] > kCandCap) s_over = 1;
-  __syncthreads();
-  if (s_over) {
-    if (tid == 0) fin[0] = 1;
-    __syncthreads();
-    return;
-  }
-  uint32_t* h2 = hist + kH2;
-  uint32_t* h3 = hist + kH3;
-  for (int i = tid; i < kBins2; i += kThreads) h2[i] = 0u;  // both packed halves (h2, h3)
-  __syncthreads();
-  for (int w = warp; w < CL; w += kWarps)
-    for (int j = lane; j < cnt[2 * w]; j += 32) hist_push(h2, (cand[w * kCandCap + j].x >> 10) & 1023u);
-  __syncthreads();
-  find_digit<kBins2>(h2, r, scratch, dig);
-  const uint32_t p2 = (b1 << 10) | (uint32_t)dig[0];
-  r -= dig[1];
-  for (int w = warp; w < CL; w += kWarps)
-    for (int j = lane; j < cnt[2 * w]; j += 32) {
-      const uint32_t key = cand[w * kCandCap + j].x;
-      if ((key >> 10) == p2) hist_push(h3, key & 1023u);
-    }
-  __syncthreads();
-  find_digit<kBins2>(h3, r, scratch, dig);
-  const uint32_t T = (p2 << 10) | (uint32_t)dig[0];
-  r -= dig[1];  // keys equal to T to take, in order
-  for (int w = warp; w < CL; w += kWarps) {
-    int gt = 0, eq = 0;
-    for (int j = lane; j < cnt[2 * w]; j += 32) {
-      const uint32_t key = cand[w * kCandCap + j].x;
-      gt += key > T;
-      eq += key == T;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      gt += __shfl_xor_sync(0xffffffffu, gt, o);
-      eq += __shfl_xor_sync(0xffffffffu, eq, o);
-    }
-    if (lane == 0) {
-      s_ge[w][0] = gt;
-      s_ge[w][1] = eq;
-    }
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const int gt = lane < CL ? cnt[2 * lane + 1] + s_ge[lane][0] : 0;
-    const int eq = lane < CL ? s_ge[lane][1] : 0;
-    const int ebefore = warp_incl_scan(eq) - eq;
-    const int take = min(max(r - ebefore, 0), eq);
-    const int nsel = gt + take;
-    const int before = warp_incl_scan(nsel) - nsel;
-    if (lane < CL) {
-      fin[2 + 2 * lane] = before;
-      fin[3 + 2 * lane] = take;
-    }
-    if (lane == 0) {
-      fin[0] = 0;
-      fin[1] = (int)T;
-    }
-  }
-  __syncthreads();
-}
 
 // the stage ring, which also holds the warps' value partials at the end
 template <typename T, int D, int GP>
@@ -494,9 +419,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
   __shared__ int scratch[33];
   __shared__ int s_dig[3];
   __shared__ int s_cnt[2];        // this CTA's keys above / at the threshold prefix
-  __shared__ int s_mine[4];       // output offset, keys at the prefix taken (+ scratch)
-  __shared__ int s_cand[2 * kMaxCluster];      // rank 0: per CTA, candidates and keys above
-  __shared__ int s_fin[2 + 2 * kMaxCluster];   // rank 0: mode, T, per CTA (offset, share)
+  __shared__ int s_mine[2];       // output offset, keys at the prefix taken
   __shared__ int s_wa[kWarps], s_wb[kWarps];
   __shared__ float s_red[kWarps][GP];
   __shared__ __align__(16) float part[PART];  // this CTA's partial o, m, l
@@ -603,14 +526,9 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
     if (!all) hist_push(h0 + kH1, key >> 20);
   }
 
-  // ---- 3. threshold: keys with (key >> shift) > P are taken, and the first
-  // rtie keys with (key >> shift) == P in pool-slot order.  Rank 0 finds the
-  // first digit's bin from the cluster histogram.  Each CTA then hands rank 0
-  // its keys in that bin (in slot order) and its count above the bin; rank 0
-  // ranks those candidates exactly and returns every CTA's output offset and
-  // share of the keys equal to the threshold T (then P = T, shift = 0).  When
-  // a CTA has more than kCandCap candidates, the digits are resolved over the
-  // whole cluster instead (remote histograms, one digit per round).
+  // ---- 3. threshold prefix P: keys with (key >> shift) > P are taken, and
+  // the first rtie keys with (key >> shift) == P in pool-slot order.  Rank 0
+  // resolves each digit from its own histograms; the others read the answer.
   uint32_t P = 0u;
   int shift = 0, rtie = 0;
   if (!all) {
@@ -627,117 +545,61 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
     };
     int r = k;
     resolve(hist + kH1, kBins1, r);
-    const uint32_t b1 = (uint32_t)s_dig[0];
-    const int c1 = s_dig[2];
+    P = (uint32_t)s_dig[0];
+    shift = 20;
     r -= s_dig[1];
-    {
-      uint2* region = reinterpret_cast<uint2*>(cluster.map_shared_rank(ring, 0)) + rank * kCandCap;
-      int base = 0, gt1 = 0;
-      for (int i0 = 0; i0 < m; i0 += kThreads) {  // CTA-uniform trip count
-        const int i = i0 + tid;
-        const uint32_t key = i < m ? keys[i] : 0u;
-        const bool cand = i < m && (key >> 20) == b1;
-        gt1 += i < m && (key >> 20) > b1;
-        const unsigned bal = __ballot_sync(0xffffffffu, cand);
-        if (lane == 0) s_wa[warp] = __popc(bal);
-        __syncthreads();
-        int before = base, tot = base;
-        for (int w = 0; w < kWarps; ++w) {
-          if (w < warp) before += s_wa[w];
-          tot += s_wa[w];
-        }
-        if (cand) {
-          const int o = before + __popc(bal & lt);
-          if (o < kCandCap) region[o] = make_uint2(key, (uint32_t)i);
-        }
-        base = tot;
-        __syncthreads();
+    if (r < s_dig[2]) {  // part of the bin: the second digit of its keys
+      for (int i = tid; i < m; i += kThreads) {
+        const uint32_t key = keys[i];
+        if ((key >> 20) == P) hist_push(h0 + kH2, (key >> 10) & 1023u);
       }
-      int gtot;
-      block_excl_scan(gt1, scratch, &gtot);
-      if (tid == 0) {
-        int* cm = cluster.map_shared_rank(s_cand, 0);
-        cm[2 * rank] = base;
-        cm[2 * rank + 1] = gtot;
-      }
-    }
-    cluster.sync();  // S2: every slice's candidates and count are with rank 0
-    if (rank == 0) rank_candidates(reinterpret_cast<const uint2*>(ring), CL, b1, r, hist, scratch, s_dig, s_cand, s_fin);
-    cluster.sync();  // S2b: rank 0's answer is ready
-    if (tid < 3) {
-      const int* f = cluster.map_shared_rank(s_fin, 0);
-      s_mine[tid] = tid == 0 ? f[0] : tid == 1 ? f[1] : f[2 + 2 * rank];
-      if (tid == 2) s_mine[3] = f[3 + 2 * rank];
-    }
-    __syncthreads();
-    const int ranked = s_mine[0] == 0;
-    const uint32_t T = (uint32_t)s_mine[1];
-    const int off_T = s_mine[2], take_T = s_mine[3];
-    __syncthreads();
-    if (ranked) {  // threshold T with this CTA's offset and share of keys equal to T
-      P = T;
-      shift = 0;
-      if (tid == 0) {
-        s_mine[0] = off_T;
-        s_mine[1] = take_T;
-      }
-      __syncthreads();
-    } else {
-      P = b1;
-      shift = 20;
-      if (r < c1) {  // part of the bin: the second digit of its keys
+      resolve(hist + kH2, kBins2, r);
+      P = (P << 10) | (uint32_t)s_dig[0];
+      shift = 10;
+      r -= s_dig[1];
+      if (r < s_dig[2]) {  // the last digit
         for (int i = tid; i < m; i += kThreads) {
           const uint32_t key = keys[i];
-          if ((key >> 20) == P) hist_push(h0 + kH2, (key >> 10) & 1023u);
+          if ((key >> 10) == P) hist_push(h0 + kH3, key & 1023u);
         }
-        resolve(hist + kH2, kBins2, r);
+        resolve(hist + kH3, kBins2, r);
         P = (P << 10) | (uint32_t)s_dig[0];
-        shift = 10;
+        shift = 0;
         r -= s_dig[1];
-        if (r < s_dig[2]) {  // the last digit
-          for (int i = tid; i < m; i += kThreads) {
-            const uint32_t key = keys[i];
-            if ((key >> 10) == P) hist_push(h0 + kH3, key & 1023u);
-          }
-          resolve(hist + kH3, kBins2, r);
-          P = (P << 10) | (uint32_t)s_dig[0];
-          shift = 0;
-          r -= s_dig[1];
-        }
       }
-      rtie = r;
-      // this CTA's counts above and at P, then every CTA's, in rank order
-      int gt = 0, eq = 0;
-      for (int i = tid; i < m; i += kThreads) {
-        const uint32_t pre = keys[i] >> shift;
-        gt += pre > P;
-        eq += pre == P;
-      }
-      int tot;
-      block_excl_scan((gt << 16) | eq, scratch, &tot);  // both counts <= 65535
-      if (tid == 0) {
-        s_cnt[0] = tot >> 16;
-        s_cnt[1] = tot & 0xFFFF;
-      }
-      cluster.sync();  // S4: every CTA's counts are published
-      if (warp == 0) {
-        int g_s = 0, e_s = 0;
-        if (lane < CL) {
-          const int* rc = cluster.map_shared_rank(s_cnt, lane);
-          g_s = rc[0];
-          e_s = rc[1];
-        }
-        const int ebefore = warp_incl_scan(e_s) - e_s;
-        const int take = min(max(rtie - ebefore, 0), e_s);
-        const int nsel_s = g_s + take;
-        const int before = warp_incl_scan(nsel_s) - nsel_s;
-        if (lane == rank) {
-          s_mine[0] = before;
-          s_mine[1] = take;
-        }
-      }
-      __syncthreads();
     }
+    rtie = r;
+    // this CTA's counts above and at P, then every CTA's, in rank order
+    int gt = 0, eq = 0;
+    for (int i = tid; i < m; i += kThreads) {
+      const uint32_t pre = keys[i] >> shift;
+      gt += pre > P;
+      eq += pre == P;
+    }
+    int tot;
+    block_excl_scan((gt << 16) | eq, scratch, &tot);  // both counts <= 65535
+    if (tid == 0) {
+      s_cnt[0] = tot >> 16;
+      s_cnt[1] = tot & 0xFFFF;
+    }
+    cluster.sync();  // S4: every CTA's counts are published
+    if (warp == 0) {
+      int g_s = 0, e_s = 0;
+      if (lane < CL) {
+        const int* rc = cluster.map_shared_rank(s_cnt, lane);
+        g_s = rc[0];
+        e_s = rc[1];
+      }
+      const int ebefore = warp_incl_scan(e_s) - e_s;
+      const int take = min(max(rtie - ebefore, 0), e_s);
+      const int nsel_s = g_s + take;
+      const int before = warp_incl_scan(nsel_s) - nsel_s;
+      if (lane == rank) {
+        s_mine[0] = before;
+        s_mine[1] = take;
+      }
+    }
+    __syncthreads();
   }
 
   // ---- 4. selected members of the slice, positions to idx (ascending)
@@ -955,11 +817,20 @@ constexpr int recv_bytes(int GP, int D) { return (GP * D + kMaxCluster + 2 * GP 
 constexpr int kDynBudget = 227 * 1024 - 8 * 1024;
 constexpr int kPairBudget = 110 * 1024;
 
+// PRISM_RD_CLUSTER=c (1..16) forces the cluster size; PRISM_RD_SOLO=1 pads
+// the shared memory request so that one CTA holds an SM.
+int env_int(const char* name, int dflt) {
+  const char* e = std::getenv(name);
+  return e && *e ? std::atoi(e) : dflt;
+}
+
 template <typename T, int D, int GP>
 cudaError_t run(const Dims& d, RDArgs a, int cl, bool overlap, cudaStream_t st) {
   auto kern = refine_decode_kernel<T, D, GP>;
-  const int smem = ring_bytes<T, D, GP>() + kHistWords * 4 + a.mc * per_member_bytes<GP>() +
-                   recv_bytes(GP, D);
+  int smem = ring_bytes<T, D, GP>() + kHistWords * 4 + a.mc * per_member_bytes<GP>() +
+             recv_bytes(GP, D);
+  static const bool solo = env_int("PRISM_RD_SOLO", 0) == 1;
+  if (solo && smem < 120 * 1024) smem = 120 * 1024;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   if (cl > 8) {
@@ -1006,6 +877,8 @@ RefineDecodePlan plan_refine_decode(const Dims& d, int kappa_p) {
   int cl = 1;
   while (cl < kMaxCluster && (int64_t)rows * cl < 2LL * d.num_sms) cl *= 2;
   while (cl < kMaxCluster && need(cl) > kPairBudget) cl *= 2;
+  static const int forced = env_int("PRISM_RD_CLUSTER", 0);
+  if (forced >= 1 && forced <= kMaxCluster && need(forced) <= kDynBudget) cl = forced;
   const bool ok = kappa_p <= kMaxCount && need(cl) <= kDynBudget;
   return RefineDecodePlan{cl, mc_of(cl), ok};
 }
