@@ -56,6 +56,14 @@ def _L():
         lib.oracle_refine_row.argtypes = [P, i32, i32, P, P, i32, i32, P, P]
         lib.oracle_refine_row.restype = i32
         lib.oracle_attend.argtypes = [P, i32, P, P, P, i32, f64, P, P]
+        lib.oracle_f32_to_f16.argtypes = [ctypes.c_float]
+        lib.oracle_f32_to_f16.restype = ctypes.c_uint16
+        lib.oracle_f16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.oracle_f16_to_f32.restype = ctypes.c_float
+        lib.oracle_quantize_int2_rows.argtypes = [P, i64, i32, P, P]
+        lib.oracle_propose_scores_int2.argtypes = [P, i32, i32, P, P, i32, P]
+        lib.oracle_propose_row_int2.argtypes = [P, i32, i32, P, P, i32, i32, P, P]
+        lib.oracle_propose_row_int2.restype = i32
         _lib = lib
     return _lib
 
@@ -144,3 +152,57 @@ def attend(q, K, V, idx, softmax_scale: float):
     lse = np.empty((1,), np.float32)
     _L().oracle_attend(_p(q), d, _p(K), _p(V), ip, n, float(softmax_scale), _p(out), _p(lse))
     return out, float(lse[0])
+
+
+# ---- INT2 proposal keys -----------------------------------------------------
+
+def f32_to_f16_bits(x: float) -> int:
+    """fp16 bits of x, round to nearest even."""
+    return int(_L().oracle_f32_to_f16(float(np.float32(x))))
+
+
+def f16_bits_to_f32(h: int) -> float:
+    return float(_L().oracle_f16_to_f32(int(h)))
+
+
+def quantize_int2_rows(k):
+    """INT2 per-group quantization -> (codes [rows, d/4] uint8 packed, params
+    [rows, d/32, 2] uint16 fp16 bits of (step S, zero point L))."""
+    k = _f32(k)
+    rows, d = k.shape
+    codes = np.empty((rows, d // 4), np.uint8)
+    params = np.empty((rows, d // 32, 2), np.uint16)
+    _L().oracle_quantize_int2_rows(_p(k), rows, d, _p(codes), _p(params))
+    return codes, params
+
+
+def unpack_int2(codes, d: int) -> np.ndarray:
+    """Packed codes [rows, d/4] -> code values [rows, d] (feature f at bits 2 (f mod 4) of byte f / 4)."""
+    codes = np.asarray(codes, np.uint8)
+    shifts = (2 * (np.arange(d) % 4)).astype(np.uint8)
+    return (codes[:, np.arange(d) // 4] >> shifts) & 3
+
+
+def propose_scores_int2(q, codes, params) -> np.ndarray:
+    """s_t = max_g sum over groups of (S * D + L * Q) (fp32, see the C source)."""
+    q = _f32(q)
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    params = np.ascontiguousarray(params, dtype=np.uint16)
+    G, d = q.shape
+    L = codes.shape[0]
+    s = np.empty((max(L, 1),), np.float32)
+    _L().oracle_propose_scores_int2(_p(q), G, d, _p(codes), _p(params), L, _p(s))
+    return s[:L].copy()
+
+
+def propose_row_int2(q, codes, params, kappa_p: int):
+    """(pool ascending int32 [min(kappa_p, L)], INT2 proposal scores [L])."""
+    q = _f32(q)
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    params = np.ascontiguousarray(params, dtype=np.uint16)
+    G, d = q.shape
+    L = codes.shape[0]
+    s = np.empty((max(L, 1),), np.float32)
+    pool = np.empty((max(min(kappa_p, L), 1),), np.int32)
+    m = _L().oracle_propose_row_int2(_p(q), G, d, _p(codes), _p(params), L, kappa_p, _p(pool), _p(s))
+    return pool[:m].copy(), s[:L].copy()

@@ -26,7 +26,7 @@ from typing import Dict, List, Optional
 
 import numpy as np
 
-from . import attend, propose_row, quantize_rows, refine_row
+from . import attend, propose_row, propose_row_int2, quantize_int2_rows, quantize_rows, refine_row
 
 
 def _np(x):
@@ -68,6 +68,37 @@ def propose_layer(q, kq, scale, cu, kappa_p: int, rows=None):
             pool[b, h, :p.size] = p
             cnt[b, h] = p.size
             scores[(b, h)] = s
+    return pool, cnt, scores
+
+
+def quantize_layer_int2(k):
+    """INT2 codes [Hkv][T][d/4] uint8 and params [Hkv][T][d/32][2] (fp16 bits)."""
+    k = _np(k).astype(np.float32)
+    Hkv, T, d = k.shape
+    codes, params = quantize_int2_rows(k.reshape(Hkv * T, d))
+    return codes.reshape(Hkv, T, d // 4), params.reshape(Hkv, T, d // 32, 2)
+
+
+def propose_layer_int2(q, codes, params, cu, kappa_p: int, rows=None):
+    """INT2 proposal: pool [B][Hkv][kappa_p] (-1 padded), pool_cnt, scores per row."""
+    q = _np(q).astype(np.float32)
+    codes, params = _np(codes), _np(params)
+    B, Hq, d = q.shape
+    Hkv = codes.shape[0]
+    G = Hq // Hkv
+    pool = np.full((B, Hkv, kappa_p), -1, np.int32)
+    cnt = np.zeros((B, Hkv), np.int32)
+    scores: Dict = {}
+    for b in range(B):
+        t0, t1 = cu[b], cu[b + 1]
+        for h in range(Hkv):
+            if rows is not None and (b, h) not in rows:
+                continue
+            p, sc = propose_row_int2(q[b, h * G:(h + 1) * G], codes[h, t0:t1],
+                                            params[h, t0:t1], kappa_p)
+            pool[b, h, :p.size] = p
+            cnt[b, h] = p.size
+            scores[(b, h)] = sc
     return pool, cnt, scores
 
 

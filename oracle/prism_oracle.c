@@ -220,3 +220,149 @@ void oracle_attend(const float* q, int32_t d, const float* K, const float* V,
   free(o);
   free(l);
 }
+
+/* ------------------------------------------------------------------------
+ * INT2 proposal keys (sec. 4.2: the pages compress the key cache read at
+ * proposal layers to INT2 for candidate scoring, without stating the
+ * scheme).  Reading used here: per (KV head, token), per group of 32
+ * consecutive features, asymmetric 2-bit codes with an fp16 zero point and
+ * an fp16 step:
+ *   lo  = min_j k_j,  hi = max_j k_j                  (group, exact in fp32)
+ *   L   = fp16(lo),   S = fp16((hi - L) / 3)          (round to nearest even)
+ *   c_j = clamp(rne((k_j - L) / S), 0, 3)             (S > 0; else c_j = 0)
+ * so the dequantized key is L + S * c_j.  Codes are packed four to a byte,
+ * feature f at bits 2 (f mod 4) of byte f / 4; (S, L) are stored as fp16
+ * bits, group by group.
+ * ------------------------------------------------------------------------ */
+
+/* fp32 -> fp16 bits, round to nearest even (IEEE 754 binary16), with
+ * overflow to infinity and gradual underflow. */
+uint16_t oracle_f32_to_f16(float f) {
+  uint32_t x;
+  memcpy(&x, &f, 4);
+  const uint32_t sign = (x >> 16) & 0x8000u;
+  const uint32_t absx = x & 0x7FFFFFFFu;
+  if (absx > 0x7F800000u) return (uint16_t)(sign | 0x7E00u);        /* NaN */
+  if (absx >= 0x47800000u) {                                         /* >= 65536: inf */
+    /* values in [65520, 65536) round to inf too; handled below */
+    return (uint16_t)(sign | 0x7C00u);
+  }
+  const int32_t e = (int32_t)(absx >> 23) - 127;                     /* unbiased exponent */
+  uint32_t mant = (absx & 0x7FFFFFu) | 0x800000u;                    /* 24-bit significand */
+  if (absx < 0x33000000u) return (uint16_t)sign;                     /* < 2^-25: rounds to 0 */
+  if (e < -14) {
+    /* subnormal half: value = mant * 2^(e-23); half ulp is 2^-24 */
+    const int shift = -14 - e + 13;                                  /* bits dropped */
+    uint32_t q = mant >> shift;
+    const uint32_t rem = mant & ((1u << shift) - 1u);
+    const uint32_t half = 1u << (shift - 1);
+    if (rem > half || (rem == half && (q & 1u))) ++q;
+    return (uint16_t)(sign | q);                                     /* q may carry into normal */
+  }
+  /* normal half: keep 11 bits of the significand */
+  uint32_t q = mant >> 13;
+  const uint32_t rem = mant & 0x1FFFu;
+  if (rem > 0x1000u || (rem == 0x1000u && (q & 1u))) ++q;
+  uint32_t he = (uint32_t)(e + 15);
+  if (q == 0x800u) {                                                 /* carry */
+    q = 0x400u;
+    ++he;
+  }
+  if (he >= 31) return (uint16_t)(sign | 0x7C00u);
+  return (uint16_t)(sign | (he << 10) | (q & 0x3FFu));
+}
+
+/* fp16 bits -> fp32 (exact). */
+float oracle_f16_to_f32(uint16_t h) {
+  const uint32_t sign = ((uint32_t)h & 0x8000u) << 16;
+  const uint32_t e = ((uint32_t)h >> 10) & 0x1Fu;
+  const uint32_t m = (uint32_t)h & 0x3FFu;
+  float f;
+  if (e == 0) {
+    f = ldexpf((float)m, -24);                                       /* subnormal or zero */
+    if (sign) f = -f;
+    return f;
+  }
+  uint32_t x;
+  if (e == 31) x = sign | 0x7F800000u | (m << 13);
+  else x = sign | ((e - 15 + 127) << 23) | (m << 13);
+  memcpy(&f, &x, 4);
+  return f;
+}
+
+void oracle_quantize_int2_rows(const float* k, int64_t rows, int32_t d, uint8_t* codes,
+                               uint16_t* params) {
+  const int32_t ng = d / 32;
+  for (int64_t r = 0; r < rows; ++r) {
+    const float* x = k + r * (int64_t)d;
+    uint8_t* cr = codes + r * (int64_t)(d / 4);
+    memset(cr, 0, (size_t)(d / 4));
+    for (int32_t g = 0; g < ng; ++g) {
+      float lo = x[32 * g], hi = x[32 * g];
+      for (int32_t j = 32 * g + 1; j < 32 * g + 32; ++j) {
+        if (x[j] < lo) lo = x[j];
+        if (x[j] > hi) hi = x[j];
+      }
+      const uint16_t lo_h = oracle_f32_to_f16(lo);
+      const float Lf = oracle_f16_to_f32(lo_h);
+      const uint16_t s_h = oracle_f32_to_f16((hi - Lf) / 3.0f);
+      const float S = oracle_f16_to_f32(s_h);
+      params[(r * ng + g) * 2] = s_h;
+      params[(r * ng + g) * 2 + 1] = lo_h;
+      for (int32_t j = 32 * g; j < 32 * g + 32; ++j) {
+        int c = 0;
+        if (S > 0.0f) {
+          float y = nearbyintf((x[j] - Lf) / S);
+          if (y < 0.0f) y = 0.0f;
+          if (y > 3.0f) y = 3.0f;
+          c = (int)y;
+        }
+        cr[j / 4] |= (uint8_t)(c << (2 * (j % 4)));
+      }
+    }
+  }
+}
+
+/*
+ * INT2 proposal scores of one (sequence, KV head) row: per query head g and
+ * feature group,
+ *   D = sum_j q[g][j] * c_j,   Q = sum_j q[g][j]      (fp32, j ascending)
+ *   term = S * D + L * Q                              (each product rounded)
+ * and score_g = sum of the terms over the groups in order (fp32), i.e. the
+ * dot product of q with the dequantized key L + S * c.  s_t = max_g score_g.
+ */
+void oracle_propose_scores_int2(const float* q, int32_t G, int32_t d, const uint8_t* codes,
+                                const uint16_t* params, int32_t L, float* s) {
+  const int32_t ng = d / 32;
+  for (int32_t t = 0; t < L; ++t) {
+    const uint8_t* cr = codes + (int64_t)t * (d / 4);
+    const uint16_t* pr = params + (int64_t)t * ng * 2;
+    float best = 0.0f;
+    for (int32_t g = 0; g < G; ++g) {
+      float acc = 0.0f;
+      for (int32_t gr = 0; gr < ng; ++gr) {
+        float D = 0.0f, Q = 0.0f;
+        for (int32_t j = 32 * gr; j < 32 * gr + 32; ++j) {
+          const int c = (cr[j / 4] >> (2 * (j % 4))) & 3;
+          D = D + q[g * d + j] * (float)c;
+          Q = Q + q[g * d + j];
+        }
+        const float S = oracle_f16_to_f32(pr[gr * 2]), Lf = oracle_f16_to_f32(pr[gr * 2 + 1]);
+        const float p1 = S * D, p2 = Lf * Q;
+        acc = acc + (p1 + p2);
+      }
+      if (g == 0 || acc > best) best = acc;
+    }
+    s[t] = best;
+  }
+}
+
+int32_t oracle_propose_row_int2(const float* q, int32_t G, int32_t d, const uint8_t* codes,
+                                const uint16_t* params, int32_t L, int32_t kappa_p,
+                                int32_t* pool, float* scores_out) {
+  float* s = scores_out ? scores_out : (float*)malloc(sizeof(float) * (size_t)(L > 0 ? L : 1));
+  oracle_propose_scores_int2(q, G, d, codes, params, L, s);
+  int32_t n = oracle_topk_ascending(s, L, kappa_p, pool);
+  if (!scores_out) free(s);
+  return n;
+}
