@@ -227,7 +227,7 @@ void oracle_attend(const float* q, int32_t d, const float* K, const float* V,
  * scheme).  Reading used here: per (KV head, token), per group of 32
  * consecutive features, asymmetric 2-bit codes with an fp16 zero point and
  * an fp16 step:
- *   lo  = min_j k_j,  hi = max_j k_j                  (group, exact in fp32)
+ *   lo  = min_j k_j,  hi = max_j k_j    (group, exact in fp32; -0 taken as +0)
  *   L   = fp16(lo),   S = fp16((hi - L) / 3)          (round to nearest even)
  *   c_j = clamp(rne((k_j - L) / S), 0, 3)             (S > 0; else c_j = 0)
  * so the dequantized key is L + S * c_j.  Codes are packed four to a byte,
@@ -303,6 +303,8 @@ void oracle_quantize_int2_rows(const float* k, int64_t rows, int32_t d, uint8_t*
         if (x[j] < lo) lo = x[j];
         if (x[j] > hi) hi = x[j];
       }
+      lo = canon(lo);  /* -0 is taken as +0, so the fp16 bits are unique */
+      hi = canon(hi);
       const uint16_t lo_h = oracle_f32_to_f16(lo);
       const float Lf = oracle_f16_to_f32(lo_h);
       const uint16_t s_h = oracle_f32_to_f16((hi - Lf) / 3.0f);
