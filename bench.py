@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true", help="skip the cpu_baseline leg")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--profile-steps", type=int, default=5)
+    ap.add_argument("--keys", default="int8", choices=["int8", "int2"],
+                    help="proposal key cache: int8 per token (the headline workload) or INT2 per 32-feature group")
     ap.add_argument("--layers", type=int, default=0,
                     help="keep only the first N layers (small cases for profiling)")
     return ap.parse_args()
@@ -66,11 +68,14 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def step_bytes(cfg) -> dict:
+def step_bytes(cfg, keys: str = "int8") -> dict:
     """Algorithmic bytes per op launch (cache reads the method must make)."""
     D, Hkv, T, B = cfg.head_dim, cfg.num_kv_heads, cfg.total_tokens, cfg.batch
     el = 2 if cfg.dtype == "bf16" else 4
-    propose = Hkv * T * (D + 4)  # int8 codes + fp32 scale per (head, position)
+    if keys == "int2":
+        propose = Hkv * T * (D // 4 + D // 32 * 4)  # 2-bit codes + fp16 (step, zero) per group
+    else:
+        propose = Hkv * T * (D + 4)  # int8 codes + fp32 scale per (head, position)
     refine = sum(min(cfg.kappa_p, L) for L in cfg.seqlens) * Hkv * D * el
     sparse = sum(min(cfg.kappa, cfg.kappa_p, L) for L in cfg.seqlens) * Hkv * D * el * 2
     dense = Hkv * T * D * el * 2
@@ -203,7 +208,7 @@ def traffic_for(op: str):
 
 # --------------------------------------------------------------------------- CPU oracle legs
 
-def oracle_units(cfg, qs, ks, vs, units, budget_s: float):
+def oracle_units(cfg, qs, ks, vs, units, budget_s: float, keys: str = "int8"):
     """Run the CPU oracle on (proposal group, KV head) units of one decode
     step until budget_s seconds of oracle time; returns (units done, seconds).
     Inputs are copied from the generated cache; untimed: host copies and the
@@ -218,14 +223,16 @@ def oracle_units(cfg, qs, ks, vs, units, budget_s: float):
         lays = list(range(lp, min(lp + cfg.group, cfg.num_layers)))
         host = {l: (qs[l][:, h * G:(h + 1) * G].float().cpu().numpy(),
                     ks[l][h].float().cpu().numpy(), vs[l][h].float().cpu().numpy()) for l in lays}
-        kq, sc = oracle.quantize_rows(host[lp][1])
+        quant = oracle.quantize_int2_rows if keys == "int2" else oracle.quantize_rows
+        propose = oracle.propose_row_int2 if keys == "int2" else oracle.propose_row
+        kq, sc = quant(host[lp][1])
         t0 = time.perf_counter()
         for b in range(cfg.batch):
             a, e = cu[b], cu[b + 1]
             if e == a:
                 continue
-            oracle.quantize_rows(host[lp][1][e - 1:e])  # the new token's key row
-            pool, _ = oracle.propose_row(host[lp][0][b], kq[a:e], sc[a:e], cfg.kappa_p)
+            quant(host[lp][1][e - 1:e])  # the new token's key row
+            pool, _ = propose(host[lp][0][b], kq[a:e], sc[a:e], cfg.kappa_p)
             for l in lays:
                 q, k, v = host[l]
                 idx, _ = oracle.refine_row(q[b], k[a:e], pool, cfg.kappa)
@@ -259,8 +266,8 @@ def run_reference(args, dist: Dist):
     vs = {x.index: x.v for x in lays}
     per_step_units = len(unit_list(cfg))
     units = [(0, h % cfg.num_kv_heads) for h in range(args.warmup + args.steps)]
-    oracle_units(cfg, qs, ks, vs, units[:args.warmup], 1e9)
-    n, secs = oracle_units(cfg, qs, ks, vs, units[args.warmup:], 1e9)
+    oracle_units(cfg, qs, ks, vs, units[:args.warmup], 1e9, args.keys)
+    n, secs = oracle_units(cfg, qs, ks, vs, units[args.warmup:], 1e9, args.keys)
     value = (n / per_step_units) / secs
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
@@ -313,16 +320,22 @@ def run_prism(args, dist: Dist):
     del layers
     dec = PrismDecoder(cfg.seqlens, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim,
                        prism.BF16 if cfg.dtype == "bf16" else prism.F32, L, cfg.group,
-                       cfg.kappa_p, cfg.kappa, device=dev)
+                       cfg.kappa_p, cfg.kappa, device=dev, keys=args.keys)
     rows = dec.new_rows.long()
     Hkv = cfg.num_kv_heads
     k_new = torch.stack([k[:, rows].transpose(0, 1).contiguous() for k in ks])  # [L][B][Hkv][d]
     v_new = torch.stack([v[:, rows].transpose(0, 1).contiguous() for v in vs])
     kqs, scs = {}, {}
     for l in cfg.proposal_layers:  # prefill: quantize the whole key cache (untimed)
-        kqs[l] = torch.empty(ks[l].shape, dtype=torch.int8, device=dev)
-        scs[l] = torch.empty(ks[l].shape[:2], dtype=torch.float32, device=dev)
-        prism.quantize_k(dec.p, ks[l], kqs[l], scs[l])
+        if args.keys == "int2":
+            Hk, Tk, Dk = ks[l].shape
+            kqs[l] = torch.empty((Hk, Tk, Dk // 4), dtype=torch.uint8, device=dev)
+            scs[l] = torch.empty((Hk, Tk, Dk // 32, 2), dtype=torch.int16, device=dev)
+            prism.quantize_k_int2(dec.p, ks[l], kqs[l], scs[l])
+        else:
+            kqs[l] = torch.empty(ks[l].shape, dtype=torch.int8, device=dev)
+            scs[l] = torch.empty(ks[l].shape[:2], dtype=torch.float32, device=dev)
+            prism.quantize_k(dec.p, ks[l], kqs[l], scs[l])
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream()
@@ -392,9 +405,14 @@ def run_prism(args, dist: Dist):
 
         def f_prop(l=l):
             prism.append_kv(dec.p, k_new[l], v_new[l], ks[l], vs[l])
-            prism.quantize_k(dec.p, ks[l], kqs[l], scs[l], tok_rows=dec.new_rows, ws=dec.ws_q)
-            prism.propose(dec.p, q_layers[l], kqs[l], scs[l], cfg.kappa_p, dec.pool[l],
-                          dec.pool_cnt[l], dec.ws_prop)
+            if args.keys == "int2":
+                prism.quantize_k_int2(dec.p, ks[l], kqs[l], scs[l], tok_rows=dec.new_rows, ws=dec.ws_q)
+                prism.propose_int2(dec.p, q_layers[l], kqs[l], scs[l], cfg.kappa_p, dec.pool[l],
+                                   dec.pool_cnt[l], dec.ws_prop)
+            else:
+                prism.quantize_k(dec.p, ks[l], kqs[l], scs[l], tok_rows=dec.new_rows, ws=dec.ws_q)
+                prism.propose(dec.p, q_layers[l], kqs[l], scs[l], cfg.kappa_p, dec.pool[l],
+                              dec.pool_cnt[l], dec.ws_prop)
 
         def f_rd(l=l):
             src = l - l % cfg.group
@@ -426,7 +444,7 @@ def run_prism(args, dist: Dist):
         for name, a, b in evs:
             per_op.setdefault(name, []).append(a.elapsed_time(b) * 1e3)  # us
     del gate
-    nbytes = step_bytes(cfg)
+    nbytes = step_bytes(cfg, args.keys)
     per_step_us = {n: sum(v) / args.profile_steps for n, v in per_op.items()}
     dominant = max(per_step_us, key=per_step_us.get)
     avg_us = statistics.mean(per_op[dominant])
@@ -468,7 +486,7 @@ def run_prism(args, dist: Dist):
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
         units = unit_list(cfg)
-        n, s = oracle_units(cfg, q_layers, ks, vs, units, args.cpu_seconds)
+        n, s = oracle_units(cfg, q_layers, ks, vs, units, args.cpu_seconds, args.keys)
         cpu = {"value": (n / len(units)) / s, "unit": "steps/s", "cores": 1, "kind": "oracle",
                "sample": f"{n} of the {len(units)} (proposal group, KV head) units of one "
                          f"{cfg.name} decode step ({s:.1f} s of single-thread oracle time)"}
@@ -483,6 +501,8 @@ def run_prism(args, dist: Dist):
             "config": dict(workload_config(cfg), l2="inputs larger than L2: a step touches "
                            f"{nbytes['step'] / 1e9:.2f} GB of distinct cache rows (L2 126 MB)",
                            refined_layers="fused refine+select+sparse-decode (prism_refine_decode)",
+                           proposal_keys="int8 per token" if args.keys == "int8"
+                           else "INT2 per 32-feature group (fp16 step and zero point)",
                            graph="one CUDA graph per step"),
             "roofline": roofline,
             "step_roofline": {"achieved": round(step_achieved, 1), "peak": peak, "unit": "GB/s",

@@ -158,6 +158,38 @@ PRISM_API prism_status prism_propose(const prism_shape* shape, const void* q, co
                            int32_t* pool_cnt, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * INT2 proposal keys (sec. 4.2: the pages compress the proposal layers' key
+ * cache to INT2 without stating the scheme; this is the library's scheme).
+ * Per KV head h, token t and group of 32 consecutive features (d = 128: four
+ * groups), with lo / hi the group's min / max (-0 taken as +0):
+ *   L = fp16(lo),  S = fp16((hi - L) / 3)          (round to nearest even)
+ *   c_j = clamp(round_half_even((K_j - L) / S), 0, 3)   (all 0 when S = 0)
+ * in IEEE fp32 arithmetic, so the dequantized key is L + S * c.
+ * Layouts: codes [Hkv][T][d/4] uint8, feature f at bits 2 (f mod 4) of byte
+ * f / 4; params [Hkv][T][d/32][2] uint16 holding the fp16 bits of (S, L).
+ * 48 bytes per key row at d = 128 (int8: 132).  tok_rows, n_rows, ws as for
+ * prism_quantize_k.  bf16 or fp32 keys, d = 64 or 128; |K| < 65504.
+ */
+PRISM_API prism_status prism_quantize_k_int2(const prism_shape* shape, const void* k,
+                                             uint8_t* codes, uint16_t* params,
+                                             const int32_t* tok_rows, int32_t n_rows, void* ws,
+                                             size_t ws_bytes, void* stream);
+
+/*
+ * prism_propose on INT2 keys: per position t < L_b and query head g,
+ *   score_g = sum over groups of (S * D + L * Q),
+ *   D = sum_{j in group} q[g][j] * c_j,   Q = sum_{j in group} q[g][j],
+ * i.e. q . (L + S c), and s_t = max_g score_g; the pool is the top
+ * min(kappa_p, L_b) positions as in prism_propose.  The workspace is
+ * PRISM_OP_PROPOSE's.  bf16 queries and d = 128 only (else
+ * PRISM_ERR_UNSUPPORTED); L_b <= PRISM_MAX_SELECT_ROW.
+ */
+PRISM_API prism_status prism_propose_int2(const prism_shape* shape, const void* q,
+                                          const uint8_t* codes, const uint16_t* params,
+                                          int32_t kappa_p, int32_t* pool_idx, int32_t* pool_cnt,
+                                          void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Refined layer (sec. 4.1; sec. 6: refined layers re-select their own top
  * kappa inside the proposed region, at a cost independent of context
  * length, sec. 5.3 "End-to-end latency"): exact scores of the pool members

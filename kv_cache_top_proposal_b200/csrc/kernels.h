@@ -31,6 +31,11 @@ cudaError_t launch_append(const Dims& d, const void* k_new, const void* v_new, v
 cudaError_t launch_quantize(const Dims& d, const void* k, int8_t* kq, float* scale,
                             const int32_t* tok_rows, int64_t n_rows, int32_t* status,
                             cudaStream_t st);
+// INT2 codes [Hkv][T][d/4] (four per byte) and (step, zero point) fp16 bits
+// [Hkv][T][d/32][2] of the listed token rows (quantize.cu).
+cudaError_t launch_quantize_int2(const Dims& d, const void* k, uint8_t* codes, uint16_t* params,
+                                 const int32_t* tok_rows, int64_t n_rows, int32_t* status,
+                                 cudaStream_t st);
 
 // Proposal scores s[h][t] (fp32, [Hkv][T]).  use_mma selects the tensor-core
 // (mma.sync, fp16 operands) scorer, valid for bf16 queries only.
@@ -39,6 +44,11 @@ cudaError_t launch_quantize(const Dims& d, const void* k, int8_t* kq, float* sca
 cudaError_t launch_propose_scores(const Dims& d, const void* q, const int8_t* kq,
                                   const float* scale, float* scores, uint32_t* hist, bool use_mma,
                                   int32_t* status, cudaStream_t st);
+// INT2 proposal scores from packed codes and (step, zero point) pairs, with
+// the first-digit histogram (bf16 queries, d = 128; score.cu).
+cudaError_t launch_propose_scores_int2(const Dims& d, const void* q, const uint8_t* codes,
+                                       const uint16_t* params, float* scores, uint32_t* hist,
+                                       int32_t* status, cudaStream_t st);
 
 // Cluster radix top-k.  mode 0 (propose): keys scores[h][cu[b] + i], row
 // length L_b, output position i.  mode 1 (refine): keys r[row][i], row length

@@ -206,6 +206,60 @@ prism_status prism_propose(const prism_shape* shape, const void* q, const int8_t
   return cuda_status(launch_select(d, a, d.max_len, st));
 }
 
+prism_status prism_quantize_k_int2(const prism_shape* shape, const void* k, uint8_t* codes,
+                                   uint16_t* params, const int32_t* tok_rows, int32_t n_rows,
+                                   void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!k || !codes || !params) return PRISM_ERR_INVALID_ARG;
+  if (tok_rows && n_rows < 0) return PRISM_ERR_INVALID_ARG;
+  if (ws && (ws_bytes < kWsHeader || ((uintptr_t)ws % kAlign) != 0)) return PRISM_ERR_WORKSPACE;
+  if ((s = set_live_sms(&d)) != PRISM_OK) return s;
+  const int64_t rows = tok_rows ? (int64_t)n_rows : d.T;
+  return cuda_status(launch_quantize_int2(d, k, codes, params, tok_rows, rows,
+                                          static_cast<int32_t*>(ws), static_cast<cudaStream_t>(stream)));
+}
+
+prism_status prism_propose_int2(const prism_shape* shape, const void* q, const uint8_t* codes,
+                                const uint16_t* params, int32_t kappa_p, int32_t* pool_idx,
+                                int32_t* pool_cnt, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!q || !codes || !params || !pool_idx || !pool_cnt || kappa_p < 1) return PRISM_ERR_INVALID_ARG;
+  if (!d.bf16 || d.D != 128) return PRISM_ERR_UNSUPPORTED;
+  if (((uintptr_t)codes | (uintptr_t)params) % 16) return PRISM_ERR_INVALID_ARG;
+  if (d.max_len > select_capacity_per_row()) return PRISM_ERR_UNSUPPORTED;
+  const Layout L = layout(d, PRISM_OP_PROPOSE, kappa_p, 0);
+  if (!ws_ok(ws, ws_bytes, L)) return PRISM_ERR_WORKSPACE;
+  if ((s = set_live_sms(&d)) != PRISM_OK) return s;
+  char* w = static_cast<char*>(ws);
+  int32_t* status = reinterpret_cast<int32_t*>(w);
+  float* scores = reinterpret_cast<float*>(w + L.a);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(w + L.b);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t rows = (size_t)d.B * d.Hkv;
+  if (cudaMemsetAsync(hist, 0, rows * 4096 * 4, st) != cudaSuccess) return PRISM_ERR_CUDA;
+  cudaError_t e = launch_propose_scores_int2(d, q, codes, params, scores, hist, status, st);
+  if (e != cudaSuccess) return PRISM_ERR_CUDA;
+  if (d.max_len <= propose_select_max_row())
+    return cuda_status(launch_propose_select(d, scores, hist, kappa_p, pool_idx, pool_cnt, status, st));
+  SelectArgs a{};
+  a.mode = 0;
+  a.Hkv = d.Hkv;
+  a.G = d.G;
+  a.Hq = d.Hq;
+  a.T = d.T;
+  a.cu = d.cu_dev;
+  a.keys = scores;
+  a.k_req = kappa_p;
+  a.out = pool_idx;
+  a.out_cnt = pool_cnt;
+  a.status = status;
+  return cuda_status(launch_select(d, a, d.max_len, st));
+}
+
 prism_status prism_refine(const prism_shape* shape, const void* q, const void* k,
                           const int32_t* pool_idx, const int32_t* pool_cnt, int32_t kappa_p,
                           int32_t kappa, int32_t* idx, int32_t* cnt, float* logits_opt, void* ws,

@@ -6,6 +6,8 @@
 // 16-byte vector: a coalesced read of the row, a shuffle max for amax, IEEE
 // divisions and round-half-even, one 8- or 4-byte store of codes per lane.
 // HBM bound: reads d*sizeof(T) and writes d + 4 bytes per row.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -144,6 +146,94 @@ cudaError_t launch_quantize(const Dims& d, const void* k, int8_t* kq, float* sca
   }
   return d.D == 128 ? run<float, 128>(d, k, kq, scale, tok_rows, n_rows, status, st)
                     : run<float, 64>(d, k, kq, scale, tok_rows, n_rows, status, st);
+}
+
+// ---- INT2 proposal keys ------------------------------------------------------
+// Per (KV head, token) and per group of 32 consecutive features (sec. 4.2
+// names INT2 for the proposal key cache; this is the scheme the library
+// defines for it): L = fp16(min), S = fp16((max - L) / 3) and
+// c = clamp(rne((k - L) / S), 0, 3) (all codes 0 when S is 0), with the
+// same IEEE operations in the same order as the definition, so codes and
+// (S, L) are bit-exact.  One warp per group: lane j holds feature j, a
+// shuffle min/max, four lanes' codes packed per byte (feature f at bits
+// 2 (f mod 4) of byte f / 4), (S, L) as fp16 bits.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) quantize_int2_kernel(const T* __restrict__ k,
+                                                            uint8_t* __restrict__ codes,
+                                                            uint16_t* __restrict__ params,
+                                                            int64_t T_tok, int Hkv,
+                                                            const int32_t* __restrict__ tok_rows,
+                                                            int64_t n_rows, int32_t* status) {
+  constexpr int NG = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t groups = (int64_t)Hkv * n_rows * NG;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t gi = warp0; gi < groups; gi += nwarps) {  // warp-uniform
+    const int64_t r = gi / NG;
+    const int grp = (int)(gi - r * NG);
+    const int64_t h = r / n_rows, i = r - h * n_rows;
+    const int64_t t = tok_rows ? (int64_t)tok_rows[i] : i;
+    if (t < 0 || t >= T_tok) {
+      if (lane == 0 && grp == 0) flag_status(status, PRISM_DEV_BAD_INDEX);
+      continue;
+    }
+    const int64_t row = h * T_tok + t;
+    float x;
+    if constexpr (sizeof(T) == 2) {
+      x = __bfloat162float(k[row * D + grp * 32 + lane]);
+    } else {
+      x = k[row * D + grp * 32 + lane];
+    }
+    float lo = x, hi = x;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    lo = __fadd_rn(lo, 0.0f);  // -0 is taken as +0 (unique fp16 bits)
+    hi = __fadd_rn(hi, 0.0f);
+    const __half lo_h = __float2half_rn(lo);
+    const float L = __half2float(lo_h);
+    const __half s_h = __float2half_rn(__fdiv_rn(__fsub_rn(hi, L), 3.0f));
+    const float S = __half2float(s_h);
+    int c = 0;
+    if (S > 0.0f) c = (int)fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(x, L), S)), 0.0f), 3.0f);
+    uint32_t b = (uint32_t)c;
+    b |= (uint32_t)__shfl_down_sync(0xffffffffu, c, 1) << 2;
+    b |= (uint32_t)__shfl_down_sync(0xffffffffu, c, 2) << 4;
+    b |= (uint32_t)__shfl_down_sync(0xffffffffu, c, 3) << 6;
+    if ((lane & 3) == 0) codes[row * (D / 4) + grp * 8 + (lane >> 2)] = (uint8_t)b;
+    if (lane == 0) {
+      params[(row * NG + grp) * 2] = __half_as_ushort(s_h);
+      params[(row * NG + grp) * 2 + 1] = __half_as_ushort(lo_h);
+    }
+  }
+}
+
+template <typename T, int D>
+static cudaError_t run_int2(const Dims& d, const void* k, uint8_t* codes, uint16_t* params,
+                            const int32_t* tok, int64_t n_rows, int32_t* status, cudaStream_t st) {
+  const int64_t groups = (int64_t)d.Hkv * n_rows * (D / 32);
+  int64_t blocks = cdiv(groups, 8);
+  const int64_t cap = (int64_t)d.num_sms * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  quantize_int2_kernel<T, D><<<(unsigned)blocks, 256, 0, st>>>(
+      static_cast<const T*>(k), codes, params, d.T, d.Hkv, tok, n_rows, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_int2(const Dims& d, const void* k, uint8_t* codes, uint16_t* params,
+                                 const int32_t* tok_rows, int64_t n_rows, int32_t* status,
+                                 cudaStream_t st) {
+  if (n_rows == 0 || d.Hkv == 0) return cudaSuccess;
+  if (d.bf16) {
+    return d.D == 128 ? run_int2<__nv_bfloat16, 128>(d, k, codes, params, tok_rows, n_rows, status, st)
+                      : run_int2<__nv_bfloat16, 64>(d, k, codes, params, tok_rows, n_rows, status, st);
+  }
+  return d.D == 128 ? run_int2<float, 128>(d, k, codes, params, tok_rows, n_rows, status, st)
+                    : run_int2<float, 64>(d, k, codes, params, tok_rows, n_rows, status, st);
 }
 
 }  // namespace prism

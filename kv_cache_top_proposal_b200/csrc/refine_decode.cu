@@ -36,8 +36,6 @@
 // value rows, d * sizeof(T) each.
 #include <cooperative_groups.h>
 
-#include <cstdlib>
-
 #include "common.cuh"
 #include "kernels.h"
 
@@ -118,17 +116,21 @@ struct RowStream {
       : base(base_), nrow(nrow_), npos(npos_), spos(spos_), list(list_), rows(rows_),
         nchunk((rows_ + SR - 1) / SR), ring(ring_) {}
 
+  // thread t always copies 16-byte chunk t % VPR of rows t / VPR, t / VPR +
+  // kThreads / VPR, ... (the row step is a multiple of 8, so the chunk's
+  // swizzled position within a row is fixed too)
   __device__ __forceinline__ void issue(int c, bool defer_new) {
+    static_assert(kThreads % VPR == 0 && (kThreads / VPR) % 8 == 0, "row step");
     if (c < nchunk) {
       const int r0 = c * SR, n = min(SR, rows - r0);
       unsigned char* buf = ring + (c % kStages) * kStageBytes;
-      for (int x = threadIdx.x; x < n * VPR; x += kThreads) {
-        const int r = x / VPR, vv = x - r * VPR;
+      const int vv = threadIdx.x % VPR;
+      const T* col = base + vv * (16 / (int)sizeof(T));
+      for (int r = threadIdx.x / VPR; r < n; r += kThreads / VPR) {
         const int pos = spos[list ? list[r0 + r] : r0 + r];
         const bool fresh = nrow && pos == npos;
         if (fresh && defer_new) continue;
-        const T* src = (fresh ? nrow : base + (int64_t)(pos >= 0 ? pos : 0) * D) +
-                       vv * (16 / (int)sizeof(T));
+        const T* src = fresh ? nrow + vv * (16 / (int)sizeof(T)) : col + (int64_t)(pos >= 0 ? pos : 0) * D;
         cp_async16(smem_u32(buf + swz<RB>(r, vv)), src, pos >= 0);
       }
     }
@@ -817,20 +819,11 @@ constexpr int recv_bytes(int GP, int D) { return (GP * D + kMaxCluster + 2 * GP 
 constexpr int kDynBudget = 227 * 1024 - 8 * 1024;
 constexpr int kPairBudget = 110 * 1024;
 
-// PRISM_RD_CLUSTER=c (1..16) forces the cluster size; PRISM_RD_SOLO=1 pads
-// the shared memory request so that one CTA holds an SM.
-int env_int(const char* name, int dflt) {
-  const char* e = std::getenv(name);
-  return e && *e ? std::atoi(e) : dflt;
-}
-
 template <typename T, int D, int GP>
 cudaError_t run(const Dims& d, RDArgs a, int cl, bool overlap, cudaStream_t st) {
   auto kern = refine_decode_kernel<T, D, GP>;
-  int smem = ring_bytes<T, D, GP>() + kHistWords * 4 + a.mc * per_member_bytes<GP>() +
-             recv_bytes(GP, D);
-  static const bool solo = env_int("PRISM_RD_SOLO", 0) == 1;
-  if (solo && smem < 120 * 1024) smem = 120 * 1024;
+  const int smem = ring_bytes<T, D, GP>() + kHistWords * 4 + a.mc * per_member_bytes<GP>() +
+                   recv_bytes(GP, D);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   if (cl > 8) {
@@ -877,8 +870,6 @@ RefineDecodePlan plan_refine_decode(const Dims& d, int kappa_p) {
   int cl = 1;
   while (cl < kMaxCluster && (int64_t)rows * cl < 2LL * d.num_sms) cl *= 2;
   while (cl < kMaxCluster && need(cl) > kPairBudget) cl *= 2;
-  static const int forced = env_int("PRISM_RD_CLUSTER", 0);
-  if (forced >= 1 && forced <= kMaxCluster && need(forced) <= kDynBudget) cl = forced;
   const bool ok = kappa_p <= kMaxCount && need(cl) <= kDynBudget;
   return RefineDecodePlan{cl, mc_of(cl), ok};
 }

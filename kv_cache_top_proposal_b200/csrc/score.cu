@@ -49,6 +49,8 @@ struct ScoreArgs {
   int64_t T;
   int B, Hkv, G;
   int32_t* status;
+  const uint8_t* codes;    // INT2 keys: [Hkv][T][d/4], four codes per byte
+  const uint16_t* params;  // INT2 keys: [Hkv][T][d/32][2] fp16 bits of (step, zero point)
 };
 
 // s_pref[b] = number of work items of sequences before b (per KV head).
@@ -573,6 +575,263 @@ __global__ void __launch_bounds__(kThreads, 3) score_tma_kernel(const __grid_con
   flush();
 }
 
+// INT2 scorer (bf16 queries, d = 128).  Per key row and query head the
+// score is sum over 32-feature groups of (S * D + L * Q), with D = q . c over
+// the group's 2-bit codes and Q = sum of q over the group (the dot product
+// with the dequantized key L + S c).  Rows stream through a cp.async ring
+// of 128-row stages (codes, then (S, L) pairs); warp w takes 16-row tile w.
+// The contraction D runs on tensor cores: a code c enters as the fp16
+// subnormal c * 2^-24 (its bits are c), the query is scaled by a power of
+// two into fp16 range as in the int8 scorer, so every product and sum is
+// exact up to fp32 rounding and one power of two undoes both scalings; each
+// k-step of 16 stays inside one group (two k-steps per group, one
+// accumulator per group).  Thread (g, tig)
+// takes, at k-step s, word s of its rows' codes (features 16 s .. 16 s + 15,
+// feature f at bits 2 (f mod 16)) and from it features 16 s + 2 tig + {0, 8}
+// and 16 s + 2 tig + {1, 9}: the query fragments follow the same features.
+// The query rows of a (sequence, KV head) go to shared memory once; Q is
+// summed there in feature order, and the group terms combine in the
+// definition's order, without fused multiply-adds.
+constexpr int kInt2Stages = 6;
+
+template <int D>
+struct Int2Layout {
+  static constexpr int CB = D / 4;                   // code bytes per row
+  static constexpr int NG = D / 32;                  // groups per row
+  static constexpr int PB = NG * 4;                  // (S, L) bytes per row
+  static constexpr int CODES = kStageRows * CB;
+  static constexpr int BYTES = CODES + kStageRows * PB;
+};
+
+// two codes (bits 0-1 and 16-17 of w) as fp16 subnormals c * 2^-24
+__device__ __forceinline__ uint32_t int2_pair(uint32_t w) { return w & 0x00030003u; }
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 3) score_int2_kernel(ScoreArgs a) {
+  constexpr int D = 128;
+  constexpr int KS = D / 16;
+  using IL = Int2Layout<D>;
+  constexpr int NG = IL::NG;
+  extern __shared__ __align__(16) unsigned char ring[];  // stages, hist, s_pref[B+1], cu[B+1]
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(ring + kInt2Stages * IL::BYTES);  // [kHist / 2]
+  int* s_pref = reinterpret_cast<int*>(s_hist + kHist / 2);
+  int* s_cu = s_pref + a.B + 1;
+  __shared__ float sq[NT * 8 * D];   // the (b, h) group's query rows, fp32
+  __shared__ float sQ[NT * 8 * NG];  // per head and group: sum of q (features in order)
+  __shared__ float s_mx[kThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, tig = lane & 3;
+  for (int i = tid; i <= a.B; i += kThreads) s_cu[i] = a.cu[i];
+  for (int i = tid; i < kHist / 2; i += kThreads) s_hist[i] = 0u;
+  chunk_prefix(a.cu, a.B, kStageRows, s_pref);
+  const int per_head = s_pref[a.B];
+  const int64_t total = (int64_t)a.Hkv * per_head;
+  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
+  const int64_t s_begin = total * blockIdx.x / gridDim.x;
+  const int64_t s_end = total * (blockIdx.x + 1) / gridDim.x;
+  const int nk = (int)(s_end - s_begin);
+  StageIter it_issue, it_comp;
+  {
+    const int h = (int)(s_begin / per_head);
+    const int cc = (int)(s_begin - (int64_t)h * per_head);
+    const int b = find_seq(s_pref, a.B, cc);
+    it_issue = StageIter{h, b, (cc - s_pref[b]) * kStageRows};
+    it_comp = it_issue;
+  }
+  auto issue = [&](int kk) {
+    if (kk < nk) {
+      const int L = s_cu[it_issue.b + 1] - s_cu[it_issue.b];
+      const int rows = min(kStageRows, L - it_issue.r0);
+      const int64_t rowbase = (int64_t)it_issue.h * a.T + s_cu[it_issue.b] + it_issue.r0;
+      unsigned char* buf = ring + (kk % kInt2Stages) * IL::BYTES;
+      const unsigned char* cs = a.codes + rowbase * IL::CB;
+      const unsigned char* ps = reinterpret_cast<const unsigned char*>(a.params) + rowbase * IL::PB;
+      for (int x = tid; x < rows * (IL::CB / 16); x += kThreads)
+        cp_async16(smem_u32(buf + x * 16), cs + x * 16, true);
+      for (int x = tid; x < rows * (IL::PB / 16); x += kThreads)
+        cp_async16(smem_u32(buf + IL::CODES + x * 16), ps + x * 16, true);
+      it_issue.advance(s_cu, a.B);
+    }
+    cp_async_commit();
+  };
+
+  uint32_t bq[NT][KS][2];
+  float Qv[NT][NG][2];  // sum of q over each group, heads nt*8 + 2 tig, + 1
+  float unscale = 1.0f;
+  int cur_b = -1, cur_h = -1;
+  int hist_row = -1, since_flush = 0;
+  auto flush = [&]() {  // packed shared histogram -> global (non-zero bins), then clear
+    if (a.hist && hist_row >= 0) {
+      uint32_t* gh = a.hist + (int64_t)hist_row * kHist;
+      for (int i = tid; i < kHist / 2; i += kThreads) {
+        const uint32_t c = s_hist[i];
+        if (c) {
+          if (c & 0xFFFFu) atomicAdd(gh + 2 * i, c & 0xFFFFu);
+          if (c >> 16) atomicAdd(gh + 2 * i + 1, c >> 16);
+          s_hist[i] = 0u;
+        }
+      }
+    }
+    since_flush = 0;
+    __syncthreads();
+  };
+#pragma unroll 1
+  for (int kk = 0; kk < kInt2Stages; ++kk) issue(kk);
+#pragma unroll 1
+  for (int kk = 0; kk < nk; ++kk) {
+    const int L = s_cu[it_comp.b + 1] - s_cu[it_comp.b];
+    const int rows = min(kStageRows, L - it_comp.r0);
+    const int64_t rowbase = (int64_t)it_comp.h * a.T + s_cu[it_comp.b] + it_comp.r0;
+    if (it_comp.b != cur_b || it_comp.h != cur_h) {  // CTA-uniform
+      cur_b = it_comp.b;
+      cur_h = it_comp.h;
+      // the group's query rows into shared memory (fp32), then the fragments,
+      // the power-of-two scale and the per-group sums Q from there
+      const __nv_bfloat16* qb = q + ((int64_t)cur_b * a.Hkv * a.G + (int64_t)cur_h * a.G) * D;
+      __syncthreads();  // the previous (b, h)'s sq / sQ are no longer read
+      float mxl = 0.0f;
+      for (int i = tid; i < a.G * D; i += kThreads) {
+        const float v = __bfloat162float(qb[i]);
+        sq[i] = v;
+        mxl = fmaxf(mxl, fabsf(v));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mxl = fmaxf(mxl, __shfl_xor_sync(0xffffffffu, mxl, o));
+      if (lane == 0) s_mx[warp] = mxl;
+      __syncthreads();
+      float mx = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kThreads / 32; ++w) mx = fmaxf(mx, s_mx[w]);
+      if (tid < a.G * NG) {  // Q of head tid / NG, group tid % NG, features in order
+        const float* qr = sq + (tid / NG) * D + (tid % NG) * 32;
+        float acc = 0.0f;
+        for (int j = 0; j < 32; ++j) acc = __fadd_rn(acc, qr[j]);
+        sQ[tid] = acc;
+      }
+      int qexp = 0;
+      if (mx > 0.0f) {
+        const int e2 = ((__float_as_int(mx) >> 23) & 0xFF) - 126;  // mx < 2^e2
+        qexp = min(103, max(-103, 15 - e2));  // 2^qexp and 2^(24 - qexp) stay normal
+      }
+      const float up = pow2f(qexp);
+      // codes enter the tensor cores as fp16 subnormals c * 2^-24: undo both
+      unscale = pow2f(24 - qexp);
+      __syncthreads();
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int n = nt * 8 + g;
+#pragma unroll
+        for (int s2 = 0; s2 < KS; ++s2) {
+          const int f = 16 * s2 + 2 * tig;
+          float v0 = 0.0f, v1 = 0.0f, v2 = 0.0f, v3 = 0.0f;
+          if (n < a.G) {
+            const float* qr = sq + n * D;
+            v0 = qr[f];
+            v1 = qr[f + 8];
+            v2 = qr[f + 1];
+            v3 = qr[f + 9];
+          }
+          bq[nt][s2][0] = pack_f16(v0 * up, v1 * up);
+          bq[nt][s2][1] = pack_f16(v2 * up, v3 * up);
+        }
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int head = nt * 8 + 2 * tig + c;
+#pragma unroll
+          for (int gr = 0; gr < NG; ++gr) Qv[nt][gr][c] = head < a.G ? sQ[head * NG + gr] : 0.0f;
+        }
+      }
+    }
+    const int row_id = it_comp.b * a.Hkv + it_comp.h;  // CTA-uniform
+    if (row_id != hist_row || since_flush == kTmaFlushStages) {
+      flush();
+      hist_row = row_id;
+    }
+    ++since_flush;
+    it_comp.advance(s_cu, a.B);
+    cp_async_wait<kInt2Stages - 1>();
+    __syncthreads();
+    const unsigned char* buf = ring + (kk % kInt2Stages) * IL::BYTES;
+    const int t = warp;  // one 16-row tile per warp
+    if (t * 16 < rows) {
+      const int rA = t * 16 + g, rB = rA + 8;
+      uint32_t wa[KS], wb[KS];
+      {
+        const uint4* ca = reinterpret_cast<const uint4*>(buf + rA * IL::CB);
+        const uint4* cb = reinterpret_cast<const uint4*>(buf + rB * IL::CB);
+        const uint4 a0 = ca[0], a1 = ca[1], b0 = cb[0], b1 = cb[1];
+        wa[0] = a0.x; wa[1] = a0.y; wa[2] = a0.z; wa[3] = a0.w;
+        wa[4] = a1.x; wa[5] = a1.y; wa[6] = a1.z; wa[7] = a1.w;
+        wb[0] = b0.x; wb[1] = b0.y; wb[2] = b0.z; wb[3] = b0.w;
+        wb[4] = b1.x; wb[5] = b1.y; wb[6] = b1.z; wb[7] = b1.w;
+      }
+      float acc[NG][NT][4];
+#pragma unroll
+      for (int gr = 0; gr < NG; ++gr)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) acc[gr][nt][0] = acc[gr][nt][1] = acc[gr][nt][2] = acc[gr][nt][3] = 0.0f;
+      const int sh = 4 * tig;
+#pragma unroll
+      for (int s2 = 0; s2 < KS; ++s2) {
+        const uint32_t xa = wa[s2] >> sh, xb = wb[s2] >> sh;
+        const uint32_t a0 = int2_pair(xa), a2 = int2_pair(xa >> 2);
+        const uint32_t a1 = int2_pair(xb), a3 = int2_pair(xb >> 2);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          mma16816(acc[s2 / 2][nt], a0, a1, a2, a3, bq[nt][s2][0], bq[nt][s2][1]);
+      }
+      // (S, L) of the two rows, group by group
+      const uint4 pA4 = *reinterpret_cast<const uint4*>(buf + IL::CODES + rA * IL::PB);
+      const uint4 pB4 = *reinterpret_cast<const uint4*>(buf + IL::CODES + rB * IL::PB);
+      const uint32_t pA[4] = {pA4.x, pA4.y, pA4.z, pA4.w}, pB[4] = {pB4.x, pB4.y, pB4.z, pB4.w};
+      float mA = -INFINITY, mB = -INFINITY;
+      // S' = S * unscale is exact (a power of two), and S' * D_mma = S * D
+      float SA[NG], LA[NG], SB[NG], LB[NG];
+#pragma unroll
+      for (int gr = 0; gr < NG; ++gr) {
+        const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&pA[gr]));
+        const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&pB[gr]));
+        SA[gr] = fa.x * unscale;
+        LA[gr] = fa.y;
+        SB[gr] = fb.x * unscale;
+        LB[gr] = fb.y;
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float sc[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // c0..c3
+#pragma unroll
+        for (int gr = 0; gr < NG; ++gr) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float S = e < 2 ? SA[gr] : SB[gr], Lz = e < 2 ? LA[gr] : LB[gr];
+            const float term = __fadd_rn(__fmul_rn(S, acc[gr][nt][e]), __fmul_rn(Lz, Qv[nt][gr][e & 1]));
+            sc[e] = __fadd_rn(sc[e], term);
+          }
+        }
+        const int col = nt * 8 + 2 * tig;
+        if (col < a.G) { mA = fmaxf(mA, sc[0]); mB = fmaxf(mB, sc[2]); }
+        if (col + 1 < a.G) { mA = fmaxf(mA, sc[1]); mB = fmaxf(mB, sc[3]); }
+      }
+      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
+      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
+      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
+      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
+      const int rs = t * 16 + g + 8 * tig;  // tig 0: row g, tig 1: row g + 8
+      const bool mine = tig < 2 && rs < rows;
+      float score = 0.0f;
+      if (mine) {
+        score = tig == 0 ? mA : mB;
+        a.scores[rowbase + rs] = score;
+      }
+      if (a.hist) warp_hist_add_packed(s_hist, ord_key(score) >> 20, mine);
+    }
+    __syncthreads();
+    issue(kk + kInt2Stages);
+  }
+  cp_async_wait<0>();
+  flush();
+}
+
 // CUDA-core scorer: one thread per key row, query in shared memory (fp32).
 template <typename T, int D, int GP>
 __global__ void __launch_bounds__(kThreads) score_simt_kernel(ScoreArgs a) {
@@ -700,6 +959,17 @@ bool run_tma(const Dims& d, const ScoreArgs& a, int64_t total, cudaError_t* err,
   return true;
 }
 
+template <int NT>
+cudaError_t run_int2(const Dims& d, const ScoreArgs& a, int64_t total, cudaStream_t st) {
+  const int smem = kInt2Stages * Int2Layout<128>::BYTES + kHist / 2 * 4 + 2 * (d.B + 1) * (int)sizeof(int);
+  auto k = score_int2_kernel<NT>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int grid = grid_for(k, smem, d.num_sms, total);
+  k<<<grid, kThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
 template <typename T, int D, int GP>
 cudaError_t run_simt(const Dims& d, const ScoreArgs& a, int64_t total, cudaStream_t st) {
   const int smem = (((d.B + 1 + 3) & ~3) + GP * D) * (int)sizeof(int);
@@ -733,7 +1003,7 @@ cudaError_t launch_propose_scores(const Dims& d, const void* q, const int8_t* kq
   for (int b = 0; b < d.B; ++b) per_head += cdiv(d.cu_host[b + 1] - d.cu_host[b], kChunkRows);
   const int64_t total = per_head * d.Hkv;
   if (total == 0) return cudaSuccess;
-  ScoreArgs a{q, kq, scale, scores, hist, d.cu_dev, d.T, d.B, d.Hkv, d.G, status};
+  ScoreArgs a{q, kq, scale, scores, hist, d.cu_dev, d.T, d.B, d.Hkv, d.G, status, nullptr, nullptr};
   if (use_mma && d.bf16 && d.D == 128 && use_tma_scorer()) {
     int64_t stages = 0;
     for (int b = 0; b < d.B; ++b) stages += cdiv(d.cu_host[b + 1] - d.cu_host[b], kStageRows);
@@ -752,6 +1022,17 @@ cudaError_t launch_propose_scores(const Dims& d, const void* q, const int8_t* kq
   }
   return d.D == 128 ? simt_by_group<float, 128>(d, a, total, st)
                     : simt_by_group<float, 64>(d, a, total, st);
+}
+
+cudaError_t launch_propose_scores_int2(const Dims& d, const void* q, const uint8_t* codes,
+                                       const uint16_t* params, float* scores, uint32_t* hist,
+                                       int32_t* status, cudaStream_t st) {
+  if (!d.bf16 || d.D != 128) return cudaErrorInvalidValue;
+  int64_t stages = 0;
+  for (int b = 0; b < d.B; ++b) stages += cdiv(d.cu_host[b + 1] - d.cu_host[b], kStageRows);
+  if (stages == 0) return cudaSuccess;
+  ScoreArgs a{q, nullptr, nullptr, scores, hist, d.cu_dev, d.T, d.B, d.Hkv, d.G, status, codes, params};
+  return d.G <= 8 ? run_int2<1>(d, a, stages * d.Hkv, st) : run_int2<2>(d, a, stages * d.Hkv, st);
 }
 
 }  // namespace prism

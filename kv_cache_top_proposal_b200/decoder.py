@@ -29,7 +29,7 @@ from . import prism
 class PrismDecoder:
     def __init__(self, seqlens, num_q_heads: int, num_kv_heads: int, head_dim: int, dtype: int,
                  num_layers: int, group: int, kappa_p: int, kappa: int, device="cuda",
-                 softmax_scale: Optional[float] = None, fused: bool = True):
+                 softmax_scale: Optional[float] = None, fused: bool = True, keys: str = "int8"):
         self.dev = torch.device(device)
         self.p = prism.Problem(seqlens, num_q_heads, num_kv_heads, head_dim, dtype, device=self.dev)
         self.B, self.Hq, self.Hkv, self.D = len(seqlens), num_q_heads, num_kv_heads, head_dim
@@ -66,6 +66,10 @@ class PrismDecoder:
         self.ws_dense = None
         # refined layers in one fused call (refine -> select -> sparse decode)
         self.fused = fused
+        # proposal keys: "int8" (kq int8 [Hkv][T][d], k_scale fp32 [Hkv][T]) or
+        # "int2" (codes uint8 [Hkv][T][d/4], params int16 [Hkv][T][d/32][2])
+        assert keys in ("int8", "int2")
+        self.keys = keys
 
     def workspaces(self) -> List[torch.Tensor]:
         return [w for w in (self.ws_q, self.ws_prop, self.ws_ref, self.ws_dec, self.ws_rd,
@@ -73,7 +77,8 @@ class PrismDecoder:
 
     def layer(self, l: int, q, k, v, kq=None, k_scale=None, quantize_new: bool = True,
               k_new=None, v_new=None, k_next=None, overlap: bool = False, stream=None):
-        """Enqueue one layer of the step (kq/k_scale required at proposal layers).
+        """Enqueue one layer of the step (kq/k_scale -- or INT2 codes/params --
+        required at proposal layers).
 
         k_new / v_new ([B][Hkv][d]), when given, are first written to the last
         position of every sequence (the token being decoded).  overlap: the
@@ -86,10 +91,18 @@ class PrismDecoder:
         if k_new is not None and not fused_append:
             prism.append_kv(p, k_new, v_new, k, v, stream=stream)
         if proposal:
-            if quantize_new and self.new_rows.numel():
-                prism.quantize_k(p, k, kq, k_scale, tok_rows=self.new_rows, ws=self.ws_q, stream=stream)
-            prism.propose(p, q, kq, k_scale, self.kappa_p, self.pool[l], self.pool_cnt[l],
-                          self.ws_prop, stream=stream)
+            if self.keys == "int2":
+                if quantize_new and self.new_rows.numel():
+                    prism.quantize_k_int2(p, k, kq, k_scale, tok_rows=self.new_rows, ws=self.ws_q,
+                                          stream=stream)
+                prism.propose_int2(p, q, kq, k_scale, self.kappa_p, self.pool[l], self.pool_cnt[l],
+                                   self.ws_prop, stream=stream)
+            else:
+                if quantize_new and self.new_rows.numel():
+                    prism.quantize_k(p, k, kq, k_scale, tok_rows=self.new_rows, ws=self.ws_q,
+                                     stream=stream)
+                prism.propose(p, q, kq, k_scale, self.kappa_p, self.pool[l], self.pool_cnt[l],
+                              self.ws_prop, stream=stream)
         src = l - l % self.group
         if self.fused:
             prism.refine_decode(p, q, k, v, self.pool[src], self.pool_cnt[src], self.kappa_p,

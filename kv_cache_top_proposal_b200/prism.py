@@ -29,7 +29,8 @@ WS_HEADER = 256
 EXPORTS = ("prism_workspace_size", "prism_append_kv", "prism_quantize_k", "prism_propose", "prism_refine",
            "prism_sparse_decode", "prism_refine_decode", "prism_dense_decode",
            "prism_clear_device_status",
-           "prism_get_device_status", "prism_status_str", "prism_sparse_decode_noalloc")
+           "prism_get_device_status", "prism_status_str", "prism_sparse_decode_noalloc",
+           "prism_quantize_k_int2", "prism_propose_int2")
 
 
 class PrismError(RuntimeError):
@@ -65,6 +66,8 @@ def _load():
         "prism_clear_device_status": [P, S, P],
         "prism_get_device_status": [P, S, P, ctypes.POINTER(ctypes.c_int32)],
         "prism_sparse_decode_noalloc": [sp, P, P, P, P, P, i32, ctypes.c_float, P, P, P, P],
+        "prism_quantize_k_int2": [sp, P, P, P, P, i32, P, S, P],
+        "prism_propose_int2": [sp, P, P, P, i32, P, P, P, S, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -155,6 +158,19 @@ def quantize_k(p: Problem, k, kq, k_scale, tok_rows=None, ws=None, stream=None):
 def propose(p: Problem, q, kq, k_scale, kappa_p: int, pool, pool_cnt, ws, stream=None):
     _check(_lib.prism_propose(p.ref, _ptr(q), _ptr(kq), _ptr(k_scale), kappa_p, _ptr(pool),
                               _ptr(pool_cnt), _ptr(ws), _nbytes(ws), _stream(stream)), "propose")
+
+
+def quantize_k_int2(p: Problem, k, codes, params, tok_rows=None, ws=None, stream=None):
+    """INT2 keys: codes [Hkv][T][d/4] uint8, params [Hkv][T][d/32][2] int16/uint16 (fp16 bits of step, zero point)."""
+    n = 0 if tok_rows is None else int(tok_rows.numel())
+    _check(_lib.prism_quantize_k_int2(p.ref, _ptr(k), _ptr(codes), _ptr(params), _ptr(tok_rows), n,
+                                      _ptr(ws), _nbytes(ws), _stream(stream)), "quantize_k_int2")
+
+
+def propose_int2(p: Problem, q, codes, params, kappa_p: int, pool, pool_cnt, ws, stream=None):
+    _check(_lib.prism_propose_int2(p.ref, _ptr(q), _ptr(codes), _ptr(params), kappa_p, _ptr(pool),
+                                   _ptr(pool_cnt), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "propose_int2")
 
 
 def refine(p: Problem, q, k, pool, pool_cnt, kappa_p: int, kappa: int, idx, cnt, ws, logits=None,

@@ -540,3 +540,87 @@ def test_refine_decode_large_ties(P, kp, kap):
         assert np.array_equal(_np(idx)[0, h], np.arange(0, 4 * kap, 4))
     oout, _ = pipeline.attend_layer(q, k, v, [0, 40000], _np(idx), _np(cnt), 0.1)
     assert np.abs(_np(out) - oout).max() <= 2e-3
+
+
+# ------------------------------------------------------------------ INT2 keys
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("bf16", 64), ("f32", 128)])
+def test_quantize_int2_bit_exact(P, dtype, d):
+    seqlens, hq, hkv = [3000, 1], 8, 2
+    prob = problem(P, seqlens, hq, hkv, d, dtype)
+    _, k, _ = make_case(seqlens, hq, hkv, d, dtype, seed=24, scale_rows=True)
+    k[0, 5] = 0.0            # a constant (zero) row: step 0
+    k[1, 9, :32] = -0.0      # signed zeros in one group
+    k[1, 9, 32:64] = 3.0
+    T = prob.total_tokens
+    codes = torch.full((hkv, T, d // 4), 0xAB, dtype=torch.uint8, device=DEV)
+    params = torch.full((hkv, T, d // 32, 2), -1, dtype=torch.int16, device=DEV)
+    ws = ws_for(P, prob, P.OP_QUANTIZE)
+    P.quantize_k_int2(prob, k, codes, params, ws=ws)
+    torch.cuda.synchronize()
+    assert P.get_device_status(ws) == 0
+    oc, op = oracle.quantize_int2_rows(_np(k).reshape(hkv * T, d))
+    assert np.array_equal(codes.cpu().numpy().reshape(hkv * T, d // 4), oc)
+    assert np.array_equal(params.cpu().numpy().view(np.uint16).reshape(hkv * T, d // 32, 2), op)
+    # only the listed rows change when tok_rows is given
+    rows = torch.tensor([0, 2999], dtype=torch.int32, device=DEV)
+    codes2 = torch.zeros_like(codes)
+    params2 = torch.zeros_like(params)
+    P.quantize_k_int2(prob, k, codes2, params2, tok_rows=rows, ws=ws)
+    torch.cuda.synchronize()
+    c2 = codes2.cpu().numpy()
+    assert np.array_equal(c2[:, [0, 2999]], codes.cpu().numpy()[:, [0, 2999]])
+    assert not c2[:, 1:2999].any()
+
+
+INT2_CASES = [
+    ([8192], 32, 8, 2048),
+    ([5000, 1031, 0, 300], 8, 2, 1024),
+    ([40000], 16, 4, 4096),
+    ([1024, 1025], 8, 2, 1024),
+]
+
+
+@pytest.mark.parametrize("case", INT2_CASES, ids=lambda c: f"{c[0]}-{c[1]}/{c[2]}-kp{c[3]}")
+def test_propose_int2_vs_oracle(P, case):
+    seqlens, hq, hkv, kp = case
+    d = 128
+    prob = problem(P, seqlens, hq, hkv, d, "bf16")
+    q, k, _ = make_case(seqlens, hq, hkv, d, "bf16", seed=25)
+    T = prob.total_tokens
+    codes = torch.zeros((hkv, T, d // 4), dtype=torch.uint8, device=DEV)
+    params = torch.zeros((hkv, T, d // 32, 2), dtype=torch.int16, device=DEV)
+    P.quantize_k_int2(prob, k, codes, params)
+    pool = torch.full((len(seqlens), hkv, kp), -7, dtype=torch.int32, device=DEV)
+    cnt = torch.full((len(seqlens), hkv), -7, dtype=torch.int32, device=DEV)
+    ws = ws_for(P, prob, P.OP_PROPOSE, kp)
+    P.propose_int2(prob, q, codes, params, kp, pool, cnt, ws)
+    torch.cuda.synchronize()
+    assert P.get_device_status(ws) == 0
+    gscores = _np(ws[256:256 + hkv * T * 4].view(torch.float32)).reshape(hkv, T)
+    opool, ocnt, oscores = pipeline.propose_layer_int2(q, codes.cpu().numpy(), params.cpu().numpy().view(np.uint16),
+                                                       prob.cu_host.tolist(), kp)
+    gp, gc = _np(pool), _np(cnt)
+    assert np.array_equal(gc, ocnt)
+    cu = prob.cu_host
+    for b in range(len(seqlens)):
+        for h in range(hkv):
+            s = oscores[(b, h)]
+            n = int(ocnt[b, h])
+            if n:
+                gs = gscores[h, cu[b]:cu[b + 1]]
+                assert np.allclose(gs, s, rtol=2e-6, atol=2e-6 * np.abs(s).max()), (b, h)
+            check_index_set(gp[b, h, :n], opool[b, h, :n], lambda t: s[t], f"int2 pool b{b} h{h}")
+            assert np.all(gp[b, h, n:] == -1)
+
+
+def test_propose_int2_unsupported_shapes(P):
+    prob = problem(P, [1000], 8, 2, 64, "bf16")
+    q, k, _ = make_case([1000], 8, 2, 64, "bf16", seed=26)
+    codes = torch.zeros((2, 1000, 16), dtype=torch.uint8, device=DEV)
+    params = torch.zeros((2, 1000, 2, 2), dtype=torch.int16, device=DEV)
+    pool = torch.zeros((1, 2, 100), dtype=torch.int32, device=DEV)
+    cnt = torch.zeros((1, 2), dtype=torch.int32, device=DEV)
+    with pytest.raises(P.PrismError) as e:
+        P.propose_int2(prob, q, codes, params, 100, pool, cnt, ws_for(P, prob, P.OP_PROPOSE, 100))
+    assert e.value.status == P.ERR_UNSUPPORTED

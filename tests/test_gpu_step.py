@@ -131,3 +131,50 @@ def test_step_full_size_sampled(prism_lib, name):
         _check_layer(dec, cfg2, lay.index, lay, kqs[0], scs[0], rows)
     del layers, dec
     torch.cuda.empty_cache()
+
+
+def test_step_int2_keys_c8k_every_row(prism_lib):
+    """A whole c8k step with INT2 proposal keys: pools against the INT2
+    oracle, then refine and attention as in the int8 path."""
+    P = prism_lib
+    cfg = workload.config("c8k")
+    layers = list(workload.generate(cfg, DEV))
+    dec = PrismDecoder(cfg.seqlens, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, P.BF16,
+                       cfg.num_layers, cfg.group, cfg.kappa_p, cfg.kappa, device=DEV, keys="int2")
+    codes, params = {}, {}
+    for lay in layers:
+        if cfg.is_proposal(lay.index):
+            H, T, D = lay.k.shape
+            codes[lay.index] = torch.zeros((H, T, D // 4), dtype=torch.uint8, device=DEV)
+            params[lay.index] = torch.zeros((H, T, D // 32, 2), dtype=torch.int16, device=DEV)
+            P.quantize_k_int2(dec.p, lay.k, codes[lay.index], params[lay.index])
+    dec.step([x.q for x in layers], [x.k for x in layers], [x.v for x in layers], codes, params)
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    cu = cfg.cu_seqlens
+    rows = _all_rows(cfg)
+    for lay in layers:
+        l = lay.index
+        _invariants(dec, cfg, l)
+        src = l - l % cfg.group
+        if l == src:
+            opool, ocnt, osc = pipeline.propose_layer_int2(lay.q, codes[l].cpu().numpy(),
+                                                           params[l].cpu().numpy().view(np.uint16), cu,
+                                                           cfg.kappa_p, rows=rows)
+            gpool, gpc = _np(dec.pool[src]), _np(dec.pool_cnt[src])
+            for (b, h) in rows:
+                n = int(ocnt[b, h])
+                assert int(gpc[b, h]) == n
+                check_index_set(gpool[b, h, :n], opool[b, h, :n], lambda t: osc[(b, h)][t],
+                                f"L{l} int2 pool {b},{h}")
+        # refine + attention on the GPU's own pool (cascade control)
+        gpool, gpc = _np(dec.pool[src]), _np(dec.pool_cnt[src])
+        gidx, gcnt = _np(dec.idx[l]), _np(dec.cnt[l])
+        oidx, ocnt, orr = pipeline.refine_layer(lay.q, lay.k, cu, gpool, gpc, cfg.kappa, rows=rows)
+        for (b, h) in rows:
+            n = int(gpc[b, h])
+            r = dict(zip(gpool[b, h, :n].tolist(), orr[(b, h)].tolist()))
+            c = int(ocnt[b, h])
+            check_index_set(gidx[b, h, :c], oidx[b, h, :c], lambda t: r[t], f"L{l} idx {b},{h}")
+        oout, _ = pipeline.attend_layer(lay.q, lay.k, lay.v, cu, gidx, gcnt, dec.scale, rows=rows)
+        assert np.abs(_np(dec.out[l]) - oout).max() <= atol_for(cfg.dtype)
