@@ -14,11 +14,12 @@
 //      mma.sync (bf16 operands, fp32 accumulation, exact bf16 products) from
 //      ldmatrix fragments -- an fp32 cache takes a CUDA-core path; the logits
 //      stay in shared memory;
-//   2. the selection key of a member is ord(max_g q_g . k); the first 12
-//      bits of every key go into one cluster histogram held by rank 0
-//      (remote shared-memory atomics, two 16-bit counts per word);
-//   3. rank 0 finds the bin of that histogram holding the kappa-th largest
-//      key and every CTA reads the answer.  Unless the whole bin is taken,
+//   2. the selection key of a member is ord(max_g q_g . k); its first 12
+//      bits go into the CTA's own histogram (two 16-bit counts per word);
+//   3. CTA c sums slice c of every CTA's histogram (distributed shared
+//      memory reads, no remote atomics), and every CTA finds, from the
+//      slice totals and then the right slice, the bin holding the kappa-th
+//      largest key.  Unless the whole bin is taken,
 //      the keys in it build a histogram of the next 10 bits in rank 0, and
 //      then of the last 10: this gives the threshold prefix P (12, 22 or 32
 //      bits) and how many keys at P are taken.  Keys at P are taken in
@@ -422,6 +423,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
   __shared__ int s_dig[3];
   __shared__ int s_cnt[2];        // this CTA's keys above / at the threshold prefix
   __shared__ int s_mine[2];       // output offset, keys at the prefix taken
+  __shared__ int s_slice;         // keys in this CTA's slice of the first-digit bins
   __shared__ int s_wa[kWarps], s_wb[kWarps];
   __shared__ float s_red[kWarps][GP];
   __shared__ __align__(16) float part[PART];  // this CTA's partial o, m, l
@@ -465,8 +467,8 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
     if (!ok) flag_status(a.status, PRISM_DEV_BAD_INDEX);
     spos[i] = ok ? p : -1;
   }
-  if (rank == 0 && !all)
-    for (int i = tid; i < kHistWords; i += kThreads) hist[i] = 0u;
+  if (!all)  // this CTA's first-digit histogram; rank 0 also the cluster's later digits
+    for (int i = tid; i < (rank == 0 ? kHistWords : kH2); i += kThreads) hist[i] = 0u;
   __syncthreads();
   cluster_arrive();  // rank 0's histograms are cleared once every CTA has arrived
   RowStream<T, D> kst(kb, knew, L - 1, spos, nullptr, m, ring);
@@ -525,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
     }
     const uint32_t key = ord_key(best);
     keys[i] = key;
-    if (!all) hist_push(h0 + kH1, key >> 20);
+    if (!all) hist_push(hist + kH1, key >> 20);  // this CTA's own histogram
   }
 
   // ---- 3. threshold prefix P: keys with (key >> shift) > P are taken, and
@@ -546,7 +548,73 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
       __syncthreads();
     };
     int r = k;
-    resolve(hist + kH1, kBins1, r);
+    if (CL == 1) {
+      resolve(hist + kH1, kBins1, r);
+    } else {
+      // first digit without remote atomics: CTA c sums slice c of every CTA's
+      // histogram (words c * WS .. + WS) into its ring, with the slice total;
+      // then every CTA picks the slice, and the bin within it, that holds
+      // the r-th largest key
+      const int WS = (kBins1 / 2) / CL;  // packed words per slice
+      uint32_t* sw = reinterpret_cast<uint32_t*>(ring);
+      __syncthreads();
+      cluster.sync();  // S1: every CTA's histogram is complete
+      int part = 0;
+      for (int x = tid; x < WS; x += kThreads) {
+        uint32_t acc = 0u;  // 16-bit halves: a bin never holds more than kappa_p keys
+        for (int c = 0; c < CL; ++c) acc += cluster.map_shared_rank(hist + kH1, c)[rank * WS + x];
+        sw[x] = acc;
+        part += (int)(acc & 0xFFFFu) + (int)(acc >> 16);
+      }
+      int tot;
+      block_excl_scan(part, scratch, &tot);
+      if (tid == 0) s_slice = tot;
+      cluster.sync();  // S1b: every slice and its total are ready
+      if (warp == 0) {
+        const int t = lane < CL ? *cluster.map_shared_rank(&s_slice, lane) : 0;
+        // slices rank in descending bin order: count above slice `lane`
+        const int incl = warp_incl_scan(t);
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        const int above = total - incl;
+        const unsigned hit = __ballot_sync(0xffffffffu, lane < CL && above < r && r <= above + t);
+        const int src = hit ? __ffs(hit) - 1 : 0;  // always exactly one lane when counts are right
+        const int above_src = __shfl_sync(0xffffffffu, above, src);
+        if (lane == 0) {
+          s_dig[0] = src;
+          s_dig[1] = above_src;
+        }
+      }
+      __syncthreads();
+      const int src = s_dig[0], above_s = s_dig[1];
+      const uint32_t* swr = reinterpret_cast<const uint32_t*>(cluster.map_shared_rank(ring, src));
+      const int nb = 2 * WS;         // bins in the slice
+      const int per = (nb + kThreads - 1) / kThreads;
+      uint32_t cnt[8];
+      int v = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int bin = tid * per + j;
+        cnt[j] = 0u;
+        if (j < per && bin < nb) cnt[j] = (swr[bin >> 1] >> ((bin & 1) * 16)) & 0xFFFFu;
+        v += (int)cnt[j];
+      }
+      int total2;
+      const int excl = block_excl_scan(v, scratch, &total2);
+      int above = above_s + total2 - excl - v;
+      const int rr = r;
+      __syncthreads();
+#pragma unroll
+      for (int j = 7; j >= 0; --j) {
+        const int c = (int)cnt[j];
+        if (j < per && above < rr && rr <= above + c) {
+          s_dig[0] = src * nb + tid * per + j;
+          s_dig[1] = above;
+          s_dig[2] = c;
+        }
+        above += c;
+      }
+      __syncthreads();
+    }
     P = (uint32_t)s_dig[0];
     shift = 20;
     r -= s_dig[1];
