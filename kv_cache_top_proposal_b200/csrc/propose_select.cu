@@ -9,14 +9,16 @@
 // slice r of positions and keeps its keys in registers (KPT per thread,
 // coalesced: key u of thread t is slice position u * kThreads + t):
 //   1. every CTA reads the row's histogram and locates the bin holding the
-//      kappa_p-th largest key (same answer in every CTA).  Each CTA hands
-//      rank 0 its keys in that bin, in position order, with its count above
-//      the bin; rank 0 ranks these candidates exactly (two more 10-bit
-//      digits over its own histograms) and returns the threshold key T,
-//      each CTA's output offset and its share of the keys equal to T ("lower
-//      index wins").  If a CTA has more candidates than rank 0 holds, the
-//      digits are resolved over the cluster instead, one barrier per digit;
-//   2. every CTA writes its kept positions in ascending order (ballot counts
+//      kappa_p-th largest key (same answer in every CTA).  Unless the whole
+//      bin is taken, the CTAs histogram the next 10 bits of their keys in
+//      it, each into its own shared memory; CTA c sums slice c of those
+//      histograms over distributed shared memory and every CTA finds the
+//      next bin from the slice totals and the right slice; then the last 10
+//      bits.  This gives the threshold prefix P and how many keys at P are
+//      taken, in position order ("lower index wins");
+//   2. the CTAs exchange their counts above and at P, which gives each one
+//      its share of the keys at P and its output offset;
+//   3. every CTA writes its kept positions in ascending order (ballot counts
 //      per (key block, warp), one block scan, placement).
 #include <cooperative_groups.h>
 
@@ -36,7 +38,6 @@ constexpr int kKPT = 16;                      // keys per thread
 constexpr int kMaxSlice = kKPT * kThreads;    // keys per CTA
 constexpr int kHist = 4096;                   // first digit (from the scorer)
 constexpr int kBins = 1024;                   // second and third digits
-constexpr int kCandCap = 512;                 // first-digit candidates per CTA ranked by rank 0
 
 struct PSArgs {
   const float* scores;   // [Hkv][T]
@@ -97,95 +98,16 @@ __device__ __forceinline__ void scan_table(int* tab, int base, int* scratch) {
   __syncthreads();
 }
 
-// Rank 0: the candidates are every CTA's keys of first-digit bin b1, CTA w's
-// in cand[w * kCandCap ..] in position order, cnt[3w] of them, with
-// cnt[3w + 1] of its keys above the bin.  Finds the r-th largest candidate T
-// (two 10-bit digits over local histograms) and writes fin = {0, T, then per
-// CTA (output offset, keys equal to T it takes, keys equal to T it holds)}:
-// keys equal to T are taken in CTA order, then position order.  fin[0] = 1
-// (nothing else written) when a CTA had more than kCandCap candidates.
-// Whole CTA.
-__device__ void rank_candidates(const uint2* cand, uint32_t b1, int r, uint32_t* h2, uint32_t* h3,
-                                int* scratch, int* dig, const int* cnt, int* fin) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  __shared__ int s_over;
-  __shared__ int s_ge[kCL][2];
-  if (tid == 0) s_over = 0;
-  __syncthreads();
-  if (tid < kCL && cnt[3 * tid] > kCandCap) s_over = 1;
-  __syncthreads();
-  if (s_over) {
-    if (tid == 0) fin[0] = 1;
-    __syncthreads();
-    return;
-  }
-  constexpr int WPR = kWarps / kCL;  // warps per CTA region
-  const int w = warp / WPR, sub = warp % WPR;
-  const int nw = cnt[3 * w];
-  const uint2* cw = cand + w * kCandCap;
-  for (int j = sub * 32 + lane; j < nw; j += WPR * 32) atomicAdd(h2 + ((cw[j].x >> 10) & (kBins - 1)), 1u);
-  __syncthreads();
-  find_digit<kBins / kThreads>([&](int bin) { return h2[bin]; }, r, scratch, dig);
-  const uint32_t p2 = (b1 << 10) | (uint32_t)dig[0];
-  r -= dig[1];
-  for (int j = sub * 32 + lane; j < nw; j += WPR * 32) {
-    const uint32_t key = cw[j].x;
-    if ((key >> 10) == p2) atomicAdd(h3 + (key & (kBins - 1)), 1u);
-  }
-  __syncthreads();
-  find_digit<kBins / kThreads>([&](int bin) { return h3[bin]; }, r, scratch, dig);
-  const uint32_t T = (p2 << 10) | (uint32_t)dig[0];
-  r -= dig[1];  // keys equal to T to take, in order
-  if (tid < kCL * 2) (&s_ge[0][0])[tid] = 0;
-  __syncthreads();
-  {
-    int gt = 0, eq = 0;
-    for (int j = sub * 32 + lane; j < nw; j += WPR * 32) {
-      const uint32_t key = cw[j].x;
-      gt += key > T;
-      eq += key == T;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      gt += __shfl_xor_sync(0xffffffffu, gt, o);
-      eq += __shfl_xor_sync(0xffffffffu, eq, o);
-    }
-    if (lane == 0) {
-      atomicAdd(&s_ge[w][0], gt);
-      atomicAdd(&s_ge[w][1], eq);
-    }
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const int gt = lane < kCL ? cnt[3 * lane + 1] + s_ge[lane][0] : 0;
-    const int eq = lane < kCL ? s_ge[lane][1] : 0;
-    const int ebefore = warp_incl_scan(eq) - eq;
-    const int take = min(max(r - ebefore, 0), eq);
-    const int nsel = gt + take;
-    const int before = warp_incl_scan(nsel) - nsel;
-    if (lane < kCL) {
-      fin[2 + 3 * lane] = before;
-      fin[3 + 3 * lane] = take;
-      fin[4 + 3 * lane] = eq;
-    }
-    if (lane == 0) {
-      fin[0] = 0;
-      fin[1] = (int)T;
-    }
-  }
-  __syncthreads();
-}
-
 __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArgs a) {
-  extern __shared__ __align__(16) uint2 cand[];      // rank 0: [kCL][kCandCap] (key, position)
-  __shared__ __align__(16) uint32_t hist2[kBins];  // rank 0: digit-2 counts
-  __shared__ __align__(16) uint32_t hist3[kBins];  // rank 0: digit-3 counts
+  __shared__ __align__(16) uint32_t hist2[kBins];  // this CTA's digit-2 counts
+  __shared__ __align__(16) uint32_t hist3[kBins];  // this CTA's digit-3 counts
   __shared__ int tabE[kKPT * kWarps];  // per (key block, warp): keys at P, then their prefix
   __shared__ int tabK[kKPT * kWarps];  // per (key block, warp): kept keys, then output slots
+  __shared__ uint32_t s_sw[kBins / kCL];  // this CTA's slice of the cluster's digit counts
+  __shared__ int s_slice;
   __shared__ int scratch[33];
   __shared__ int s_dig[3];
-  __shared__ int s_cnt[3 * kCL];    // rank 0: per CTA, candidates, keys above, (spare)
-  __shared__ int s_fin[2 + 3 * kCL];  // rank 0: mode, T, per CTA (offset, share, at T)
+  __shared__ int s_cnt[2];   // this CTA's keys above / at the prefix
   __shared__ int s_mine[3];  // output offset, keys at the prefix taken, keys at the prefix
 
   cg::cluster_group cluster = cg::this_cluster();
@@ -215,16 +137,12 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
     return;
   }
   const int k = a.kp;
-  uint32_t* h2 = cluster.map_shared_rank(hist2, 0);
-  uint32_t* h3 = cluster.map_shared_rank(hist3, 0);
-  if (rank == 0) {
-    for (int i = tid; i < kBins; i += kThreads) {
-      hist2[i] = 0u;
-      hist3[i] = 0u;
-    }
+  for (int i = tid; i < kBins; i += kThreads) {
+    hist2[i] = 0u;
+    hist3[i] = 0u;
   }
   __syncthreads();
-  cluster_arrive();  // rank 0's histograms are cleared once every CTA has arrived
+  cluster_arrive();  // pairs with the wait below (every CTA is running)
 
   // ---- the slice's keys, kKPT loads in flight per thread
   uint32_t key[kKPT];
@@ -243,95 +161,81 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
 
   // ---- 1. threshold: keys with (key >> shift) > P are taken, and the first
   // rtie keys with (key >> shift) == P in position order.  Every CTA finds
-  // the first digit's bin b1 from the row's histogram.  Each CTA hands rank 0
-  // its keys in b1 (in position order) and its count above b1; rank 0 ranks
-  // the candidates exactly and returns the threshold T with every CTA's
-  // offset and share of the keys equal to T (then P = T, shift = 0).  When a
-  // CTA has more than kCandCap candidates, the last two digits are resolved
-  // over the whole cluster instead (remote histograms, one digit per round).
+  // the first digit's bin b1 from the row's histogram.  Unless the whole
+  // bin is taken, each CTA counts the next 10 bits of its keys in b1 into its
+  // own histogram; CTA c sums slice c of all of them (distributed shared
+  // memory reads, no remote atomics) and every CTA finds the next bin from
+  // the slice totals and the right slice; then the same for the last 10
+  // bits.  Finally the CTAs exchange their counts above and at P.
   const uint32_t* gh = a.hist + (int64_t)row * kHist;
   find_digit<kHist / kThreads>([&](int bin) { return __ldcg(gh + bin); }, k, scratch, s_dig);
-  const uint32_t b1 = (uint32_t)s_dig[0];
+  uint32_t P = (uint32_t)s_dig[0];
+  int shift = 20;
   const int c1 = s_dig[2];
   int r = k - s_dig[1];
   cluster_wait();
-  {
-    // candidates in position order: counts per (key block, warp), one scan
-    int gt1 = 0;
-#pragma unroll
-    for (int u = 0; u < kKPT; ++u) {
-      const bool c = in(u) && (key[u] >> 20) == b1;
-      gt1 += in(u) && (key[u] >> 20) > b1;
-      const unsigned bal = __ballot_sync(0xffffffffu, c);
-      if (lane == 0) tabE[u * kWarps + warp] = __popc(bal);
-    }
+  auto cluster_digit = [&](const uint32_t* hl, int rr) {
+    constexpr int WS = kBins / kCL;  // bins per slice
     __syncthreads();
-    const int v = tid < kKPT * kWarps ? tabE[tid] : 0;
-    int ncand;
-    const int excl = block_excl_scan(v, scratch, &ncand);
-    if (tid < kKPT * kWarps) tabE[tid] = excl;
-    int gtot;
-    block_excl_scan(gt1, scratch, &gtot);  // (also orders the table writes)
-    uint2* region = cluster.map_shared_rank(cand, 0) + rank * kCandCap;
-#pragma unroll
-    for (int u = 0; u < kKPT; ++u) {
-      const bool c = in(u) && (key[u] >> 20) == b1;
-      const unsigned bal = __ballot_sync(0xffffffffu, c);
-      if (c) {
-        const int o = tabE[u * kWarps + warp] + __popc(bal & lt);
-        if (o < kCandCap) region[o] = make_uint2(key[u], (uint32_t)(lo + u * kThreads + tid));
+    cluster.sync();  // every CTA's histogram is complete
+    int part = 0;
+    for (int x = tid; x < WS; x += kThreads) {
+      uint32_t acc = 0u;
+      for (int c = 0; c < kCL; ++c) acc += cluster.map_shared_rank(hl, c)[rank * WS + x];
+      s_sw[x] = acc;
+      part += (int)acc;
+    }
+    int tot;
+    block_excl_scan(part, scratch, &tot);
+    if (tid == 0) s_slice = tot;
+    cluster.sync();  // every slice and its total are ready
+    if (warp == 0) {
+      const int t = lane < kCL ? *cluster.map_shared_rank(&s_slice, lane) : 0;
+      const int incl = warp_incl_scan(t);  // slices rank in descending bin order
+      const int above = __shfl_sync(0xffffffffu, incl, 31) - incl;
+      const unsigned hit = __ballot_sync(0xffffffffu, lane < kCL && above < rr && rr <= above + t);
+      const int src = hit ? __ffs(hit) - 1 : 0;  // exactly one lane when counts are right
+      const int above_src = __shfl_sync(0xffffffffu, above, src);
+      if (lane == 0) {
+        s_dig[0] = src;
+        s_dig[1] = above_src;
       }
     }
-    if (tid == 0) {
-      int* cm = cluster.map_shared_rank(s_cnt, 0);
-      cm[3 * rank] = ncand;
-      cm[3 * rank + 1] = gtot;
-    }
-  }
-  cluster.sync();  // S1: every slice's candidates and count are with rank 0
-  if (rank == 0) rank_candidates(cand, b1, r, hist2, hist3, scratch, s_dig, s_cnt, s_fin);
-  cluster.sync();  // S2: rank 0's answer is ready
-  uint32_t P;
-  int shift;
-  {
-    if (tid < 5) {
-      const int* f = cluster.map_shared_rank(s_fin, 0);
-      const int v = tid == 0 ? f[0] : tid == 1 ? f[1] : f[tid + 3 * rank];
-      if (tid < 2) s_dig[tid] = v;
-      else s_mine[tid - 2] = v;
+    __syncthreads();
+    const int src = s_dig[0], above_s = s_dig[1];
+    const uint32_t* swr = cluster.map_shared_rank(s_sw, src);
+    const int v = tid < WS ? (int)swr[tid] : 0;  // one bin per thread (WS <= kThreads)
+    int total2;
+    const int excl = block_excl_scan(v, scratch, &total2);
+    const int above = above_s + total2 - excl - v;
+    if (tid < WS && above < rr && rr <= above + v) {
+      s_dig[0] = src * WS + tid;
+      s_dig[1] = above;
+      s_dig[2] = v;
     }
     __syncthreads();
-  }
-  const bool ranked = s_dig[0] == 0;
-  if (ranked) {
-    P = (uint32_t)s_dig[1];
-    shift = 0;
-  } else {
-    P = b1;
-    shift = 20;
-    __syncthreads();  // s_dig is rewritten below
-    if (r < c1) {  // part of the bin: the second digit of its keys
+  };
+  if (r < c1) {  // part of the bin: the second digit of its keys
+#pragma unroll
+    for (int u = 0; u < kKPT; ++u)
+      if (in(u) && (key[u] >> 20) == P) atomicAdd(hist2 + ((key[u] >> 10) & (kBins - 1)), 1u);
+    cluster_digit(hist2, r);
+    P = (P << 10) | (uint32_t)s_dig[0];
+    shift = 10;
+    r -= s_dig[1];
+    if (r < s_dig[2]) {  // the last digit
 #pragma unroll
       for (int u = 0; u < kKPT; ++u)
-        if (in(u) && (key[u] >> 20) == P) atomicAdd(h2 + ((key[u] >> 10) & (kBins - 1)), 1u);
-      cluster.sync();
-      find_digit<kBins / kThreads>([&](int bin) { return h2[bin]; }, r, scratch, s_dig);
+        if (in(u) && (key[u] >> 10) == P) atomicAdd(hist3 + (key[u] & (kBins - 1)), 1u);
+      cluster_digit(hist3, r);
       P = (P << 10) | (uint32_t)s_dig[0];
-      shift = 10;
+      shift = 0;
       r -= s_dig[1];
-      if (r < s_dig[2]) {  // the last digit
-#pragma unroll
-        for (int u = 0; u < kKPT; ++u)
-          if (in(u) && (key[u] >> 10) == P) atomicAdd(h3 + (key[u] & (kBins - 1)), 1u);
-        cluster.sync();
-        find_digit<kBins / kThreads>([&](int bin) { return h3[bin]; }, r, scratch, s_dig);
-        P = (P << 10) | (uint32_t)s_dig[0];
-        shift = 0;
-        r -= s_dig[1];
-      }
     }
-    const int rtie = r;
-    // counts above / at P, then every CTA's, in rank order
+  }
+  const int rtie = r;
+  // counts above / at P, then every CTA's, in rank order
+  {
     int gt = 0, eq = 0;
 #pragma unroll
     for (int u = 0; u < kKPT; ++u) {
@@ -347,26 +251,26 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
       s_cnt[0] = tot >> 16;
       s_cnt[1] = tot & 0xFFFF;
     }
-    cluster.sync();  // every CTA's counts are published
-    if (warp == 0) {
-      int g_s = 0, e_s = 0;
-      if (lane < kCL) {
-        const int* rc = cluster.map_shared_rank(s_cnt, lane);
-        g_s = rc[0];
-        e_s = rc[1];
-      }
-      const int ebefore = warp_incl_scan(e_s) - e_s;
-      const int take = min(max(rtie - ebefore, 0), e_s);
-      const int nsel = g_s + take;
-      const int before = warp_incl_scan(nsel) - nsel;
-      if (lane == rank) {
-        s_mine[0] = before;
-        s_mine[1] = take;
-        s_mine[2] = e_s;
-      }
-    }
-    __syncthreads();
   }
+  cluster.sync();  // every CTA's counts are published
+  if (warp == 0) {
+    int g_s = 0, e_s = 0;
+    if (lane < kCL) {
+      const int* rc = cluster.map_shared_rank(s_cnt, lane);
+      g_s = rc[0];
+      e_s = rc[1];
+    }
+    const int ebefore = warp_incl_scan(e_s) - e_s;
+    const int take = min(max(rtie - ebefore, 0), e_s);
+    const int nsel = g_s + take;
+    const int before = warp_incl_scan(nsel) - nsel;
+    if (lane == rank) {
+      s_mine[0] = before;
+      s_mine[1] = take;
+      s_mine[2] = e_s;
+    }
+  }
+  __syncthreads();
   const int off = s_mine[0], take = s_mine[1];
   const bool part = take < s_mine[2];  // the slice keeps only some of its keys at P
 
@@ -434,13 +338,10 @@ cudaError_t launch_propose_select(const Dims& d, const float* scores, const uint
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(rows * kCL));
   cfg.blockDim = dim3(kThreads);
-  const int smem = kCL * kCandCap * (int)sizeof(uint2);
-  cudaError_t e = cudaFuncSetAttribute(propose_select_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e =
+      cudaFuncSetAttribute(propose_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(propose_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  if (e != cudaSuccess) return e;
-  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;

@@ -547,29 +547,27 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
       if (rank != 0 && tid < 3) s_dig[tid] = dig0[tid];
       __syncthreads();
     };
-    int r = k;
-    if (CL == 1) {
-      resolve(hist + kH1, kBins1, r);
-    } else {
-      // first digit without remote atomics: CTA c sums slice c of every CTA's
-      // histogram (words c * WS .. + WS) into its ring, with the slice total;
-      // then every CTA picks the slice, and the bin within it, that holds
-      // the r-th largest key
-      const int WS = (kBins1 / 2) / CL;  // packed words per slice
+    // Without remote atomics: every CTA holds a packed histogram hl of nb
+    // bins; CTA c sums slice c of all of them into its ring, with the slice
+    // total; then every CTA finds, from the slice totals and the right
+    // slice, the bin holding the r-th largest key (s_dig = bin, keys above
+    // it, keys in it).  Two cluster barriers; the first orders the hl writes.
+    auto cluster_digit = [&](const uint32_t* hl, int nb, int r) {
+      const int WS = (nb / 2) / CL;  // packed words per slice
       uint32_t* sw = reinterpret_cast<uint32_t*>(ring);
       __syncthreads();
-      cluster.sync();  // S1: every CTA's histogram is complete
+      cluster.sync();  // every CTA's histogram is complete
       int part = 0;
       for (int x = tid; x < WS; x += kThreads) {
         uint32_t acc = 0u;  // 16-bit halves: a bin never holds more than kappa_p keys
-        for (int c = 0; c < CL; ++c) acc += cluster.map_shared_rank(hist + kH1, c)[rank * WS + x];
+        for (int c = 0; c < CL; ++c) acc += cluster.map_shared_rank(hl, c)[rank * WS + x];
         sw[x] = acc;
         part += (int)(acc & 0xFFFFu) + (int)(acc >> 16);
       }
       int tot;
       block_excl_scan(part, scratch, &tot);
       if (tid == 0) s_slice = tot;
-      cluster.sync();  // S1b: every slice and its total are ready
+      cluster.sync();  // every slice and its total are ready
       if (warp == 0) {
         const int t = lane < CL ? *cluster.map_shared_rank(&s_slice, lane) : 0;
         // slices rank in descending bin order: count above slice `lane`
@@ -587,43 +585,56 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
       __syncthreads();
       const int src = s_dig[0], above_s = s_dig[1];
       const uint32_t* swr = reinterpret_cast<const uint32_t*>(cluster.map_shared_rank(ring, src));
-      const int nb = 2 * WS;         // bins in the slice
-      const int per = (nb + kThreads - 1) / kThreads;
+      const int sb = 2 * WS;  // bins in the slice
+      const int per = (sb + kThreads - 1) / kThreads;
       uint32_t cnt[8];
       int v = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int bin = tid * per + j;
         cnt[j] = 0u;
-        if (j < per && bin < nb) cnt[j] = (swr[bin >> 1] >> ((bin & 1) * 16)) & 0xFFFFu;
+        if (j < per && bin < sb) cnt[j] = (swr[bin >> 1] >> ((bin & 1) * 16)) & 0xFFFFu;
         v += (int)cnt[j];
       }
       int total2;
       const int excl = block_excl_scan(v, scratch, &total2);
       int above = above_s + total2 - excl - v;
-      const int rr = r;
       __syncthreads();
 #pragma unroll
       for (int j = 7; j >= 0; --j) {
         const int c = (int)cnt[j];
-        if (j < per && above < rr && rr <= above + c) {
-          s_dig[0] = src * nb + tid * per + j;
+        if (j < per && above < r && r <= above + c) {
+          s_dig[0] = src * sb + tid * per + j;
           s_dig[1] = above;
           s_dig[2] = c;
         }
         above += c;
       }
       __syncthreads();
-    }
+    };
+    int r = k;
+    if (CL == 1) resolve(hist + kH1, kBins1, r);
+    else cluster_digit(hist + kH1, kBins1, r);
     P = (uint32_t)s_dig[0];
     shift = 20;
     r -= s_dig[1];
     if (r < s_dig[2]) {  // part of the bin: the second digit of its keys
-      for (int i = tid; i < m; i += kThreads) {
-        const uint32_t key = keys[i];
-        if ((key >> 20) == P) hist_push(h0 + kH2, (key >> 10) & 1023u);
+      if (CL == 1) {
+        for (int i = tid; i < m; i += kThreads) {
+          const uint32_t key = keys[i];
+          if ((key >> 20) == P) hist_push(h0 + kH2, (key >> 10) & 1023u);
+        }
+        resolve(hist + kH2, kBins2, r);
+      } else {
+        // this CTA's own histogram again (no CTA reads the first one any more)
+        for (int i = tid; i < kBins2 / 2; i += kThreads) hist[kH1 + i] = 0u;
+        __syncthreads();
+        for (int i = tid; i < m; i += kThreads) {
+          const uint32_t key = keys[i];
+          if ((key >> 20) == P) hist_push(hist + kH1, (key >> 10) & 1023u);
+        }
+        cluster_digit(hist + kH1, kBins2, r);
       }
-      resolve(hist + kH2, kBins2, r);
       P = (P << 10) | (uint32_t)s_dig[0];
       shift = 10;
       r -= s_dig[1];
