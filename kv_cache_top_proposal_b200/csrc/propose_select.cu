@@ -180,8 +180,12 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
     cluster.sync();  // every CTA's histogram is complete
     int part = 0;
     for (int x = tid; x < WS; x += kThreads) {
+      uint32_t v[kCL];  // every CTA's count, all loads in flight at once
+#pragma unroll
+      for (int c = 0; c < kCL; ++c) v[c] = cluster.map_shared_rank(hl, c)[rank * WS + x];
       uint32_t acc = 0u;
-      for (int c = 0; c < kCL; ++c) acc += cluster.map_shared_rank(hl, c)[rank * WS + x];
+#pragma unroll
+      for (int c = 0; c < kCL; ++c) acc += v[c];
       s_sw[x] = acc;
       part += (int)acc;
     }

@@ -559,8 +559,13 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
       cluster.sync();  // every CTA's histogram is complete
       int part = 0;
       for (int x = tid; x < WS; x += kThreads) {
+        uint32_t v[kMaxCluster];  // every CTA's word, all loads in flight at once
+#pragma unroll
+        for (int c = 0; c < kMaxCluster; ++c)
+          v[c] = c < CL ? cluster.map_shared_rank(hl, c)[rank * WS + x] : 0u;
         uint32_t acc = 0u;  // 16-bit halves: a bin never holds more than kappa_p keys
-        for (int c = 0; c < CL; ++c) acc += cluster.map_shared_rank(hl, c)[rank * WS + x];
+#pragma unroll
+        for (int c = 0; c < kMaxCluster; ++c) acc += v[c];
         sw[x] = acc;
         part += (int)(acc & 0xFFFFu) + (int)(acc >> 16);
       }
@@ -618,23 +623,12 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
     P = (uint32_t)s_dig[0];
     shift = 20;
     r -= s_dig[1];
-    if (r < s_dig[2]) {  // part of the bin: the second digit of its keys
-      if (CL == 1) {
-        for (int i = tid; i < m; i += kThreads) {
-          const uint32_t key = keys[i];
-          if ((key >> 20) == P) hist_push(h0 + kH2, (key >> 10) & 1023u);
-        }
-        resolve(hist + kH2, kBins2, r);
-      } else {
-        // this CTA's own histogram again (no CTA reads the first one any more)
-        for (int i = tid; i < kBins2 / 2; i += kThreads) hist[kH1 + i] = 0u;
-        __syncthreads();
-        for (int i = tid; i < m; i += kThreads) {
-          const uint32_t key = keys[i];
-          if ((key >> 20) == P) hist_push(hist + kH1, (key >> 10) & 1023u);
-        }
-        cluster_digit(hist + kH1, kBins2, r);
+    if (r < s_dig[2]) {  // part of the bin: the second digit of its (few) keys, in rank 0
+      for (int i = tid; i < m; i += kThreads) {
+        const uint32_t key = keys[i];
+        if ((key >> 20) == P) hist_push(h0 + kH2, (key >> 10) & 1023u);
       }
+      resolve(hist + kH2, kBins2, r);
       P = (P << 10) | (uint32_t)s_dig[0];
       shift = 10;
       r -= s_dig[1];
