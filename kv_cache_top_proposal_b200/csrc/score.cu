@@ -575,6 +575,249 @@ __global__ void __launch_bounds__(kThreads, 3) score_tma_kernel(const __grid_con
   flush();
 }
 
+// Integer tensor-core scorer (bf16 queries, d = 128), on the tensor-copy
+// pipeline above.  The int8 codes enter mma.sync.m16n8k32 (s8 x s8 -> s32)
+// as stored: no conversion.  Each query head is held in fixed point,
+// Q = rint(q * 2^sh) with sh per head such that its largest |q| lands in
+// [2^29, 2^30), written as four signed base-256 digits (limbs)
+// Q = l0 2^24 + l1 2^16 + l2 2^8 + l3, each an int8.  A bf16 element within
+// 2^-22 of its head's largest lies on that grid exactly; a smaller one rounds
+// to it (by less than 2^-30 of the largest).  Code x limb products and their
+// sums over a row are exact in int32 (at most 128 * 128 * 127 < 2^21 in
+// magnitude); the four limb sums combine exactly in 64-bit integers and are
+// rounded to fp32 once, then taken back by 2^-sh and multiplied by the row's
+// scale.  Head quad j uses two n8 tiles: column 2 t + i of tile u holds limb
+// 2 u + i of head 4 j + t, so thread (g, t) ends with all four limb sums of
+// head 4 j + t for its rows g and g + 8.  At k-step s thread (g, t) covers
+// features 32 t + 8 s .. + 7: words 2 (s & 1) and 2 (s & 1) + 1 of its chunk
+// s / 2 (the tensor-copy scorer's chunk assignment).
+__device__ __forceinline__ void mma_s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                       uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// low byte of x as a signed value in [-128, 127]
+__device__ __forceinline__ int sbyte(int x) { return ((x & 0xFF) ^ 0x80) - 0x80; }
+
+template <int NH>
+__global__ void __launch_bounds__(kThreads, 3) score_i8_kernel(const __grid_constant__ CUtensorMap tm,
+                                                              ScoreArgs a) {
+  constexpr int D = 128;
+  extern __shared__ unsigned char dsm_raw[];
+  unsigned char* ring =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(ring + kTmaStages * kTmaStageBytes);  // [kHist / 2]
+  int* s_pref = reinterpret_cast<int*>(s_hist + kHist / 2);
+  int* s_cu = s_pref + a.B + 1;
+  __shared__ __align__(8) uint64_t full[kTmaStages];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, tig = lane & 3;
+  for (int i = tid; i <= a.B; i += kThreads) s_cu[i] = a.cu[i];
+  for (int i = tid; i < kHist / 2; i += kThreads) s_hist[i] = 0u;
+  if (tid == 0) {
+    for (int i = 0; i < kTmaStages; ++i) mbar_init(&full[i], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  chunk_prefix(a.cu, a.B, kStageRows, s_pref);  // ends with __syncthreads
+  const int per_head = s_pref[a.B];
+  const int64_t total = (int64_t)a.Hkv * per_head;
+  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
+  const int64_t s_begin = total * blockIdx.x / gridDim.x;
+  const int64_t s_end = total * (blockIdx.x + 1) / gridDim.x;
+  const int nk = (int)(s_end - s_begin);
+  StageIter it_issue, it_comp;
+  {
+    const int h = (int)(s_begin / per_head);
+    const int cc = (int)(s_begin - (int64_t)h * per_head);
+    const int b = find_seq(s_pref, a.B, cc);
+    it_issue = StageIter{h, b, (cc - s_pref[b]) * kStageRows};
+    it_comp = it_issue;
+  }
+  auto issue = [&](int kk) {  // thread 0
+    if (kk < nk) {
+      const int64_t y = (int64_t)it_issue.h * a.T + s_cu[it_issue.b] + it_issue.r0;
+      tma_rows(ring + (kk % kTmaStages) * kTmaStageBytes, &tm, (int)y, &full[kk % kTmaStages]);
+      it_issue.advance(s_cu, a.B);
+    }
+  };
+  if (tid == 0) {
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tm)) : "memory");
+    for (int kk = 0; kk < kTmaStages; ++kk) issue(kk);
+  }
+
+  uint32_t bq[NH][2][4][2];  // [quad][tile][k-step][b0, b1]
+  float us1[NH], us2[NH];    // 2^-sh of head 4 j + tig, as two exact factors
+  int cur_b = -1, cur_h = -1;
+  int hist_row = -1, since_flush = 0;
+  const int rs = warp * 16 + g + 8 * tig;
+  auto load_scale = [&](const StageIter& it) {
+    if (tig >= 2 || it.h >= a.Hkv) return 0.0f;
+    const int L = s_cu[it.b + 1] - s_cu[it.b];
+    if (rs >= min(kStageRows, L - it.r0)) return 0.0f;
+    return __ldg(a.scale + (int64_t)it.h * a.T + s_cu[it.b] + it.r0 + rs);
+  };
+  float sc_next = nk > 0 ? load_scale(it_comp) : 0.0f;
+  auto flush = [&]() {
+    if (a.hist && hist_row >= 0) {
+      uint32_t* gh = a.hist + (int64_t)hist_row * kHist;
+      for (int i = tid; i < kHist / 2; i += kThreads) {
+        const uint32_t c = s_hist[i];
+        if (c) {
+          if (c & 0xFFFFu) atomicAdd(gh + 2 * i, c & 0xFFFFu);
+          if (c >> 16) atomicAdd(gh + 2 * i + 1, c >> 16);
+          s_hist[i] = 0u;
+        }
+      }
+    }
+    since_flush = 0;
+    __syncthreads();
+  };
+#pragma unroll 1
+  for (int kk = 0; kk < nk; ++kk) {
+    const int L = s_cu[it_comp.b + 1] - s_cu[it_comp.b];
+    const int rows = min(kStageRows, L - it_comp.r0);
+    const int64_t rowbase = (int64_t)it_comp.h * a.T + s_cu[it_comp.b] + it_comp.r0;
+    if (it_comp.b != cur_b || it_comp.h != cur_h) {
+      // limbs of the query heads of (b, h): thread (g, tig) supplies column g
+      // of both tiles of each quad -- head 4 j + g / 2, limbs g % 2 and
+      // 2 + g % 2 -- at its features 32 tig .. + 31
+      cur_b = it_comp.b;
+      cur_h = it_comp.h;
+#pragma unroll
+      for (int j = 0; j < NH; ++j) {
+        const int hd = 4 * j + (g >> 1);
+        float qv[32];
+        if (hd < a.G) {
+          const uint4* src = reinterpret_cast<const uint4*>(
+              q + ((int64_t)cur_b * a.Hkv * a.G + (int64_t)cur_h * a.G + hd) * D + 32 * tig);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 w = src[c];
+            qv[8 * c + 0] = bf16lo(w.x); qv[8 * c + 1] = bf16hi(w.x);
+            qv[8 * c + 2] = bf16lo(w.y); qv[8 * c + 3] = bf16hi(w.y);
+            qv[8 * c + 4] = bf16lo(w.z); qv[8 * c + 5] = bf16hi(w.z);
+            qv[8 * c + 6] = bf16lo(w.w); qv[8 * c + 7] = bf16hi(w.w);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) qv[e] = 0.0f;
+        }
+        float mx = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, fabsf(qv[e]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));  // the head's four feature quarters
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        int sh = 0;
+        if (mx > 0.0f) sh = 30 - (((__float_as_int(mx) >> 23) & 0xFF) - 126);  // mx * 2^sh < 2^30
+        // sh lies in [-98, 156]: each factor is an exact power of two
+        const float up1 = pow2f(min(sh, 126)), up2 = pow2f(max(sh - 126, 0));
+        const float dn1 = pow2f(-min(sh, 126)), dn2 = pow2f(-max(sh - 126, 0));
+        const int li = g & 1;
+#pragma unroll
+        for (int st = 0; st < 4; ++st)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t w0 = 0u, w1 = 0u;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int Q = __float2int_rn(qv[8 * st + 4 * hf + e] * up1 * up2);
+              const int d3 = sbyte(Q);
+              const int q1 = (Q - d3) >> 8;
+              const int d2 = sbyte(q1);
+              const int q2 = (q1 - d2) >> 8;
+              const int d1 = sbyte(q2);
+              const int d0 = (q2 - d1) >> 8;
+              const int t0 = li ? d1 : d0, t1 = li ? d3 : d2;  // tile 0: limb li, tile 1: limb 2 + li
+              w0 |= (uint32_t)(t0 & 0xFF) << (8 * e);
+              w1 |= (uint32_t)(t1 & 0xFF) << (8 * e);
+            }
+            bq[j][0][st][hf] = w0;
+            bq[j][1][st][hf] = w1;
+          }
+        // head 4 j + tig was prepared by the lanes with g = 2 tig
+        us1[j] = __shfl_sync(0xffffffffu, dn1, 8 * tig);
+        us2[j] = __shfl_sync(0xffffffffu, dn2, 8 * tig);
+      }
+    }
+    const int row_id = it_comp.b * a.Hkv + it_comp.h;  // CTA-uniform
+    if (row_id != hist_row || since_flush == kTmaFlushStages) {
+      flush();
+      hist_row = row_id;
+    }
+    ++since_flush;
+    it_comp.advance(s_cu, a.B);
+    const float sc = sc_next;
+    if (kk + 1 < nk) sc_next = load_scale(it_comp);
+    const int slot = kk % kTmaStages;
+    {
+      uint32_t it = 0;
+      while (!mbar_try_wait(&full[slot], (uint32_t)(kk / kTmaStages) & 1u)) {
+        if (++it == kWaitLimit) {
+          if (tid == 0) flag_status(a.status, PRISM_DEV_TIMEOUT);
+          break;
+        }
+      }
+    }
+    const unsigned char* buf = ring + slot * kTmaStageBytes;
+    const int t = warp;  // one 16-row tile per warp
+    if (t * 16 < rows) {
+      const bool mine = tig < 2 && rs < rows;  // tig 0: row g, tig 1: row g + 8
+      uint4 cur[2][2];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int r = t * 16 + g + 8 * half;  // r & 7 == g
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch)
+          cur[half][ch] = *reinterpret_cast<const uint4*>(buf + r * 128 + (((2 * tig + ch) ^ g) << 4));
+      }
+      int acc[NH][2][4];
+#pragma unroll
+      for (int j = 0; j < NH; ++j)
+#pragma unroll
+        for (int u = 0; u < 2; ++u) acc[j][u][0] = acc[j][u][1] = acc[j][u][2] = acc[j][u][3] = 0;
+#pragma unroll
+      for (int st = 0; st < 4; ++st) {
+        const uint32_t a0 = word_of(cur[0][st >> 1], 2 * (st & 1));      // row g
+        const uint32_t a2 = word_of(cur[0][st >> 1], 2 * (st & 1) + 1);
+        const uint32_t a1 = word_of(cur[1][st >> 1], 2 * (st & 1));      // row g + 8
+        const uint32_t a3 = word_of(cur[1][st >> 1], 2 * (st & 1) + 1);
+#pragma unroll
+        for (int j = 0; j < NH; ++j)
+#pragma unroll
+          for (int u = 0; u < 2; ++u) mma_s8(acc[j][u], a0, a1, a2, a3, bq[j][u][st][0], bq[j][u][st][1]);
+      }
+      float mA = -INFINITY, mB = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < NH; ++j) {
+        if (4 * j + tig < a.G) {
+          const long long sA = ((long long)(acc[j][0][0] * 256 + acc[j][0][1]) << 16) +
+                               (long long)(acc[j][1][0] * 256 + acc[j][1][1]);
+          const long long sB = ((long long)(acc[j][0][2] * 256 + acc[j][0][3]) << 16) +
+                               (long long)(acc[j][1][2] * 256 + acc[j][1][3]);
+          mA = fmaxf(mA, __ll2float_rn(sA) * us1[j] * us2[j]);
+          mB = fmaxf(mB, __ll2float_rn(sB) * us1[j] * us2[j]);
+        }
+      }
+      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
+      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
+      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
+      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
+      float score = 0.0f;
+      if (mine) {
+        score = sc * (tig == 0 ? mA : mB);
+        a.scores[rowbase + rs] = score;
+      }
+      if (a.hist) warp_hist_add_packed(s_hist, ord_key(score) >> 20, mine);
+    }
+    __syncthreads();  // every warp is done with the stage
+    if (tid == 0) issue(kk + kTmaStages);
+  }
+  flush();
+}
+
 // INT2 scorer (bf16 queries, d = 128).  Per key row and query head the
 // score is sum over 32-feature groups of (S * D + L * Q), with D = q . c over
 // the group's 2-bit codes and Q = sum of q over the group (the dot product
@@ -911,10 +1154,13 @@ cudaError_t run_mma(const Dims& d, const ScoreArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// PRISM_PROPOSE_SCORER=mma selects the cp.async tensor-core scorer instead
-bool use_tma_scorer() {
+// PRISM_PROPOSE_SCORER=mma selects the cp.async fp16 tensor-core scorer,
+// =tma the tensor-copy fp16 one; by default the integer one runs (G <= 8)
+int scorer_choice() {
   const char* e = std::getenv("PRISM_PROPOSE_SCORER");
-  return !(e && std::strcmp(e, "mma") == 0);
+  if (e && std::strcmp(e, "mma") == 0) return 0;
+  if (e && std::strcmp(e, "tma") == 0) return 1;
+  return 2;
 }
 
 // cuTensorMapEncodeTiled from the driver, looked up once
@@ -930,10 +1176,12 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// Launches the TMA scorer when the code tensor can be described by a tensor
-// map (d = 128, 16-byte aligned base); returns false to fall back.
-template <int NT>
-bool run_tma(const Dims& d, const ScoreArgs& a, int64_t total, cudaError_t* err, cudaStream_t st) {
+using TmaScoreKernel = void (*)(const CUtensorMap, ScoreArgs);
+
+// Launches a tensor-copy scorer when the code tensor can be described by a
+// tensor map (d = 128, 16-byte aligned base); returns false to fall back.
+bool run_tma(TmaScoreKernel k, const Dims& d, const ScoreArgs& a, int64_t total, cudaError_t* err,
+             cudaStream_t st) {
   const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode || d.D != 128 || (reinterpret_cast<uintptr_t>(a.kq) & 15) != 0) return false;
   const uint64_t nrows = (uint64_t)d.Hkv * (uint64_t)d.T;
@@ -948,7 +1196,6 @@ bool run_tma(const Dims& d, const ScoreArgs& a, int64_t total, cudaError_t* err,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
   const int smem = 1024 + kTmaStages * kTmaStageBytes + kHist / 2 * 4 + 2 * (d.B + 1) * (int)sizeof(int);
-  auto k = score_tma_kernel<NT>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess) {
     const int grid = grid_for(k, smem, d.num_sms, total);
@@ -1004,13 +1251,16 @@ cudaError_t launch_propose_scores(const Dims& d, const void* q, const int8_t* kq
   const int64_t total = per_head * d.Hkv;
   if (total == 0) return cudaSuccess;
   ScoreArgs a{q, kq, scale, scores, hist, d.cu_dev, d.T, d.B, d.Hkv, d.G, status, nullptr, nullptr};
-  if (use_mma && d.bf16 && d.D == 128 && use_tma_scorer()) {
+  const int choice = scorer_choice();
+  if (use_mma && d.bf16 && d.D == 128 && choice > 0) {
     int64_t stages = 0;
     for (int b = 0; b < d.B; ++b) stages += cdiv(d.cu_host[b + 1] - d.cu_host[b], kStageRows);
+    TmaScoreKernel k = d.G <= 8 ? score_tma_kernel<1> : score_tma_kernel<2>;
+    // the integer scorer reads query rows in 16-byte pieces
+    if (choice == 2 && d.G <= 8 && (reinterpret_cast<uintptr_t>(q) & 15) == 0)
+      k = d.G <= 4 ? score_i8_kernel<1> : score_i8_kernel<2>;
     cudaError_t e = cudaSuccess;
-    const bool ran = d.G <= 8 ? run_tma<1>(d, a, stages * d.Hkv, &e, st)
-                              : run_tma<2>(d, a, stages * d.Hkv, &e, st);
-    if (ran) return e;
+    if (run_tma(k, d, a, stages * d.Hkv, &e, st)) return e;
   }
   if (use_mma && d.bf16) {
     if (d.D == 128) return d.G <= 8 ? run_mma<128, 1>(d, a, st) : run_mma<128, 2>(d, a, st);

@@ -97,22 +97,26 @@ PROPOSE_CASES = [
     ([1024, 1025, 1023], 16, 4, 128, "bf16", 1024),  # L == kappa_p, +-1
     ([40000], 8, 2, 128, "bf16", 4096),         # many tiles and chunks
     ([9000], 12, 3, 128, "f32", 700),           # G = 4, fp32
+    ([1500, 77], 4, 4, 128, "bf16", 300),       # G = 1 at d = 128 (one head of the quad)
+    ([2049, 100], 6, 2, 128, "bf16", 512),      # G = 3
+    ([1700], 12, 2, 128, "bf16", 400),          # G = 6 (two quads, the second partial)
 ]
 
 
 @pytest.mark.parametrize("case", PROPOSE_CASES, ids=lambda c: f"{c[0]}-{c[1]}/{c[2]}-d{c[3]}-{c[4]}-kp{c[5]}")
-@pytest.mark.parametrize("scorer", ["tma", "mma", "simt"])
+@pytest.mark.parametrize("scorer", ["i8", "tma", "mma", "simt"])
 def test_propose_vs_oracle(P, case, scorer, monkeypatch):
-    """tma: the default tensor-core scorer, fed by tensor copies (d = 128;
-    d = 64 takes the cp.async one); mma: the cp.async tensor-core scorer;
-    simt: CUDA cores."""
+    """i8: the default scorer, integer tensor cores on the stored codes with
+    the query in fixed point, fed by tensor copies (d = 128 and G <= 8; d = 64
+    takes the cp.async fp16 one, G > 8 the tensor-copy fp16 one); tma: the
+    tensor-copy fp16 scorer; mma: the cp.async fp16 scorer; simt: CUDA cores."""
     seqlens, hq, hkv, d, dtype, kp = case
     if scorer == "simt":
         monkeypatch.setenv("PRISM_PROPOSE_SCORER", "simt")
     elif dtype != "bf16":
         pytest.skip("the tensor-core scorers take bf16 queries")
-    elif scorer == "mma":
-        monkeypatch.setenv("PRISM_PROPOSE_SCORER", "mma")
+    elif scorer in ("mma", "tma"):
+        monkeypatch.setenv("PRISM_PROPOSE_SCORER", scorer)
     prob = problem(P, seqlens, hq, hkv, d, dtype)
     q, k, _ = make_case(seqlens, hq, hkv, d, dtype, seed=2)
     T = prob.total_tokens
@@ -139,6 +143,47 @@ def test_propose_vs_oracle(P, case, scorer, monkeypatch):
                 assert np.allclose(gs, s, rtol=2e-6, atol=2e-6 * np.abs(s).max()), (b, h)
             check_index_set(gp[b, h, :n], opool[b, h, :n], lambda t: s[t], f"pool b{b} h{h}")
             assert np.all(gp[b, h, n:] == -1)
+
+
+def test_propose_query_ranges(P):
+    """Query heads far from unit scale, where the integer scorer's fixed-point
+    query needs care: a group at 2^-110 (shift above 126, taken in two
+    factors), one at 2^100, one whose heads mix elements 2^-40 apart (the
+    small ones off the grid), and one with an all-zero head and an all-negative
+    one.  Scores and pools are checked against the oracle as above."""
+    seqlens, hq, hkv, d, kp = [3000, 1200], 16, 4, 128, 700
+    prob = problem(P, seqlens, hq, hkv, d, "bf16")
+    q, k, _ = make_case(seqlens, hq, hkv, d, "bf16", seed=11)
+    qf = q.float().cpu().view(len(seqlens), hkv, hq // hkv, d)
+    qf[:, 0] *= 2.0 ** -110
+    qf[:, 1] *= 2.0 ** 100
+    qf[:, 2, :, ::2] *= 2.0 ** -40
+    qf[:, 3, 0] = 0.0
+    qf[:, 3, 1] = -qf[:, 3, 1].abs()
+    q = qf.view(len(seqlens), hq, d).to(torch.bfloat16).to(DEV)
+    T = prob.total_tokens
+    kq = torch.zeros((hkv, T, d), dtype=torch.int8, device=DEV)
+    sc = torch.zeros((hkv, T), dtype=torch.float32, device=DEV)
+    P.quantize_k(prob, k, kq, sc)
+    pool = torch.full((len(seqlens), hkv, kp), -7, dtype=torch.int32, device=DEV)
+    cnt = torch.full((len(seqlens), hkv), -7, dtype=torch.int32, device=DEV)
+    ws = ws_for(P, prob, P.OP_PROPOSE, kp)
+    P.propose(prob, q, kq, sc, kp, pool, cnt, ws)
+    torch.cuda.synchronize()
+    assert P.get_device_status(ws) == 0
+    gscores = _np(ws[256:256 + hkv * T * 4].view(torch.float32)).reshape(hkv, T)
+    opool, ocnt, oscores = pipeline.propose_layer(q, kq, sc, prob.cu_host.tolist(), kp)
+    gp, gc = _np(pool), _np(cnt)
+    assert np.array_equal(gc, ocnt)
+    cu = prob.cu_host
+    for b in range(len(seqlens)):
+        for h in range(hkv):
+            s = oscores[(b, h)]
+            n = int(ocnt[b, h])
+            gs = gscores[h, cu[b]:cu[b + 1]]
+            assert np.all(np.isfinite(gs)) and np.abs(s).max() > 0, (b, h)
+            assert np.allclose(gs, s, rtol=2e-6, atol=2e-6 * np.abs(s).max()), (b, h)
+            check_index_set(gp[b, h, :n], opool[b, h, :n], lambda t: s[t], f"pool b{b} h{h}")
 
 
 @pytest.mark.parametrize("L0,kp", [(3000, 1000), (60000, 8192)], ids=["small", "many-candidates"])
