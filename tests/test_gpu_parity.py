@@ -145,6 +145,43 @@ def test_propose_vs_oracle(P, case, scorer, monkeypatch):
             assert np.all(gp[b, h, n:] == -1)
 
 
+@pytest.mark.parametrize("keys", ["int8", "int2"])
+def test_propose_workspace_reuse(P, keys):
+    """Calls on one propose workspace (here three, on different queries) each
+    match the oracle: nothing a call leaves in the workspace (scores,
+    first-digit histograms) leaks into the next."""
+    seqlens, hq, hkv, d, kp = [5000, 2100], 8, 2, 128, 900
+    prob = problem(P, seqlens, hq, hkv, d, "bf16")
+    T = prob.total_tokens
+    ws = ws_for(P, prob, P.OP_PROPOSE, kp)
+    for it in range(3):
+        q, k, _ = make_case(seqlens, hq, hkv, d, "bf16", seed=40 + it)
+        pool = torch.full((len(seqlens), hkv, kp), -7, dtype=torch.int32, device=DEV)
+        cnt = torch.full((len(seqlens), hkv), -7, dtype=torch.int32, device=DEV)
+        if keys == "int8":
+            kq = torch.zeros((hkv, T, d), dtype=torch.int8, device=DEV)
+            sc = torch.zeros((hkv, T), dtype=torch.float32, device=DEV)
+            P.quantize_k(prob, k, kq, sc)
+            P.propose(prob, q, kq, sc, kp, pool, cnt, ws)
+            opool, ocnt, oscores = pipeline.propose_layer(q, kq, sc, prob.cu_host.tolist(), kp)
+        else:
+            codes = torch.zeros((hkv, T, d // 4), dtype=torch.uint8, device=DEV)
+            params = torch.zeros((hkv, T, d // 32, 2), dtype=torch.int16, device=DEV)
+            P.quantize_k_int2(prob, k, codes, params)
+            P.propose_int2(prob, q, codes, params, kp, pool, cnt, ws)
+            opool, ocnt, oscores = pipeline.propose_layer_int2(
+                q, codes.cpu().numpy(), params.cpu().numpy().view(np.uint16), prob.cu_host.tolist(), kp)
+        torch.cuda.synchronize()
+        assert P.get_device_status(ws) == 0
+        gp, gc = _np(pool), _np(cnt)
+        assert np.array_equal(gc, ocnt)
+        for b in range(len(seqlens)):
+            for h in range(hkv):
+                n = int(ocnt[b, h])
+                sc_of = oscores[(b, h)]
+                check_index_set(gp[b, h, :n], opool[b, h, :n], lambda t: sc_of[t], f"call {it} b{b} h{h}")
+
+
 def test_propose_query_ranges(P):
     """Query heads far from unit scale, where the integer scorer's fixed-point
     query needs care: a group at 2^-110 (shift above 126, taken in two
