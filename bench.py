@@ -404,6 +404,10 @@ def run_prism(args, dist: Dist):
         pl = cfg.is_proposal(l)
 
         def f_prop(l=l):
+            if dec.scorer_appends:  # the scorer quantizes the new key rows; the refined layer appends
+                prism.propose_append(dec.p, q_layers[l], k_new[l], kqs[l], scs[l], cfg.kappa_p,
+                                     dec.pool[l], dec.pool_cnt[l], dec.ws_prop)
+                return
             prism.append_kv(dec.p, k_new[l], v_new[l], ks[l], vs[l])
             if args.keys == "int2":
                 prism.quantize_k_int2(dec.p, ks[l], kqs[l], scs[l], tok_rows=dec.new_rows, ws=dec.ws_q)
@@ -416,7 +420,9 @@ def run_prism(args, dist: Dist):
 
         def f_rd(l=l):
             src = l - l % cfg.group
-            fa = not cfg.is_proposal(l)  # refined layers append their new rows themselves
+            # refined layers append their new rows themselves, and so do proposal
+            # layers whose scorer took the new key rows
+            fa = not cfg.is_proposal(l) or dec.scorer_appends
             prism.refine_decode(dec.p, q_layers[l], ks[l], vs[l], dec.pool[src], dec.pool_cnt[src],
                                 cfg.kappa_p, cfg.kappa, dec.scale, dec.idx[l], dec.cnt[l],
                                 dec.out[l], dec.ws_rd, lse=dec.lse[l],

@@ -158,6 +158,22 @@ PRISM_API prism_status prism_propose(const prism_shape* shape, const void* q, co
                            int32_t* pool_cnt, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * prism_propose for a decode step whose new key rows are not in the codes
+ * yet: k_new [B][Hkv][d] (the token's key rows, cache dtype) are quantized as
+ * prism_quantize_k does and written to kq / k_scale at position L_b - 1 of
+ * every non-empty sequence by the scorer itself, which then scores them with
+ * the rest -- one launch fewer than prism_quantize_k + prism_propose, and the
+ * K cache itself is not read (the new row may be appended to it later, e.g.
+ * by prism_refine_decode).  Same outputs, workspace and rules as
+ * prism_propose.  bf16, d = 128, G <= 8 and L_b <= PRISM_MAX_SELECT_ROW only
+ * (else PRISM_ERR_UNSUPPORTED); q, k_new and kq 16-byte aligned.
+ */
+PRISM_API prism_status prism_propose_append(const prism_shape* shape, const void* q,
+                                            const void* k_new, int8_t* kq, float* k_scale,
+                                            int32_t kappa_p, int32_t* pool_idx, int32_t* pool_cnt,
+                                            void* ws, size_t ws_bytes, void* stream);
+
+/*
  * INT2 proposal keys (sec. 4.2: the pages compress the proposal layers' key
  * cache to INT2 without stating the scheme; this is the library's scheme).
  * Per KV head h, token t and group of 32 consecutive features (d = 128: four

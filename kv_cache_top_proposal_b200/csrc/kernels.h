@@ -46,6 +46,13 @@ cudaError_t launch_propose_scores(const Dims& d, const void* q, const int8_t* kq
                                   int32_t* status, cudaStream_t st);
 // INT2 proposal scores from packed codes and (step, zero point) pairs, with
 // the first-digit histogram (bf16 queries, d = 128; score.cu).
+// The integer scorer with this token's key rows k_new [B][Hkv][d] (bf16),
+// quantized by the scorer into kq / scale at position L_b - 1 of every
+// non-empty sequence before that position is scored.  bf16, d = 128, G <= 8
+// only (cudaErrorInvalidValue otherwise).
+cudaError_t launch_propose_scores_new_rows(const Dims& d, const void* q, int8_t* kq, float* scale,
+                                           const void* k_new, float* scores, uint32_t* hist,
+                                           int32_t* status, cudaStream_t st);
 cudaError_t launch_propose_scores_int2(const Dims& d, const void* q, const uint8_t* codes,
                                        const uint16_t* params, float* scores, uint32_t* hist,
                                        int32_t* status, cudaStream_t st);

@@ -206,6 +206,33 @@ prism_status prism_propose(const prism_shape* shape, const void* q, const int8_t
   return cuda_status(launch_select(d, a, d.max_len, st));
 }
 
+prism_status prism_propose_append(const prism_shape* shape, const void* q, const void* k_new,
+                                  int8_t* kq, float* k_scale, int32_t kappa_p, int32_t* pool_idx,
+                                  int32_t* pool_cnt, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!q || !k_new || !kq || !k_scale || !pool_idx || !pool_cnt || kappa_p < 1)
+    return PRISM_ERR_INVALID_ARG;
+  if (!d.bf16 || d.D != 128 || d.G > 8 || d.max_len > propose_select_max_row())
+    return PRISM_ERR_UNSUPPORTED;
+  if (((uintptr_t)q | (uintptr_t)k_new | (uintptr_t)kq) % 16) return PRISM_ERR_INVALID_ARG;
+  const Layout L = layout(d, PRISM_OP_PROPOSE, kappa_p, 0);
+  if (!ws_ok(ws, ws_bytes, L)) return PRISM_ERR_WORKSPACE;
+  if ((s = set_live_sms(&d)) != PRISM_OK) return s;
+  char* w = static_cast<char*>(ws);
+  int32_t* status = reinterpret_cast<int32_t*>(w);
+  float* scores = reinterpret_cast<float*>(w + L.a);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(w + L.b);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t rows = (size_t)d.B * d.Hkv;
+  if (cudaMemsetAsync(hist, 0, rows * 4096 * 4, st) != cudaSuccess) return PRISM_ERR_CUDA;
+  cudaError_t e = launch_propose_scores_new_rows(d, q, kq, k_scale, k_new, scores, hist, status, st);
+  if (e == cudaErrorInvalidValue) return PRISM_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return PRISM_ERR_CUDA;
+  return cuda_status(launch_propose_select(d, scores, hist, kappa_p, pool_idx, pool_cnt, status, st));
+}
+
 prism_status prism_quantize_k_int2(const prism_shape* shape, const void* k, uint8_t* codes,
                                    uint16_t* params, const int32_t* tok_rows, int32_t n_rows,
                                    void* ws, size_t ws_bytes, void* stream) {

@@ -51,6 +51,9 @@ struct ScoreArgs {
   int32_t* status;
   const uint8_t* codes;    // INT2 keys: [Hkv][T][d/4], four codes per byte
   const uint16_t* params;  // INT2 keys: [Hkv][T][d/32][2] fp16 bits of (step, zero point)
+  const void* k_new;       // integer scorer: [B][Hkv][d] new key rows to quantize at L_b - 1, or null
+  int8_t* kq_w;            // with k_new: where its codes go (the same codes as kq)
+  float* scale_w;          // with k_new: where its scales go
 };
 
 // s_pref[b] = number of work items of sequences before b (per KV head).
@@ -613,6 +616,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_i8_kernel(const __grid_cons
   int* s_pref = reinterpret_cast<int*>(s_hist + kHist / 2);
   int* s_cu = s_pref + a.B + 1;
   __shared__ __align__(8) uint64_t full[kTmaStages];
+  __shared__ float s_newscale;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tig = lane & 3;
   for (int i = tid; i <= a.B; i += kThreads) s_cu[i] = a.cu[i];
@@ -679,6 +683,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_i8_kernel(const __grid_cons
   for (int kk = 0; kk < nk; ++kk) {
     const int L = s_cu[it_comp.b + 1] - s_cu[it_comp.b];
     const int rows = min(kStageRows, L - it_comp.r0);
+    const int nr = L - 1 - it_comp.r0;  // the stage row of position L - 1 when nr < rows
     const int64_t rowbase = (int64_t)it_comp.h * a.T + s_cu[it_comp.b] + it_comp.r0;
     if (it_comp.b != cur_b || it_comp.h != cur_h) {
       // limbs of the query heads of (b, h): thread (g, tig) supplies column g
@@ -749,7 +754,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_i8_kernel(const __grid_cons
     }
     ++since_flush;
     it_comp.advance(s_cu, a.B);
-    const float sc = sc_next;
+    float sc = sc_next;
     if (kk + 1 < nk) sc_next = load_scale(it_comp);
     const int slot = kk % kTmaStages;
     {
@@ -761,7 +766,40 @@ __global__ void __launch_bounds__(kThreads, 3) score_i8_kernel(const __grid_cons
         }
       }
     }
-    const unsigned char* buf = ring + slot * kTmaStageBytes;
+    unsigned char* buf = ring + slot * kTmaStageBytes;
+    if (a.k_new && nr < rows) {  // CTA-uniform
+      // this token's key row, not in the codes yet: warp 0 quantizes it as
+      // the quantizer does (amax / 127, round half to even, clamp to 127)
+      // into the stage and into the cache's codes and scales
+      if (warp == 0) {
+        const __nv_bfloat16* kn =
+            static_cast<const __nv_bfloat16*>(a.k_new) + ((int64_t)cur_b * a.Hkv + cur_h) * D;
+        const uint2 w = *reinterpret_cast<const uint2*>(kn + 4 * lane);
+        const float f[4] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y)};
+        float amax = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float sq = __fdiv_rn(amax, 127.0f);
+        uint32_t packed = 0u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          int c = 0;
+          if (amax != 0.0f) c = (int)fminf(fmaxf(rintf(__fdiv_rn(f[e], sq)), -127.0f), 127.0f);
+          packed |= ((uint32_t)(c & 0xFF)) << (8 * e);
+        }
+        // features 4 lane .. + 3: chunk lane / 4 of the row, swizzled as the copy lays it out
+        *reinterpret_cast<uint32_t*>(buf + nr * 128 + ((((lane >> 2) ^ (nr & 7)) << 4) | ((lane & 3) << 2))) =
+            packed;
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // before the slot's next copy
+        *reinterpret_cast<uint32_t*>(a.kq_w + (rowbase + nr) * D + 4 * lane) = packed;
+        if (lane == 0) {
+          s_newscale = amax != 0.0f ? sq : 0.0f;
+          a.scale_w[rowbase + nr] = s_newscale;
+        }
+      }
+      __syncthreads();
+      if (rs == nr) sc = s_newscale;
+    }
     const int t = warp;  // one 16-row tile per warp
     if (t * 16 < rows) {
       const bool mine = tig < 2 && rs < rows;  // tig 0: row g, tig 1: row g + 8
@@ -1250,7 +1288,8 @@ cudaError_t launch_propose_scores(const Dims& d, const void* q, const int8_t* kq
   for (int b = 0; b < d.B; ++b) per_head += cdiv(d.cu_host[b + 1] - d.cu_host[b], kChunkRows);
   const int64_t total = per_head * d.Hkv;
   if (total == 0) return cudaSuccess;
-  ScoreArgs a{q, kq, scale, scores, hist, d.cu_dev, d.T, d.B, d.Hkv, d.G, status, nullptr, nullptr};
+  ScoreArgs a{q, kq, scale, scores, hist, d.cu_dev, d.T, d.B, d.Hkv, d.G, status, nullptr, nullptr,
+              nullptr, nullptr, nullptr};
   const int choice = scorer_choice();
   if (use_mma && d.bf16 && d.D == 128 && choice > 0) {
     int64_t stages = 0;
@@ -1274,6 +1313,23 @@ cudaError_t launch_propose_scores(const Dims& d, const void* q, const int8_t* kq
                     : simt_by_group<float, 64>(d, a, total, st);
 }
 
+cudaError_t launch_propose_scores_new_rows(const Dims& d, const void* q, int8_t* kq, float* scale,
+                                           const void* k_new, float* scores, uint32_t* hist,
+                                           int32_t* status, cudaStream_t st) {
+  if (!d.bf16 || d.D != 128 || d.G > 8 || (reinterpret_cast<uintptr_t>(q) & 15) != 0 ||
+      (reinterpret_cast<uintptr_t>(k_new) & 7) != 0)
+    return cudaErrorInvalidValue;
+  int64_t stages = 0;
+  for (int b = 0; b < d.B; ++b) stages += cdiv(d.cu_host[b + 1] - d.cu_host[b], kStageRows);
+  if (stages == 0) return cudaSuccess;
+  ScoreArgs a{q, kq, scale, scores, hist, d.cu_dev, d.T, d.B, d.Hkv, d.G, status, nullptr, nullptr,
+              k_new, kq, scale};
+  cudaError_t e = cudaSuccess;
+  if (!run_tma(d.G <= 4 ? score_i8_kernel<1> : score_i8_kernel<2>, d, a, stages * d.Hkv, &e, st))
+    return cudaErrorInvalidValue;
+  return e;
+}
+
 cudaError_t launch_propose_scores_int2(const Dims& d, const void* q, const uint8_t* codes,
                                        const uint16_t* params, float* scores, uint32_t* hist,
                                        int32_t* status, cudaStream_t st) {
@@ -1281,7 +1337,8 @@ cudaError_t launch_propose_scores_int2(const Dims& d, const void* q, const uint8
   int64_t stages = 0;
   for (int b = 0; b < d.B; ++b) stages += cdiv(d.cu_host[b + 1] - d.cu_host[b], kStageRows);
   if (stages == 0) return cudaSuccess;
-  ScoreArgs a{q, nullptr, nullptr, scores, hist, d.cu_dev, d.T, d.B, d.Hkv, d.G, status, codes, params};
+  ScoreArgs a{q, nullptr, nullptr, scores, hist, d.cu_dev, d.T, d.B, d.Hkv, d.G, status, codes, params,
+              nullptr, nullptr, nullptr};
   return d.G <= 8 ? run_int2<1>(d, a, stages * d.Hkv, st) : run_int2<2>(d, a, stages * d.Hkv, st);
 }
 

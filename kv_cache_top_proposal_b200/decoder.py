@@ -70,6 +70,11 @@ class PrismDecoder:
         # "int2" (codes uint8 [Hkv][T][d/4], params int16 [Hkv][T][d/32][2])
         assert keys in ("int8", "int2")
         self.keys = keys
+        # int8 proposal layers of a fused step hand the new key rows to the
+        # scorer (prism_propose_append), which quantizes them itself; the
+        # fused refined layer after it appends the rows to the cache
+        self.scorer_appends = (fused and keys == "int8" and dtype == prism.BF16 and head_dim == 128
+                               and num_q_heads // num_kv_heads <= 8)
 
     def workspaces(self) -> List[torch.Tensor]:
         return [w for w in (self.ws_q, self.ws_prop, self.ws_ref, self.ws_dec, self.ws_rd,
@@ -86,11 +91,16 @@ class PrismDecoder:
         one, so this layer's launch may begin before it ends."""
         p = self.p
         proposal = l % self.group == 0
+        # the scorer quantizes the new key rows itself (int8 keys, fused step)
+        scorer_new = proposal and self.scorer_appends and k_new is not None and quantize_new
         # a fused refined layer appends the new rows itself
-        fused_append = self.fused and not proposal and k_new is not None
+        fused_append = self.fused and k_new is not None and (not proposal or scorer_new)
         if k_new is not None and not fused_append:
             prism.append_kv(p, k_new, v_new, k, v, stream=stream)
-        if proposal:
+        if scorer_new:
+            prism.propose_append(p, q, k_new, kq, k_scale, self.kappa_p, self.pool[l], self.pool_cnt[l],
+                                 self.ws_prop, stream=stream)
+        elif proposal:
             if self.keys == "int2":
                 if quantize_new and self.new_rows.numel():
                     prism.quantize_k_int2(p, k, kq, k_scale, tok_rows=self.new_rows, ws=self.ws_q,
@@ -134,9 +144,11 @@ class PrismDecoder:
         score, select, attend, merge)."""
         n = 0
         for l in range(self.num_layers):
-            n += 1 if append and (l % self.group == 0 or not self.fused) else 0
-            if l % self.group == 0:
-                n += (1 if self.new_rows.numel() else 0) + 2
+            proposal = l % self.group == 0
+            scorer_new = proposal and self.scorer_appends and append
+            n += 1 if append and ((proposal and not scorer_new) or not self.fused) else 0
+            if proposal:
+                n += (1 if self.new_rows.numel() and not scorer_new else 0) + 2
             n += 1 if self.fused else 2 + 2
         return n
 

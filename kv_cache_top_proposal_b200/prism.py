@@ -26,7 +26,8 @@ MAX_SELECT_ROW = 393216
 RD_OVERLAP = 0x1
 WS_HEADER = 256
 
-EXPORTS = ("prism_workspace_size", "prism_append_kv", "prism_quantize_k", "prism_propose", "prism_refine",
+EXPORTS = ("prism_workspace_size", "prism_append_kv", "prism_quantize_k", "prism_propose",
+           "prism_propose_append", "prism_refine",
            "prism_sparse_decode", "prism_refine_decode", "prism_dense_decode",
            "prism_clear_device_status",
            "prism_get_device_status", "prism_status_str", "prism_sparse_decode_noalloc",
@@ -58,6 +59,7 @@ def _load():
         "prism_append_kv": [sp, P, P, P, P, P],
         "prism_quantize_k": [sp, P, P, P, P, i32, P, S, P],
         "prism_propose": [sp, P, P, P, i32, P, P, P, S, P],
+        "prism_propose_append": [sp, P, P, P, P, i32, P, P, P, S, P],
         "prism_refine": [sp, P, P, P, P, i32, i32, P, P, P, P, S, P],
         "prism_sparse_decode": [sp, P, P, P, P, P, i32, ctypes.c_float, P, P, P, S, P],
         "prism_refine_decode": [sp, P, P, P, P, P, i32, i32, ctypes.c_float, P, P, P, P, P, P, P,
@@ -158,6 +160,14 @@ def quantize_k(p: Problem, k, kq, k_scale, tok_rows=None, ws=None, stream=None):
 def propose(p: Problem, q, kq, k_scale, kappa_p: int, pool, pool_cnt, ws, stream=None):
     _check(_lib.prism_propose(p.ref, _ptr(q), _ptr(kq), _ptr(k_scale), kappa_p, _ptr(pool),
                               _ptr(pool_cnt), _ptr(ws), _nbytes(ws), _stream(stream)), "propose")
+
+
+def propose_append(p: Problem, q, k_new, kq, k_scale, kappa_p: int, pool, pool_cnt, ws, stream=None):
+    """propose with this token's key rows k_new [B][Hkv][d] quantized into kq / k_scale at
+    position L_b - 1 by the scorer itself (bf16, d = 128, G <= 8)."""
+    _check(_lib.prism_propose_append(p.ref, _ptr(q), _ptr(k_new), _ptr(kq), _ptr(k_scale), kappa_p,
+                                     _ptr(pool), _ptr(pool_cnt), _ptr(ws), _nbytes(ws),
+                                     _stream(stream)), "propose_append")
 
 
 def quantize_k_int2(p: Problem, k, codes, params, tok_rows=None, ws=None, stream=None):

@@ -182,6 +182,78 @@ def test_propose_workspace_reuse(P, keys):
                 check_index_set(gp[b, h, :n], opool[b, h, :n], lambda t: sc_of[t], f"call {it} b{b} h{h}")
 
 
+PROPOSE_APPEND_CASES = [
+    # seqlens, hq, hkv, kappa_p
+    ([5000, 1031, 0, 300, 1], 8, 2, 1024),  # ragged, an empty sequence, one of length 1
+    ([2500, 129, 128], 64, 8, 333),          # G = 8; the new row alone in a stage, and at its end
+    ([3000, 777], 8, 8, 200),                # G = 1
+]
+
+
+@pytest.mark.parametrize("case", PROPOSE_APPEND_CASES, ids=lambda c: f"{c[0]}-{c[1]}/{c[2]}-kp{c[3]}")
+def test_propose_append_vs_oracle(P, case):
+    """prism_propose_append: the scorer quantizes this token's key rows into
+    kq / k_scale at L_b - 1 (bit-exact with the oracle's quantizer; every
+    other row untouched) and scores them with the rest; the pool matches the
+    oracle's proposal over the codes with the new rows in place.  The cache
+    row at L_b - 1 holds something else (the new row is appended later)."""
+    seqlens, hq, hkv, kp = case
+    d = 128
+    prob = problem(P, seqlens, hq, hkv, d, "bf16")
+    q, k, _ = make_case(seqlens, hq, hkv, d, "bf16", seed=31)
+    g = torch.Generator(device="cpu").manual_seed(32)
+    k_new = (torch.randn((len(seqlens), hkv, d), generator=g) * 1.5).to(torch.bfloat16).to(DEV)
+    k_new[0, 0, :] = 0  # an all-zero new row: scale 0, codes 0
+    T = prob.total_tokens
+    kq = torch.zeros((hkv, T, d), dtype=torch.int8, device=DEV)
+    sc = torch.zeros((hkv, T), dtype=torch.float32, device=DEV)
+    P.quantize_k(prob, k, kq, sc)  # the cache's codes, stale at L_b - 1
+    kq_before, sc_before = _np(kq).copy(), _np(sc).copy()
+    pool = torch.full((len(seqlens), hkv, kp), -7, dtype=torch.int32, device=DEV)
+    cnt = torch.full((len(seqlens), hkv), -7, dtype=torch.int32, device=DEV)
+    ws = ws_for(P, prob, P.OP_PROPOSE, kp)
+    P.propose_append(prob, q, k_new, kq, sc, kp, pool, cnt, ws)
+    torch.cuda.synchronize()
+    assert P.get_device_status(ws) == 0
+    cu = prob.cu_host
+    want_kq, want_sc = kq_before.copy(), sc_before.copy()
+    okq, osc = oracle.quantize_rows(_np(k_new).reshape(-1, d))
+    okq, osc = okq.reshape(len(seqlens), hkv, d), osc.reshape(len(seqlens), hkv)
+    for b in range(len(seqlens)):
+        if cu[b + 1] > cu[b]:
+            want_kq[:, cu[b + 1] - 1] = okq[b]
+            want_sc[:, cu[b + 1] - 1] = osc[b]
+    assert np.array_equal(_np(kq), want_kq)
+    assert np.array_equal(_np(sc).view(np.uint32), want_sc.view(np.uint32))
+    opool, ocnt, oscores = pipeline.propose_layer(q, want_kq, want_sc, cu.tolist(), kp)
+    gp, gc = _np(pool), _np(cnt)
+    assert np.array_equal(gc, ocnt)
+    gscores = _np(ws[256:256 + hkv * T * 4].view(torch.float32)).reshape(hkv, T)
+    for b in range(len(seqlens)):
+        for h in range(hkv):
+            n = int(ocnt[b, h])
+            s_ = oscores[(b, h)]
+            if n:
+                gs = gscores[h, cu[b]:cu[b + 1]]
+                assert np.allclose(gs, s_, rtol=2e-6, atol=2e-6 * np.abs(s_).max()), (b, h)
+            check_index_set(gp[b, h, :n], opool[b, h, :n], lambda t: s_[t], f"pool b{b} h{h}")
+            assert np.all(gp[b, h, n:] == -1)
+
+
+def test_propose_append_unsupported(P):
+    """Shapes the integer scorer does not take are refused, not computed."""
+    prob = problem(P, [300], 8, 2, 64, "bf16")  # d = 64
+    q, k, _ = make_case([300], 8, 2, 64, "bf16", seed=3)
+    kq = torch.zeros((2, 300, 64), dtype=torch.int8, device=DEV)
+    sc = torch.zeros((2, 300), dtype=torch.float32, device=DEV)
+    pool = torch.zeros((1, 2, 100), dtype=torch.int32, device=DEV)
+    cnt = torch.zeros((1, 2), dtype=torch.int32, device=DEV)
+    k_new = torch.zeros((1, 2, 64), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(P.PrismError) as e:
+        P.propose_append(prob, q, k_new, kq, sc, 100, pool, cnt, ws_for(P, prob, P.OP_PROPOSE, 100))
+    assert e.value.status == P.ERR_UNSUPPORTED
+
+
 def test_propose_query_ranges(P):
     """Query heads far from unit scale, where the integer scorer's fixed-point
     query needs care: a group at 2^-110 (shift above 126, taken in two
