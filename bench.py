@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--profile-steps", type=int, default=5)
     ap.add_argument("--keys", default="int8", choices=["int8", "int2"],
                     help="proposal key cache: int8 per token (the headline workload) or INT2 per 32-feature group")
+    ap.add_argument("--grow", action="store_true",
+                    help="decode loop over the growing sequence: every replayed step appends one "
+                         "token (batch-1 configs); the cache starts short by the replays")
     ap.add_argument("--layers", type=int, default=0,
                     help="keep only the first N layers (small cases for profiling)")
     return ap.parse_args()
@@ -318,9 +321,16 @@ def run_prism(args, dist: Dist):
     ks = [x.k for x in layers]
     vs = [x.v for x in layers]
     del layers
-    dec = PrismDecoder(cfg.seqlens, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim,
+    # --grow: a decode loop over one growing sequence; every replay of the step
+    # graph appends one token, so it starts short by the number of replays
+    n_grow = 1 + 2 * args.warmup + args.steps + max(10, args.steps // 2) if args.grow else 0
+    if args.grow and cfg.batch != 1:
+        raise SystemExit("--grow decodes one sequence (batch 1)")
+    seqlens0 = (cfg.seqlens[0] - n_grow,) if args.grow else cfg.seqlens
+    dec = PrismDecoder(seqlens0, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim,
                        prism.BF16 if cfg.dtype == "bf16" else prism.F32, L, cfg.group,
-                       cfg.kappa_p, cfg.kappa, device=dev, keys=args.keys)
+                       cfg.kappa_p, cfg.kappa, device=dev, keys=args.keys,
+                       capacity=cfg.total_tokens)
     rows = dec.new_rows.long()
     Hkv = cfg.num_kv_heads
     k_new = torch.stack([k[:, rows].transpose(0, 1).contiguous() for k in ks])  # [L][B][Hkv][d]
@@ -343,6 +353,8 @@ def run_prism(args, dist: Dist):
     q_layers = [q_all[l] for l in range(L)]
 
     def step():
+        if args.grow:
+            dec.advance_on_device(1)
         dec.step(q_layers, ks, vs, kqs, scs, quantize_new=True, k_new=k_new, v_new=v_new)
 
     step()  # eager once (validates arguments before capture)
@@ -396,6 +408,9 @@ def run_prism(args, dist: Dist):
     h2d = (q_h.numel() * q_h.element_size() + kn_h.numel() * kn_h.element_size()
            + vn_h.numel() * vn_h.element_size())
     d2h = out_h.numel() * out_h.element_size()
+
+    if args.grow:
+        dec.lengths_from_device()  # the dense comparison sizes its splits from the host copy
 
     # ---- per-op durations (one graph per op; the queue is filled behind a
     # long memset so every event pair brackets device time only)
@@ -509,7 +524,10 @@ def run_prism(args, dist: Dist):
                            refined_layers="fused refine+select+sparse-decode (prism_refine_decode)",
                            proposal_keys="int8 per token" if args.keys == "int8"
                            else "INT2 per 32-feature group (fp16 step and zero point)",
-                           graph="one CUDA graph per step"),
+                           graph="one CUDA graph per step",
+                           **({"growth": f"decode loop: every replayed step appends one token, "
+                                         f"from L = {seqlens0[0]} to {seqlens0[0] + n_grow}"}
+                              if args.grow else {})),
             "roofline": roofline,
             "step_roofline": {"achieved": round(step_achieved, 1), "peak": peak, "unit": "GB/s",
                               "frac": round(step_achieved / peak, 4),

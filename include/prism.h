@@ -88,10 +88,21 @@ typedef enum prism_op {
 #define PRISM_DEV_TIMEOUT   0x4   /* a bounded device-side wait gave up        */
 
 /* Shape of one layer's decode problem.  cu_seqlens_host mirrors
- * cu_seqlens_dev (B+1 entries, cu[0] = 0, non-decreasing, cu[B] =
+ * cu_seqlens_dev (B+1 entries, cu[0] = 0, non-decreasing, cu[B] <=
  * total_tokens); the host copy sizes grids and is validated, the device copy
- * is what kernels read.  head_dim is 64 or 128; num_q_heads is a multiple of
- * num_kv_heads with G <= 16; batch <= 4096. */
+ * is what kernels read.  total_tokens is the number of rows of every
+ * per-token array ([Hkv][total_tokens][...]: K, V, kq, k_scale, INT2 codes
+ * and params); rows past cu[B] are spare capacity, which a decode loop fills
+ * by growing the last sequence (cu[B] += 1 per step, device copy included).
+ * Kernels read the lengths from the device copy when they run, so a captured
+ * CUDA graph of the decode path (prism_append_kv, prism_quantize_k,
+ * prism_propose, prism_propose_append, prism_refine_decode, prism_refine,
+ * prism_sparse_decode) stays valid while the last sequence grows, as long as
+ * it stays within 131072 positions when the graph was captured at or below
+ * that (the proposal selection then takes the same path).
+ * prism_dense_decode sizes its split grid from the host copy,
+ * which must be current for it.  head_dim is 64 or 128; num_q_heads is a
+ * multiple of num_kv_heads with G <= 16; batch <= 4096. */
 typedef struct prism_shape {
   int32_t batch;
   int32_t num_q_heads;

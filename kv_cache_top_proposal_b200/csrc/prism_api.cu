@@ -39,7 +39,7 @@ prism_status check_shape(const prism_shape* s, Dims* d) {
     const int L = cu[b + 1] - cu[b];
     if (L > max_len) max_len = L;
   }
-  if ((int64_t)cu[s->batch] != s->total_tokens) return PRISM_ERR_INVALID_ARG;
+  if ((int64_t)cu[s->batch] > s->total_tokens) return PRISM_ERR_INVALID_ARG;  // spare rows allowed
   d->B = s->batch;
   d->Hq = s->num_q_heads;
   d->Hkv = s->num_kv_heads;

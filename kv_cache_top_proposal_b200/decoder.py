@@ -18,6 +18,7 @@ so it can be captured in a CUDA graph.
 """
 from __future__ import annotations
 
+import contextlib
 import math
 from typing import List, Optional
 
@@ -29,9 +30,11 @@ from . import prism
 class PrismDecoder:
     def __init__(self, seqlens, num_q_heads: int, num_kv_heads: int, head_dim: int, dtype: int,
                  num_layers: int, group: int, kappa_p: int, kappa: int, device="cuda",
-                 softmax_scale: Optional[float] = None, fused: bool = True, keys: str = "int8"):
+                 softmax_scale: Optional[float] = None, fused: bool = True, keys: str = "int8",
+                 capacity: Optional[int] = None):
         self.dev = torch.device(device)
-        self.p = prism.Problem(seqlens, num_q_heads, num_kv_heads, head_dim, dtype, device=self.dev)
+        self.p = prism.Problem(seqlens, num_q_heads, num_kv_heads, head_dim, dtype, device=self.dev,
+                               capacity=capacity)
         self.B, self.Hq, self.Hkv, self.D = len(seqlens), num_q_heads, num_kv_heads, head_dim
         self.num_layers, self.group = num_layers, group
         self.kappa_p, self.kappa = kappa_p, kappa
@@ -50,9 +53,12 @@ class PrismDecoder:
         self.lse_all = torch.zeros((num_layers, B, Hq), **f32)
         self.out = [self.out_all[l] for l in range(num_layers)]
         self.lse = [self.lse_all[l] for l in range(num_layers)]
-        # the newly appended token of every sequence (packed row index)
-        last = [c - 1 for c in self.p.cu_host[1:].tolist() if True]
-        self.new_rows = torch.tensor([r for r, L in zip(last, seqlens) if L > 0], **i32)
+        # the newly appended token of every sequence (packed row index), with
+        # a page-locked host mirror that grow() advances
+        last = [c - 1 for c in self.p.cu_host[1:].tolist()]
+        rows = torch.tensor([r for r, L in zip(last, seqlens) if L > 0], dtype=torch.int32)
+        self._new_rows_host = rows.pin_memory() if self.dev.type == "cuda" else rows.clone()
+        self.new_rows = rows.to(self.dev)
 
         def ws(op, kp=0, k=0):
             n = prism.workspace_size(self.p, op, kp, k)
@@ -138,6 +144,42 @@ class PrismDecoder:
                        k_new=None if k_new is None else k_new[l],
                        v_new=None if v_new is None else v_new[l],
                        overlap=self.fused and not pl and l > 0, stream=stream)
+
+    def grow(self, n: int = 1):
+        """Decode loop over one growing sequence: the last sequence gets n more
+        tokens (the next step appends its token at the new last position).
+        Host mirrors only; lengths_to_device() sends them, on the stream,
+        ahead of the step's kernels (inside a captured step graph, each
+        replay copies the mirrors as they are then)."""
+        assert self.p.seqlens[-1] > 0, "the last sequence is empty"
+        self.p.grow(n)
+        self._new_rows_host[-1] += n
+
+    def lengths_to_device(self, stream=None):
+        """Enqueue the copies of cu_seqlens and of the new-token rows from
+        their host mirrors to the device."""
+        ctx = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+        with ctx:
+            self.p.cu_dev.copy_(self.p.cu_pin, non_blocking=True)
+            self.new_rows.copy_(self._new_rows_host, non_blocking=True)
+
+    def advance_on_device(self, n: int = 1):
+        """The device-only form of grow(): the last sequence's length and
+        new-token row move on by n on the current stream, so that a captured
+        step graph that starts with this call advances the loop on every
+        replay without the host (whose mirrors then keep the capture-time
+        lengths)."""
+        self.p.cu_dev[-1:].add_(n)
+        self.new_rows[-1:].add_(n)
+
+    def lengths_from_device(self):
+        """Bring the host mirrors back in line with the device lengths (after
+        advance_on_device), for calls that size their work from the host
+        copy (dense decode)."""
+        cu = self.p.cu_dev.cpu()
+        self.p.cu_pin.copy_(cu)
+        self.p.seqlens = [int(x) for x in (cu[1:] - cu[:-1]).tolist()]
+        self._new_rows_host.copy_(self.new_rows.cpu())
 
     def launches_per_step(self, append: bool) -> int:
         """Kernels one step enqueues (append, quantize, score, select, refine

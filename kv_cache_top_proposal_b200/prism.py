@@ -110,22 +110,32 @@ class Problem:
     """A layer-shape descriptor (the C ``prism_shape``) plus its cu_seqlens.
 
     ``seqlens`` are the per-sequence context lengths; the device copy of
-    cu_seqlens lives on ``device`` and the host mirror in a numpy array that
-    this object keeps alive.
+    cu_seqlens lives on ``device`` and the host mirror in an array that this
+    object keeps alive (page-locked when ``device`` is a GPU, so a captured
+    graph can copy it).  ``capacity`` (default: the total length) is the row
+    count of every per-token array; rows past the last sequence are spare,
+    for a decode loop that grows the last sequence (``grow``).
     """
 
     def __init__(self, seqlens: Sequence[int], num_q_heads: int, num_kv_heads: int, head_dim: int,
-                 dtype: int, device="cuda", cu_dev=None):
+                 dtype: int, device="cuda", cu_dev=None, capacity: Optional[int] = None):
         import torch
 
         cu = np.zeros(len(seqlens) + 1, np.int32)
         cu[1:] = np.cumsum(np.asarray(seqlens, np.int64)).astype(np.int32)
-        self.cu_host = cu
-        self.cu_dev = cu_dev if cu_dev is not None else torch.tensor(cu, dtype=torch.int32, device=device)
+        host = torch.from_numpy(cu)
+        if torch.device(device).type == "cuda":
+            host = host.pin_memory()
+        self.cu_pin = host                # host mirror (the C shape points at it)
+        self.cu_host = host.numpy()       # the same memory, as numpy
+        self.cu_dev = cu_dev if cu_dev is not None else host.to(device)
         self.seqlens = [int(x) for x in seqlens]
+        self.capacity = int(cu[-1]) if capacity is None else int(capacity)
+        if self.capacity < int(cu[-1]):
+            raise ValueError("capacity below the total length")
         self.shape = Shape(len(seqlens), num_q_heads, num_kv_heads, head_dim, dtype,
                            ctypes.c_void_p(self.cu_dev.data_ptr()),
-                           ctypes.c_void_p(cu.ctypes.data), int(cu[-1]))
+                           ctypes.c_void_p(host.data_ptr()), self.capacity)
 
     @property
     def ref(self):
@@ -133,7 +143,17 @@ class Problem:
 
     @property
     def total_tokens(self) -> int:
-        return int(self.cu_host[-1])
+        """Rows of every per-token array (the capacity)."""
+        return self.capacity
+
+    def grow(self, n: int = 1):
+        """The last sequence gets n more tokens, in the host mirror only; copy
+        ``cu_pin`` to ``cu_dev`` on the stream before the kernels that should
+        see it (decoder.PrismDecoder.lengths_to_device)."""
+        if int(self.cu_host[-1]) + n > self.capacity:
+            raise ValueError("the last sequence would outgrow the capacity")
+        self.cu_host[-1] += n
+        self.seqlens[-1] += n
 
 
 def workspace_size(p: Problem, op: int, kappa_p: int = 0, kappa: int = 0) -> int:

@@ -73,8 +73,11 @@ def test_bad_cu_seqlens_rejected(prism_lib):
     cu[1] = 200  # not monotone
     assert _ws(P, s, P.OP_PROPOSE, 16)[0] == P.ERR_INVALID_ARG
     s, cu = _shape(P, [100, 50])
-    s.total_tokens = 151  # disagrees with cu[B]
+    s.total_tokens = 149  # fewer rows than cu[B]
     assert _ws(P, s, P.OP_PROPOSE, 16)[0] == P.ERR_INVALID_ARG
+    s, cu = _shape(P, [100, 50])
+    s.total_tokens = 151  # one spare row past cu[B]: accepted
+    assert _ws(P, s, P.OP_PROPOSE, 16)[0] == P.OK
     s, cu = _shape(P, [100])
     cu[0] = 1
     assert _ws(P, s, P.OP_PROPOSE, 16)[0] == P.ERR_INVALID_ARG

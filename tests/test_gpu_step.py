@@ -178,3 +178,67 @@ def test_step_int2_keys_c8k_every_row(prism_lib):
             check_index_set(gidx[b, h, :c], oidx[b, h, :c], lambda t: r[t], f"L{l} idx {b},{h}")
         oout, _ = pipeline.attend_layer(lay.q, lay.k, lay.v, cu, gidx, gcnt, dec.scale, rows=rows)
         assert np.abs(_np(dec.out[l]) - oout).max() <= atol_for(cfg.dtype)
+
+
+def test_decode_loop_grows_one_sequence(prism_lib):
+    """A decode loop over one growing sequence: the cache holds spare rows,
+    one step graph is captured once, and before each replay the sequence
+    grows by one token, whose K/V rows every layer appends (the proposal
+    layer's scorer quantizes its key row).  After every step the proposal
+    codes match the oracle's quantizer bit for bit, and pools, index sets
+    and outputs match the oracle at that length (c8k shapes, four layers)."""
+    P = prism_lib
+    steps = 3
+    cfg = workload.config("c8k").replace(num_layers=4)
+    layers = list(workload.generate(cfg, DEV))
+    cap = cfg.seqlens[0]
+    L0 = cap - steps
+    # the rows the loop appends: kept aside, then overwritten in the cache
+    news = [(lay.k[:, L0:].clone(), lay.v[:, L0:].clone()) for lay in layers]
+    for lay in layers:
+        lay.k[:, L0:] = 7.0
+        lay.v[:, L0:] = -7.0
+    dec = PrismDecoder([L0], cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, P.BF16,
+                       cfg.num_layers, cfg.group, cfg.kappa_p, cfg.kappa, device=DEV, capacity=cap)
+    assert dec.scorer_appends
+    kqs, scs = {}, {}
+    for lay in layers:
+        if cfg.is_proposal(lay.index):
+            kqs[lay.index], scs[lay.index] = _prefill_kq(P, dec, cfg, lay)
+    qbuf = [lay.q.clone() for lay in layers]
+    knbuf = [torch.empty((1, cfg.num_kv_heads, cfg.head_dim), dtype=torch.bfloat16, device=DEV)
+             for _ in layers]
+    vnbuf = [torch.empty_like(x) for x in knbuf]
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        dec.lengths_to_device()
+        dec.step(qbuf, [x.k for x in layers], [x.v for x in layers], kqs, scs, k_new=knbuf,
+                 v_new=vnbuf)
+    gen = torch.Generator(device="cpu").manual_seed(77)
+    for t in range(steps):
+        dec.grow(1)
+        L = L0 + t + 1
+        for l, lay in enumerate(layers):
+            qbuf[l].copy_((lay.q.float().cpu() + 0.3 * torch.randn(lay.q.shape, generator=gen))
+                          .to(torch.bfloat16))
+            knbuf[l].copy_(news[l][0][:, t][None])
+            vnbuf[l].copy_(news[l][1][:, t][None])
+        g.replay()
+        torch.cuda.synchronize()
+        assert dec.device_status() == 0
+        assert int(dec.p.cu_dev[-1]) == L
+        cfg_t = cfg.replace(seqlens=(L,))
+        for l, lay in enumerate(layers):
+            # the cache as the step left it: rows < L with this step's token at L - 1
+            assert torch.equal(lay.k[:, L - 1], news[l][0][:, t])
+            assert torch.equal(lay.v[:, L - 1], news[l][1][:, t])
+            view = workload.Layer(l, qbuf[l], lay.k[:, :L], lay.v[:, :L])
+            if cfg.is_proposal(l):
+                okq, osc = pipeline.quantize_layer(view.k)
+                assert np.array_equal(_np(kqs[l][:, :L]), okq)
+                assert np.array_equal(_np(scs[l][:, :L]).view(np.uint32), osc.view(np.uint32))
+            src = l - l % cfg.group
+            _invariants(dec, cfg_t, l)
+            _check_layer(dec, cfg_t, l, view, kqs[src][:, :L], scs[src][:, :L], _all_rows(cfg_t))
+    del g
