@@ -5,16 +5,20 @@ in the "g x" setting one layer in every x is a proposal layer; the pages
 inherit the partition from an offline calibration, sec. 4 Overview, which is
 replaced here by the periodic map ``layer % group == 0``):
 
-  proposal layer l:  quantize the newly appended key row of every sequence
-                     (prism_quantize_k on the last position), then
-                     prism_propose -> candidate pool of kappa_p positions;
-  every layer l:     prism_refine on the latest pool -> kappa positions,
-                     prism_sparse_decode over them -> out[l], lse[l].
+  proposal layer l:  the token's key rows are quantized into the proposal
+                     codes and the codes are scored (prism_propose_append,
+                     or prism_quantize_k then prism_propose / their INT2
+                     forms) -> candidate pool of kappa_p positions;
+  every layer l:     prism_refine_decode on the latest pool: exact rescoring,
+                     top kappa, sparse flash-decode and merge in one launch,
+                     appending the layer's new K/V rows -> out[l], lse[l]
+                     (or prism_refine then prism_sparse_decode).
 
 A proposal layer also refines its own pool and attends over the refined set
 (every layer attends over kappa exactly rescored tokens).  All buffers are
 allocated once by torch; a step only enqueues library calls on one stream,
-so it can be captured in a CUDA graph.
+so it can be captured in a CUDA graph.  A decode loop over one growing
+sequence (grow / advance_on_device) replays one captured step per token.
 """
 from __future__ import annotations
 
