@@ -382,6 +382,21 @@ __device__ __forceinline__ void tma_rows(void* dst, const CUtensorMap* tm, int y
       : "memory");
 }
 
+// The same copy marked evict-first in L2: the code stream is read once, and
+// should not push out of L2 the scores and histograms the selection reads
+// right after the scorer.
+__device__ __forceinline__ void tma_rows_stream(void* dst, const CUtensorMap* tm, int y, uint64_t* bar,
+                                                uint64_t policy) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
+               "r"(kTmaStageBytes)
+               : "memory");
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;\n" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(0), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 3) score_tma_kernel(const __grid_constant__ CUtensorMap tm,
                                                                 ScoreArgs a) {
@@ -643,7 +658,10 @@ __global__ void __launch_bounds__(kThreads, 3) score_i8_kernel(const __grid_cons
   auto issue = [&](int kk) {  // thread 0
     if (kk < nk) {
       const int64_t y = (int64_t)it_issue.h * a.T + s_cu[it_issue.b] + it_issue.r0;
-      tma_rows(ring + (kk % kTmaStages) * kTmaStageBytes, &tm, (int)y, &full[kk % kTmaStages]);
+      uint64_t evict_first;
+      asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(evict_first));
+      tma_rows_stream(ring + (kk % kTmaStages) * kTmaStageBytes, &tm, (int)y, &full[kk % kTmaStages],
+                      evict_first);
       it_issue.advance(s_cu, a.B);
     }
   };
