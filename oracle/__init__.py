@@ -56,6 +56,12 @@ def _L():
         lib.oracle_refine_row.argtypes = [P, i32, i32, P, P, i32, i32, P, P]
         lib.oracle_refine_row.restype = i32
         lib.oracle_attend.argtypes = [P, i32, P, P, P, i32, f64, P, P]
+        lib.oracle_propose_scores_sum.argtypes = [P, i32, i32, P, P, i32, P]
+        lib.oracle_propose_row_sum.argtypes = [P, i32, i32, P, P, i32, i32, P, P]
+        lib.oracle_propose_row_sum.restype = i32
+        lib.oracle_refine_scores_sum.argtypes = [P, i32, i32, P, P, i32, P]
+        lib.oracle_refine_row_sum.argtypes = [P, i32, i32, P, P, i32, i32, P, P]
+        lib.oracle_refine_row_sum.restype = i32
         lib.oracle_f32_to_f16.argtypes = [ctypes.c_float]
         lib.oracle_f32_to_f16.restype = ctypes.c_uint16
         lib.oracle_f16_to_f32.argtypes = [ctypes.c_uint16]
@@ -98,44 +104,55 @@ def topk_ascending(s, k: int) -> np.ndarray:
     return out[:m].copy()
 
 
-def propose_scores(q, kq, scale) -> np.ndarray:
-    """s_t = scale_t * max_g sum_j q[g, j] * kq[t, j] (fp32, j ascending)."""
+AGGS = ("max", "sum")  # how the G query heads of a KV head combine into one selection score
+
+
+def _sfx(agg: str) -> str:
+    if agg not in AGGS:
+        raise ValueError(f"agg must be one of {AGGS}")
+    return "" if agg == "max" else "_sum"
+
+
+def propose_scores(q, kq, scale, agg: str = "max") -> np.ndarray:
+    """s_t = scale_t * max_g (or sum_g) sum_j q[g, j] * kq[t, j] (fp32, j ascending)."""
     q, kq, scale = _f32(q), np.ascontiguousarray(kq, dtype=np.int8), _f32(scale)
     G, d = q.shape
     L = kq.shape[0]
     s = np.empty((L,), np.float32)
-    _L().oracle_propose_scores(_p(q), G, d, _p(kq), _p(scale), L, _p(s))
+    getattr(_L(), "oracle_propose_scores" + _sfx(agg))(_p(q), G, d, _p(kq), _p(scale), L, _p(s))
     return s
 
 
-def propose_row(q, kq, scale, kappa_p: int):
+def propose_row(q, kq, scale, kappa_p: int, agg: str = "max"):
     """(pool ascending int32 [min(kappa_p, L)], proposal scores [L])."""
     q, kq, scale = _f32(q), np.ascontiguousarray(kq, dtype=np.int8), _f32(scale)
     G, d = q.shape
     L = kq.shape[0]
     s = np.empty((max(L, 1),), np.float32)
     pool = np.empty((max(min(kappa_p, L), 1),), np.int32)
-    m = _L().oracle_propose_row(_p(q), G, d, _p(kq), _p(scale), L, kappa_p, _p(pool), _p(s))
+    m = getattr(_L(), "oracle_propose_row" + _sfx(agg))(_p(q), G, d, _p(kq), _p(scale), L, kappa_p,
+                                                        _p(pool), _p(s))
     return pool[:m].copy(), s[:L].copy()
 
 
-def refine_scores(q, K, pool) -> np.ndarray:
-    """r_i = max_g sum_j q[g, j] * K[pool_i, j] (fp32, j ascending)."""
+def refine_scores(q, K, pool, agg: str = "max") -> np.ndarray:
+    """r_i = max_g (or sum_g) sum_j q[g, j] * K[pool_i, j] (fp32, j ascending)."""
     q, K, pool = _f32(q), _f32(K), _i32(pool)
     G, d = q.shape
     r = np.empty((max(pool.size, 1),), np.float32)
-    _L().oracle_refine_scores(_p(q), G, d, _p(K), _p(pool), pool.size, _p(r))
+    getattr(_L(), "oracle_refine_scores" + _sfx(agg))(_p(q), G, d, _p(K), _p(pool), pool.size, _p(r))
     return r[:pool.size].copy()
 
 
-def refine_row(q, K, pool, kappa: int):
+def refine_row(q, K, pool, kappa: int, agg: str = "max"):
     """(refined positions ascending int32 [min(kappa, |pool|)], exact pool scores)."""
     q, K, pool = _f32(q), _f32(K), _i32(pool)
     G, d = q.shape
     n = pool.size
     r = np.empty((max(n, 1),), np.float32)
     idx = np.empty((max(min(kappa, n), 1),), np.int32)
-    m = _L().oracle_refine_row(_p(q), G, d, _p(K), _p(pool), n, kappa, _p(idx), _p(r))
+    m = getattr(_L(), "oracle_refine_row" + _sfx(agg))(_p(q), G, d, _p(K), _p(pool), n, kappa,
+                                                       _p(idx), _p(r))
     return idx[:m].copy(), r[:n].copy()
 
 

@@ -49,8 +49,9 @@ def quantize_layer(k):
     return kq.reshape(Hkv, T, d), sc.reshape(Hkv, T)
 
 
-def propose_layer(q, kq, scale, cu, kappa_p: int, rows=None):
-    """pool [B][Hkv][kappa_p] (-1 padded), pool_cnt [B][Hkv], scores per row."""
+def propose_layer(q, kq, scale, cu, kappa_p: int, rows=None, agg: str = "max"):
+    """pool [B][Hkv][kappa_p] (-1 padded), pool_cnt [B][Hkv], scores per row
+    (agg: how the group's query heads combine, "max" or "sum")."""
     q = _np(q).astype(np.float32)
     kq, scale = _np(kq), _np(scale).astype(np.float32)
     B, Hq, d = q.shape
@@ -64,7 +65,7 @@ def propose_layer(q, kq, scale, cu, kappa_p: int, rows=None):
         for h in range(Hkv):
             if rows is not None and (b, h) not in rows:
                 continue
-            p, s = propose_row(q[b, h * G:(h + 1) * G], kq[h, t0:t1], scale[h, t0:t1], kappa_p)
+            p, s = propose_row(q[b, h * G:(h + 1) * G], kq[h, t0:t1], scale[h, t0:t1], kappa_p, agg)
             pool[b, h, :p.size] = p
             cnt[b, h] = p.size
             scores[(b, h)] = s
@@ -102,8 +103,9 @@ def propose_layer_int2(q, codes, params, cu, kappa_p: int, rows=None):
     return pool, cnt, scores
 
 
-def refine_layer(q, k, cu, pool, pool_cnt, kappa: int, rows=None):
-    """idx [B][Hkv][kappa] (-1 padded), cnt [B][Hkv], exact pool scores per row."""
+def refine_layer(q, k, cu, pool, pool_cnt, kappa: int, rows=None, agg: str = "max"):
+    """idx [B][Hkv][kappa] (-1 padded), cnt [B][Hkv], exact pool scores per row
+    (agg as in propose_layer)."""
     q = _np(q).astype(np.float32)
     k = _np(k).astype(np.float32)
     pool, pool_cnt = _np(pool), _np(pool_cnt)
@@ -119,7 +121,7 @@ def refine_layer(q, k, cu, pool, pool_cnt, kappa: int, rows=None):
             if rows is not None and (b, h) not in rows:
                 continue
             n = int(pool_cnt[b, h])
-            sel, r = refine_row(q[b, h * G:(h + 1) * G], k[h, t0:t1], pool[b, h, :n], kappa)
+            sel, r = refine_row(q[b, h * G:(h + 1) * G], k[h, t0:t1], pool[b, h, :n], kappa, agg)
             idx[b, h, :sel.size] = sel
             cnt[b, h] = sel.size
             scores[(b, h)] = r

@@ -184,6 +184,65 @@ int32_t oracle_refine_row(const float* q, int32_t G, int32_t d, const float* K,
 }
 
 /*
+ * Group aggregation by sum, the selection variant next to the maximum above
+ * (the pages leave open how the G query heads of a KV head share one set;
+ * the sum is the other plain reading):
+ *   proposal: s_t = scale_t * sum_g D_g(t)                  g ascending, fp32
+ *   refine:   r_i = sum_g sum_j q[g][j] * K[pool_i][j]      g, j ascending, fp32
+ * The selections over them are those of the maximum forms.
+ */
+void oracle_propose_scores_sum(const float* q, int32_t G, int32_t d, const int8_t* kq,
+                               const float* scale, int32_t L, float* s) {
+  for (int32_t t = 0; t < L; ++t) {
+    const int8_t* kr = kq + (int64_t)t * d;
+    float tot = 0.0f;
+    for (int32_t g = 0; g < G; ++g) {
+      float acc = 0.0f;
+      for (int32_t j = 0; j < d; ++j) acc = acc + q[g * d + j] * (float)kr[j];
+      tot = tot + acc;
+    }
+    s[t] = scale[t] * tot;
+  }
+}
+
+int32_t oracle_propose_row_sum(const float* q, int32_t G, int32_t d, const int8_t* kq,
+                               const float* scale, int32_t L, int32_t kappa_p, int32_t* pool,
+                               float* scores_out) {
+  float* s = scores_out ? scores_out : (float*)malloc(sizeof(float) * (size_t)(L > 0 ? L : 1));
+  oracle_propose_scores_sum(q, G, d, kq, scale, L, s);
+  int32_t n = oracle_topk_ascending(s, L, kappa_p, pool);
+  if (!scores_out) free(s);
+  return n;
+}
+
+void oracle_refine_scores_sum(const float* q, int32_t G, int32_t d, const float* K,
+                              const int32_t* pool, int32_t n, float* r) {
+  for (int32_t i = 0; i < n; ++i) {
+    const float* kr = K + (int64_t)pool[i] * d;
+    float tot = 0.0f;
+    for (int32_t g = 0; g < G; ++g) {
+      float acc = 0.0f;
+      for (int32_t j = 0; j < d; ++j) acc = acc + q[g * d + j] * kr[j];
+      tot = tot + acc;
+    }
+    r[i] = tot;
+  }
+}
+
+int32_t oracle_refine_row_sum(const float* q, int32_t G, int32_t d, const float* K,
+                              const int32_t* pool, int32_t n, int32_t kappa, int32_t* idx,
+                              float* r_out) {
+  float* r = r_out ? r_out : (float*)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
+  oracle_refine_scores_sum(q, G, d, K, pool, n, r);
+  int32_t* slot = (int32_t*)malloc(sizeof(int32_t) * (size_t)(n > 0 ? n : 1));
+  int32_t m = oracle_topk_ascending(r, n, kappa, slot);
+  for (int32_t i = 0; i < m; ++i) idx[i] = pool[slot[i]];
+  free(slot);
+  if (!r_out) free(r);
+  return m;
+}
+
+/*
  * Softmax attention of one query head over the rows listed in idx (all rows
  * 0..n-1 when idx is NULL), in fp64:
  *   l_t = softmax_scale * sum_j q_j k_tj
