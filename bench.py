@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--profile-steps", type=int, default=5)
     ap.add_argument("--keys", default="int8", choices=["int8", "int2"],
                     help="proposal key cache: int8 per token (the headline workload) or INT2 per 32-feature group")
+    ap.add_argument("--group-agg", default="max", choices=["max", "sum"],
+                    help="how the query heads of a KV head combine into the selection score")
     ap.add_argument("--grow", action="store_true",
                     help="decode loop over the growing sequence: every replayed step appends one "
                          "token (batch-1 configs); the cache starts short by the replays")
@@ -211,7 +213,7 @@ def traffic_for(op: str):
 
 # --------------------------------------------------------------------------- CPU oracle legs
 
-def oracle_units(cfg, qs, ks, vs, units, budget_s: float, keys: str = "int8"):
+def oracle_units(cfg, qs, ks, vs, units, budget_s: float, keys: str = "int8", agg: str = "max"):
     """Run the CPU oracle on (proposal group, KV head) units of one decode
     step until budget_s seconds of oracle time; returns (units done, seconds).
     Inputs are copied from the generated cache; untimed: host copies and the
@@ -235,10 +237,13 @@ def oracle_units(cfg, qs, ks, vs, units, budget_s: float, keys: str = "int8"):
             if e == a:
                 continue
             quant(host[lp][1][e - 1:e])  # the new token's key row
-            pool, _ = propose(host[lp][0][b], kq[a:e], sc[a:e], cfg.kappa_p)
+            if keys == "int2":
+                pool, _ = propose(host[lp][0][b], kq[a:e], sc[a:e], cfg.kappa_p)
+            else:
+                pool, _ = propose(host[lp][0][b], kq[a:e], sc[a:e], cfg.kappa_p, agg=agg)
             for l in lays:
                 q, k, v = host[l]
-                idx, _ = oracle.refine_row(q[b], k[a:e], pool, cfg.kappa)
+                idx, _ = oracle.refine_row(q[b], k[a:e], pool, cfg.kappa, agg=agg)
                 for g in range(G):
                     oracle.attend(q[b, g], k[a:e], v[a:e], idx, scale)
         spent += time.perf_counter() - t0
@@ -269,8 +274,8 @@ def run_reference(args, dist: Dist):
     vs = {x.index: x.v for x in lays}
     per_step_units = len(unit_list(cfg))
     units = [(0, h % cfg.num_kv_heads) for h in range(args.warmup + args.steps)]
-    oracle_units(cfg, qs, ks, vs, units[:args.warmup], 1e9, args.keys)
-    n, secs = oracle_units(cfg, qs, ks, vs, units[args.warmup:], 1e9, args.keys)
+    oracle_units(cfg, qs, ks, vs, units[:args.warmup], 1e9, args.keys, args.group_agg)
+    n, secs = oracle_units(cfg, qs, ks, vs, units[args.warmup:], 1e9, args.keys, args.group_agg)
     value = (n / per_step_units) / secs
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
@@ -330,7 +335,7 @@ def run_prism(args, dist: Dist):
     dec = PrismDecoder(seqlens0, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim,
                        prism.BF16 if cfg.dtype == "bf16" else prism.F32, L, cfg.group,
                        cfg.kappa_p, cfg.kappa, device=dev, keys=args.keys,
-                       capacity=cfg.total_tokens)
+                       capacity=cfg.total_tokens, group_agg=args.group_agg)
     rows = dec.new_rows.long()
     Hkv = cfg.num_kv_heads
     k_new = torch.stack([k[:, rows].transpose(0, 1).contiguous() for k in ks])  # [L][B][Hkv][d]
@@ -421,7 +426,7 @@ def run_prism(args, dist: Dist):
         def f_prop(l=l):
             if dec.scorer_appends:  # the scorer quantizes the new key rows; the refined layer appends
                 prism.propose_append(dec.p, q_layers[l], k_new[l], kqs[l], scs[l], cfg.kappa_p,
-                                     dec.pool[l], dec.pool_cnt[l], dec.ws_prop)
+                                     dec.pool[l], dec.pool_cnt[l], dec.ws_prop, sum_group=dec.sum_group)
                 return
             prism.append_kv(dec.p, k_new[l], v_new[l], ks[l], vs[l])
             if args.keys == "int2":
@@ -441,7 +446,8 @@ def run_prism(args, dist: Dist):
             prism.refine_decode(dec.p, q_layers[l], ks[l], vs[l], dec.pool[src], dec.pool_cnt[src],
                                 cfg.kappa_p, cfg.kappa, dec.scale, dec.idx[l], dec.cnt[l],
                                 dec.out[l], dec.ws_rd, lse=dec.lse[l],
-                                k_new=k_new[l] if fa else None, v_new=v_new[l] if fa else None)
+                                k_new=k_new[l] if fa else None, v_new=v_new[l] if fa else None,
+                                sum_group=dec.sum_group)
 
         if pl:
             ops.append(("propose", graph_of(f_prop, stream)))
@@ -507,7 +513,7 @@ def run_prism(args, dist: Dist):
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
         units = unit_list(cfg)
-        n, s = oracle_units(cfg, q_layers, ks, vs, units, args.cpu_seconds, args.keys)
+        n, s = oracle_units(cfg, q_layers, ks, vs, units, args.cpu_seconds, args.keys, args.group_agg)
         cpu = {"value": (n / len(units)) / s, "unit": "steps/s", "cores": 1, "kind": "oracle",
                "sample": f"{n} of the {len(units)} (proposal group, KV head) units of one "
                          f"{cfg.name} decode step ({s:.1f} s of single-thread oracle time)"}
@@ -525,6 +531,7 @@ def run_prism(args, dist: Dist):
                            proposal_keys="int8 per token" if args.keys == "int8"
                            else "INT2 per 32-feature group (fp16 step and zero point)",
                            graph="one CUDA graph per step",
+                           group_aggregation=args.group_agg,
                            **({"growth": f"decode loop: every replayed step appends one token, "
                                          f"from L = {seqlens0[0]} to {seqlens0[0] + n_grow}"}
                               if args.grow else {})),

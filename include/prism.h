@@ -176,13 +176,18 @@ PRISM_API prism_status prism_propose(const prism_shape* shape, const void* q, co
  * the rest -- one launch fewer than prism_quantize_k + prism_propose, and the
  * K cache itself is not read (the new row may be appended to it later, e.g.
  * by prism_refine_decode).  Same outputs, workspace and rules as
- * prism_propose.  bf16, d = 128, G <= 8 and L_b <= PRISM_MAX_SELECT_ROW only
- * (else PRISM_ERR_UNSUPPORTED); q, k_new and kq 16-byte aligned.
+ * prism_propose.  bf16, d = 128, G <= 8 and L_b <= 131072 only (else
+ * PRISM_ERR_UNSUPPORTED); q, k_new and kq 16-byte aligned.
+ * flags: PRISM_PROPOSE_SUM_GROUP selects the group-sum variant,
+ *   s_t = k_scale[h][t] * sum_{g<G} sum_j q[b][h*G+g][j] * kq[h][t][j];
+ * other bits are rejected (PRISM_ERR_INVALID_ARG).
  */
+#define PRISM_PROPOSE_SUM_GROUP 0x1u
 PRISM_API prism_status prism_propose_append(const prism_shape* shape, const void* q,
                                             const void* k_new, int8_t* kq, float* k_scale,
                                             int32_t kappa_p, int32_t* pool_idx, int32_t* pool_cnt,
-                                            void* ws, size_t ws_bytes, void* stream);
+                                            uint32_t flags, void* ws, size_t ws_bytes,
+                                            void* stream);
 
 /*
  * INT2 proposal keys (sec. 4.2: the pages compress the proposal layers' key
@@ -275,8 +280,12 @@ PRISM_API prism_status prism_sparse_decode(const prism_shape* shape, const void*
  * status word; it touches q, v, k_new_opt, v_new_opt and its outputs only
  * afterwards.  Set it only when the previous kernel writes none of the
  * former (e.g. the refined layer before this one, on the same pool).
+ * PRISM_RD_SUM_GROUP selects the group-sum variant of the exact score:
+ * r_i = sum_g sum_j q[g][j] * K[pool_i][j] in place of the maximum over g
+ * (the selection and the attention are unchanged).
  */
 #define PRISM_RD_OVERLAP 0x1u
+#define PRISM_RD_SUM_GROUP 0x2u
 PRISM_API prism_status prism_refine_decode(const prism_shape* shape, const void* q, void* k,
                                            void* v, const int32_t* pool_idx,
                                            const int32_t* pool_cnt, int32_t kappa_p,

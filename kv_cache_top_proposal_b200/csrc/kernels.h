@@ -48,11 +48,12 @@ cudaError_t launch_propose_scores(const Dims& d, const void* q, const int8_t* kq
 // the first-digit histogram (bf16 queries, d = 128; score.cu).
 // The integer scorer with this token's key rows k_new [B][Hkv][d] (bf16),
 // quantized by the scorer into kq / scale at position L_b - 1 of every
-// non-empty sequence before that position is scored.  bf16, d = 128, G <= 8
-// only (cudaErrorInvalidValue otherwise).
+// non-empty sequence before that position is scored; sum_group: the
+// selection score sums the group's query heads instead of taking their
+// maximum.  bf16, d = 128, G <= 8 only (cudaErrorInvalidValue otherwise).
 cudaError_t launch_propose_scores_new_rows(const Dims& d, const void* q, int8_t* kq, float* scale,
                                            const void* k_new, float* scores, uint32_t* hist,
-                                           int32_t* status, cudaStream_t st);
+                                           bool sum_group, int32_t* status, cudaStream_t st);
 cudaError_t launch_propose_scores_int2(const Dims& d, const void* q, const uint8_t* codes,
                                        const uint16_t* params, float* scores, uint32_t* hist,
                                        int32_t* status, cudaStream_t st);
@@ -106,7 +107,8 @@ cudaError_t launch_refine_decode(const Dims& d, const RefineDecodePlan& p, const
                                  const void* v_new, const void* k_next, const int32_t* pool,
                                  const int32_t* pool_cnt, int kappa_p, int kappa,
                                  float softmax_scale, int32_t* idx, int32_t* cnt, float* out,
-                                 float* lse, int32_t* status, bool overlap, cudaStream_t st);
+                                 float* lse, int32_t* status, bool overlap, bool sum_group,
+                                 cudaStream_t st);
 
 // Split-K attention partials over idx rows (idx == nullptr: every position).
 struct AttendPlan {

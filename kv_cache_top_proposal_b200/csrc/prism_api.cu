@@ -208,12 +208,14 @@ prism_status prism_propose(const prism_shape* shape, const void* q, const int8_t
 
 prism_status prism_propose_append(const prism_shape* shape, const void* q, const void* k_new,
                                   int8_t* kq, float* k_scale, int32_t kappa_p, int32_t* pool_idx,
-                                  int32_t* pool_cnt, void* ws, size_t ws_bytes, void* stream) {
+                                  int32_t* pool_cnt, uint32_t flags, void* ws, size_t ws_bytes,
+                                  void* stream) {
   Dims d;
   prism_status s = check_shape(shape, &d);
   if (s != PRISM_OK) return s;
   if (!q || !k_new || !kq || !k_scale || !pool_idx || !pool_cnt || kappa_p < 1)
     return PRISM_ERR_INVALID_ARG;
+  if (flags & ~PRISM_PROPOSE_SUM_GROUP) return PRISM_ERR_INVALID_ARG;
   if (!d.bf16 || d.D != 128 || d.G > 8 || d.max_len > propose_select_max_row())
     return PRISM_ERR_UNSUPPORTED;
   if (((uintptr_t)q | (uintptr_t)k_new | (uintptr_t)kq) % 16) return PRISM_ERR_INVALID_ARG;
@@ -227,7 +229,8 @@ prism_status prism_propose_append(const prism_shape* shape, const void* q, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t rows = (size_t)d.B * d.Hkv;
   if (cudaMemsetAsync(hist, 0, rows * 4096 * 4, st) != cudaSuccess) return PRISM_ERR_CUDA;
-  cudaError_t e = launch_propose_scores_new_rows(d, q, kq, k_scale, k_new, scores, hist, status, st);
+  cudaError_t e = launch_propose_scores_new_rows(d, q, kq, k_scale, k_new, scores, hist,
+                                                 (flags & PRISM_PROPOSE_SUM_GROUP) != 0, status, st);
   if (e == cudaErrorInvalidValue) return PRISM_ERR_UNSUPPORTED;
   if (e != cudaSuccess) return PRISM_ERR_CUDA;
   return cuda_status(launch_propose_select(d, scores, hist, kappa_p, pool_idx, pool_cnt, status, st));
@@ -359,7 +362,7 @@ prism_status prism_refine_decode(const prism_shape* shape, const void* q, void* 
   if (!q || !k || !v || !pool_idx || !pool_cnt || !idx || !cnt || !out) return PRISM_ERR_INVALID_ARG;
   if (kappa_p < 1 || kappa < 1 || kappa > kappa_p) return PRISM_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale)) return PRISM_ERR_INVALID_ARG;
-  if (flags & ~PRISM_RD_OVERLAP) return PRISM_ERR_INVALID_ARG;
+  if (flags & ~(PRISM_RD_OVERLAP | PRISM_RD_SUM_GROUP)) return PRISM_ERR_INVALID_ARG;
   if ((k_new_opt == nullptr) != (v_new_opt == nullptr)) return PRISM_ERR_INVALID_ARG;
   if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v) % 16) return PRISM_ERR_INVALID_ARG;
   if (k_new_opt && (((uintptr_t)k_new_opt | (uintptr_t)v_new_opt | (uintptr_t)k | (uintptr_t)v) % 16))
@@ -372,6 +375,7 @@ prism_status prism_refine_decode(const prism_shape* shape, const void* q, void* 
                                           pool_cnt, kappa_p, kappa, softmax_scale, idx, cnt, out,
                                           lse_opt, static_cast<int32_t*>(ws),
                                           (flags & PRISM_RD_OVERLAP) != 0,
+                                          (flags & PRISM_RD_SUM_GROUP) != 0,
                                           static_cast<cudaStream_t>(stream)));
 }
 

@@ -82,6 +82,7 @@ struct RDArgs {
   float* out;
   float* lse;
   int32_t* status;
+  int sum_group;  // selection score: sum over the group's query heads instead of the maximum
 };
 
 // Byte offset of 16-byte chunk `c` of row `r` in a stage: chunks are XOR
@@ -515,14 +516,15 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
 
   // ---- 2. selection keys; their first digit into the cluster histogram
   constexpr bool kSplit = ScorePick<T, D, GP>::type::kSplit;  // second half-sums in pw
+  const bool sum_group = a.sum_group != 0;  // the group's heads summed, not maxed
   for (int i = tid; i < m; i += kThreads) {
-    float best = -INFINITY;
+    float best = sum_group ? 0.0f : -INFINITY;
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
       if (g < a.G) {
         float v = dots[g * a.mc + i];
         if (kSplit) dots[g * a.mc + i] = v = v + pw[g * a.mc + i];
-        best = fmaxf(best, v);
+        best = sum_group ? best + v : fmaxf(best, v);
       }
     }
     const uint32_t key = ord_key(best);
@@ -952,10 +954,11 @@ cudaError_t launch_refine_decode(const Dims& d, const RefineDecodePlan& p, const
                                  const void* v_new, const void* k_next, const int32_t* pool,
                                  const int32_t* pool_cnt, int kappa_p, int kappa,
                                  float softmax_scale, int32_t* idx, int32_t* cnt, float* out,
-                                 float* lse, int32_t* status, bool overlap, cudaStream_t st) {
+                                 float* lse, int32_t* status, bool overlap, bool sum_group,
+                                 cudaStream_t st) {
   if (d.B * d.Hkv == 0) return cudaSuccess;
   RDArgs a{q, k, v, k_next, k_new, v_new, d.cu_dev, pool, pool_cnt, kappa_p, kappa, d.Hkv, d.G, d.Hq, d.T, p.mc,
-           softmax_scale * 1.4426950408889634f, idx, cnt, out, lse, status};
+           softmax_scale * 1.4426950408889634f, idx, cnt, out, lse, status, sum_group ? 1 : 0};
   if (d.bf16)
     return d.D == 128 ? by_group<__nv_bfloat16, 128>(d, a, p.cluster, overlap, st)
                       : by_group<__nv_bfloat16, 64>(d, a, p.cluster, overlap, st);

@@ -54,6 +54,7 @@ struct ScoreArgs {
   const void* k_new;       // integer scorer: [B][Hkv][d] new key rows to quantize at L_b - 1, or null
   int8_t* kq_w;            // with k_new: where its codes go (the same codes as kq)
   float* scale_w;          // with k_new: where its scales go
+  int sum_group;           // integer scorer: sum over the group's query heads, not the maximum
 };
 
 // s_pref[b] = number of work items of sequences before b (per KV head).
@@ -845,7 +846,8 @@ __global__ void __launch_bounds__(kThreads, 3) score_i8_kernel(const __grid_cons
 #pragma unroll
           for (int u = 0; u < 2; ++u) mma_s8(acc[j][u], a0, a1, a2, a3, bq[j][u][st][0], bq[j][u][st][1]);
       }
-      float mA = -INFINITY, mB = -INFINITY;
+      const bool sum = a.sum_group != 0;  // CTA-uniform
+      float mA = sum ? 0.0f : -INFINITY, mB = mA;
 #pragma unroll
       for (int j = 0; j < NH; ++j) {
         if (4 * j + tig < a.G) {
@@ -853,14 +855,18 @@ __global__ void __launch_bounds__(kThreads, 3) score_i8_kernel(const __grid_cons
                                (long long)(acc[j][1][0] * 256 + acc[j][1][1]);
           const long long sB = ((long long)(acc[j][0][2] * 256 + acc[j][0][3]) << 16) +
                                (long long)(acc[j][1][2] * 256 + acc[j][1][3]);
-          mA = fmaxf(mA, __ll2float_rn(sA) * us1[j] * us2[j]);
-          mB = fmaxf(mB, __ll2float_rn(sB) * us1[j] * us2[j]);
+          const float vA = __ll2float_rn(sA) * us1[j] * us2[j], vB = __ll2float_rn(sB) * us1[j] * us2[j];
+          mA = sum ? mA + vA : fmaxf(mA, vA);
+          mB = sum ? mB + vB : fmaxf(mB, vB);
         }
       }
-      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 1));
-      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, 2));
-      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
-      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
+      // over the heads held by the four lanes of a row (head 4 j + tig)
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        const float xA = __shfl_xor_sync(0xffffffffu, mA, o), xB = __shfl_xor_sync(0xffffffffu, mB, o);
+        mA = sum ? mA + xA : fmaxf(mA, xA);
+        mB = sum ? mB + xB : fmaxf(mB, xB);
+      }
       float score = 0.0f;
       if (mine) {
         score = sc * (tig == 0 ? mA : mB);
@@ -1307,7 +1313,7 @@ cudaError_t launch_propose_scores(const Dims& d, const void* q, const int8_t* kq
   const int64_t total = per_head * d.Hkv;
   if (total == 0) return cudaSuccess;
   ScoreArgs a{q, kq, scale, scores, hist, d.cu_dev, d.T, d.B, d.Hkv, d.G, status, nullptr, nullptr,
-              nullptr, nullptr, nullptr};
+              nullptr, nullptr, nullptr, 0};
   const int choice = scorer_choice();
   if (use_mma && d.bf16 && d.D == 128 && choice > 0) {
     int64_t stages = 0;
@@ -1333,7 +1339,7 @@ cudaError_t launch_propose_scores(const Dims& d, const void* q, const int8_t* kq
 
 cudaError_t launch_propose_scores_new_rows(const Dims& d, const void* q, int8_t* kq, float* scale,
                                            const void* k_new, float* scores, uint32_t* hist,
-                                           int32_t* status, cudaStream_t st) {
+                                           bool sum_group, int32_t* status, cudaStream_t st) {
   if (!d.bf16 || d.D != 128 || d.G > 8 || (reinterpret_cast<uintptr_t>(q) & 15) != 0 ||
       (reinterpret_cast<uintptr_t>(k_new) & 7) != 0)
     return cudaErrorInvalidValue;
@@ -1341,7 +1347,7 @@ cudaError_t launch_propose_scores_new_rows(const Dims& d, const void* q, int8_t*
   for (int b = 0; b < d.B; ++b) stages += cdiv(d.cu_host[b + 1] - d.cu_host[b], kStageRows);
   if (stages == 0) return cudaSuccess;
   ScoreArgs a{q, kq, scale, scores, hist, d.cu_dev, d.T, d.B, d.Hkv, d.G, status, nullptr, nullptr,
-              k_new, kq, scale};
+              k_new, kq, scale, sum_group ? 1 : 0};
   cudaError_t e = cudaSuccess;
   if (!run_tma(d.G <= 4 ? score_i8_kernel<1> : score_i8_kernel<2>, d, a, stages * d.Hkv, &e, st))
     return cudaErrorInvalidValue;
@@ -1356,7 +1362,7 @@ cudaError_t launch_propose_scores_int2(const Dims& d, const void* q, const uint8
   for (int b = 0; b < d.B; ++b) stages += cdiv(d.cu_host[b + 1] - d.cu_host[b], kStageRows);
   if (stages == 0) return cudaSuccess;
   ScoreArgs a{q, nullptr, nullptr, scores, hist, d.cu_dev, d.T, d.B, d.Hkv, d.G, status, codes, params,
-              nullptr, nullptr, nullptr};
+              nullptr, nullptr, nullptr, 0};
   return d.G <= 8 ? run_int2<1>(d, a, stages * d.Hkv, st) : run_int2<2>(d, a, stages * d.Hkv, st);
 }
 

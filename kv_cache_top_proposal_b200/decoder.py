@@ -35,7 +35,7 @@ class PrismDecoder:
     def __init__(self, seqlens, num_q_heads: int, num_kv_heads: int, head_dim: int, dtype: int,
                  num_layers: int, group: int, kappa_p: int, kappa: int, device="cuda",
                  softmax_scale: Optional[float] = None, fused: bool = True, keys: str = "int8",
-                 capacity: Optional[int] = None):
+                 capacity: Optional[int] = None, group_agg: str = "max"):
         self.dev = torch.device(device)
         self.p = prism.Problem(seqlens, num_q_heads, num_kv_heads, head_dim, dtype, device=self.dev,
                                capacity=capacity)
@@ -85,6 +85,13 @@ class PrismDecoder:
         # fused refined layer after it appends the rows to the cache
         self.scorer_appends = (fused and keys == "int8" and dtype == prism.BF16 and head_dim == 128
                                and num_q_heads // num_kv_heads <= 8)
+        # how the G query heads of a KV head combine into its selection
+        # score: "max" (the default reading) or "sum" (the variant, carried
+        # by the scorer that takes the new rows and by the fused refined layer)
+        assert group_agg in ("max", "sum")
+        if group_agg == "sum" and not self.scorer_appends:
+            raise ValueError("group_agg='sum' needs the fused step with int8 keys (bf16, d = 128, G <= 8)")
+        self.sum_group = group_agg == "sum"
 
     def workspaces(self) -> List[torch.Tensor]:
         return [w for w in (self.ws_q, self.ws_prop, self.ws_ref, self.ws_dec, self.ws_rd,
@@ -109,8 +116,10 @@ class PrismDecoder:
             prism.append_kv(p, k_new, v_new, k, v, stream=stream)
         if scorer_new:
             prism.propose_append(p, q, k_new, kq, k_scale, self.kappa_p, self.pool[l], self.pool_cnt[l],
-                                 self.ws_prop, stream=stream)
+                                 self.ws_prop, sum_group=self.sum_group, stream=stream)
         elif proposal:
+            if self.sum_group:
+                raise ValueError("group_agg='sum' proposals need this token's key rows (k_new)")
             if self.keys == "int2":
                 if quantize_new and self.new_rows.numel():
                     prism.quantize_k_int2(p, k, kq, k_scale, tok_rows=self.new_rows, ws=self.ws_q,
@@ -130,7 +139,7 @@ class PrismDecoder:
                                 self.ws_rd, lse=self.lse[l],
                                 k_new=k_new if fused_append else None,
                                 v_new=v_new if fused_append else None, k_prefetch=k_next,
-                                overlap=overlap, stream=stream)
+                                overlap=overlap, sum_group=self.sum_group, stream=stream)
             return
         prism.refine(p, q, k, self.pool[src], self.pool_cnt[src], self.kappa_p, self.kappa,
                      self.idx[l], self.cnt[l], self.ws_ref, stream=stream)

@@ -24,6 +24,8 @@ NOALLOC_SCRATCH_BYTES = 4 << 20
 DEV_BAD_INDEX, DEV_TOO_LONG, DEV_TIMEOUT = 0x1, 0x2, 0x4
 MAX_SELECT_ROW = 393216
 RD_OVERLAP = 0x1
+RD_SUM_GROUP = 0x2
+PROPOSE_SUM_GROUP = 0x1
 WS_HEADER = 256
 
 EXPORTS = ("prism_workspace_size", "prism_append_kv", "prism_quantize_k", "prism_propose",
@@ -59,7 +61,7 @@ def _load():
         "prism_append_kv": [sp, P, P, P, P, P],
         "prism_quantize_k": [sp, P, P, P, P, i32, P, S, P],
         "prism_propose": [sp, P, P, P, i32, P, P, P, S, P],
-        "prism_propose_append": [sp, P, P, P, P, i32, P, P, P, S, P],
+        "prism_propose_append": [sp, P, P, P, P, i32, P, P, ctypes.c_uint32, P, S, P],
         "prism_refine": [sp, P, P, P, P, i32, i32, P, P, P, P, S, P],
         "prism_sparse_decode": [sp, P, P, P, P, P, i32, ctypes.c_float, P, P, P, S, P],
         "prism_refine_decode": [sp, P, P, P, P, P, i32, i32, ctypes.c_float, P, P, P, P, P, P, P,
@@ -182,11 +184,14 @@ def propose(p: Problem, q, kq, k_scale, kappa_p: int, pool, pool_cnt, ws, stream
                               _ptr(pool_cnt), _ptr(ws), _nbytes(ws), _stream(stream)), "propose")
 
 
-def propose_append(p: Problem, q, k_new, kq, k_scale, kappa_p: int, pool, pool_cnt, ws, stream=None):
+def propose_append(p: Problem, q, k_new, kq, k_scale, kappa_p: int, pool, pool_cnt, ws,
+                   sum_group: bool = False, stream=None):
     """propose with this token's key rows k_new [B][Hkv][d] quantized into kq / k_scale at
-    position L_b - 1 by the scorer itself (bf16, d = 128, G <= 8)."""
+    position L_b - 1 by the scorer itself (bf16, d = 128, G <= 8).  sum_group: the
+    group's query heads are summed instead of maxed (PRISM_PROPOSE_SUM_GROUP)."""
     _check(_lib.prism_propose_append(p.ref, _ptr(q), _ptr(k_new), _ptr(kq), _ptr(k_scale), kappa_p,
-                                     _ptr(pool), _ptr(pool_cnt), _ptr(ws), _nbytes(ws),
+                                     _ptr(pool), _ptr(pool_cnt),
+                                     PROPOSE_SUM_GROUP if sum_group else 0, _ptr(ws), _nbytes(ws),
                                      _stream(stream)), "propose_append")
 
 
@@ -219,14 +224,17 @@ def sparse_decode(p: Problem, q, k, v, idx, cnt, kappa: int, softmax_scale: floa
 
 def refine_decode(p: Problem, q, k, v, pool, pool_cnt, kappa_p: int, kappa: int,
                   softmax_scale: float, idx, cnt, out, ws, lse=None, k_new=None, v_new=None,
-                  k_prefetch=None, overlap: bool = False, stream=None):
+                  k_prefetch=None, overlap: bool = False, sum_group: bool = False, stream=None):
     """Refined layer in one call; k_new / v_new ([B][Hkv][d]) are appended
     at the last position of every sequence first.  overlap: the launch may
-    begin before the previous kernel on the stream ends (see PRISM_RD_OVERLAP)."""
+    begin before the previous kernel on the stream ends (see PRISM_RD_OVERLAP);
+    sum_group: the exact score sums the group's query heads (PRISM_RD_SUM_GROUP)."""
     _check(_lib.prism_refine_decode(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(pool), _ptr(pool_cnt),
                                     kappa_p, kappa, float(softmax_scale), _ptr(idx), _ptr(cnt),
                                     _ptr(out), _ptr(lse), _ptr(k_new), _ptr(v_new),
-                                    _ptr(k_prefetch), RD_OVERLAP if overlap else 0, _ptr(ws),
+                                    _ptr(k_prefetch),
+                                    (RD_OVERLAP if overlap else 0) | (RD_SUM_GROUP if sum_group else 0),
+                                    _ptr(ws),
                                     _nbytes(ws), _stream(stream)),
            "refine_decode")
 

@@ -113,7 +113,7 @@ def test_calls_validate_before_launch(prism_lib):
     # fused refined layer: unknown flags, a lone new row, misaligned rows
     _, nrd = _ws(P, s, P.OP_REFINE_DECODE, 1024, 256)
     rd = lib.prism_refine_decode
-    assert rd(ref, f, f, f, f, f, 1024, 256, 0.1, f, f, f, None, None, None, None, 2, ws, nrd,
+    assert rd(ref, f, f, f, f, f, 1024, 256, 0.1, f, f, f, None, None, None, None, 4, ws, nrd,
               None) == P.ERR_INVALID_ARG
     assert rd(ref, f, f, f, f, f, 1024, 256, 0.1, f, f, f, None, f, None, None, 0, ws, nrd,
               None) == P.ERR_INVALID_ARG
@@ -122,6 +122,13 @@ def test_calls_validate_before_launch(prism_lib):
               None) == P.ERR_INVALID_ARG
     assert rd(ref, f, f, f, f, f, 1024, 2048, 0.1, f, f, f, None, None, None, None, 0, ws, nrd,
               None) == P.ERR_INVALID_ARG
+    # proposal with the new key rows: unknown flags, missing rows, unsupported head dim
+    pa = lib.prism_propose_append
+    assert pa(ref, f, f, f, f, 1024, f, f, 2, ws, nprop, None) == P.ERR_INVALID_ARG
+    assert pa(ref, f, None, f, f, 1024, f, f, 0, ws, nprop, None) == P.ERR_INVALID_ARG
+    s64, cu64 = _shape(P, [100], d=64)  # cu64 stays alive: s64 points at it
+    _, n64 = _ws(P, s64, P.OP_PROPOSE, 1024)
+    assert pa(ctypes.byref(s64), f, f, f, f, 1024, f, f, 0, ws, n64, None) == P.ERR_UNSUPPORTED
 
 
 def test_too_long_rows_unsupported(prism_lib):

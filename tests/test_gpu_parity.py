@@ -190,8 +190,9 @@ PROPOSE_APPEND_CASES = [
 ]
 
 
+@pytest.mark.parametrize("agg", ["max", "sum"])
 @pytest.mark.parametrize("case", PROPOSE_APPEND_CASES, ids=lambda c: f"{c[0]}-{c[1]}/{c[2]}-kp{c[3]}")
-def test_propose_append_vs_oracle(P, case):
+def test_propose_append_vs_oracle(P, case, agg):
     """prism_propose_append: the scorer quantizes this token's key rows into
     kq / k_scale at L_b - 1 (bit-exact with the oracle's quantizer; every
     other row untouched) and scores them with the rest; the pool matches the
@@ -212,7 +213,7 @@ def test_propose_append_vs_oracle(P, case):
     pool = torch.full((len(seqlens), hkv, kp), -7, dtype=torch.int32, device=DEV)
     cnt = torch.full((len(seqlens), hkv), -7, dtype=torch.int32, device=DEV)
     ws = ws_for(P, prob, P.OP_PROPOSE, kp)
-    P.propose_append(prob, q, k_new, kq, sc, kp, pool, cnt, ws)
+    P.propose_append(prob, q, k_new, kq, sc, kp, pool, cnt, ws, sum_group=agg == "sum")
     torch.cuda.synchronize()
     assert P.get_device_status(ws) == 0
     cu = prob.cu_host
@@ -225,7 +226,7 @@ def test_propose_append_vs_oracle(P, case):
             want_sc[:, cu[b + 1] - 1] = osc[b]
     assert np.array_equal(_np(kq), want_kq)
     assert np.array_equal(_np(sc).view(np.uint32), want_sc.view(np.uint32))
-    opool, ocnt, oscores = pipeline.propose_layer(q, want_kq, want_sc, cu.tolist(), kp)
+    opool, ocnt, oscores = pipeline.propose_layer(q, want_kq, want_sc, cu.tolist(), kp, agg=agg)
     gp, gc = _np(pool), _np(cnt)
     assert np.array_equal(gc, ocnt)
     gscores = _np(ws[256:256 + hkv * T * 4].view(torch.float32)).reshape(hkv, T)
@@ -478,10 +479,13 @@ def test_bad_indices_flagged_not_read(P):
 
 # ------------------------------------------------------------------ fused refine + decode
 
+@pytest.mark.parametrize("agg", ["max", "sum"])
 @pytest.mark.parametrize("case", REFINE_CASES + [([8192], 32, 8, 128, "bf16", 8192, 2048),
                                                   ([70000, 3], 8, 2, 64, "bf16", 6000, 1500)],
                          ids=lambda c: f"{c[0]}-{c[1]}/{c[2]}-d{c[3]}-{c[4]}-{c[5]}-{c[6]}")
-def test_refine_decode_vs_oracle(P, case):
+def test_refine_decode_vs_oracle(P, case, agg):
+    """agg: how the group's query heads combine into the exact score (the
+    maximum, or the group-sum variant, PRISM_RD_SUM_GROUP)."""
     seqlens, hq, hkv, d, dtype, kp, kap = case
     B = len(seqlens)
     prob = problem(P, seqlens, hq, hkv, d, dtype)
@@ -503,10 +507,10 @@ def test_refine_decode_vs_oracle(P, case):
     assert ws.numel() == 256
     scale = float(np.float32(1 / math.sqrt(d)))
     P.refine_decode(prob, q, k, v, torch.tensor(pool, device=DEV), torch.tensor(pcnt, device=DEV),
-                    kp, kap, scale, idx, cnt, out, ws, lse=lse)
+                    kp, kap, scale, idx, cnt, out, ws, lse=lse, sum_group=agg == "sum")
     torch.cuda.synchronize()
     assert P.get_device_status(ws) == 0
-    oidx, ocnt, oscores = pipeline.refine_layer(q, k, cu.tolist(), pool, pcnt, kap)
+    oidx, ocnt, oscores = pipeline.refine_layer(q, k, cu.tolist(), pool, pcnt, kap, agg=agg)
     gi, gc = _np(idx), _np(cnt)
     assert np.array_equal(gc, ocnt)
     for b in range(B):

@@ -26,10 +26,10 @@ def _np(t):
         else t.detach().cpu().numpy()
 
 
-def _decoder(P, cfg, fused=True):
+def _decoder(P, cfg, fused=True, group_agg="max"):
     return PrismDecoder(cfg.seqlens, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim,
                         P.F32 if cfg.dtype == "f32" else P.BF16, cfg.num_layers, cfg.group,
-                        cfg.kappa_p, cfg.kappa, device=DEV, fused=fused)
+                        cfg.kappa_p, cfg.kappa, device=DEV, fused=fused, group_agg=group_agg)
 
 
 def _prefill_kq(P, dec, cfg, lay):
@@ -39,12 +39,12 @@ def _prefill_kq(P, dec, cfg, lay):
     return kq, sc
 
 
-def _check_layer(dec, cfg, l, lay, kq, sc, rows):
+def _check_layer(dec, cfg, l, lay, kq, sc, rows, agg="max"):
     cu = cfg.cu_seqlens
     src = l - l % cfg.group
     gpool, gpc = _np(dec.pool[src]), _np(dec.pool_cnt[src])
     if l == src:
-        opool, ocnt, osc = pipeline.propose_layer(lay.q, kq, sc, cu, cfg.kappa_p, rows=rows)
+        opool, ocnt, osc = pipeline.propose_layer(lay.q, kq, sc, cu, cfg.kappa_p, rows=rows, agg=agg)
         for (b, h) in rows:
             n = int(ocnt[b, h])
             assert int(gpc[b, h]) == n
@@ -52,7 +52,7 @@ def _check_layer(dec, cfg, l, lay, kq, sc, rows):
                             f"L{l} pool {b},{h}")
             assert np.all(gpool[b, h, n:] == -1)
     gidx, gcnt = _np(dec.idx[l]), _np(dec.cnt[l])
-    oidx, ocnt, orr = pipeline.refine_layer(lay.q, lay.k, cu, gpool, gpc, cfg.kappa, rows=rows)
+    oidx, ocnt, orr = pipeline.refine_layer(lay.q, lay.k, cu, gpool, gpc, cfg.kappa, rows=rows, agg=agg)
     for (b, h) in rows:
         n = int(gpc[b, h])
         r = dict(zip(gpool[b, h, :n].tolist(), orr[(b, h)].tolist()))
@@ -242,3 +242,32 @@ def test_decode_loop_grows_one_sequence(prism_lib):
             _invariants(dec, cfg_t, l)
             _check_layer(dec, cfg_t, l, view, kqs[src][:, :L], scs[src][:, :L], _all_rows(cfg_t))
     del g
+
+
+def test_step_group_sum_c8k_every_row(prism_lib):
+    """A whole c8k step with the group-sum selection variant (the proposal
+    scorer and the refined layers sum the group's query heads): every row of
+    every layer against the oracle's sum mode.  The step appends the token's
+    rows (the sum variant rides on the scorer that quantizes them)."""
+    P = prism_lib
+    cfg = workload.config("c8k")
+    layers = list(workload.generate(cfg, DEV))
+    dec = _decoder(P, cfg, group_agg="sum")
+    kqs, scs = {}, {}
+    for lay in layers:
+        if cfg.is_proposal(lay.index):
+            kqs[lay.index], scs[lay.index] = _prefill_kq(P, dec, cfg, lay)
+    # this token's rows: the cache already holds them at L - 1 (generated), so
+    # appending them again leaves the cache as the oracle sees it
+    L = cfg.seqlens[0]
+    k_new = [lay.k[:, L - 1][None].clone() for lay in layers]
+    v_new = [lay.v[:, L - 1][None].clone() for lay in layers]
+    dec.step([x.q for x in layers], [x.k for x in layers], [x.v for x in layers], kqs, scs,
+             k_new=k_new, v_new=v_new)
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    for lay in layers:
+        l = lay.index
+        src = l - l % cfg.group
+        _invariants(dec, cfg, l)
+        _check_layer(dec, cfg, l, lay, kqs[src], scs[src], _all_rows(cfg), agg="sum")
