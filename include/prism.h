@@ -6,14 +6,20 @@
  * One decode step, per layer l (sec. 4 Overview, sec. 5.3 "Accuracy-efficiency
  * trade-off": in the "g x" setting one layer in every x is a proposal layer):
  *
- *   proposal layer:  prism_quantize_k (new token rows) -> prism_propose
- *   every layer:     prism_refine (on the latest pool) -> prism_sparse_decode
+ *   proposal layer:  prism_propose_append (the scorer quantizes the token's
+ *                    key rows itself), or prism_quantize_k (new token rows)
+ *                    -> prism_propose
+ *   every layer:     prism_refine_decode on the latest pool (rescoring, top
+ *                    kappa, sparse decode and merge in one launch, appending
+ *                    the token's K/V rows), or prism_refine ->
+ *                    prism_sparse_decode
  *
  * prism_dense_decode is the dense flash-decode over the same cache, the
  * comparison path (the pages compare against FlashAttention, sec. 5.3).
  *
  * Notation: B sequences, Hq query heads, Hkv KV heads, G = Hq / Hkv, head
- * dimension d, sequence b has L_b = cu[b+1] - cu[b] tokens, T = cu[B].
+ * dimension d, sequence b has L_b = cu[b+1] - cu[b] tokens, T = total_tokens
+ * (>= cu[B]: rows past cu[B] are spare capacity).
  * Query head hq reads KV head hq / G.
  *
  * Layouts (row-major, all device memory unless stated):
@@ -33,8 +39,8 @@
  * no mutable global state, and may be called from several streams at once
  * with disjoint outputs and workspaces.  The one exception is
  * prism_sparse_decode_noalloc (end of this file), which works in a fixed
- * scratch array that the library itself holds on every device.  All work is enqueued on `stream`
- * (a cudaStream_t; NULL is the legacy default stream).
+ * scratch array that the library itself holds on every device.  All work is
+ * enqueued on `stream` (a cudaStream_t; NULL is the legacy default stream).
  *
  * Errors: every argument that can be checked on the host (null pointers,
  * sizes, head_dim, kappa <= kappa_p, monotone cu_seqlens_host, workspace

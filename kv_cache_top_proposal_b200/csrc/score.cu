@@ -635,6 +635,8 @@ __global__ void __launch_bounds__(kThreads, 3) score_i8_kernel(const __grid_cons
   __shared__ float s_newscale;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tig = lane & 3;
+  // the descriptor's fetch overlaps the loads of the sequence offsets
+  if (tid == 0) asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tm)) : "memory");
   for (int i = tid; i <= a.B; i += kThreads) s_cu[i] = a.cu[i];
   for (int i = tid; i < kHist / 2; i += kThreads) s_hist[i] = 0u;
   if (tid == 0) {
@@ -666,10 +668,8 @@ __global__ void __launch_bounds__(kThreads, 3) score_i8_kernel(const __grid_cons
       it_issue.advance(s_cu, a.B);
     }
   };
-  if (tid == 0) {
-    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tm)) : "memory");
+  if (tid == 0)
     for (int kk = 0; kk < kTmaStages; ++kk) issue(kk);
-  }
 
   uint32_t bq[NH][2][4][2];  // [quad][tile][k-step][b0, b1]
   float us1[NH], us2[NH];    // 2^-sh of head 4 j + tig, as two exact factors
