@@ -856,16 +856,26 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
     const int o_lo = rank * per, o_hi = min(nout, o_lo + per);
     for (int oi = o_lo + tid; oi < o_hi; oi += kThreads) {
       const int g = oi / D, j = oi - g * D;
+      // every source's (m, l, o) loaded at once (sources past CL count as empty)
+      float mv[kMaxCluster], lv[kMaxCluster], ov[kMaxCluster];
+#pragma unroll
+      for (int src = 0; src < kMaxCluster; ++src) {
+        const bool in = src < CL;
+        mv[src] = in ? recv_ml[src * 2 * GP + g] : -INFINITY;
+        lv[src] = in ? recv_ml[src * 2 * GP + GP + g] : 0.0f;
+        ov[src] = in ? recv[src * per + (oi - o_lo)] : 0.0f;
+      }
       float M = -INFINITY;
-      for (int src = 0; src < CL; ++src) M = fmaxf(M, recv_ml[src * 2 * GP + g]);
+#pragma unroll
+      for (int src = 0; src < kMaxCluster; ++src) M = fmaxf(M, mv[src]);
       float Ls = 0.0f, O = 0.0f;
       if (M != -INFINITY) {
-        for (int src = 0; src < CL; ++src) {
-          const float mv = recv_ml[src * 2 * GP + g];
-          if (mv == -INFINITY) continue;
-          const float wt = exp2f(mv - M);
-          Ls = fmaf(wt, recv_ml[src * 2 * GP + GP + g], Ls);
-          O = fmaf(wt, recv[src * per + (oi - o_lo)], O);
+#pragma unroll
+        for (int src = 0; src < kMaxCluster; ++src) {
+          if (mv[src] == -INFINITY) continue;
+          const float wt = exp2f(mv[src] - M);
+          Ls = fmaf(wt, lv[src], Ls);
+          O = fmaf(wt, ov[src], O);
         }
       }
       const int64_t hq = (int64_t)b * a.Hq + (int64_t)h * a.G + g;
