@@ -5,22 +5,25 @@
 // for every position of every sequence, written as fp32 [Hkv][T].
 //
 // This is the bandwidth-dominant step of a decode step: d + 4 bytes per key
-// row and per KV head (132 B at d = 128).  Per row it also does G*d
-// multiply-adds plus d int8 -> float conversions, which at G = 4 is close to
-// the fp32 pipe's limit at full HBM rate, so two kernels exist:
+// row and per KV head (132 B at d = 128).  The kernels:
 //
-//  * score_mma_kernel (bf16 queries): tensor cores.  Key rows are the M
-//    dimension of mma.sync.m16n8k16 (f16 x f16 -> f32), the G query heads the
-//    N dimension.  int8 codes convert exactly to fp16 with one byte-permute
-//    and one packed subtraction per pair; the bf16 query is scaled by a power
-//    of two so that its largest element lands in [2^14, 2^15) and converted
-//    to fp16, exact for every element down to 2^-31 of the largest; products
-//    are exact and accumulate in fp32.  The feature axis is permuted so that
-//    each thread's A-fragment elements are two contiguous 16-byte pieces of
-//    its rows (the same permutation is applied to the query).  Rows stream
-//    through a ring of shared-memory stages filled by cp.async (six 16 KB
-//    stages in flight per CTA, two CTAs per SM), so the kernel keeps enough
-//    bytes in flight to run at HBM speed.
+//  * score_i8_kernel (default; bf16 queries, d = 128, G <= 8): tensor copies
+//    (cp.async.bulk.tensor, 128-row stages, evict-first in L2) feed integer
+//    tensor cores (mma.sync.m16n8k32, s8): the stored codes are the A
+//    operand as they are, each query head enters as four int8 limbs of a
+//    31-bit fixed-point value, and the int32 sums are exact.  It can also
+//    quantize this token's key rows into the codes (prism_propose_append)
+//    and sum the group's heads instead of taking their maximum.
+//  * score_tma_kernel and score_mma_kernel (bf16 queries): fp16 tensor
+//    cores.  Key rows are the M dimension of mma.sync.m16n8k16, the G query
+//    heads the N dimension; int8 codes convert exactly to fp16 with one
+//    byte-permute and one packed subtraction per pair; the bf16 query is
+//    scaled by a power of two so that its largest element lands in
+//    [2^14, 2^15) and converted to fp16; products are exact and accumulate in
+//    fp32.  The first moves stages by tensor copies, the second by cp.async
+//    (PRISM_PROPOSE_SCORER=tma / =mma select them).
+//  * score_int2_kernel: INT2 keys on fp16 tensor cores (codes as fp16
+//    subnormals), cp.async stages.
 //  * score_simt_kernel: plain fp32 FMAs on CUDA cores (fp32 queries, and the
 //    comparison kernel for bf16).
 #include <cuda.h>
