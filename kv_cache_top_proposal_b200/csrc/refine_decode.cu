@@ -14,8 +14,9 @@
 //      mma.sync (bf16 operands, fp32 accumulation, exact bf16 products) from
 //      ldmatrix fragments -- an fp32 cache takes a CUDA-core path; the logits
 //      stay in shared memory;
-//   2. the selection key of a member is ord(max_g q_g . k); its first 12
-//      bits go into the CTA's own histogram (two 16-bit counts per word);
+//   2. the selection key of a member is ord(max_g q_g . k) (or of the sum
+//      over g, the group-sum variant); its first 12 bits go into the CTA's
+//      own histogram (two 16-bit counts per word);
 //   3. CTA c sums slice c of every CTA's histogram (distributed shared
 //      memory reads, no remote atomics), and every CTA finds, from the
 //      slice totals and then the right slice, the bin holding the kappa-th
@@ -32,7 +33,11 @@
 //      value rows are streamed (same ring);
 //   6. every CTA owns one slice of the G x d outputs: the others store the
 //      matching slices of their partials (o, m, l) into it, and it merges
-//      them and writes out and lse.
+//      them (every source's partial loaded at once) and writes out and lse.
+// The same launch can append this token's K and V rows (rank 0 writes them
+// into the cache; reads of that position take them directly), and may start
+// while the previous refined layer still runs (programmatic dependent
+// launch): until that layer ends it reads only the pool and the key rows.
 // Nothing goes to global scratch.  Bytes per row: kappa_p key rows and kappa
 // value rows, d * sizeof(T) each.
 #include <cooperative_groups.h>
