@@ -213,56 +213,124 @@ def traffic_for(op: str):
 
 # --------------------------------------------------------------------------- CPU oracle legs
 
-def oracle_units(cfg, qs, ks, vs, units, budget_s: float, keys: str = "int8", agg: str = "max"):
-    """Run the CPU oracle on (proposal group, KV head) units of one decode
-    step until budget_s seconds of oracle time; returns (units done, seconds).
-    Inputs are copied from the generated cache; untimed: host copies and the
-    prefill quantization of the unit's key cache."""
+def unit_list(cfg):
+    """The (proposal group, KV head) units of one decode step: a unit is one
+    KV head's proposal and every layer of the group that uses its pool."""
+    groups = len(cfg.proposal_layers)
+    return [(g, h) for h in range(cfg.num_kv_heads) for g in range(groups)]
+
+
+def unit_bytes(cfg) -> int:
+    """Host bytes one prepared unit holds (fp32 K and V of one head, every
+    layer of a group)."""
+    return cfg.group * 2 * cfg.total_tokens * cfg.head_dim * 4
+
+
+def unit_inputs(cfg, qs, ks, vs, unit, keys: str = "int8"):
+    """Host copies of one unit's inputs and the prefill quantization of its
+    key cache (untimed preparation)."""
+    import oracle
+
+    grp, h = unit
+    G = cfg.G
+    lp = grp * cfg.group
+    lays = list(range(lp, min(lp + cfg.group, cfg.num_layers)))
+    host = {l: (qs[l][:, h * G:(h + 1) * G].float().cpu().numpy(),
+                ks[l][h].float().cpu().numpy(), vs[l][h].float().cpu().numpy()) for l in lays}
+    quant = oracle.quantize_int2_rows if keys == "int2" else oracle.quantize_rows
+    kq, sc = quant(host[lp][1])
+    return {"lays": lays, "lp": lp, "host": host, "kq": kq, "sc": sc}
+
+
+def unit_run(cfg, u, keys: str = "int8", agg: str = "max"):
+    """The oracle's work for one unit of a decode step, every sequence: the
+    new token's key row quantized, the proposal over the whole sequence, and
+    per layer of the group the refine and the attention of every query head."""
     import oracle
 
     G, D, cu = cfg.G, cfg.head_dim, cfg.cu_seqlens
     scale = float(torch.tensor(1.0 / math.sqrt(D), dtype=torch.float32))
-    done, spent = 0, 0.0
-    for (grp, h) in units:
-        lp = grp * cfg.group
-        lays = list(range(lp, min(lp + cfg.group, cfg.num_layers)))
-        host = {l: (qs[l][:, h * G:(h + 1) * G].float().cpu().numpy(),
-                    ks[l][h].float().cpu().numpy(), vs[l][h].float().cpu().numpy()) for l in lays}
-        quant = oracle.quantize_int2_rows if keys == "int2" else oracle.quantize_rows
-        propose = oracle.propose_row_int2 if keys == "int2" else oracle.propose_row
-        kq, sc = quant(host[lp][1])
+    host, lp, kq, sc = u["host"], u["lp"], u["kq"], u["sc"]
+    quant = oracle.quantize_int2_rows if keys == "int2" else oracle.quantize_rows
+    for b in range(cfg.batch):
+        a, e = cu[b], cu[b + 1]
+        if e == a:
+            continue
+        quant(host[lp][1][e - 1:e])  # the new token's key row
+        if keys == "int2":
+            pool, _ = oracle.propose_row_int2(host[lp][0][b], kq[a:e], sc[a:e], cfg.kappa_p)
+        else:
+            pool, _ = oracle.propose_row(host[lp][0][b], kq[a:e], sc[a:e], cfg.kappa_p, agg=agg)
+        for l in u["lays"]:
+            q, k, v = host[l]
+            idx, _ = oracle.refine_row(q[b], k[a:e], pool, cfg.kappa, agg=agg)
+            for g in range(G):
+                oracle.attend(q[b, g], k[a:e], v[a:e], idx, scale)
+
+
+def oracle_threads(cfg, want: int) -> int:
+    """Threads for the oracle: at most the host's cores, the units of a step,
+    and what host memory holds (one prepared unit per thread)."""
+    n = min(want, len(unit_list(cfg)))
+    try:
+        import psutil
+
+        n = min(n, max(1, int(0.5 * psutil.virtual_memory().available // unit_bytes(cfg))))
+    except Exception:
+        pass
+    return max(1, n)
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+class OracleRounds:
+    """`threads` units of one decode step, prepared once; a round runs each
+    of them once, one per thread, and is timed by the wall clock (the C
+    oracle releases the interpreter lock while it computes)."""
+
+    def __init__(self, cfg, qs, ks, vs, threads: int, keys: str = "int8", agg: str = "max"):
+        from concurrent.futures import ThreadPoolExecutor
+
+        self.cfg, self.keys, self.agg, self.threads = cfg, keys, agg, threads
+        self.units = unit_list(cfg)[:threads]
+        self.pool = ThreadPoolExecutor(threads)
+        self.inputs = list(self.pool.map(lambda u: unit_inputs(cfg, qs, ks, vs, u, keys), self.units))
+
+    def round(self) -> float:
         t0 = time.perf_counter()
-        for b in range(cfg.batch):
-            a, e = cu[b], cu[b + 1]
-            if e == a:
-                continue
-            quant(host[lp][1][e - 1:e])  # the new token's key row
-            if keys == "int2":
-                pool, _ = propose(host[lp][0][b], kq[a:e], sc[a:e], cfg.kappa_p)
-            else:
-                pool, _ = propose(host[lp][0][b], kq[a:e], sc[a:e], cfg.kappa_p, agg=agg)
-            for l in lays:
-                q, k, v = host[l]
-                idx, _ = oracle.refine_row(q[b], k[a:e], pool, cfg.kappa, agg=agg)
-                for g in range(G):
-                    oracle.attend(q[b, g], k[a:e], v[a:e], idx, scale)
-        spent += time.perf_counter() - t0
-        done += 1
-        if spent >= budget_s:
-            break
-    return done, spent
+        list(self.pool.map(lambda u: unit_run(self.cfg, u, self.keys, self.agg), self.inputs))
+        return time.perf_counter() - t0
+
+    def close(self):
+        self.pool.shutdown()
+        self.inputs = None
 
 
-def unit_list(cfg):
-    groups = len(cfg.proposal_layers)
-    return [(g, h) for h in range(cfg.num_kv_heads) for g in range(groups)]
+def oracle_rate(cfg, qs, ks, vs, threads: int, budget_s: float, keys: str = "int8", agg: str = "max"):
+    """(decode steps/s, units timed, seconds) of the oracle on `threads`
+    threads, timed rounds repeated until budget_s seconds."""
+    r = OracleRounds(cfg, qs, ks, vs, threads, keys, agg)
+    spent, rounds = 0.0, 0
+    while spent < budget_s or rounds == 0:
+        spent += r.round()
+        rounds += 1
+    r.close()
+    n = rounds * len(r.units)
+    return (n / len(unit_list(cfg))) / spent, n, spent
 
 
 # --------------------------------------------------------------------------- reference arm
 
 def run_reference(args, dist: Dist):
-    """The oracle, as it stands, timed on host cores: each step is one
-    (proposal group, KV head) unit, i.e. 1/(groups*Hkv) of a decode step."""
+    """The oracle, as it stands, timed on host cores.  A timed step is one
+    round: `threads` (proposal group, KV head) units of the decode step, one
+    per thread, so ms_per_step is the time of that sample and value is the
+    whole-step rate it implies (units/s over units per decode step)."""
     if dist.rank != 0:
         return
     cfg = workload.config(args.config)
@@ -273,23 +341,52 @@ def run_reference(args, dist: Dist):
     ks = {x.index: x.k for x in lays}
     vs = {x.index: x.v for x in lays}
     per_step_units = len(unit_list(cfg))
-    units = [(0, h % cfg.num_kv_heads) for h in range(args.warmup + args.steps)]
-    oracle_units(cfg, qs, ks, vs, units[:args.warmup], 1e9, args.keys, args.group_agg)
-    n, secs = oracle_units(cfg, qs, ks, vs, units[args.warmup:], 1e9, args.keys, args.group_agg)
-    value = (n / per_step_units) / secs
+    threads = oracle_threads(cfg.replace(num_layers=len(first)), host_cores())
+    # units of the first proposal group only (its layers are the ones generated)
+    r = OracleRounds(cfg.replace(num_layers=len(first)), qs, ks, vs, threads, args.keys,
+                     args.group_agg)
+    del lays, qs, ks, vs
+    for _ in range(args.warmup):
+        r.round()
+    secs = sum(r.round() for _ in range(args.steps))
+    n_units = args.steps * len(r.units)
+    r.close()
+    value = (n_units / per_step_units) / secs
+    sample = (f"each timed step = {len(r.units)} of the {per_step_units} (proposal group, KV head) "
+              f"units of one {cfg.name} decode step, one per thread on {threads} threads; "
+              f"{n_units} units in {secs:.2f} s; value = units/s / {per_step_units}")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32 selection / f64 attention (CPU oracle)",
-        "data": "synthetic (seeded drifting-Gaussian RoPE keys, planted salient tokens)",
-        "config": workload_config(cfg),
-        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": 1, "kind": "oracle",
-                         "sample": f"each timed step = 1 of {per_step_units} (proposal group, KV head) "
-                                   f"units of one {cfg.name} decode step; {n} units timed"},
+        "data": DATA,
+        "config": line_config(cfg, args),
+        "step_sample": {"units_per_timed_step": len(r.units), "units_per_decode_step": per_step_units,
+                        "ms_per_decode_step": 1e3 / value},
+        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+DATA = "synthetic (seeded drifting-Gaussian RoPE keys, planted salient tokens)"
+
+
+def line_config(cfg, args, seqlens0=None, n_grow=0):
+    """The `config` object of the JSON line, the same for both arms."""
+    nbytes = step_bytes(cfg, args.keys)
+    return dict(workload_config(cfg), l2="inputs larger than L2: a step touches "
+                f"{nbytes['step'] / 1e9:.2f} GB of distinct cache rows (L2 126 MB)",
+                refined_layers="fused refine+select+sparse-decode (prism_refine_decode)",
+                proposal_keys="int8 per token" if args.keys == "int8"
+                else "INT2 per 32-feature group (fp16 step and zero point)",
+                graph="one CUDA graph per step",
+                group_aggregation=args.group_agg,
+                **({"growth": f"decode loop: every replayed step appends one token, "
+                              f"from L = {seqlens0[0]} to {seqlens0[0] + n_grow}"}
+                   if args.grow and seqlens0 else {}))
 
 
 def workload_config(cfg):
@@ -474,14 +571,43 @@ def run_prism(args, dist: Dist):
     nbytes = step_bytes(cfg, args.keys)
     per_step_us = {n: sum(v) / args.profile_steps for n, v in per_op.items()}
     dominant = max(per_step_us, key=per_step_us.get)
-    avg_us = statistics.mean(per_op[dominant])
+    iso_us = statistics.mean(per_op[dominant])
+
+    # ---- the dominant kernel as it runs inside the step: every refined-layer
+    # launch of the step, in step order with the step's flags (overlapped
+    # launches, in-kernel appends), and nothing else; one graph, timed like
+    # the step
+    def rd_chain():
+        for l in range(L):
+            pl = cfg.is_proposal(l)
+            fa = not pl or dec.scorer_appends
+            src = l - l % cfg.group
+            prism.refine_decode(dec.p, q_layers[l], ks[l], vs[l], dec.pool[src], dec.pool_cnt[src],
+                                cfg.kappa_p, cfg.kappa, dec.scale, dec.idx[l], dec.cnt[l],
+                                dec.out[l], dec.ws_rd, lse=dec.lse[l],
+                                k_new=k_new[l] if fa else None, v_new=v_new[l] if fa else None,
+                                overlap=dec.fused and not pl and l > 0, sum_group=dec.sum_group)
+
+    g_rd = graph_of(rd_chain, stream)
+    rd_reps = max(20, args.steps)
+    rd_secs = dist.max(timed(g_rd.replay, rd_reps, args.warmup))
+    del g_rd
+    instep_us = rd_secs * 1e6 / (rd_reps * L)
     peak, peak_kind = hbm_peak()
-    achieved = nbytes[dominant] / (avg_us * 1e-6) / 1e9
-    roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1),
+    achieved = nbytes["refine_decode"] / (instep_us * 1e-6) / 1e9
+    roofline = {"bound": "hbm", "kernel": "refine_decode", "achieved": round(achieved, 1),
                 "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic_for(dominant),
-                "algorithmic_bytes_per_launch": nbytes[dominant], "avg_launch_us": round(avg_us, 2),
-                "share_of_step": round(per_step_us[dominant] / sum(per_step_us.values()), 3)}
+                "frac": round(achieved / peak, 4), "traffic": traffic_for("refine_decode"),
+                "algorithmic_bytes_per_launch": nbytes["refine_decode"],
+                "avg_launch_us": round(instep_us, 3), "launches_per_step": L,
+                "timing": "in step: a graph of the step's refined-layer launches in step order "
+                          "with the step's flags, CUDA events on the launching stream, "
+                          f"{rd_reps} replays / ({rd_reps} x {L} launches)",
+                "share_of_step": round(L * instep_us / (ms_per_step * 1e3), 3),
+                "isolated_launch_us": round(statistics.mean(per_op["refine_decode"]), 2),
+                "isolated_frac": round(nbytes["refine_decode"]
+                                       / (statistics.mean(per_op["refine_decode"]) * 1e-6) / 1e9 / peak, 4),
+                "largest_isolated_op": dominant, "largest_isolated_op_us": round(iso_us, 2)}
     ops_summary = {n: {"us_per_launch": round(statistics.mean(v), 2),
                        "launches_per_step": len(v) // args.profile_steps,
                        "GB/s": round(nbytes[n] / (statistics.mean(v) * 1e-6) / 1e9, 1)}
@@ -509,14 +635,23 @@ def run_prism(args, dist: Dist):
 
     status |= dec.device_status()
 
-    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1)
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1), on one
+    # thread and on as many threads as the host has cores (memory permitting)
     cpu = None
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu:
         units = unit_list(cfg)
-        n, s = oracle_units(cfg, q_layers, ks, vs, units, args.cpu_seconds, args.keys, args.group_agg)
-        cpu = {"value": (n / len(units)) / s, "unit": "steps/s", "cores": 1, "kind": "oracle",
-               "sample": f"{n} of the {len(units)} (proposal group, KV head) units of one "
-                         f"{cfg.name} decode step ({s:.1f} s of single-thread oracle time)"}
+        nt = oracle_threads(cfg, host_cores())
+        v_n, n_n, s_n = oracle_rate(cfg, q_layers, ks, vs, nt, args.cpu_seconds, args.keys,
+                                    args.group_agg)
+        v_1, n_1, s_1 = oracle_rate(cfg, q_layers, ks, vs, 1, args.cpu_seconds / 3, args.keys,
+                                    args.group_agg)
+        cpu = {"value": v_n, "unit": "steps/s", "cores": nt, "kind": "oracle",
+               "sample": f"{n_n} (proposal group, KV head) units of a {cfg.name} decode step "
+                         f"({len(units)} per step), {nt} at a time on {nt} threads, "
+                         f"{s_n:.1f} s wall; value = units/s / {len(units)}",
+               "host_cores": host_cores(),
+               "single_thread": {"value": v_1, "cores": 1,
+                                 "sample": f"{n_1} units on one thread, {s_1:.1f} s"}}
 
     if dist.rank == 0:
         peak, peak_kind = hbm_peak()
@@ -524,17 +659,8 @@ def run_prism(args, dist: Dist):
             "metric": METRIC, "value": round(value, 3), "unit": "steps/s", "n_gpus": dist.world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded drifting-Gaussian RoPE keys, planted salient tokens)",
-            "config": dict(workload_config(cfg), l2="inputs larger than L2: a step touches "
-                           f"{nbytes['step'] / 1e9:.2f} GB of distinct cache rows (L2 126 MB)",
-                           refined_layers="fused refine+select+sparse-decode (prism_refine_decode)",
-                           proposal_keys="int8 per token" if args.keys == "int8"
-                           else "INT2 per 32-feature group (fp16 step and zero point)",
-                           graph="one CUDA graph per step",
-                           group_aggregation=args.group_agg,
-                           **({"growth": f"decode loop: every replayed step appends one token, "
-                                         f"from L = {seqlens0[0]} to {seqlens0[0] + n_grow}"}
-                              if args.grow else {})),
+            "data": DATA,
+            "config": line_config(cfg, args, seqlens0, n_grow),
             "roofline": roofline,
             "step_roofline": {"achieved": round(step_achieved, 1), "peak": peak, "unit": "GB/s",
                               "frac": round(step_achieved / peak, 4),

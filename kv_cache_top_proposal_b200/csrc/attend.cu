@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendArgs a) {
   float* s_m = sm + SLOTS * GP * D;      // [SLOTS][GP]
   float* s_l = s_m + SLOTS * GP;         // [SLOTS][GP]
 
-  const int row = blockIdx.y, split = blockIdx.x;
+  const int row = blockIdx.x, split = blockIdx.y;  // rows on x: B * Hkv may exceed 65535
   const int b = row / a.Hkv, h = row - b * a.Hkv;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int sub = lane / LPR, li = lane % LPR;
@@ -260,7 +260,7 @@ cudaError_t run(const Dims& d, const AttendPlan& p, const AttendArgs& a, cudaStr
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
   }
-  k<<<dim3(p.splits, d.B * d.Hkv), kThreads, smem, st>>>(a);
+  k<<<dim3(d.B * d.Hkv, p.splits), kThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -444,6 +444,16 @@ __global__ void __launch_bounds__(kThreads, 3) score_tma_kernel(const __grid_con
       it_issue.advance(s_cu, a.B);
     }
   };
+  // A stage that never arrived: report it, wait (bounded) for the copies
+  // still in flight into this CTA's ring, issue nothing more.
+  auto abandon = [&](int kk) {
+    if (tid == 0) flag_status(a.status, PRISM_DEV_TIMEOUT);
+    for (int j = kk; j < nk && j < kk + kTmaStages; ++j) {
+      uint32_t it = 0;
+      while (!mbar_try_wait(&full[j % kTmaStages], (uint32_t)(j / kTmaStages) & 1u) && ++it < kWaitLimit) {
+      }
+    }
+  };
   if (tid == 0) {
     asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tm)) : "memory");
     for (int kk = 0; kk < kTmaStages; ++kk) issue(kk);
@@ -536,11 +546,12 @@ __global__ void __launch_bounds__(kThreads, 3) score_tma_kernel(const __grid_con
     const float sc = sc_next;
     if (kk + 1 < nk) sc_next = load_scale(it_comp);
     const int slot = kk % kTmaStages;
+    bool late = false;  // this thread gave up waiting for the stage
     {
       uint32_t it = 0;
       while (!mbar_try_wait(&full[slot], (uint32_t)(kk / kTmaStages) & 1u)) {
         if (++it == kWaitLimit) {
-          if (tid == 0) flag_status(a.status, PRISM_DEV_TIMEOUT);
+          late = true;
           break;
         }
       }
@@ -585,13 +596,17 @@ __global__ void __launch_bounds__(kThreads, 3) score_tma_kernel(const __grid_con
       mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 1));
       mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, 2));
       float score = 0.0f;
-      if (mine) {
+      if (mine && !late) {
         score = sc * ((tig == 0 ? mA : mB) * unscale);
         a.scores[rowbase + rs] = score;
       }
-      if (a.hist) warp_hist_add_packed(s_hist, ord_key(score) >> 20, mine);
+      if (a.hist) warp_hist_add_packed(s_hist, ord_key(score) >> 20, mine && !late);
     }
-    __syncthreads();  // every warp is done with the stage
+    // every warp is done with the stage; a stage that never arrived ends the CTA
+    if (__syncthreads_or(late)) {
+      abandon(kk);
+      return;
+    }
     if (tid == 0) issue(kk + kTmaStages);
   }
   flush();
@@ -669,6 +684,16 @@ __global__ void __launch_bounds__(kThreads, 3) score_i8_kernel(const __grid_cons
       tma_rows_stream(ring + (kk % kTmaStages) * kTmaStageBytes, &tm, (int)y, &full[kk % kTmaStages],
                       evict_first);
       it_issue.advance(s_cu, a.B);
+    }
+  };
+  // A stage that never arrived: report it, wait (bounded) for the copies
+  // still in flight into this CTA's ring, issue nothing more.
+  auto abandon = [&](int kk) {
+    if (tid == 0) flag_status(a.status, PRISM_DEV_TIMEOUT);
+    for (int j = kk; j < nk && j < kk + kTmaStages; ++j) {
+      uint32_t it = 0;
+      while (!mbar_try_wait(&full[j % kTmaStages], (uint32_t)(j / kTmaStages) & 1u) && ++it < kWaitLimit) {
+      }
     }
   };
   if (tid == 0)
@@ -779,11 +804,12 @@ __global__ void __launch_bounds__(kThreads, 3) score_i8_kernel(const __grid_cons
     float sc = sc_next;
     if (kk + 1 < nk) sc_next = load_scale(it_comp);
     const int slot = kk % kTmaStages;
+    bool late = false;  // this thread gave up waiting for the stage
     {
       uint32_t it = 0;
       while (!mbar_try_wait(&full[slot], (uint32_t)(kk / kTmaStages) & 1u)) {
         if (++it == kWaitLimit) {
-          if (tid == 0) flag_status(a.status, PRISM_DEV_TIMEOUT);
+          late = true;
           break;
         }
       }
@@ -871,13 +897,17 @@ __global__ void __launch_bounds__(kThreads, 3) score_i8_kernel(const __grid_cons
         mB = sum ? mB + xB : fmaxf(mB, xB);
       }
       float score = 0.0f;
-      if (mine) {
+      if (mine && !late) {
         score = sc * (tig == 0 ? mA : mB);
         a.scores[rowbase + rs] = score;
       }
-      if (a.hist) warp_hist_add_packed(s_hist, ord_key(score) >> 20, mine);
+      if (a.hist) warp_hist_add_packed(s_hist, ord_key(score) >> 20, mine && !late);
     }
-    __syncthreads();  // every warp is done with the stage
+    // every warp is done with the stage; a stage that never arrived ends the CTA
+    if (__syncthreads_or(late)) {
+      abandon(kk);
+      return;
+    }
     if (tid == 0) issue(kk + kTmaStages);
   }
   flush();

@@ -28,3 +28,9 @@ def test_reference_arm_json_line(extra):
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    # a timed step is a sample of units; ms_per_step is that sample's time and
+    # value the whole-step rate it implies
+    ss = line["step_sample"]
+    frac = ss["units_per_timed_step"] / ss["units_per_decode_step"]
+    assert 0 < frac <= 1 and ss["units_per_timed_step"] == cb["cores"]
+    assert abs(line["ms_per_step"] - 1e3 * frac / line["value"]) <= 1e-6 * line["ms_per_step"]

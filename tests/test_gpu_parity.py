@@ -630,7 +630,16 @@ def test_refine_decode_appends_new_rows(P, dtype):
     # result matches the oracle on the appended cache
     gi, gc = _np(i1), _np(c1)
     assert any((gi[b, h, :gc[b, h]] == seqlens[b] - 1).any() for b in range(B) for h in range(hkv))
-    oout, _ = pipeline.attend_layer(q, k1, v1, prob.cu_host.tolist(), gi, gc, scale)
+    # the index sets against the oracle's refine on the appended cache
+    cu = prob.cu_host.tolist()
+    oidx, ocnt, orr = pipeline.refine_layer(q, k1, cu, pool, pcnt, kap)
+    for b in range(B):
+        for h in range(hkv):
+            n, c = int(pcnt[b, h]), int(ocnt[b, h])
+            assert int(gc[b, h]) == c
+            r = dict(zip(pool[b, h, :n].tolist(), orr[(b, h)].tolist()))
+            check_index_set(gi[b, h, :c], oidx[b, h, :c], lambda t: r[t], f"append idx {b},{h}")
+    oout, _ = pipeline.attend_layer(q, k1, v1, cu, gi, gc, scale)
     assert np.abs(_np(o1) - oout).max() <= atol_for(dtype)
 
 

@@ -1,10 +1,12 @@
 """Whole decode steps through the layer driver vs the oracle.
 
 Small configurations are checked on every (sequence, KV head) row of every
-layer.  The full-size configurations run in the launch configuration the
-benchmark times (same kernels, same split plans) and are checked on sampled
-rows the oracle computes one by one, plus invariants on every row.  Each
-stage is checked on the GPU's own upstream set (cascade control).
+layer.  The full-size configurations run the call sequence the benchmark
+times (captured step graph, the token's rows appended inside the kernels,
+overlapped refined layers) and are checked on every row of a whole proposal
+group; a second test samples rows of a step whose caches already hold the
+token (no appends).
+Each stage is checked on the GPU's own upstream set (cascade control).
 """
 import math
 
@@ -271,3 +273,94 @@ def test_step_group_sum_c8k_every_row(prism_lib):
         src = l - l % cfg.group
         _invariants(dec, cfg, l)
         _check_layer(dec, cfg, l, lay, kqs[src], scs[src], _all_rows(cfg), agg="sum")
+
+
+def _spoil_last_rows(layers, cu, kqs, scs):
+    """Overwrite every sequence's last cache row (K, V, and the proposal codes
+    and scales) so that only the step's own appends can restore them."""
+    for lay in layers:
+        for b in range(len(cu) - 1):
+            if cu[b + 1] > cu[b]:
+                lay.k[:, cu[b + 1] - 1] = 7.0
+                lay.v[:, cu[b + 1] - 1] = -7.0
+                if lay.index in kqs:
+                    kqs[lay.index][:, cu[b + 1] - 1] = 99
+                    scs[lay.index][:, cu[b + 1] - 1] = 5.0
+
+
+@pytest.mark.parametrize("name", ["c128k", "ragged16", "c32k_b4"])
+def test_step_timed_sequence_full_size_every_row(prism_lib, name):
+    """The call sequence the benchmark times, at full size, on every row of a
+    whole proposal group: the token's K/V rows are handed in (k_new/v_new),
+    so the proposal layer's scorer quantizes the new key rows itself
+    (prism_propose_append) and every refined layer appends its rows inside
+    the fused kernel; consecutive refined layers overlap through programmatic
+    dependent launch; the step is one captured CUDA graph, replayed twice.
+    Before each replay the cache's last rows (K, V, codes, scales) are
+    spoiled, so the checks see only what the replay itself wrote.  Every
+    (sequence, KV head) row of every layer is then compared with the
+    oracle: codes bit for bit, pools and index sets exactly up to near-ties,
+    outputs within the bf16 tolerance."""
+    P = prism_lib
+    full = workload.config(name)
+    cfg = full.replace(num_layers=full.group)
+    layers = list(workload.generate(cfg, DEV))
+    cu = cfg.cu_seqlens
+    nz = [b for b in range(cfg.batch) if cu[b + 1] > cu[b]]
+    saved = [({b: lay.k[:, cu[b + 1] - 1].clone() for b in nz},
+              {b: lay.v[:, cu[b + 1] - 1].clone() for b in nz}) for lay in layers]
+    # this token's rows, [B][Hkv][d] per layer, as bench.py builds them
+    rows = torch.tensor([cu[b + 1] - 1 for b in nz], dtype=torch.long, device=DEV)
+    k_new = [lay.k[:, rows].transpose(0, 1).contiguous() for lay in layers]
+    v_new = [lay.v[:, rows].transpose(0, 1).contiguous() for lay in layers]
+    dec = PrismDecoder(cfg.seqlens, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, P.BF16,
+                       cfg.num_layers, cfg.group, cfg.kappa_p, cfg.kappa, device=DEV,
+                       capacity=cfg.total_tokens)
+    assert dec.scorer_appends
+    kqs, scs = {}, {}
+    for lay in layers:
+        if cfg.is_proposal(lay.index):
+            kqs[lay.index], scs[lay.index] = _prefill_kq(P, dec, cfg, lay)
+    qs, ks, vs = [x.q for x in layers], [x.k for x in layers], [x.v for x in layers]
+    s = torch.cuda.Stream()
+
+    def step():
+        dec.step(qs, ks, vs, kqs, scs, quantize_new=True, k_new=k_new, v_new=v_new)
+
+    with torch.cuda.stream(s):
+        _spoil_last_rows(layers, cu, kqs, scs)
+        step()  # eager once, as the benchmark does before capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step()
+    for rep in range(2):
+        for x in dec.idx + dec.out:
+            x.fill_(-3)
+        for lp in dec.pool:
+            dec.pool[lp].fill_(-3)
+        _spoil_last_rows(layers, cu, kqs, scs)
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        assert dec.device_status() == 0
+    # the appends: the cache's last rows are this token's rows again
+    for lay, (kl, vl) in zip(layers, saved):
+        for b in nz:
+            assert torch.equal(lay.k[:, cu[b + 1] - 1], kl[b]), (lay.index, b)
+            assert torch.equal(lay.v[:, cu[b + 1] - 1], vl[b]), (lay.index, b)
+    every = _all_rows(cfg)
+    okq = {}
+    for lay in layers:
+        l = lay.index
+        if cfg.is_proposal(l):
+            okq[l] = pipeline.quantize_layer(lay.k)
+            assert np.array_equal(_np(kqs[l]), okq[l][0]), f"L{l} codes"
+            assert np.array_equal(_np(scs[l]).view(np.uint32), okq[l][1].view(np.uint32)), f"L{l} scales"
+    for lay in layers:
+        l = lay.index
+        src = l - l % cfg.group
+        _invariants(dec, cfg, l)
+        _check_layer(dec, cfg, l, lay, okq[src][0], okq[src][1], every)
+    del g, layers, dec
+    torch.cuda.empty_cache()

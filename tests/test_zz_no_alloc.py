@@ -14,8 +14,6 @@ import numpy as np
 import pytest
 import torch
 
-from parity_util import atol_for
-
 DEV = "cuda"
 
 
@@ -46,32 +44,58 @@ CASES = [
 ]
 
 
+def _both(P, prob, q, k, v, idx, cnt, kap, scale, B, hq, d):
+    """(workspace status, out, lse) of prism_sparse_decode and (status_dev,
+    out, lse) of the no-allocation entry point on the same inputs."""
+    ws = torch.zeros(P.workspace_size(prob, P.OP_SPARSE_DECODE, 0, kap), dtype=torch.uint8,
+                     device=DEV)
+    ref_out = torch.full((B, hq, d), 77.0, device=DEV)
+    ref_lse = torch.full((B, hq), 77.0, device=DEV)
+    P.sparse_decode(prob, q, k, v, idx, cnt, kap, scale, ref_out, ws, lse=ref_lse)
+    out = torch.full((B, hq, d), -55.0, device=DEV)
+    lse = torch.full((B, hq), -55.0, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    P.sparse_decode_noalloc(prob, q, k, v, idx, cnt, kap, scale, out, status, lse=lse)
+    torch.cuda.synchronize()
+    return (P.get_device_status(ws), ref_out, ref_lse), (int(status.item()), out, lse)
+
+
 @pytest.mark.gpu
 def test_noalloc_matches_workspace_entry_point_twice(prism_lib):
+    """Same kernels, same split plan and summation order as the workspace
+    entry point, so the results must be identical, bit for bit."""
     P = prism_lib
     for i, (seqlens, hq, hkv, d, dtype, kap) in enumerate(CASES):
         prob = P.Problem(seqlens, hq, hkv, d, P.BF16 if dtype == "bf16" else P.F32, device=DEV)
         q, k, v, idx, cnt = _inputs(seqlens, hq, hkv, d, dtype, kap, seed=40 + i)
         scale = float(np.float32(1 / math.sqrt(d)))
-        B = len(seqlens)
-        ws = torch.zeros(P.workspace_size(prob, P.OP_SPARSE_DECODE, 0, kap), dtype=torch.uint8,
-                         device=DEV)
-        ref_out = torch.full((B, hq, d), 77.0, device=DEV)
-        ref_lse = torch.full((B, hq), 77.0, device=DEV)
-        P.sparse_decode(prob, q, k, v, idx, cnt, kap, scale, ref_out, ws, lse=ref_lse)
-        out = torch.full((B, hq, d), -55.0, device=DEV)
-        lse = torch.full((B, hq), -55.0, device=DEV)
-        status = torch.zeros(1, dtype=torch.int32, device=DEV)
-        P.sparse_decode_noalloc(prob, q, k, v, idx, cnt, kap, scale, out, status, lse=lse)
-        torch.cuda.synchronize()
-        assert P.get_device_status(ws) == 0
-        assert int(status.item()) == 0
-        tol = atol_for(dtype)
-        assert (out - ref_out).abs().max().item() <= tol, i
-        r, g = ref_lse.cpu().numpy(), lse.cpu().numpy()
-        fin = np.isfinite(r)
-        assert np.array_equal(np.isfinite(g), fin), i
-        assert np.abs(g[fin] - r[fin]).max() <= 10 * tol, i
+        (ws_st, ref_out, ref_lse), (st, out, lse) = _both(P, prob, q, k, v, idx, cnt, kap, scale,
+                                                          len(seqlens), hq, d)
+        assert ws_st == 0 and st == 0, i
+        assert torch.equal(out, ref_out), i
+        assert torch.equal(lse, ref_lse), i
+
+
+@pytest.mark.gpu
+def test_noalloc_reports_bad_indices_in_status_dev(prism_lib):
+    """An index past its sequence and a count above kappa: the kernels skip
+    the bad index and clamp the count without touching memory outside the
+    arrays, and the no-allocation call reports both in the caller's status
+    word exactly as the workspace entry point reports them in its header."""
+    P = prism_lib
+    seqlens, hq, hkv, d, kap = [3000, 1200], 8, 2, 128, 256
+    prob = P.Problem(seqlens, hq, hkv, d, P.BF16, device=DEV)
+    q, k, v, idx, cnt = _inputs(seqlens, hq, hkv, d, "bf16", kap, seed=9)
+    idx[0, 1, 5] = seqlens[0]       # one position at L: skipped
+    cnt[1, 0] = kap + 7             # one count above kappa: clamped to kappa
+    idx[1, 0, :] = torch.arange(kap, dtype=torch.int32, device=DEV)
+    scale = float(np.float32(1 / math.sqrt(d)))
+    (ws_st, ref_out, ref_lse), (st, out, lse) = _both(P, prob, q, k, v, idx, cnt, kap, scale,
+                                                      len(seqlens), hq, d)
+    assert ws_st == P.DEV_BAD_INDEX
+    assert st == P.DEV_BAD_INDEX
+    assert torch.equal(out, ref_out)
+    assert torch.equal(lse, ref_lse)
 
 
 def test_noalloc_rejects_requests_beyond_the_scratch(prism_lib):
