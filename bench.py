@@ -55,6 +55,12 @@ def parse():
                     help="proposal key cache: int8 per token (the headline workload) or INT2 per 32-feature group")
     ap.add_argument("--group-agg", default="max", choices=["max", "sum"],
                     help="how the query heads of a KV head combine into the selection score")
+    ap.add_argument("--proposal-select", default="exact", choices=["exact", "quantized"],
+                    help="what a proposal layer attends over: its own pool refined with exact scores "
+                         "(the default reading) or the top kappa of its quantized scores")
+    ap.add_argument("--sets", default="kv_head", choices=["kv_head", "q_head", "sequence"],
+                    help="selection granularity: one pool and set per (sequence, KV head), a set per "
+                         "query head, or one pool and set per sequence shared by every head")
     ap.add_argument("--grow", action="store_true",
                     help="decode loop over the growing sequence: every replayed step appends one "
                          "token (batch-1 configs); the cache starts short by the replays")
@@ -242,7 +248,7 @@ def unit_inputs(cfg, qs, ks, vs, unit, keys: str = "int8"):
     return {"lays": lays, "lp": lp, "host": host, "kq": kq, "sc": sc}
 
 
-def unit_run(cfg, u, keys: str = "int8", agg: str = "max"):
+def unit_run(cfg, u, keys: str = "int8", agg: str = "max", proposal_select: str = "exact"):
     """The oracle's work for one unit of a decode step, every sequence: the
     new token's key row quantized, the proposal over the whole sequence, and
     per layer of the group the refine and the attention of every query head."""
@@ -258,12 +264,15 @@ def unit_run(cfg, u, keys: str = "int8", agg: str = "max"):
             continue
         quant(host[lp][1][e - 1:e])  # the new token's key row
         if keys == "int2":
-            pool, _ = oracle.propose_row_int2(host[lp][0][b], kq[a:e], sc[a:e], cfg.kappa_p)
+            pool, ps = oracle.propose_row_int2(host[lp][0][b], kq[a:e], sc[a:e], cfg.kappa_p)
         else:
-            pool, _ = oracle.propose_row(host[lp][0][b], kq[a:e], sc[a:e], cfg.kappa_p, agg=agg)
+            pool, ps = oracle.propose_row(host[lp][0][b], kq[a:e], sc[a:e], cfg.kappa_p, agg=agg)
         for l in u["lays"]:
             q, k, v = host[l]
-            idx, _ = oracle.refine_row(q[b], k[a:e], pool, cfg.kappa, agg=agg)
+            if l == lp and proposal_select == "quantized":
+                idx = oracle.pool_topk(ps, pool, cfg.kappa)
+            else:
+                idx, _ = oracle.refine_row(q[b], k[a:e], pool, cfg.kappa, agg=agg)
             for g in range(G):
                 oracle.attend(q[b, g], k[a:e], v[a:e], idx, scale)
 
@@ -293,17 +302,20 @@ class OracleRounds:
     of them once, one per thread, and is timed by the wall clock (the C
     oracle releases the interpreter lock while it computes)."""
 
-    def __init__(self, cfg, qs, ks, vs, threads: int, keys: str = "int8", agg: str = "max"):
+    def __init__(self, cfg, qs, ks, vs, threads: int, keys: str = "int8", agg: str = "max",
+                 proposal_select: str = "exact"):
         from concurrent.futures import ThreadPoolExecutor
 
         self.cfg, self.keys, self.agg, self.threads = cfg, keys, agg, threads
+        self.proposal_select = proposal_select
         self.units = unit_list(cfg)[:threads]
         self.pool = ThreadPoolExecutor(threads)
         self.inputs = list(self.pool.map(lambda u: unit_inputs(cfg, qs, ks, vs, u, keys), self.units))
 
     def round(self) -> float:
         t0 = time.perf_counter()
-        list(self.pool.map(lambda u: unit_run(self.cfg, u, self.keys, self.agg), self.inputs))
+        list(self.pool.map(lambda u: unit_run(self.cfg, u, self.keys, self.agg, self.proposal_select),
+                           self.inputs))
         return time.perf_counter() - t0
 
     def close(self):
@@ -311,10 +323,11 @@ class OracleRounds:
         self.inputs = None
 
 
-def oracle_rate(cfg, qs, ks, vs, threads: int, budget_s: float, keys: str = "int8", agg: str = "max"):
+def oracle_rate(cfg, qs, ks, vs, threads: int, budget_s: float, keys: str = "int8", agg: str = "max",
+                proposal_select: str = "exact"):
     """(decode steps/s, units timed, seconds) of the oracle on `threads`
     threads, timed rounds repeated until budget_s seconds."""
-    r = OracleRounds(cfg, qs, ks, vs, threads, keys, agg)
+    r = OracleRounds(cfg, qs, ks, vs, threads, keys, agg, proposal_select)
     spent, rounds = 0.0, 0
     while spent < budget_s or rounds == 0:
         spent += r.round()
@@ -335,16 +348,18 @@ def run_reference(args, dist: Dist):
         return
     cfg = workload.config(args.config)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    first = list(range(0, min(cfg.group, cfg.num_layers)))
+    per_step_units = len(unit_list(cfg))
+    threads = oracle_threads(cfg, host_cores())
+    # the layers of as many proposal groups as the threads' units need
+    n_groups = min(len(cfg.proposal_layers), -(-threads // cfg.num_kv_heads))
+    first = list(range(0, min(n_groups * cfg.group, cfg.num_layers)))
+    sub = cfg.replace(num_layers=len(first))
     lays = list(workload.generate(cfg, dev, layers=first))
     qs = {x.index: x.q for x in lays}
     ks = {x.index: x.k for x in lays}
     vs = {x.index: x.v for x in lays}
-    per_step_units = len(unit_list(cfg))
-    threads = oracle_threads(cfg.replace(num_layers=len(first)), host_cores())
-    # units of the first proposal group only (its layers are the ones generated)
-    r = OracleRounds(cfg.replace(num_layers=len(first)), qs, ks, vs, threads, args.keys,
-                     args.group_agg)
+    threads = min(threads, len(unit_list(sub)))
+    r = OracleRounds(sub, qs, ks, vs, threads, args.keys, args.group_agg, args.proposal_select)
     del lays, qs, ks, vs
     for _ in range(args.warmup):
         r.round()
@@ -379,7 +394,9 @@ def line_config(cfg, args, seqlens0=None, n_grow=0):
     nbytes = step_bytes(cfg, args.keys)
     return dict(workload_config(cfg), l2="inputs larger than L2: a step touches "
                 f"{nbytes['step'] / 1e9:.2f} GB of distinct cache rows (L2 126 MB)",
-                refined_layers="fused refine+select+sparse-decode (prism_refine_decode)",
+                refined_layers="fused refine+select+sparse-decode (prism_refine_decode)"
+                if args.sets == "kv_head" else "refine and sparse decode (two calls)",
+                proposal_select=args.proposal_select, selection_sets=args.sets,
                 proposal_keys="int8 per token" if args.keys == "int8"
                 else "INT2 per 32-feature group (fp16 step and zero point)",
                 graph="one CUDA graph per step",
@@ -432,7 +449,8 @@ def run_prism(args, dist: Dist):
     dec = PrismDecoder(seqlens0, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim,
                        prism.BF16 if cfg.dtype == "bf16" else prism.F32, L, cfg.group,
                        cfg.kappa_p, cfg.kappa, device=dev, keys=args.keys,
-                       capacity=cfg.total_tokens, group_agg=args.group_agg)
+                       capacity=cfg.total_tokens, group_agg=args.group_agg,
+                       proposal_select=args.proposal_select, sets=args.sets)
     rows = dec.new_rows.long()
     Hkv = cfg.num_kv_heads
     k_new = torch.stack([k[:, rows].transpose(0, 1).contiguous() for k in ks])  # [L][B][Hkv][d]
@@ -514,104 +532,133 @@ def run_prism(args, dist: Dist):
     if args.grow:
         dec.lengths_from_device()  # the dense comparison sizes its splits from the host copy
 
-    # ---- per-op durations (one graph per op; the queue is filled behind a
-    # long memset so every event pair brackets device time only)
-    ops = []
-    for l in range(L):
-        pl = cfg.is_proposal(l)
-
-        def f_prop(l=l):
-            if dec.scorer_appends:  # the scorer quantizes the new key rows; the refined layer appends
-                prism.propose_append(dec.p, q_layers[l], k_new[l], kqs[l], scs[l], cfg.kappa_p,
-                                     dec.pool[l], dec.pool_cnt[l], dec.ws_prop, sum_group=dec.sum_group)
-                return
-            prism.append_kv(dec.p, k_new[l], v_new[l], ks[l], vs[l])
-            if args.keys == "int2":
-                prism.quantize_k_int2(dec.p, ks[l], kqs[l], scs[l], tok_rows=dec.new_rows, ws=dec.ws_q)
-                prism.propose_int2(dec.p, q_layers[l], kqs[l], scs[l], cfg.kappa_p, dec.pool[l],
-                                   dec.pool_cnt[l], dec.ws_prop)
-            else:
-                prism.quantize_k(dec.p, ks[l], kqs[l], scs[l], tok_rows=dec.new_rows, ws=dec.ws_q)
-                prism.propose(dec.p, q_layers[l], kqs[l], scs[l], cfg.kappa_p, dec.pool[l],
-                              dec.pool_cnt[l], dec.ws_prop)
-
-        def f_rd(l=l):
-            src = l - l % cfg.group
-            # refined layers append their new rows themselves, and so do proposal
-            # layers whose scorer took the new key rows
-            fa = not cfg.is_proposal(l) or dec.scorer_appends
-            prism.refine_decode(dec.p, q_layers[l], ks[l], vs[l], dec.pool[src], dec.pool_cnt[src],
-                                cfg.kappa_p, cfg.kappa, dec.scale, dec.idx[l], dec.cnt[l],
-                                dec.out[l], dec.ws_rd, lse=dec.lse[l],
-                                k_new=k_new[l] if fa else None, v_new=v_new[l] if fa else None,
-                                sum_group=dec.sum_group)
-
-        if pl:
-            ops.append(("propose", graph_of(f_prop, stream)))
-        ops.append(("refine_decode", graph_of(f_rd, stream)))
-    # ~30 MB of memset per queued graph launch keeps the device busy while the
-    # host enqueues the profiled sequence
-    gate = torch.empty(min(6 << 30, max(256 << 20, len(ops) * (30 << 20))), dtype=torch.uint8,
-                       device=dev)
-    per_op = {}
-    for _ in range(args.profile_steps):
-        gate.zero_()
-        evs = []
-        for name, og in ops:
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            og.replay()
-            b.record(stream)
-            evs.append((name, a, b))
-        torch.cuda.synchronize()
-        for name, a, b in evs:
-            per_op.setdefault(name, []).append(a.elapsed_time(b) * 1e3)  # us
-    del gate
+    variant = args.sets != "kv_head" or args.proposal_select != "exact"
     nbytes = step_bytes(cfg, args.keys)
-    per_step_us = {n: sum(v) / args.profile_steps for n, v in per_op.items()}
-    dominant = max(per_step_us, key=per_step_us.get)
-    iso_us = statistics.mean(per_op[dominant])
-
-    # ---- the dominant kernel as it runs inside the step: every refined-layer
-    # launch of the step, in step order with the step's flags (overlapped
-    # launches, in-kernel appends), and nothing else; one graph, timed like
-    # the step
-    def rd_chain():
+    if not variant:
+        # ---- per-op durations (one graph per op; the queue is filled behind a
+        # long memset so every event pair brackets device time only)
+        ops = []
         for l in range(L):
             pl = cfg.is_proposal(l)
-            fa = not pl or dec.scorer_appends
-            src = l - l % cfg.group
-            prism.refine_decode(dec.p, q_layers[l], ks[l], vs[l], dec.pool[src], dec.pool_cnt[src],
-                                cfg.kappa_p, cfg.kappa, dec.scale, dec.idx[l], dec.cnt[l],
-                                dec.out[l], dec.ws_rd, lse=dec.lse[l],
-                                k_new=k_new[l] if fa else None, v_new=v_new[l] if fa else None,
-                                overlap=dec.fused and not pl and l > 0, sum_group=dec.sum_group)
 
-    g_rd = graph_of(rd_chain, stream)
-    rd_reps = max(20, args.steps)
-    rd_secs = dist.max(timed(g_rd.replay, rd_reps, args.warmup))
-    del g_rd
-    instep_us = rd_secs * 1e6 / (rd_reps * L)
-    peak, peak_kind = hbm_peak()
-    achieved = nbytes["refine_decode"] / (instep_us * 1e-6) / 1e9
-    roofline = {"bound": "hbm", "kernel": "refine_decode", "achieved": round(achieved, 1),
-                "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic_for("refine_decode"),
-                "algorithmic_bytes_per_launch": nbytes["refine_decode"],
-                "avg_launch_us": round(instep_us, 3), "launches_per_step": L,
-                "timing": "in step: a graph of the step's refined-layer launches in step order "
-                          "with the step's flags, CUDA events on the launching stream, "
-                          f"{rd_reps} replays / ({rd_reps} x {L} launches)",
-                "share_of_step": round(L * instep_us / (ms_per_step * 1e3), 3),
-                "isolated_launch_us": round(statistics.mean(per_op["refine_decode"]), 2),
-                "isolated_frac": round(nbytes["refine_decode"]
-                                       / (statistics.mean(per_op["refine_decode"]) * 1e-6) / 1e9 / peak, 4),
-                "largest_isolated_op": dominant, "largest_isolated_op_us": round(iso_us, 2)}
-    ops_summary = {n: {"us_per_launch": round(statistics.mean(v), 2),
-                       "launches_per_step": len(v) // args.profile_steps,
-                       "GB/s": round(nbytes[n] / (statistics.mean(v) * 1e-6) / 1e9, 1)}
-                   for n, v in per_op.items()}
+            def f_prop(l=l):
+                if dec.scorer_appends:  # the scorer quantizes the new key rows; the refined layer appends
+                    prism.propose_append(dec.p, q_layers[l], k_new[l], kqs[l], scs[l], cfg.kappa_p,
+                                         dec.pool[l], dec.pool_cnt[l], dec.ws_prop, sum_group=dec.sum_group)
+                    return
+                prism.append_kv(dec.p, k_new[l], v_new[l], ks[l], vs[l])
+                if args.keys == "int2":
+                    prism.quantize_k_int2(dec.p, ks[l], kqs[l], scs[l], tok_rows=dec.new_rows, ws=dec.ws_q)
+                    prism.propose_int2(dec.p, q_layers[l], kqs[l], scs[l], cfg.kappa_p, dec.pool[l],
+                                       dec.pool_cnt[l], dec.ws_prop)
+                else:
+                    prism.quantize_k(dec.p, ks[l], kqs[l], scs[l], tok_rows=dec.new_rows, ws=dec.ws_q)
+                    prism.propose(dec.p, q_layers[l], kqs[l], scs[l], cfg.kappa_p, dec.pool[l],
+                                  dec.pool_cnt[l], dec.ws_prop)
+
+            def f_rd(l=l):
+                src = l - l % cfg.group
+                # refined layers append their new rows themselves, and so do proposal
+                # layers whose scorer took the new key rows
+                fa = not cfg.is_proposal(l) or dec.scorer_appends
+                prism.refine_decode(dec.p, q_layers[l], ks[l], vs[l], dec.pool[src], dec.pool_cnt[src],
+                                    cfg.kappa_p, cfg.kappa, dec.scale, dec.idx[l], dec.cnt[l],
+                                    dec.out[l], dec.ws_rd, lse=dec.lse[l],
+                                    k_new=k_new[l] if fa else None, v_new=v_new[l] if fa else None,
+                                    sum_group=dec.sum_group)
+
+            if pl:
+                ops.append(("propose", graph_of(f_prop, stream)))
+            ops.append(("refine_decode", graph_of(f_rd, stream)))
+        # ~30 MB of memset per queued graph launch keeps the device busy while the
+        # host enqueues the profiled sequence
+        gate = torch.empty(min(6 << 30, max(256 << 20, len(ops) * (30 << 20))), dtype=torch.uint8,
+                           device=dev)
+        per_op = {}
+        for _ in range(args.profile_steps):
+            gate.zero_()
+            evs = []
+            for name, og in ops:
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                og.replay()
+                b.record(stream)
+                evs.append((name, a, b))
+            torch.cuda.synchronize()
+            for name, a, b in evs:
+                per_op.setdefault(name, []).append(a.elapsed_time(b) * 1e3)  # us
+        del gate
+        per_step_us = {n: sum(v) / args.profile_steps for n, v in per_op.items()}
+        dominant = max(per_step_us, key=per_step_us.get)
+        iso_us = statistics.mean(per_op[dominant])
+
+        # ---- the dominant kernel as it runs inside the step: every refined-layer
+        # launch of the step, in step order with the step's flags (overlapped
+        # launches, in-kernel appends), and nothing else; one graph, timed like
+        # the step
+        def rd_chain():
+            for l in range(L):
+                pl = cfg.is_proposal(l)
+                fa = not pl or dec.scorer_appends
+                src = l - l % cfg.group
+                prism.refine_decode(dec.p, q_layers[l], ks[l], vs[l], dec.pool[src], dec.pool_cnt[src],
+                                    cfg.kappa_p, cfg.kappa, dec.scale, dec.idx[l], dec.cnt[l],
+                                    dec.out[l], dec.ws_rd, lse=dec.lse[l],
+                                    k_new=k_new[l] if fa else None, v_new=v_new[l] if fa else None,
+                                    overlap=dec.fused and not pl and l > 0, sum_group=dec.sum_group)
+
+        g_rd = graph_of(rd_chain, stream)
+        rd_reps = max(20, args.steps)
+        rd_secs = dist.max(timed(g_rd.replay, rd_reps, args.warmup))
+        del g_rd
+        instep_us = rd_secs * 1e6 / (rd_reps * L)
+        peak, peak_kind = hbm_peak()
+        achieved = nbytes["refine_decode"] / (instep_us * 1e-6) / 1e9
+        roofline = {"bound": "hbm", "kernel": "refine_decode", "achieved": round(achieved, 1),
+                    "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
+                    "frac": round(achieved / peak, 4), "traffic": traffic_for("refine_decode"),
+                    "algorithmic_bytes_per_launch": nbytes["refine_decode"],
+                    "avg_launch_us": round(instep_us, 3), "launches_per_step": L,
+                    "timing": "in step: a graph of the step's refined-layer launches in step order "
+                              "with the step's flags, CUDA events on the launching stream, "
+                              f"{rd_reps} replays / ({rd_reps} x {L} launches)",
+                    "share_of_step": round(L * instep_us / (ms_per_step * 1e3), 3),
+                    "isolated_launch_us": round(statistics.mean(per_op["refine_decode"]), 2),
+                    "isolated_frac": round(nbytes["refine_decode"]
+                                           / (statistics.mean(per_op["refine_decode"]) * 1e-6) / 1e9 / peak, 4),
+                    "largest_isolated_op": dominant, "largest_isolated_op_us": round(iso_us, 2)}
+        ops_summary = {n: {"us_per_launch": round(statistics.mean(v), 2),
+                           "launches_per_step": len(v) // args.profile_steps,
+                           "GB/s": round(nbytes[n] / (statistics.mean(v) * 1e-6) / 1e9, 1)}
+                       for n, v in per_op.items()}
+    else:
+        # the variants: the refined (non-proposal) layers of the step, in step
+        # order through the layer driver, timed as one graph
+        def layer_chain():
+            for l in range(L):
+                if not cfg.is_proposal(l):
+                    dec.layer(l, q_layers[l], ks[l], vs[l], k_new=k_new[l], v_new=v_new[l],
+                              overlap=dec.fused and l > 0)
+
+        g_lc = graph_of(layer_chain, stream)
+        nref = sum(1 for l in range(L) if not cfg.is_proposal(l))
+        reps = max(20, args.steps)
+        lc_secs = dist.max(timed(g_lc.replay, reps, args.warmup))
+        del g_lc
+        per_us = lc_secs * 1e6 / (reps * nref)
+        peak, peak_kind = hbm_peak()
+        lb = nbytes["refine_decode"] if dec.fused else nbytes["refine"] + nbytes["sparse_decode"]
+        achieved = lb / (per_us * 1e-6) / 1e9
+        roofline = {"bound": "hbm", "kernel": "refined_layer" if not dec.fused else "refine_decode",
+                    "achieved": round(achieved, 1), "peak": peak, "peak_source": peak_kind,
+                    "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                    "algorithmic_bytes_per_launch": lb, "avg_launch_us": round(per_us, 3),
+                    "launches_per_step": nref,
+                    "timing": "in step: a graph of the step's refined layers through the layer "
+                              f"driver, {reps} replays / ({reps} x {nref} layers)",
+                    "share_of_step": round(nref * per_us / (ms_per_step * 1e3), 3)}
+        ops_summary = None
     step_achieved = nbytes["step"] / (ms_per_step * 1e-3) / 1e9
 
     # ---- dense flash-decode over the identical cache (comparison path)
@@ -642,14 +689,16 @@ def run_prism(args, dist: Dist):
         units = unit_list(cfg)
         nt = oracle_threads(cfg, host_cores())
         v_n, n_n, s_n = oracle_rate(cfg, q_layers, ks, vs, nt, args.cpu_seconds, args.keys,
-                                    args.group_agg)
+                                    args.group_agg, args.proposal_select)
         v_1, n_1, s_1 = oracle_rate(cfg, q_layers, ks, vs, 1, args.cpu_seconds / 3, args.keys,
-                                    args.group_agg)
+                                    args.group_agg, args.proposal_select)
         cpu = {"value": v_n, "unit": "steps/s", "cores": nt, "kind": "oracle",
                "sample": f"{n_n} (proposal group, KV head) units of a {cfg.name} decode step "
                          f"({len(units)} per step), {nt} at a time on {nt} threads, "
                          f"{s_n:.1f} s wall; value = units/s / {len(units)}",
                "host_cores": host_cores(),
+               "reading": "per (sequence, KV head) sets" if args.sets == "kv_head" else
+               "per (sequence, KV head) sets (the oracle's units do not split by the variant's granularity)",
                "single_thread": {"value": v_1, "cores": 1,
                                  "sample": f"{n_1} units on one thread, {s_1:.1f} s"}}
 

@@ -244,6 +244,64 @@ PRISM_API prism_status prism_refine(const prism_shape* shape, const void* q, con
                           void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Selection granularity (sec. 4.1 shares index sets under GQA without saying
+ * at which granularity; sec. 3 analyses attention per head; sec. 2 "Related
+ * Work" names a set shared by all heads).  The plain calls use one pool and
+ * one set per (sequence, KV head), the scores of its G query heads combined
+ * by their maximum.  The _ex calls take `sets`:
+ *   PRISM_SETS_KV_HEAD   that default (the _ex calls forward to the plain ones);
+ *   PRISM_SETS_Q_HEAD    the pool stays per (sequence, KV head); each query
+ *                        head keeps its own top kappa of that pool by its own
+ *                        exact score q_hq . K and attends over it: idx / cnt
+ *                        are [B][Hq][kappa] / [B][Hq];
+ *   PRISM_SETS_SEQUENCE  one pool and one set per sequence, shared by every
+ *                        head: a position's score is the maximum over all KV
+ *                        heads of the per-KV-head score; pool / pool_cnt are
+ *                        [B][kappa_p] / [B], idx / cnt [B][kappa] / [B], and
+ *                        every query head attends over the sequence's set
+ *                        with its own KV head's rows.
+ * Workspaces are those of the plain calls (prism_workspace_size covers every
+ * granularity).  Other `sets` values: PRISM_ERR_INVALID_ARG.
+ */
+#define PRISM_SETS_KV_HEAD 0u
+#define PRISM_SETS_Q_HEAD 1u
+#define PRISM_SETS_SEQUENCE 2u
+PRISM_API prism_status prism_propose_ex(const prism_shape* shape, const void* q, const int8_t* kq,
+                                        const float* k_scale, int32_t kappa_p, int32_t* pool_idx,
+                                        int32_t* pool_cnt, uint32_t sets, void* ws,
+                                        size_t ws_bytes, void* stream);
+PRISM_API prism_status prism_refine_ex(const prism_shape* shape, const void* q, const void* k,
+                                       const int32_t* pool_idx, const int32_t* pool_cnt,
+                                       int32_t kappa_p, int32_t kappa, int32_t* idx, int32_t* cnt,
+                                       uint32_t sets, void* ws, size_t ws_bytes, void* stream);
+PRISM_API prism_status prism_sparse_decode_ex(const prism_shape* shape, const void* q,
+                                              const void* k, const void* v, const int32_t* idx,
+                                              const int32_t* cnt, int32_t kappa,
+                                              float softmax_scale, uint32_t sets, float* out,
+                                              float* lse_opt, void* ws, size_t ws_bytes,
+                                              void* stream);
+
+/*
+ * The proposal layer's own index set under the other reading of sec. 4.1
+ * (refined layers re-select inside the pool; what the proposal layer itself
+ * attends over is not stated): the top min(kappa, pool_cnt) members of the
+ * pool by the proposal scores the proposal call just computed -- no exact
+ * rescoring -- written as ascending positions to idx [B][Hkv][kappa] and cnt
+ * [B][Hkv] (ties to the lower position).  The default reading is
+ * prism_refine / prism_refine_decode on the proposal layer's own pool.
+ * propose_ws is the workspace of the prism_propose, prism_propose_append or
+ * prism_propose_int2 call that produced pool_idx / pool_cnt, on the same
+ * stream and shape, with no call on that workspace in between (its scores
+ * are read); ws is sized by PRISM_OP_REFINE for (kappa_p, kappa).  Follow
+ * with prism_sparse_decode on idx for the layer's attention.
+ */
+PRISM_API prism_status prism_propose_topk(const prism_shape* shape, const void* propose_ws,
+                                          size_t propose_ws_bytes, const int32_t* pool_idx,
+                                          const int32_t* pool_cnt, int32_t kappa_p, int32_t kappa,
+                                          int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes,
+                                          void* stream);
+
+/*
  * Token-level sparse attention over the selected rows (sec. 1, sec. 2.1):
  * for every query head hq of sequence b, with h = hq / G and the rows
  * t in idx[b][h][0 .. cnt[b][h]),
@@ -308,6 +366,23 @@ PRISM_API prism_status prism_refine_decode(const prism_shape* shape, const void*
 PRISM_API prism_status prism_dense_decode(const prism_shape* shape, const void* q, const void* k,
                                 const void* v, float softmax_scale, float* out, float* lse_opt,
                                 void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Index overlap of two selections, per row (sec. 3 "Observations", Figure 1:
+ * the overlap ratio between a reference layer's index set and the set of a
+ * layer at some offset; Figure 12: the share of one layer's top-kappa that an
+ * expanded top-rho*kappa set of another layer covers).  A diagnostic outside
+ * the decode step.  a [rows][stride_a] and b [rows][stride_b] are device
+ * index sets, row r holding cnt_a[r] / cnt_b[r] members (clamped to
+ * [0, stride]) in strictly ascending order, as every selection of this
+ * library is written; out[r] = |a_r intersect b_r| (device int32 [rows]).
+ * Rows whose lists are not ascending give an unspecified count (no memory
+ * outside the rows is read).  rows = 0 enqueues nothing.
+ */
+PRISM_API prism_status prism_index_overlap(int32_t rows, const int32_t* a, const int32_t* cnt_a,
+                                           int32_t stride_a, const int32_t* b,
+                                           const int32_t* cnt_b, int32_t stride_b, int32_t* out,
+                                           void* stream);
 
 /* Zero the workspace header (status word) on `stream`. */
 PRISM_API prism_status prism_clear_device_status(void* ws, size_t ws_bytes, void* stream);

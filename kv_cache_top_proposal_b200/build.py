@@ -20,7 +20,8 @@ SO = os.path.join(LIBDIR, "libprism.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "prism.h")
 
 SOURCES = ["prism_api.cu", "quantize.cu", "score.cu", "select.cu", "refine.cu", "attend.cu",
-           "refine_decode.cu", "propose_select.cu"]
+           "refine_decode.cu", "propose_select.cu", "overlap.cu",
+           "sets.cu"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-std=c++17", "-lineinfo",

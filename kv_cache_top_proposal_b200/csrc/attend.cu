@@ -22,6 +22,8 @@ namespace {
 
 constexpr int kThreads = 128;
 constexpr int kWarps = kThreads / 32;
+// rows a lane group loads before it computes (a deeper unroll costs
+// registers, hence resident warps, and moved no more bytes per SM)
 constexpr int kUnroll = 2;
 
 struct AttendArgs {
@@ -39,6 +41,8 @@ struct AttendArgs {
   float* part_o;
   float* part_ml;
   int32_t* status;
+  int kv_div;   // row (b, h) reads K/V head h / kv_div
+  int idx_div;  // and idx / cnt row (b Hkv + h) / idx_div
 };
 
 template <typename T, int D, int GP>
@@ -60,8 +64,9 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendArgs a) {
   const int t0 = a.cu[b];
   const int L = a.cu[b + 1] - t0;
   int n = L;
+  const int irow = row / a.idx_div;
   if (a.idx) {
-    n = a.cnt[row];
+    n = a.cnt[irow];
     if (n < 0 || n > a.idx_stride) {
       if (threadIdx.x == 0 && split == 0) flag_status(a.status, PRISM_DEV_BAD_INDEX);
       n = n < 0 ? 0 : a.idx_stride;
@@ -69,10 +74,10 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendArgs a) {
   }
   const int e0 = split * a.per_split;
   const int e1 = min(n, e0 + a.per_split);
-  const int64_t off = ((int64_t)h * a.T + t0) * D + li * E;
+  const int64_t off = ((int64_t)(h / a.kv_div) * a.T + t0) * D + li * E;
   const T* kbase = static_cast<const T*>(a.k) + off;
   const T* vbase = static_cast<const T*>(a.v) + off;
-  const int32_t* idx = a.idx ? a.idx + (int64_t)row * a.idx_stride : nullptr;
+  const int32_t* idx = a.idx ? a.idx + (int64_t)irow * a.idx_stride : nullptr;
 
   float qf[GP][E];
   {
@@ -196,6 +201,226 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(const AttendArgs a) {
   }
 }
 
+// ---- dense pass (the comparison path): contiguous rows staged by bulk copies
+//
+// Split s of row (b, h) covers positions [s*per, (s+1)*per) of sequence b.
+// Thread 0 keeps kDStages stages in flight, each one 1D bulk copy of kDRows
+// K rows and one of kDRows V rows (8 KB each, contiguous in the cache) into
+// shared memory, completing on the stage's mbarrier; the CTA computes on the
+// oldest stage with the same lane-group math as attend_kernel (two rows per
+// lane group per stage pass) and hands the stage back.  Bytes in flight per
+// SM come from the stage ring, not from registers.  A stage wait is bounded:
+// past kDWaitLimit polls the CTA flags PRISM_DEV_TIMEOUT, waits (bounded) for
+// its copies in flight and returns.
+constexpr int kDThreads = 256;
+constexpr int kDWarps = kDThreads / 32;
+constexpr int kDStages = 6;
+constexpr int kDPartBytes = 8192;  // K (or V) bytes of one stage
+constexpr uint32_t kDWaitLimit = 1u << 24;
+
+__device__ __forceinline__ void d_mbar_init(uint64_t* bar) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool d_mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void d_bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <typename T, int D, int GP>
+__global__ void __launch_bounds__(kDThreads, GP <= 4 ? 2 : 1) dense_kernel(const AttendArgs a) {
+  constexpr int E = Vec16<T>::E;
+  constexpr int LPR = D / E;            // lanes per row
+  constexpr int RPW = 32 / LPR;         // rows per warp per pass
+  constexpr int RB = D * (int)sizeof(T);
+  constexpr int R = kDPartBytes / RB;   // rows per stage
+  constexpr int PASS = kDWarps * RPW;   // rows per CTA pass
+  static_assert(R == 2 * PASS, "two passes per stage");
+  constexpr int SLOTS = kDWarps * RPW;
+  extern __shared__ __align__(128) unsigned char dsm[];
+  __shared__ __align__(8) uint64_t full[kDStages];
+
+  const int row = blockIdx.x, split = blockIdx.y;
+  const int b = row / a.Hkv, h = row - b * a.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int sub = lane / LPR, li = lane % LPR;
+  const int slot = warp * RPW + sub;
+  const int t0 = a.cu[b];
+  const int L = a.cu[b + 1] - t0;
+  const int e0 = split * a.per_split;
+  const int e1 = min(L, e0 + a.per_split);
+  const int nst = e1 > e0 ? (e1 - e0 + R - 1) / R : 0;
+  const unsigned char* kg = reinterpret_cast<const unsigned char*>(static_cast<const T*>(a.k) +
+                                                                   ((int64_t)h * a.T + t0) * D);
+  const unsigned char* vg = reinterpret_cast<const unsigned char*>(static_cast<const T*>(a.v) +
+                                                                   ((int64_t)h * a.T + t0) * D);
+  auto stage_k = [&](int i) { return dsm + (i % kDStages) * 2 * kDPartBytes; };
+  auto issue = [&](int i) {  // thread 0
+    if (i < nst) {
+      const int r0 = e0 + i * R, n = min(R, e1 - r0);
+      uint64_t* bar = &full[i % kDStages];
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
+                   "r"(2 * n * RB)
+                   : "memory");
+      d_bulk_load(stage_k(i), kg + (int64_t)r0 * RB, n * RB, bar);
+      d_bulk_load(stage_k(i) + kDPartBytes, vg + (int64_t)r0 * RB, n * RB, bar);
+    }
+  };
+  if (tid == 0) {
+    for (int i = 0; i < kDStages; ++i) d_mbar_init(&full[i]);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    for (int i = 0; i < kDStages; ++i) issue(i);
+  }
+  __syncthreads();
+
+  float qf[GP][E];
+  {
+    const T* q = static_cast<const T*>(a.q) + ((int64_t)b * a.Hq + (int64_t)h * a.G) * D + li * E;
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      if (g < a.G) {
+        Vec16<T>::unpack(ld16(q + (int64_t)g * D), qf[g]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) qf[g][e] = 0.0f;
+      }
+    }
+  }
+  float m[GP], l[GP], o[GP][E];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    m[g] = -INFINITY;
+    l[g] = 0.0f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) o[g][e] = 0.0f;
+  }
+
+  for (int i = 0; i < nst; ++i) {
+    bool late = false;
+    {
+      uint32_t it = 0;
+      while (!d_mbar_try_wait(&full[i % kDStages], (uint32_t)(i / kDStages) & 1u)) {
+        if (++it == kDWaitLimit) {
+          late = true;
+          break;
+        }
+      }
+    }
+    if (__syncthreads_or(late)) {  // a stage never arrived: report, drain, stop
+      if (tid == 0) {
+        flag_status(a.status, PRISM_DEV_TIMEOUT);
+        for (int j = i; j < nst && j < i + kDStages; ++j) {
+          uint32_t it = 0;
+          while (!d_mbar_try_wait(&full[j % kDStages], (uint32_t)(j / kDStages) & 1u) && ++it < kDWaitLimit) {
+          }
+        }
+      }
+      return;
+    }
+    const unsigned char* ks = stage_k(i);
+    const unsigned char* vs = ks + kDPartBytes;
+    const int r0 = e0 + i * R, n = min(R, e1 - r0);
+    uint4 kr[2], vr[2];
+    bool ok[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int r = u * PASS + slot;
+      ok[u] = r < n;
+      kr[u] = ok[u] ? *reinterpret_cast<const uint4*>(ks + r * RB + li * 16) : make_uint4(0, 0, 0, 0);
+      vr[u] = ok[u] ? *reinterpret_cast<const uint4*>(vs + r * RB + li * 16) : make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();  // the stage is in registers: hand it back
+    if (tid == 0) issue(i + kDStages);
+    float lg[2][GP];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      float f[E];
+      Vec16<T>::unpack(kr[u], f);
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float sdot = 0.0f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) sdot = fmaf(qf[g][e], f[e], sdot);
+        sdot = group_sum<LPR>(sdot);
+        lg[u][g] = ok[u] ? sdot * a.scale_log2 : -INFINITY;
+      }
+    }
+    float vf[2][E];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) Vec16<T>::unpack(vr[u], vf[u]);
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      const float mx = fmaxf(m[g], fmaxf(lg[0][g], lg[1][g]));
+      if (mx == -INFINITY) continue;
+      const float alpha = exp2f(m[g] - mx);
+      const float p0 = exp2f(lg[0][g] - mx), p1 = exp2f(lg[1][g] - mx);
+      l[g] = l[g] * alpha + (p0 + p1);
+#pragma unroll
+      for (int e = 0; e < E; ++e) o[g][e] = fmaf(p1, vf[1][e], fmaf(p0, vf[0][e], o[g][e] * alpha));
+      m[g] = mx;
+    }
+  }
+
+  // combine the CTA's lane groups in slot order (the ring is free now)
+  float* s_o = reinterpret_cast<float*>(dsm);  // [SLOTS][GP][D]
+  float* s_m = s_o + SLOTS * GP * D;           // [SLOTS][GP]
+  float* s_l = s_m + SLOTS * GP;               // [SLOTS][GP]
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) s_o[(slot * GP + g) * D + li * E + e] = o[g][e];
+    if (li == 0) {
+      s_m[slot * GP + g] = m[g];
+      s_l[slot * GP + g] = l[g];
+    }
+  }
+  __syncthreads();
+  for (int x = tid; x < a.G * D; x += kDThreads) {
+    const int g = x / D, j = x - g * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int sl = 0; sl < SLOTS; ++sl) M = fmaxf(M, s_m[sl * GP + g]);
+    float Ls = 0.0f, O = 0.0f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int sl = 0; sl < SLOTS; ++sl) {
+        const float ms = s_m[sl * GP + g];
+        const float w = ms == -INFINITY ? 0.0f : exp2f(ms - M);
+        Ls = fmaf(w, s_l[sl * GP + g], Ls);
+        O = fmaf(w, s_o[(sl * GP + g) * D + j], O);
+      }
+    }
+    const int64_t pr = ((int64_t)b * a.Hq + (int64_t)h * a.G + g) * a.splits + split;
+    a.part_o[pr * D + j] = O;
+    if (j == 0) {
+      a.part_ml[pr * 2] = M;
+      a.part_ml[pr * 2 + 1] = Ls;
+    }
+  }
+}
+
+// dense shared memory: the stage ring, which also holds the lane groups'
+// partials at the end
+template <typename T, int D, int GP>
+constexpr int dense_smem() {
+  constexpr int ring = kDStages * 2 * kDPartBytes;
+  constexpr int slots = kDWarps * (32 / (D / Vec16<T>::E));
+  constexpr int comb = (slots * GP * D + 2 * slots * GP) * 4;
+  return ring > comb ? ring : comb;
+}
+
 // One CTA of D threads per (sequence, query head): the split weights
 // 2^(m_s - M) are computed in parallel into shared memory, then thread j sums
 // its feature over the splits with independent (pipelined) loads.
@@ -252,6 +477,14 @@ __global__ void __launch_bounds__(D) merge_kernel(int splits, const float* __res
 
 template <typename T, int D, int GP>
 cudaError_t run(const Dims& d, const AttendPlan& p, const AttendArgs& a, cudaStream_t st) {
+  if (!a.idx) {  // dense: the staged kernel
+    constexpr int smem = dense_smem<T, D, GP>();
+    auto kd = dense_kernel<T, D, GP>;
+    cudaError_t e = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kd<<<dim3(d.B * d.Hkv, p.splits), kDThreads, smem, st>>>(a);
+    return cudaGetLastError();
+  }
   constexpr int RPW = 32 / (D / Vec16<T>::E);
   constexpr int SLOTS = kWarps * RPW;
   const int smem = (SLOTS * GP * D + 2 * SLOTS * GP) * (int)sizeof(float);
@@ -277,10 +510,14 @@ cudaError_t by_group(const Dims& d, const AttendPlan& p, const AttendArgs& a, cu
 
 }  // namespace
 
-AttendPlan plan_attend(const Dims& d, int64_t max_rows_per_seq) {
-  constexpr int step = 16;  // rows one CTA covers per iteration (bf16, d = 128)
+AttendPlan plan_attend(const Dims& d, int64_t max_rows_per_seq, bool dense) {
+  // rows one CTA covers per iteration: a sparse pass step (bf16, d = 128), or
+  // a dense stage (the largest, fp32 d = 64: 64 rows, so every dtype's
+  // stage divides it)
+  const int step = dense ? 64 : 16;
   const int64_t rows = (int64_t)d.B * d.Hkv;
-  const int64_t target = 4LL * d.num_sms;
+  // dense: one wave of two CTAs per SM; sparse: four CTAs per SM
+  const int64_t target = (dense ? 2LL : 4LL) * d.num_sms;
   int64_t splits = rows > 0 ? cdiv(target, rows) : 1;
   const int64_t max_splits = cdiv(max_rows_per_seq > 0 ? max_rows_per_seq : 1, step);
   if (splits > max_splits) splits = max_splits;
@@ -294,10 +531,11 @@ AttendPlan plan_attend(const Dims& d, int64_t max_rows_per_seq) {
 cudaError_t launch_attend(const Dims& d, const AttendPlan& p, const void* q, const void* k,
                           const void* v, const int32_t* idx, const int32_t* cnt, int idx_stride,
                           float softmax_scale, float* part_o, float* part_ml, float* out,
-                          float* lse, int32_t* status, cudaStream_t st) {
+                          float* lse, int32_t* status, cudaStream_t st, int kv_div, int idx_div) {
   if (d.B * d.Hq == 0) return cudaSuccess;
   AttendArgs a{q, k, v, d.cu_dev, idx, cnt, idx_stride, d.Hkv, d.G, d.Hq, d.T,
-               p.per_split, p.splits, softmax_scale * 1.4426950408889634f, part_o, part_ml, status};
+               p.per_split, p.splits, softmax_scale * 1.4426950408889634f, part_o, part_ml, status,
+               kv_div > 1 ? kv_div : 1, idx_div > 1 ? idx_div : 1};
   cudaError_t e;
   if (d.bf16)
     e = d.D == 128 ? by_group<__nv_bfloat16, 128>(d, p, a, st) : by_group<__nv_bfloat16, 64>(d, p, a, st);

@@ -76,6 +76,7 @@ struct SelectArgs {
   const float* dots;
   float* logits;
   int32_t* status;
+  int pool_div;  // mode 1: pool row = row / pool_div (0 or 1: the row itself)
 };
 int select_capacity_per_row();  // longest row one cluster can select from
 
@@ -88,10 +89,21 @@ cudaError_t launch_propose_select(const Dims& d, const float* scores, const uint
                                   cudaStream_t st);
 cudaError_t launch_select(const Dims& d, const SelectArgs& a, int max_row_len, cudaStream_t st);
 
-// Exact pool scores r[row][i] = max_g q_g . K[pool_i] (+ per-head dots).
+// Exact pool scores r[row][i] = max_g q_g . K[pool_i] (+ per-head dots);
+// row (b, h) reads pool row (b * Hkv + h) / pool_div (pool_div = Hkv: one
+// pool per sequence shared by its KV heads).
 cudaError_t launch_refine_scores(const Dims& d, const void* q, const void* k, const int32_t* pool,
                                  const int32_t* pool_cnt, int pool_stride, float* r, float* dots,
-                                 int32_t* status, cudaStream_t st);
+                                 int32_t* status, cudaStream_t st, int pool_div = 1);
+// out[o][i] = max_h in[(o * H + h) * inner + i] over h < H, for o < outer,
+// i < inner (the maximum of per-head scores over the heads; sets.cu).
+cudaError_t launch_head_max(const float* in, int H, int64_t outer, int64_t inner, float* out,
+                            cudaStream_t st);
+
+// Proposal scores of the pool members: r[row][i] = scores[h][cu[b] + pool[row][i]].
+cudaError_t launch_pool_gather(const Dims& d, const float* scores, const int32_t* pool,
+                               const int32_t* pool_cnt, int pool_stride, float* r, int32_t* status,
+                               cudaStream_t st);
 
 // Fused refine -> top-kappa -> sparse decode, one cluster of `cluster` CTAs
 // per (sequence, KV head); mc = pool members per CTA.  ok = false when the
@@ -115,10 +127,20 @@ struct AttendPlan {
   int splits;
   int per_split;
 };
-AttendPlan plan_attend(const Dims& d, int64_t max_rows_per_seq);
+AttendPlan plan_attend(const Dims& d, int64_t max_rows_per_seq, bool dense);
+// kv_div: row (b, h) of d reads K/V head h / kv_div (d.Hkv = Hq, G = 1 for
+// one set per query head); idx_div: it reads idx / cnt row (b Hkv + h) /
+// idx_div (idx_div = Hkv for one set per sequence).
 cudaError_t launch_attend(const Dims& d, const AttendPlan& p, const void* q, const void* k,
                           const void* v, const int32_t* idx, const int32_t* cnt, int idx_stride,
                           float softmax_scale, float* part_o, float* part_ml, float* out,
-                          float* lse, int32_t* status, cudaStream_t st);
+                          float* lse, int32_t* status, cudaStream_t st, int kv_div = 1,
+                          int idx_div = 1);
+
+// |a_row intersect b_row| per row of two ascending index-set arrays
+// (overlap.cu); counts are clamped to [0, stride].
+cudaError_t launch_overlap(int rows, const int32_t* a, const int32_t* cnt_a, int stride_a,
+                           const int32_t* b, const int32_t* cnt_b, int stride_b, int32_t* out,
+                           cudaStream_t st);
 
 }  // namespace prism

@@ -77,21 +77,27 @@ Layout layout(const Dims& d, int op, int kappa_p, int kappa) {
   switch (op) {
     case PRISM_OP_QUANTIZE:
       break;
-    case PRISM_OP_PROPOSE:  // scores [Hkv][T] fp32, first-digit histogram [rows][4096] u32
+    case PRISM_OP_PROPOSE:  // scores [Hkv][T] fp32, first-digit histogram [rows][4096] u32,
+                            // per-sequence head maxima [T] fp32
       L.a = off;
       off = align_up(off + (size_t)d.Hkv * (size_t)d.T * sizeof(float));
       L.b = off;
       off = align_up(off + rows * 4096 * 4);
+      L.c = off;
+      off = align_up(off + (size_t)d.T * sizeof(float));
       break;
-    case PRISM_OP_REFINE:  // r [rows][kappa_p], dots [rows][G][kappa_p]
+    case PRISM_OP_REFINE:  // r [rows][kappa_p], dots [rows][G][kappa_p], head maxima [B][kappa_p]
       L.a = off;
       off = align_up(off + rows * (size_t)kappa_p * sizeof(float));
       L.b = off;
       off = align_up(off + rows * (size_t)d.G * (size_t)kappa_p * sizeof(float));
+      L.c = off;
+      off = align_up(off + (size_t)d.B * (size_t)kappa_p * sizeof(float));
       break;
     case PRISM_OP_SPARSE_DECODE:
     case PRISM_OP_DENSE_DECODE: {
-      const AttendPlan p = plan_attend(d, op == PRISM_OP_SPARSE_DECODE ? kappa : d.max_len);
+      const AttendPlan p = plan_attend(d, op == PRISM_OP_SPARSE_DECODE ? kappa : d.max_len,
+                                      op == PRISM_OP_DENSE_DECODE);
       const size_t parts = (size_t)d.B * d.Hq * (size_t)p.splits;
       L.a = off;  // partial o [B][Hq][splits][D]
       off = align_up(off + parts * (size_t)d.D * sizeof(float));
@@ -330,6 +336,185 @@ prism_status prism_refine(const prism_shape* shape, const void* q, const void* k
   return cuda_status(launch_select(d, a, kappa_p, st));
 }
 
+prism_status prism_propose_topk(const prism_shape* shape, const void* propose_ws,
+                                size_t propose_ws_bytes, const int32_t* pool_idx,
+                                const int32_t* pool_cnt, int32_t kappa_p, int32_t kappa,
+                                int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes,
+                                void* stream) {
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!pool_idx || !pool_cnt || !idx || !cnt) return PRISM_ERR_INVALID_ARG;
+  if (kappa_p < 1 || kappa < 1 || kappa > kappa_p) return PRISM_ERR_INVALID_ARG;
+  if (kappa_p > select_capacity_per_row()) return PRISM_ERR_UNSUPPORTED;
+  const Layout P = layout(d, PRISM_OP_PROPOSE, kappa_p, 0);
+  if (!ws_ok(propose_ws, propose_ws_bytes, P)) return PRISM_ERR_WORKSPACE;
+  const Layout L = layout(d, PRISM_OP_REFINE, kappa_p, kappa);
+  if (!ws_ok(ws, ws_bytes, L)) return PRISM_ERR_WORKSPACE;
+  if ((s = set_live_sms(&d)) != PRISM_OK) return s;
+  char* w = static_cast<char*>(ws);
+  int32_t* status = reinterpret_cast<int32_t*>(w);
+  float* r = reinterpret_cast<float*>(w + L.a);
+  const float* scores = reinterpret_cast<const float*>(static_cast<const char*>(propose_ws) + P.a);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_pool_gather(d, scores, pool_idx, pool_cnt, kappa_p, r, status, st);
+  if (e != cudaSuccess) return PRISM_ERR_CUDA;
+  SelectArgs a{};
+  a.mode = 1;
+  a.Hkv = d.Hkv;
+  a.G = d.G;
+  a.Hq = d.Hq;
+  a.T = d.T;
+  a.cu = d.cu_dev;
+  a.keys = r;
+  a.pool = pool_idx;
+  a.pool_cnt = pool_cnt;
+  a.pool_stride = kappa_p;
+  a.k_req = kappa;
+  a.out = idx;
+  a.out_cnt = cnt;
+  a.status = status;
+  return cuda_status(launch_select(d, a, kappa_p, st));
+}
+
+prism_status prism_propose_ex(const prism_shape* shape, const void* q, const int8_t* kq,
+                              const float* k_scale, int32_t kappa_p, int32_t* pool_idx,
+                              int32_t* pool_cnt, uint32_t sets, void* ws, size_t ws_bytes,
+                              void* stream) {
+  if (sets == PRISM_SETS_KV_HEAD || sets == PRISM_SETS_Q_HEAD)
+    return prism_propose(shape, q, kq, k_scale, kappa_p, pool_idx, pool_cnt, ws, ws_bytes, stream);
+  if (sets != PRISM_SETS_SEQUENCE) return PRISM_ERR_INVALID_ARG;
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!q || !kq || !k_scale || !pool_idx || !pool_cnt || kappa_p < 1) return PRISM_ERR_INVALID_ARG;
+  if (d.max_len > select_capacity_per_row()) return PRISM_ERR_UNSUPPORTED;
+  const Layout L = layout(d, PRISM_OP_PROPOSE, kappa_p, 0);
+  if (!ws_ok(ws, ws_bytes, L)) return PRISM_ERR_WORKSPACE;
+  if ((s = set_live_sms(&d)) != PRISM_OK) return s;
+  char* w = static_cast<char*>(ws);
+  int32_t* status = reinterpret_cast<int32_t*>(w);
+  float* scores = reinterpret_cast<float*>(w + L.a);
+  float* smax = reinterpret_cast<float*>(w + L.c);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_propose_scores(d, q, kq, k_scale, scores, nullptr, use_mma_scorer() && d.bf16,
+                                        status, st);
+  if (e != cudaSuccess) return PRISM_ERR_CUDA;
+  if ((e = launch_head_max(scores, d.Hkv, 1, d.T, smax, st)) != cudaSuccess) return PRISM_ERR_CUDA;
+  Dims d1 = d;  // one selection row per sequence over the head maxima
+  d1.Hkv = 1;
+  d1.G = d.Hq;
+  SelectArgs a{};
+  a.mode = 0;
+  a.Hkv = 1;
+  a.G = d.Hq;
+  a.Hq = d.Hq;
+  a.T = d.T;
+  a.cu = d.cu_dev;
+  a.keys = smax;
+  a.k_req = kappa_p;
+  a.out = pool_idx;
+  a.out_cnt = pool_cnt;
+  a.status = status;
+  return cuda_status(launch_select(d1, a, d.max_len, st));
+}
+
+prism_status prism_refine_ex(const prism_shape* shape, const void* q, const void* k,
+                             const int32_t* pool_idx, const int32_t* pool_cnt, int32_t kappa_p,
+                             int32_t kappa, int32_t* idx, int32_t* cnt, uint32_t sets, void* ws,
+                             size_t ws_bytes, void* stream) {
+  if (sets == PRISM_SETS_KV_HEAD)
+    return prism_refine(shape, q, k, pool_idx, pool_cnt, kappa_p, kappa, idx, cnt, nullptr, ws,
+                        ws_bytes, stream);
+  if (sets != PRISM_SETS_Q_HEAD && sets != PRISM_SETS_SEQUENCE) return PRISM_ERR_INVALID_ARG;
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!q || !k || !pool_idx || !pool_cnt || !idx || !cnt) return PRISM_ERR_INVALID_ARG;
+  if (kappa_p < 1 || kappa < 1 || kappa > kappa_p) return PRISM_ERR_INVALID_ARG;
+  if (kappa_p > select_capacity_per_row()) return PRISM_ERR_UNSUPPORTED;
+  const Layout L = layout(d, PRISM_OP_REFINE, kappa_p, kappa);
+  if (!ws_ok(ws, ws_bytes, L)) return PRISM_ERR_WORKSPACE;
+  if ((s = set_live_sms(&d)) != PRISM_OK) return s;
+  char* w = static_cast<char*>(ws);
+  int32_t* status = reinterpret_cast<int32_t*>(w);
+  float* r = reinterpret_cast<float*>(w + L.a);
+  float* dots = reinterpret_cast<float*>(w + L.b);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SelectArgs a{};
+  a.mode = 1;
+  a.T = d.T;
+  a.cu = d.cu_dev;
+  a.pool = pool_idx;
+  a.pool_cnt = pool_cnt;
+  a.pool_stride = kappa_p;
+  a.k_req = kappa;
+  a.out = idx;
+  a.out_cnt = cnt;
+  a.status = status;
+  Dims d1 = d;
+  if (sets == PRISM_SETS_Q_HEAD) {
+    // per-head exact scores dots [B][Hkv][G][kappa_p] = [B Hq][kappa_p]: one
+    // selection row per query head over its group's pool
+    cudaError_t e = launch_refine_scores(d, q, k, pool_idx, pool_cnt, kappa_p, r, dots, status, st);
+    if (e != cudaSuccess) return PRISM_ERR_CUDA;
+    d1.Hkv = d.Hq;
+    d1.G = 1;
+    a.keys = dots;
+    a.pool_div = d.G;
+  } else {
+    // every KV head scores the sequence's pool; the head maxima select
+    float* rmax = reinterpret_cast<float*>(w + L.c);
+    cudaError_t e = launch_refine_scores(d, q, k, pool_idx, pool_cnt, kappa_p, r, nullptr, status, st,
+                                         d.Hkv);
+    if (e != cudaSuccess) return PRISM_ERR_CUDA;
+    if ((e = launch_head_max(r, d.Hkv, d.B, kappa_p, rmax, st)) != cudaSuccess) return PRISM_ERR_CUDA;
+    d1.Hkv = 1;
+    d1.G = d.Hq;
+    a.keys = rmax;
+  }
+  a.Hkv = d1.Hkv;
+  a.G = d1.G;
+  a.Hq = d.Hq;
+  return cuda_status(launch_select(d1, a, kappa_p, st));
+}
+
+prism_status prism_sparse_decode_ex(const prism_shape* shape, const void* q, const void* k,
+                                    const void* v, const int32_t* idx, const int32_t* cnt,
+                                    int32_t kappa, float softmax_scale, uint32_t sets, float* out,
+                                    float* lse_opt, void* ws, size_t ws_bytes, void* stream) {
+  if (sets == PRISM_SETS_KV_HEAD)
+    return prism_sparse_decode(shape, q, k, v, idx, cnt, kappa, softmax_scale, out, lse_opt, ws,
+                               ws_bytes, stream);
+  if (sets != PRISM_SETS_Q_HEAD && sets != PRISM_SETS_SEQUENCE) return PRISM_ERR_INVALID_ARG;
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!q || !k || !v || !idx || !cnt || !out || kappa < 1) return PRISM_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return PRISM_ERR_INVALID_ARG;
+  const Layout L = layout(d, PRISM_OP_SPARSE_DECODE, 0, kappa);
+  if (!ws_ok(ws, ws_bytes, L)) return PRISM_ERR_WORKSPACE;
+  Dims d1 = d;
+  int kv_div = 1, idx_div = 1;
+  if (sets == PRISM_SETS_Q_HEAD) {  // a row per query head, reading its group's K/V head
+    d1.Hkv = d.Hq;
+    d1.G = 1;
+    kv_div = d.G;
+  } else {  // every KV head reads the sequence's one set
+    idx_div = d.Hkv;
+  }
+  // the per-query-head rows split no finer than the per-KV-head plan the
+  // workspace is sized for: B Hq splits' <= B Hq splits
+  const AttendPlan p = plan_attend(d1, kappa, false);
+  if ((s = set_live_sms(&d)) != PRISM_OK) return s;
+  char* w = static_cast<char*>(ws);
+  return cuda_status(launch_attend(d1, p, q, k, v, idx, cnt, kappa, softmax_scale,
+                                   reinterpret_cast<float*>(w + L.a),
+                                   reinterpret_cast<float*>(w + L.b), out, lse_opt,
+                                   reinterpret_cast<int32_t*>(w), static_cast<cudaStream_t>(stream),
+                                   kv_div, idx_div));
+}
+
 prism_status prism_sparse_decode(const prism_shape* shape, const void* q, const void* k,
                                  const void* v, const int32_t* idx, const int32_t* cnt,
                                  int32_t kappa, float softmax_scale, float* out, float* lse_opt,
@@ -341,7 +526,7 @@ prism_status prism_sparse_decode(const prism_shape* shape, const void* q, const 
   if (!std::isfinite(softmax_scale)) return PRISM_ERR_INVALID_ARG;
   const Layout L = layout(d, PRISM_OP_SPARSE_DECODE, 0, kappa);
   if (!ws_ok(ws, ws_bytes, L)) return PRISM_ERR_WORKSPACE;
-  const AttendPlan p = plan_attend(d, kappa);
+  const AttendPlan p = plan_attend(d, kappa, false);
   if ((s = set_live_sms(&d)) != PRISM_OK) return s;
   char* w = static_cast<char*>(ws);
   return cuda_status(launch_attend(d, p, q, k, v, idx, cnt, kappa, softmax_scale,
@@ -386,16 +571,27 @@ prism_status prism_dense_decode(const prism_shape* shape, const void* q, const v
   prism_status s = check_shape(shape, &d);
   if (s != PRISM_OK) return s;
   if (!q || !k || !v || !out) return PRISM_ERR_INVALID_ARG;
+  if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v) % 16) return PRISM_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale)) return PRISM_ERR_INVALID_ARG;
   const Layout L = layout(d, PRISM_OP_DENSE_DECODE, 0, 0);
   if (!ws_ok(ws, ws_bytes, L)) return PRISM_ERR_WORKSPACE;
-  const AttendPlan p = plan_attend(d, d.max_len);
+  const AttendPlan p = plan_attend(d, d.max_len, true);
   if ((s = set_live_sms(&d)) != PRISM_OK) return s;
   char* w = static_cast<char*>(ws);
   return cuda_status(launch_attend(d, p, q, k, v, nullptr, nullptr, 0, softmax_scale,
                                    reinterpret_cast<float*>(w + L.a),
                                    reinterpret_cast<float*>(w + L.b), out, lse_opt,
                                    reinterpret_cast<int32_t*>(w), static_cast<cudaStream_t>(stream)));
+}
+
+prism_status prism_index_overlap(int32_t rows, const int32_t* a, const int32_t* cnt_a,
+                                 int32_t stride_a, const int32_t* b, const int32_t* cnt_b,
+                                 int32_t stride_b, int32_t* out, void* stream) {
+  if (rows < 0 || stride_a < 1 || stride_b < 1) return PRISM_ERR_INVALID_ARG;
+  if (rows == 0) return PRISM_OK;
+  if (!a || !cnt_a || !b || !cnt_b || !out) return PRISM_ERR_INVALID_ARG;
+  return cuda_status(launch_overlap(rows, a, cnt_a, stride_a, b, cnt_b, stride_b, out,
+                                    static_cast<cudaStream_t>(stream)));
 }
 
 prism_status prism_clear_device_status(void* ws, size_t ws_bytes, void* stream) {
@@ -483,7 +679,7 @@ extern "C" prism_status prism_sparse_decode_noalloc(const prism_shape* shape, co
   // header bytes at its start stay unused (the status goes to status_dev).
   const Layout L = layout(d, PRISM_OP_SPARSE_DECODE, 0, kappa);
   if (L.total > (size_t)PRISM_NOALLOC_SCRATCH_BYTES) return PRISM_ERR_SCRATCH_LIMIT;
-  const AttendPlan p = plan_attend(d, kappa);
+  const AttendPlan p = plan_attend(d, kappa, false);
   if ((s = set_live_sms(&d)) != PRISM_OK) return s;
   char* w = nullptr;
   if ((s = noalloc_scratch_ptr(&w)) != PRISM_OK) return s;

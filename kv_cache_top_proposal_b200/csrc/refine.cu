@@ -33,6 +33,7 @@ struct RefineArgs {
   float* r;
   float* dots;
   int32_t* status;
+  int pool_div;  // row (b, h) reads pool row (b Hkv + h) / pool_div
 };
 
 template <typename T, int D, int GP>
@@ -44,7 +45,8 @@ __global__ void __launch_bounds__(kThreads) refine_score_kernel(const RefineArgs
   const int b = row / a.Hkv, h = row - b * a.Hkv;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int sub = lane / LPR, li = lane % LPR;
-  int n = a.pool_cnt[row];
+  const int prow = row / a.pool_div;
+  int n = a.pool_cnt[prow];
   n = n < 0 ? 0 : (n > a.pool_stride ? a.pool_stride : n);
   const int e0 = blockIdx.x * a.per_cta;
   const int e1 = min(n, e0 + a.per_cta);
@@ -53,7 +55,7 @@ __global__ void __launch_bounds__(kThreads) refine_score_kernel(const RefineArgs
   const int L = a.cu[b + 1] - t0;
   const T* kbase = static_cast<const T*>(a.k) + ((int64_t)h * a.T + t0) * D + li * E;
   const T* q = static_cast<const T*>(a.q) + ((int64_t)b * a.Hkv * a.G + (int64_t)h * a.G) * D;
-  const int32_t* pool = a.pool + (int64_t)row * a.pool_stride;
+  const int32_t* pool = a.pool + (int64_t)prow * a.pool_stride;
 
   float qf[GP][E];
 #pragma unroll
@@ -137,13 +139,53 @@ cudaError_t by_group(const Dims& d, const RefineArgs& a, cudaStream_t st) {
   }
 }
 
+// The proposal scores of the pool members, r[row][i] = scores[h][cu[b] +
+// pool[row][i]] (the selection keys of a proposal layer that takes its own
+// set from its quantized scores); a position outside its sequence is flagged
+// and ranks last.  4 B gathered per member (the scores are L2-resident after
+// the proposal).
+__global__ void __launch_bounds__(kThreads) pool_gather_kernel(const float* __restrict__ scores,
+                                                               const int32_t* __restrict__ cu,
+                                                               const int32_t* __restrict__ pool,
+                                                               const int32_t* __restrict__ pool_cnt,
+                                                               int pool_stride, int Hkv, int64_t T,
+                                                               float* __restrict__ r,
+                                                               int32_t* status) {
+  const int row = blockIdx.y;
+  const int b = row / Hkv, h = row - b * Hkv;
+  int n = pool_cnt[row];
+  n = n < 0 ? 0 : (n > pool_stride ? pool_stride : n);
+  const int t0 = cu[b], L = cu[b + 1] - t0;
+  const float* sb = scores + (int64_t)h * T + t0;
+  const int32_t* pr = pool + (int64_t)row * pool_stride;
+  float* rr = r + (int64_t)row * pool_stride;
+  for (int i = blockIdx.x * kThreads + threadIdx.x; i < n; i += gridDim.x * kThreads) {
+    const int p = pr[i];
+    const bool ok = p >= 0 && p < L;
+    if (!ok) flag_status(status, PRISM_DEV_BAD_INDEX);
+    rr[i] = ok ? sb[p] : -INFINITY;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_pool_gather(const Dims& d, const float* scores, const int32_t* pool,
+                               const int32_t* pool_cnt, int pool_stride, float* r, int32_t* status,
+                               cudaStream_t st) {
+  const int rows = d.B * d.Hkv;
+  if (rows == 0 || pool_stride == 0) return cudaSuccess;
+  const int bx = (int)cdiv(pool_stride, kThreads) < 8 ? (int)cdiv(pool_stride, kThreads) : 8;
+  pool_gather_kernel<<<dim3(bx, rows), kThreads, 0, st>>>(scores, d.cu_dev, pool, pool_cnt, pool_stride,
+                                                          d.Hkv, d.T, r, status);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_refine_scores(const Dims& d, const void* q, const void* k, const int32_t* pool,
                                  const int32_t* pool_cnt, int pool_stride, float* r, float* dots,
-                                 int32_t* status, cudaStream_t st) {
+                                 int32_t* status, cudaStream_t st, int pool_div) {
   if (d.B * d.Hkv == 0 || pool_stride == 0) return cudaSuccess;
-  RefineArgs a{q, k, d.cu_dev, pool, pool_cnt, pool_stride, d.Hkv, d.G, d.T, 0, r, dots, status};
+  RefineArgs a{q, k, d.cu_dev, pool, pool_cnt, pool_stride, d.Hkv, d.G, d.T, 0, r, dots, status,
+               pool_div > 1 ? pool_div : 1};
   if (d.bf16)
     return d.D == 128 ? by_group<__nv_bfloat16, 128>(d, a, st) : by_group<__nv_bfloat16, 64>(d, a, st);
   return d.D == 128 ? by_group<float, 128>(d, a, st) : by_group<float, 64>(d, a, st);

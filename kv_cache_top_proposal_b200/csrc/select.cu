@@ -35,8 +35,14 @@ constexpr int kCluster = 8;
 constexpr int kThreads = 1024;
 constexpr int kMaxChunk = 49152;  // keys per CTA (192 KB of shared memory)
 
+// mode 1: selection row `row` draws from pool row row / pool_div (several
+// selection rows -- the query heads of a group -- may share one pool)
+__device__ __forceinline__ int pool_row(const SelectArgs& a, int row) {
+  return a.pool_div > 1 ? row / a.pool_div : row;
+}
+
 __device__ __forceinline__ int32_t position_of(const SelectArgs& a, int row, int i) {
-  return a.mode == 0 ? i : a.pool[(int64_t)row * a.pool_stride + i];
+  return a.mode == 0 ? i : a.pool[(int64_t)pool_row(a, row) * a.pool_stride + i];
 }
 
 __device__ __forceinline__ void emit(const SelectArgs& a, int row, int b, int h, int i, int slot,
@@ -71,7 +77,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelectArgs a)
     n = a.cu[b + 1] - t0;
     kbase = a.keys + (int64_t)h * a.T + t0;
   } else {
-    n = a.pool_cnt[row];
+    n = a.pool_cnt[pool_row(a, row)];
     if (n < 0 || n > a.pool_stride) {
       if (rank == 0 && tid == 0) flag_status(a.status, PRISM_DEV_BAD_INDEX);
       n = n < 0 ? 0 : a.pool_stride;

@@ -35,7 +35,8 @@ class PrismDecoder:
     def __init__(self, seqlens, num_q_heads: int, num_kv_heads: int, head_dim: int, dtype: int,
                  num_layers: int, group: int, kappa_p: int, kappa: int, device="cuda",
                  softmax_scale: Optional[float] = None, fused: bool = True, keys: str = "int8",
-                 capacity: Optional[int] = None, group_agg: str = "max"):
+                 capacity: Optional[int] = None, group_agg: str = "max",
+                 proposal_select: str = "exact", sets: str = "kv_head"):
         self.dev = torch.device(device)
         self.p = prism.Problem(seqlens, num_q_heads, num_kv_heads, head_dim, dtype, device=self.dev,
                                capacity=capacity)
@@ -48,10 +49,22 @@ class PrismDecoder:
         i32 = dict(dtype=torch.int32, device=self.dev)
         f32 = dict(dtype=torch.float32, device=self.dev)
         self.proposal_layers = [l for l in range(num_layers) if l % group == 0]
-        self.pool = {l: torch.full((B, Hkv, kappa_p), -1, **i32) for l in self.proposal_layers}
-        self.pool_cnt = {l: torch.zeros((B, Hkv), **i32) for l in self.proposal_layers}
-        self.idx = [torch.full((B, Hkv, kappa), -1, **i32) for _ in range(num_layers)]
-        self.cnt = [torch.zeros((B, Hkv), **i32) for _ in range(num_layers)]
+        # selection granularity: one pool and set per (sequence, KV head)
+        # ("kv_head", the default reading); a set per query head over the
+        # group's pool ("q_head"); one pool and set per sequence shared by
+        # every head ("sequence").  The last two run the two-call path.
+        assert sets in ("kv_head", "q_head", "sequence")
+        self.sets = sets
+        self.sets_code = {"kv_head": prism.SETS_KV_HEAD, "q_head": prism.SETS_Q_HEAD,
+                          "sequence": prism.SETS_SEQUENCE}[sets]
+        if sets != "kv_head":
+            fused = False
+        ph = 1 if sets == "sequence" else Hkv       # pool rows per sequence
+        sh = {"kv_head": Hkv, "q_head": Hq, "sequence": 1}[sets]  # set rows per sequence
+        self.pool = {l: torch.full((B, ph, kappa_p), -1, **i32) for l in self.proposal_layers}
+        self.pool_cnt = {l: torch.zeros((B, ph), **i32) for l in self.proposal_layers}
+        self.idx = [torch.full((B, sh, kappa), -1, **i32) for _ in range(num_layers)]
+        self.cnt = [torch.zeros((B, sh), **i32) for _ in range(num_layers)]
         # per-layer outputs are views of one buffer (one device-to-host copy)
         self.out_all = torch.zeros((num_layers, B, Hq, D), **f32)
         self.lse_all = torch.zeros((num_layers, B, Hq), **f32)
@@ -89,9 +102,16 @@ class PrismDecoder:
         # score: "max" (the default reading) or "sum" (the variant, carried
         # by the scorer that takes the new rows and by the fused refined layer)
         assert group_agg in ("max", "sum")
+        if sets != "kv_head" and (keys != "int8" or group_agg != "max"):
+            raise ValueError("the q_head / sequence granularities take int8 keys and the maximum")
         if group_agg == "sum" and not self.scorer_appends:
             raise ValueError("group_agg='sum' needs the fused step with int8 keys (bf16, d = 128, G <= 8)")
         self.sum_group = group_agg == "sum"
+        # what a proposal layer attends over: "exact" (it refines its own pool
+        # like every layer, the default reading) or "quantized" (the top kappa
+        # of its pool by the proposal scores it just computed, no rescoring)
+        assert proposal_select in ("exact", "quantized")
+        self.proposal_select = proposal_select
 
     def workspaces(self) -> List[torch.Tensor]:
         return [w for w in (self.ws_q, self.ws_prop, self.ws_ref, self.ws_dec, self.ws_rd,
@@ -130,9 +150,17 @@ class PrismDecoder:
                 if quantize_new and self.new_rows.numel():
                     prism.quantize_k(p, k, kq, k_scale, tok_rows=self.new_rows, ws=self.ws_q,
                                      stream=stream)
-                prism.propose(p, q, kq, k_scale, self.kappa_p, self.pool[l], self.pool_cnt[l],
-                              self.ws_prop, stream=stream)
+                prism.propose_ex(p, q, kq, k_scale, self.kappa_p, self.pool[l], self.pool_cnt[l],
+                                 self.sets_code, self.ws_prop, stream=stream)
         src = l - l % self.group
+        if proposal and self.proposal_select == "quantized":
+            prism.propose_topk(p, self.ws_prop, self.pool[l], self.pool_cnt[l], self.kappa_p, self.kappa,
+                               self.idx[l], self.cnt[l], self.ws_ref, stream=stream)
+            if fused_append:  # no refined-layer call appends this layer's rows
+                prism.append_kv(p, k_new, v_new, k, v, stream=stream)
+            prism.sparse_decode(p, q, k, v, self.idx[l], self.cnt[l], self.kappa, self.scale,
+                                self.out[l], self.ws_dec, lse=self.lse[l], stream=stream)
+            return
         if self.fused:
             prism.refine_decode(p, q, k, v, self.pool[src], self.pool_cnt[src], self.kappa_p,
                                 self.kappa, self.scale, self.idx[l], self.cnt[l], self.out[l],
@@ -141,10 +169,10 @@ class PrismDecoder:
                                 v_new=v_new if fused_append else None, k_prefetch=k_next,
                                 overlap=overlap, sum_group=self.sum_group, stream=stream)
             return
-        prism.refine(p, q, k, self.pool[src], self.pool_cnt[src], self.kappa_p, self.kappa,
-                     self.idx[l], self.cnt[l], self.ws_ref, stream=stream)
-        prism.sparse_decode(p, q, k, v, self.idx[l], self.cnt[l], self.kappa, self.scale,
-                            self.out[l], self.ws_dec, lse=self.lse[l], stream=stream)
+        prism.refine_ex(p, q, k, self.pool[src], self.pool_cnt[src], self.kappa_p, self.kappa,
+                        self.idx[l], self.cnt[l], self.sets_code, self.ws_ref, stream=stream)
+        prism.sparse_decode_ex(p, q, k, v, self.idx[l], self.cnt[l], self.kappa, self.scale,
+                               self.sets_code, self.out[l], self.ws_dec, lse=self.lse[l], stream=stream)
 
     def step(self, qs, ks, vs, kqs, scales, quantize_new: bool = True, k_new=None, v_new=None,
              stream=None):
@@ -204,7 +232,12 @@ class PrismDecoder:
             n += 1 if append and ((proposal and not scorer_new) or not self.fused) else 0
             if proposal:
                 n += (1 if self.new_rows.numel() and not scorer_new else 0) + 2
+            if proposal and self.proposal_select == "quantized":
+                n += (1 if append and self.fused and scorer_new else 0) + 2 + 2
+                continue
             n += 1 if self.fused else 2 + 2
+            if self.sets == "sequence":  # the head maxima of the pool scores (and of the proposal's)
+                n += 2 if proposal else 1
         return n
 
     def dense_layer(self, l: int, q, k, v, out, lse=None, stream=None):

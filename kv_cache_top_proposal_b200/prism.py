@@ -25,6 +25,7 @@ DEV_BAD_INDEX, DEV_TOO_LONG, DEV_TIMEOUT = 0x1, 0x2, 0x4
 MAX_SELECT_ROW = 393216
 RD_OVERLAP = 0x1
 RD_SUM_GROUP = 0x2
+SETS_KV_HEAD, SETS_Q_HEAD, SETS_SEQUENCE = 0, 1, 2
 PROPOSE_SUM_GROUP = 0x1
 WS_HEADER = 256
 
@@ -33,7 +34,8 @@ EXPORTS = ("prism_workspace_size", "prism_append_kv", "prism_quantize_k", "prism
            "prism_sparse_decode", "prism_refine_decode", "prism_dense_decode",
            "prism_clear_device_status",
            "prism_get_device_status", "prism_status_str", "prism_sparse_decode_noalloc",
-           "prism_quantize_k_int2", "prism_propose_int2")
+           "prism_quantize_k_int2", "prism_propose_int2", "prism_index_overlap",
+           "prism_propose_topk", "prism_propose_ex", "prism_refine_ex", "prism_sparse_decode_ex")
 
 
 class PrismError(RuntimeError):
@@ -72,6 +74,12 @@ def _load():
         "prism_sparse_decode_noalloc": [sp, P, P, P, P, P, i32, ctypes.c_float, P, P, P, P],
         "prism_quantize_k_int2": [sp, P, P, P, P, i32, P, S, P],
         "prism_propose_int2": [sp, P, P, P, i32, P, P, P, S, P],
+        "prism_index_overlap": [i32, P, P, i32, P, P, i32, P, P],
+        "prism_propose_topk": [sp, P, S, P, P, i32, i32, P, P, P, S, P],
+        "prism_propose_ex": [sp, P, P, P, i32, P, P, ctypes.c_uint32, P, S, P],
+        "prism_refine_ex": [sp, P, P, P, P, i32, i32, P, P, ctypes.c_uint32, P, S, P],
+        "prism_sparse_decode_ex": [sp, P, P, P, P, P, i32, ctypes.c_float, ctypes.c_uint32, P, P, P, S,
+                                   P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -215,6 +223,15 @@ def refine(p: Problem, q, k, pool, pool_cnt, kappa_p: int, kappa: int, idx, cnt,
                              _stream(stream)), "refine")
 
 
+def propose_topk(p: Problem, propose_ws, pool, pool_cnt, kappa_p: int, kappa: int, idx, cnt, ws,
+                 stream=None):
+    """The proposal layer's own top-kappa from the scores its proposal call
+    left in propose_ws (no exact rescoring); ws sized by OP_REFINE."""
+    _check(_lib.prism_propose_topk(p.ref, _ptr(propose_ws), _nbytes(propose_ws), _ptr(pool),
+                                   _ptr(pool_cnt), kappa_p, kappa, _ptr(idx), _ptr(cnt), _ptr(ws),
+                                   _nbytes(ws), _stream(stream)), "propose_topk")
+
+
 def sparse_decode(p: Problem, q, k, v, idx, cnt, kappa: int, softmax_scale: float, out, ws,
                   lse=None, stream=None):
     _check(_lib.prism_sparse_decode(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt), kappa,
@@ -268,3 +285,37 @@ def get_device_status(ws, stream=None) -> int:
     _check(_lib.prism_get_device_status(_ptr(ws), _nbytes(ws), _stream(stream), ctypes.byref(c)),
            "get_device_status")
     return c.value
+
+
+def index_overlap(a, cnt_a, b, cnt_b, out, stream=None):
+    """out[r] = |a[r, :cnt_a[r]] intersect b[r, :cnt_b[r]]| for ascending
+    index sets a [rows][stride_a], b [rows][stride_b] (int32, device)."""
+    rows = int(cnt_a.numel())
+    assert int(cnt_b.numel()) == rows and int(out.numel()) == rows
+    _check(_lib.prism_index_overlap(rows, _ptr(a), _ptr(cnt_a), int(a.shape[-1]), _ptr(b),
+                                    _ptr(cnt_b), int(b.shape[-1]), _ptr(out), _stream(stream)),
+           "index_overlap")
+
+
+def propose_ex(p: Problem, q, kq, k_scale, kappa_p: int, pool, pool_cnt, sets: int, ws, stream=None):
+    """prism_propose at a selection granularity (SETS_*); SETS_SEQUENCE
+    writes one pool per sequence, pool [B][kappa_p], pool_cnt [B]."""
+    _check(_lib.prism_propose_ex(p.ref, _ptr(q), _ptr(kq), _ptr(k_scale), kappa_p, _ptr(pool),
+                                 _ptr(pool_cnt), sets, _ptr(ws), _nbytes(ws), _stream(stream)),
+           "propose_ex")
+
+
+def refine_ex(p: Problem, q, k, pool, pool_cnt, kappa_p: int, kappa: int, idx, cnt, sets: int, ws,
+              stream=None):
+    """prism_refine at a selection granularity: SETS_Q_HEAD writes idx
+    [B][Hq][kappa], SETS_SEQUENCE idx [B][kappa] from pool [B][kappa_p]."""
+    _check(_lib.prism_refine_ex(p.ref, _ptr(q), _ptr(k), _ptr(pool), _ptr(pool_cnt), kappa_p, kappa,
+                                _ptr(idx), _ptr(cnt), sets, _ptr(ws), _nbytes(ws), _stream(stream)),
+           "refine_ex")
+
+
+def sparse_decode_ex(p: Problem, q, k, v, idx, cnt, kappa: int, softmax_scale: float, sets: int, out,
+                     ws, lse=None, stream=None):
+    _check(_lib.prism_sparse_decode_ex(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt), kappa,
+                                       float(softmax_scale), sets, _ptr(out), _ptr(lse), _ptr(ws),
+                                       _nbytes(ws), _stream(stream)), "sparse_decode_ex")

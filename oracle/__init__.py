@@ -70,6 +70,16 @@ def _L():
         lib.oracle_propose_scores_int2.argtypes = [P, i32, i32, P, P, i32, P]
         lib.oracle_propose_row_int2.argtypes = [P, i32, i32, P, P, i32, i32, P, P]
         lib.oracle_propose_row_int2.restype = i32
+        lib.oracle_set_overlap.argtypes = [P, i32, P, i32]
+        lib.oracle_set_overlap.restype = i32
+        lib.oracle_pool_topk.argtypes = [P, P, i32, i32, P]
+        lib.oracle_pool_topk.restype = i32
+        lib.oracle_refine_row_heads.argtypes = [P, i32, i32, P, P, i32, i32, P, P]
+        lib.oracle_refine_row_heads.restype = i32
+        lib.oracle_propose_row_seq.argtypes = [P, i32, i32, i32, P, P, i32, i32, P, P]
+        lib.oracle_propose_row_seq.restype = i32
+        lib.oracle_refine_row_seq.argtypes = [P, i32, i32, i32, P, i32, P, i32, i32, P, P]
+        lib.oracle_refine_row_seq.restype = i32
         _lib = lib
     return _lib
 
@@ -133,6 +143,16 @@ def propose_row(q, kq, scale, kappa_p: int, agg: str = "max"):
     m = getattr(_L(), "oracle_propose_row" + _sfx(agg))(_p(q), G, d, _p(kq), _p(scale), L, kappa_p,
                                                         _p(pool), _p(s))
     return pool[:m].copy(), s[:L].copy()
+
+
+def pool_topk(scores, pool, kappa: int) -> np.ndarray:
+    """The proposal layer's own set under the quantized-selection reading:
+    the top min(kappa, |pool|) pool members by their proposal scores
+    (scores [L], one per position), positions ascending."""
+    s, pool = _f32(scores), _i32(pool)
+    idx = np.empty((max(min(kappa, pool.size), 1),), np.int32)
+    m = _L().oracle_pool_topk(_p(s), _p(pool), pool.size, kappa, _p(idx))
+    return idx[:m].copy()
 
 
 def refine_scores(q, K, pool, agg: str = "max") -> np.ndarray:
@@ -223,3 +243,52 @@ def propose_row_int2(q, codes, params, kappa_p: int):
     pool = np.empty((max(min(kappa_p, L), 1),), np.int32)
     m = _L().oracle_propose_row_int2(_p(q), G, d, _p(codes), _p(params), L, kappa_p, _p(pool), _p(s))
     return pool[:m].copy(), s[:L].copy()
+
+
+# ---- index overlap (sec. 3 "Observations", Figure 1) -------------------------
+
+def set_overlap(a, b) -> int:
+    """|a intersect b| of two strictly ascending index sets."""
+    a, b = _i32(a), _i32(b)
+    return int(_L().oracle_set_overlap(_p(a), a.size, _p(b), b.size))
+
+
+# ---- selection granularity variants ------------------------------------------
+
+def refine_row_heads(q, K, pool, kappa: int):
+    """Per-query-head sets over a shared pool: (idx [G][min(kappa, n)]
+    positions ascending per head, exact scores [G][n])."""
+    q, K, pool = _f32(q), _f32(K), _i32(pool)
+    G, d = q.shape
+    n = pool.size
+    idx = np.empty((G, max(kappa, 1)), np.int32)
+    r = np.empty((G, max(n, 1)), np.float32)
+    m = _L().oracle_refine_row_heads(_p(q), G, d, _p(K), _p(pool), n, kappa, _p(idx), _p(r))
+    return idx[:, :m].copy(), r[:, :n].copy()
+
+
+def propose_row_seq(q, kq, scale, kappa_p: int):
+    """One pool per sequence shared by every head: q [Hq][d], kq [Hkv][L][d],
+    scale [Hkv][L] -> (pool ascending, head-max proposal scores [L])."""
+    q = _f32(q)
+    kq = np.ascontiguousarray(kq, dtype=np.int8)
+    scale = _f32(scale)
+    Hkv, L, d = kq.shape
+    G = q.shape[0] // Hkv
+    s = np.empty((max(L, 1),), np.float32)
+    pool = np.empty((max(min(kappa_p, L), 1),), np.int32)
+    m = _L().oracle_propose_row_seq(_p(q), Hkv, G, d, _p(kq), _p(scale), L, kappa_p, _p(pool), _p(s))
+    return pool[:m].copy(), s[:L].copy()
+
+
+def refine_row_seq(q, K, pool, kappa: int):
+    """One set per sequence: q [Hq][d], K [Hkv][L][d] -> (positions ascending,
+    head-max exact scores of the pool)."""
+    q, K, pool = _f32(q), _f32(K), _i32(pool)
+    Hkv, L, d = K.shape
+    G = q.shape[0] // Hkv
+    n = pool.size
+    r = np.empty((max(n, 1),), np.float32)
+    idx = np.empty((max(min(kappa, n), 1),), np.int32)
+    m = _L().oracle_refine_row_seq(_p(q), Hkv, G, d, _p(K), L, _p(pool), n, kappa, _p(idx), _p(r))
+    return idx[:m].copy(), r[:n].copy()

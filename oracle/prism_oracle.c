@@ -427,3 +427,131 @@ int32_t oracle_propose_row_int2(const float* q, int32_t G, int32_t d, const uint
   if (!scores_out) free(s);
   return n;
 }
+
+/*
+ * Index overlap of two selections (sec. 3 "Observations", Figure 1: the
+ * overlap ratio between the index sets of a reference layer and of a layer
+ * at a given offset; Figure 12: the share of a layer's top-kappa that an
+ * expanded top-rho*kappa set of another layer covers).  a[0..na) and
+ * b[0..nb) are index sets in strictly ascending order; the result is
+ * |a intersect b|, found by walking both lists once.  The ratios divide it
+ * by the set sizes the figure names.
+ */
+int32_t oracle_set_overlap(const int32_t* a, int32_t na, const int32_t* b, int32_t nb) {
+  int32_t i = 0, j = 0, c = 0;
+  while (i < na && j < nb) {
+    if (a[i] == b[j]) {
+      ++c;
+      ++i;
+      ++j;
+    } else if (a[i] < b[j]) {
+      ++i;
+    } else {
+      ++j;
+    }
+  }
+  return c;
+}
+
+/*
+ * The other reading of what a proposal layer attends over (sec. 4.1 states
+ * that refined layers re-select inside the pool, and leaves the proposal
+ * layer's own set open): the proposal layer takes the top min(kappa, n)
+ * members of its pool by their proposal scores -- the quantized-key scores
+ * it has already computed -- with no exact rescoring.  s holds the proposal
+ * score of every position of the sequence; ties go to the lower position
+ * (the pool is ascending, so the lower slot).  Positions are written in
+ * ascending order; returns the count.
+ */
+int32_t oracle_pool_topk(const float* s, const int32_t* pool, int32_t n, int32_t kappa,
+                         int32_t* idx) {
+  float* r = (float*)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
+  int32_t* slot = (int32_t*)malloc(sizeof(int32_t) * (size_t)(n > 0 ? n : 1));
+  for (int32_t i = 0; i < n; ++i) r[i] = s[pool[i]];
+  int32_t m = oracle_topk_ascending(r, n, kappa, slot);
+  for (int32_t i = 0; i < m; ++i) idx[i] = pool[slot[i]];
+  free(slot);
+  free(r);
+  return m;
+}
+
+/*
+ * Selection granularity variants (sec. 4.1 shares index sets under GQA
+ * without saying at which granularity; sec. 2 "Related Work" names a set
+ * shared by all heads, DSA; the pages analyse attention per head, sec. 3).
+ *
+ * Per query head: the proposal region stays one pool per (sequence, KV
+ * head), shared by the group; each query head g then keeps its own top
+ * min(kappa, n) pool members by its own exact score
+ *   r_g(i) = sum_j q[g][j] * K[pool_i][j]          fp32, j ascending
+ * (ties to the lower position) and attends over them.  idx is [G][kappa]
+ * (row g at idx + g * kappa, positions ascending), r_out [G][n] may be NULL.
+ * Returns the per-head count min(kappa, n).
+ */
+int32_t oracle_refine_row_heads(const float* q, int32_t G, int32_t d, const float* K,
+                                const int32_t* pool, int32_t n, int32_t kappa, int32_t* idx,
+                                float* r_out) {
+  int32_t m = 0;
+  float* r = (float*)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
+  int32_t* slot = (int32_t*)malloc(sizeof(int32_t) * (size_t)(n > 0 ? n : 1));
+  for (int32_t g = 0; g < G; ++g) {
+    for (int32_t i = 0; i < n; ++i) {
+      const float* kr = K + (int64_t)pool[i] * d;
+      float acc = 0.0f;
+      for (int32_t j = 0; j < d; ++j) acc = acc + q[g * d + j] * kr[j];
+      r[i] = acc;
+      if (r_out) r_out[(int64_t)g * n + i] = acc;
+    }
+    m = oracle_topk_ascending(r, n, kappa, slot);
+    for (int32_t i = 0; i < m; ++i) idx[(int64_t)g * kappa + i] = pool[slot[i]];
+  }
+  free(slot);
+  free(r);
+  return m;
+}
+
+/*
+ * One set per sequence, shared by every head: the selection score of a
+ * position is the maximum over all Hkv KV heads of that head's score (the
+ * maximum over its G query heads, as in the per-KV-head reading):
+ *   proposal  s_t = max_h scale[h][t] * max_g sum_j q[h G + g][j] * kq[h][t][j]
+ *   refine    r_i = max_h max_g sum_j q[h G + g][j] * K[h][pool_i][j]
+ * q is [Hkv G][d]; kq / K are [Hkv][L][d] (head h at + h * L * d), scale
+ * [Hkv][L].  The selections and their order rules are those of the
+ * per-KV-head forms.  Returns the pool / set size.
+ */
+int32_t oracle_propose_row_seq(const float* q, int32_t Hkv, int32_t G, int32_t d,
+                               const int8_t* kq, const float* scale, int32_t L, int32_t kappa_p,
+                               int32_t* pool, float* s_out) {
+  float* s = s_out ? s_out : (float*)malloc(sizeof(float) * (size_t)(L > 0 ? L : 1));
+  float* sh = (float*)malloc(sizeof(float) * (size_t)(L > 0 ? L : 1));
+  for (int32_t h = 0; h < Hkv; ++h) {
+    oracle_propose_scores(q + (int64_t)h * G * d, G, d, kq + (int64_t)h * L * d,
+                          scale + (int64_t)h * L, L, sh);
+    for (int32_t t = 0; t < L; ++t)
+      if (h == 0 || sh[t] > s[t]) s[t] = sh[t];
+  }
+  free(sh);
+  int32_t m = oracle_topk_ascending(s, L, kappa_p, pool);
+  if (!s_out) free(s);
+  return m;
+}
+
+int32_t oracle_refine_row_seq(const float* q, int32_t Hkv, int32_t G, int32_t d, const float* K,
+                              int32_t L, const int32_t* pool, int32_t n, int32_t kappa,
+                              int32_t* idx, float* r_out) {
+  float* r = r_out ? r_out : (float*)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
+  float* rh = (float*)malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
+  for (int32_t h = 0; h < Hkv; ++h) {
+    oracle_refine_scores(q + (int64_t)h * G * d, G, d, K + (int64_t)h * L * d, pool, n, rh);
+    for (int32_t i = 0; i < n; ++i)
+      if (h == 0 || rh[i] > r[i]) r[i] = rh[i];
+  }
+  free(rh);
+  int32_t* slot = (int32_t*)malloc(sizeof(int32_t) * (size_t)(n > 0 ? n : 1));
+  int32_t m = oracle_topk_ascending(r, n, kappa, slot);
+  for (int32_t i = 0; i < m; ++i) idx[i] = pool[slot[i]];
+  free(slot);
+  if (!r_out) free(r);
+  return m;
+}

@@ -144,3 +144,28 @@ def test_status_strings(prism_lib):
     for code in range(6):
         assert lib.prism_status_str(code)
     assert b"workspace" in lib.prism_status_str(prism_lib.ERR_WORKSPACE)
+
+
+def test_propose_topk_and_overlap_reject_bad_arguments(prism_lib):
+    """Host checks of prism_propose_topk (the proposal workspace and the
+    refine workspace are both sized and aligned) and prism_index_overlap."""
+    P = prism_lib
+    lib = P.library()
+    s, cu = _shape(P, [1000, 3000])
+    _, nprop = _ws(P, s, P.OP_PROPOSE, 256)
+    _, nref = _ws(P, s, P.OP_REFINE, 256, 64)
+    f = ctypes.c_void_p(FAKE)
+
+    def call(pws, pn, ws, n, kp=256, k=64):
+        return lib.prism_propose_topk(ctypes.byref(s), pws, pn, f, f, kp, k, f, f, ws, n, None)
+
+    assert call(f, nprop - 1, f, nref) == P.ERR_WORKSPACE           # proposal workspace too small
+    assert call(f, nprop, f, nref - 1) == P.ERR_WORKSPACE           # refine workspace too small
+    assert call(ctypes.c_void_p(FAKE + 16), nprop, f, nref) == P.ERR_WORKSPACE  # misaligned
+    assert call(f, nprop, f, nref, kp=64, k=256) == P.ERR_INVALID_ARG  # kappa > kappa_p
+    assert call(None, nprop, f, nref) == P.ERR_WORKSPACE
+    ov = lib.prism_index_overlap
+    assert ov(4, f, f, 0, f, f, 8, f, None) == P.ERR_INVALID_ARG     # stride 0
+    assert ov(-1, f, f, 8, f, f, 8, f, None) == P.ERR_INVALID_ARG
+    assert ov(4, None, f, 8, f, f, 8, f, None) == P.ERR_INVALID_ARG
+    assert ov(0, None, None, 8, None, None, 8, None, None) == P.OK  # nothing to do

@@ -709,6 +709,71 @@ def test_refine_decode_large_ties(P, kp, kap):
     assert np.abs(_np(out) - oout).max() <= 2e-3
 
 
+GATHER_CASES = [
+    # (seqlens, Hq, Hkv, d, kappa_p, kappa, integer keys): the c128k row
+    # shape, a ragged batch with an empty and a short sequence, the largest
+    # gathered pool and the first one past it (cluster rounds on both
+    # paths), and integer keys (many exactly equal scores at the threshold)
+    ([131072], 32, 8, 128, 8192, 2048, False),
+    ([40000, 9000, 0, 300, 12300], 32, 8, 128, 4096, 1024, False),
+    ([30000], 8, 2, 128, 8192, 3000, False),
+    ([30000], 8, 2, 128, 8193, 3000, False),
+    ([20000, 7000], 32, 8, 128, 8192, 2048, True),
+    ([2000], 4, 1, 64, 256, 64, True),
+]
+
+
+@pytest.mark.parametrize("case", GATHER_CASES, ids=lambda c: f"{len(c[0])}seq-kp{c[4]}-k{c[5]}-int{int(c[6])}")
+def test_refine_decode_gathered_selection(P, case, monkeypatch):
+    """The gathered selection (every CTA reads the row's keys and resolves
+    the threshold itself) against the cluster-wide digit rounds: the same
+    index sets and bit-identical outputs; and against the oracle."""
+    seqlens, hq, hkv, d, kp, kap, integer = case
+    B = len(seqlens)
+    prob = problem(P, seqlens, hq, hkv, d, "bf16")
+    q, k, v = make_case(seqlens, hq, hkv, d, "bf16", seed=31)
+    if integer:  # small integer keys and queries: exact, often equal, scores
+        g = torch.Generator(device="cpu").manual_seed(32)
+        k.copy_(torch.randint(-2, 3, k.shape, generator=g).to(k.dtype).to(DEV))
+        q.copy_(torch.randint(-1, 2, q.shape, generator=g).to(q.dtype).to(DEV))
+    rng = np.random.default_rng(33)
+    pool = np.full((B, hkv, kp), -1, np.int32)
+    pcnt = np.zeros((B, hkv), np.int32)
+    for b, L in enumerate(seqlens):
+        for h in range(hkv):
+            n = min(kp, L)
+            pool[b, h, :n] = np.sort(rng.choice(L, n, replace=False))
+            pcnt[b, h] = n
+    pool_t, pcnt_t = torch.tensor(pool, device=DEV), torch.tensor(pcnt, device=DEV)
+    scale = float(np.float32(1 / math.sqrt(d)))
+    ws = ws_for(P, prob, P.OP_REFINE_DECODE, kp, kap)
+    res = []
+    for mode in ("cluster", "gather"):
+        monkeypatch.setenv("PRISM_RD_SELECT", mode)
+        idx = torch.full((B, hkv, kap), -7, dtype=torch.int32, device=DEV)
+        cnt = torch.zeros((B, hkv), dtype=torch.int32, device=DEV)
+        out = torch.full((B, hq, d), 77.0, device=DEV)
+        lse = torch.full((B, hq), 77.0, device=DEV)
+        P.refine_decode(prob, q, k, v, pool_t, pcnt_t, kp, kap, scale, idx, cnt, out, ws, lse=lse)
+        torch.cuda.synchronize()
+        res.append((idx, cnt, out, lse))
+    assert P.get_device_status(ws) == 0
+    (i0, c0, o0, l0), (i1, c1, o1, l1) = res
+    assert torch.equal(i0, i1) and torch.equal(c0, c1)
+    assert torch.equal(o0, o1) and torch.equal(l0, l1)
+    oidx, ocnt, oscores = pipeline.refine_layer(q, k, prob.cu_host.tolist(), pool, pcnt, kap)
+    gi, gc = _np(i1), _np(c1)
+    assert np.array_equal(gc, ocnt)
+    for b in range(B):
+        for h in range(hkv):
+            n, c = int(pcnt[b, h]), int(ocnt[b, h])
+            r = dict(zip(pool[b, h, :n].tolist(), oscores[(b, h)].tolist()))
+            check_index_set(gi[b, h, :c], oidx[b, h, :c], lambda t: r[t], f"idx b{b} h{h}")
+            assert np.all(gi[b, h, c:] == -1)
+    oout, _ = pipeline.attend_layer(q, k, v, prob.cu_host.tolist(), gi, gc, scale)
+    assert np.abs(_np(o1) - oout).max() <= atol_for("bf16")
+
+
 # ------------------------------------------------------------------ INT2 keys
 
 @pytest.mark.parametrize("dtype,d", [("bf16", 128), ("bf16", 64), ("f32", 128)])
@@ -805,3 +870,82 @@ def test_propose_int2_unsupported_shapes(P):
     with pytest.raises(P.PrismError) as e:
         P.propose_int2(prob, q, codes, params, 100, pool, cnt, ws_for(P, prob, P.OP_PROPOSE, 100))
     assert e.value.status == P.ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------------------ selection granularity
+
+SETS_CASES = [
+    # (seqlens, Hq, Hkv, d, kappa_p, kappa): ragged with an empty and a short
+    # sequence (pools and sets shorter than their budgets), one KV head, G = 1
+    ([5000, 0, 700, 2500], 32, 8, 128, 1024, 256),
+    ([3000], 4, 1, 64, 512, 100),
+    ([1500, 4000], 8, 8, 128, 600, 600),
+]
+
+
+@pytest.mark.parametrize("case", SETS_CASES, ids=lambda c: f"{len(c[0])}seq-{c[1]}/{c[2]}-kp{c[4]}")
+@pytest.mark.parametrize("sets", ["q_head", "sequence"])
+def test_selection_granularity_calls_vs_oracle(P, case, sets):
+    seqlens, hq, hkv, d, kp, kap = case
+    B = len(seqlens)
+    prob = problem(P, seqlens, hq, hkv, d, "bf16")
+    q, k, v = make_case(seqlens, hq, hkv, d, "bf16", seed=41)
+    cu = prob.cu_host.tolist()
+    code = P.SETS_Q_HEAD if sets == "q_head" else P.SETS_SEQUENCE
+    kq = torch.zeros(k.shape, dtype=torch.int8, device=DEV)
+    sc = torch.zeros(k.shape[:2], dtype=torch.float32, device=DEV)
+    P.quantize_k(prob, k, kq, sc)
+    prow = 1 if sets == "sequence" else hkv
+    srow = hq if sets == "q_head" else 1
+    pool = torch.full((B, prow, kp), -7, dtype=torch.int32, device=DEV)
+    pcnt = torch.zeros((B, prow), dtype=torch.int32, device=DEV)
+    wp = ws_for(P, prob, P.OP_PROPOSE, kp)
+    P.propose_ex(prob, q, kq, sc, kp, pool, pcnt, code, wp)
+    idx = torch.full((B, srow, kap), -7, dtype=torch.int32, device=DEV)
+    cnt = torch.zeros((B, srow), dtype=torch.int32, device=DEV)
+    wr = ws_for(P, prob, P.OP_REFINE, kp, kap)
+    P.refine_ex(prob, q, k, pool, pcnt, kp, kap, idx, cnt, code, wr)
+    out = torch.full((B, hq, d), 77.0, device=DEV)
+    lse = torch.full((B, hq), 77.0, device=DEV)
+    wd = ws_for(P, prob, P.OP_SPARSE_DECODE, 0, kap)
+    scale = float(np.float32(1 / math.sqrt(d)))
+    P.sparse_decode_ex(prob, q, k, v, idx, cnt, kap, scale, code, out, wd, lse=lse)
+    torch.cuda.synchronize()
+    for w in (wp, wr, wd):
+        assert P.get_device_status(w) == 0
+    okq, osc = pipeline.quantize_layer(k)
+    gp, gpc, gi, gc = _np(pool), _np(pcnt), _np(idx), _np(cnt)
+    if sets == "sequence":
+        opool, ocnt, oscore = pipeline.propose_layer_seq(q, okq, osc, cu, kp)
+        for b in range(B):
+            n = int(ocnt[b])
+            assert int(gpc[b, 0]) == n == min(kp, seqlens[b])
+            check_index_set(gp[b, 0, :n], opool[b, :n], lambda t: oscore[b][t], f"pool {b}")
+            assert np.all(gp[b, 0, n:] == -1)
+        oidx, oc, orr = pipeline.refine_layer_seq(q, k, cu, gp[:, 0], gpc[:, 0], kap)
+        for b in range(B):
+            n, c = int(gpc[b, 0]), int(oc[b])
+            assert int(gc[b, 0]) == c
+            r = dict(zip(gp[b, 0, :n].tolist(), orr[b].tolist()))
+            check_index_set(gi[b, 0, :c], oidx[b, :c], lambda t: r[t], f"idx {b}")
+            assert np.all(gi[b, 0, c:] == -1)
+        oout, olse = pipeline.attend_layer_sets(q, k, v, cu, gi[:, 0], gc[:, 0], "sequence", scale)
+    else:
+        opool, ocnt, oscore = pipeline.propose_layer(q, okq, osc, cu, kp)
+        assert np.array_equal(gpc, ocnt)
+        oidx, oc, orr = pipeline.refine_layer_heads(q, k, cu, gp, gpc, kap)
+        G = hq // hkv
+        for b in range(B):
+            for h in range(hq):
+                n, c = int(gpc[b, h // G]), int(oc[b, h])
+                assert int(gc[b, h]) == c
+                r = dict(zip(gp[b, h // G, :n].tolist(), orr[(b, h)].tolist()))
+                check_index_set(gi[b, h, :c], oidx[b, h, :c], lambda t: r[t], f"idx {b},{h}")
+                assert np.all(gi[b, h, c:] == -1)
+        oout, olse = pipeline.attend_layer_sets(q, k, v, cu, gi, gc, "q_head", scale)
+    tol = atol_for("bf16")
+    assert np.abs(_np(out) - oout).max() <= tol
+    gl = _np(lse)
+    fin = np.isfinite(olse)
+    assert np.array_equal(np.isfinite(gl), fin)
+    assert np.abs(gl[fin] - olse[fin]).max() <= 10 * tol

@@ -364,3 +364,126 @@ def test_step_timed_sequence_full_size_every_row(prism_lib, name):
         _check_layer(dec, cfg, l, lay, okq[src][0], okq[src][1], every)
     del g, layers, dec
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["c8k", "ragged16"])
+def test_step_quantized_proposal_selection_every_row(prism_lib, name):
+    """The other reading of what a proposal layer attends over: its own set
+    is the top kappa of its pool by the proposal scores (prism_propose_topk,
+    no exact rescoring), and its attention runs over that set; the refined
+    layers are unchanged.  Every row of a proposal group against the oracle
+    in that mode (ragged16: the first group, four layers), with the token's
+    rows handed in as the benchmark does."""
+    P = prism_lib
+    full = workload.config(name)
+    cfg = full.replace(num_layers=full.group)
+    layers = list(workload.generate(cfg, DEV))
+    cu = cfg.cu_seqlens
+    nz = [b for b in range(cfg.batch) if cu[b + 1] > cu[b]]
+    rows = torch.tensor([cu[b + 1] - 1 for b in nz], dtype=torch.long, device=DEV)
+    k_new = [lay.k[:, rows].transpose(0, 1).contiguous() for lay in layers]
+    v_new = [lay.v[:, rows].transpose(0, 1).contiguous() for lay in layers]
+    dec = PrismDecoder(cfg.seqlens, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, P.BF16,
+                       cfg.num_layers, cfg.group, cfg.kappa_p, cfg.kappa, device=DEV,
+                       proposal_select="quantized")
+    kqs, scs = {}, {}
+    for lay in layers:
+        if cfg.is_proposal(lay.index):
+            kqs[lay.index], scs[lay.index] = _prefill_kq(P, dec, cfg, lay)
+    dec.step([x.q for x in layers], [x.k for x in layers], [x.v for x in layers], kqs, scs,
+             k_new=k_new, v_new=v_new)
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    every = _all_rows(cfg)
+    lay0 = layers[0]
+    okq, osc = pipeline.quantize_layer(lay0.k)
+    opool, ocnt, oscore = pipeline.propose_layer(lay0.q, okq, osc, cu, cfg.kappa_p)
+    gpool, gpc = _np(dec.pool[0]), _np(dec.pool_cnt[0])
+    for (b, h) in every:
+        n = int(ocnt[b, h])
+        assert int(gpc[b, h]) == n
+        check_index_set(gpool[b, h, :n], opool[b, h, :n], lambda t: oscore[(b, h)][t], f"pool {b},{h}")
+    # the proposal layer's own set on the GPU's pool, from the oracle's scores
+    oidx, ocnt2 = pipeline.pool_topk_layer(oscore, gpool, gpc, cfg.kappa)
+    gidx, gcnt = _np(dec.idx[0]), _np(dec.cnt[0])
+    for (b, h) in every:
+        c = int(ocnt2[b, h])
+        assert int(gcnt[b, h]) == c
+        check_index_set(gidx[b, h, :c], oidx[b, h, :c], lambda t: oscore[(b, h)][t], f"L0 idx {b},{h}")
+        assert set(gidx[b, h, :c].tolist()) <= set(gpool[b, h, :int(gpc[b, h])].tolist())
+    oout, olse = pipeline.attend_layer(lay0.q, lay0.k, lay0.v, cu, gidx, gcnt, dec.scale)
+    tol = atol_for(cfg.dtype)
+    assert np.abs(_np(dec.out[0]) - oout).max() <= tol
+    assert np.abs(_np(dec.lse[0]) - olse).max() <= 10 * tol
+    # the refined layers as in the default mode
+    for lay in layers[1:]:
+        _invariants(dec, cfg, lay.index)
+        _check_layer(dec, cfg, lay.index, lay, okq, osc, every)
+
+
+@pytest.mark.parametrize("sets", ["q_head", "sequence"])
+@pytest.mark.parametrize("name", ["c8k", "ragged16"])
+def test_step_selection_granularity_every_row(prism_lib, name, sets):
+    """The selection-granularity variants over a whole proposal group, every
+    row: one set per query head over the group's pool, or one pool and one
+    set per sequence shared by every head.  Pools against the oracle (its
+    proposal scores in that granularity), sets on the GPU's own pools, and
+    attention on the GPU's own sets (cascade control)."""
+    P = prism_lib
+    full = workload.config(name)
+    cfg = full.replace(num_layers=full.group)
+    layers = list(workload.generate(cfg, DEV))
+    cu = cfg.cu_seqlens
+    dec = PrismDecoder(cfg.seqlens, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, P.BF16,
+                       cfg.num_layers, cfg.group, cfg.kappa_p, cfg.kappa, device=DEV, sets=sets)
+    kqs, scs = {}, {}
+    for lay in layers:
+        if cfg.is_proposal(lay.index):
+            kqs[lay.index], scs[lay.index] = _prefill_kq(P, dec, cfg, lay)
+    dec.step([x.q for x in layers], [x.k for x in layers], [x.v for x in layers], kqs, scs)
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    lay0 = layers[0]
+    okq, osc = pipeline.quantize_layer(lay0.k)
+    gpool, gpc = _np(dec.pool[0]), _np(dec.pool_cnt[0])
+    tol = atol_for(cfg.dtype)
+    if sets == "sequence":
+        opool, ocnt, oscore = pipeline.propose_layer_seq(lay0.q, okq, osc, cu, cfg.kappa_p)
+        for b in range(cfg.batch):
+            n = int(ocnt[b])
+            assert int(gpc[b, 0]) == n
+            check_index_set(gpool[b, 0, :n], opool[b, :n], lambda t: oscore[b][t], f"seq pool {b}")
+    else:
+        opool, ocnt, oscore = pipeline.propose_layer(lay0.q, okq, osc, cu, cfg.kappa_p)
+        for (b, h) in _all_rows(cfg):
+            n = int(ocnt[b, h])
+            assert int(gpc[b, h]) == n
+            check_index_set(gpool[b, h, :n], opool[b, h, :n], lambda t: oscore[(b, h)][t], f"pool {b},{h}")
+    for lay in layers:
+        l = lay.index
+        gidx, gcnt = _np(dec.idx[l]), _np(dec.cnt[l])
+        if sets == "sequence":
+            oidx, ocnt2, orr = pipeline.refine_layer_seq(lay.q, lay.k, cu, gpool[:, 0], gpc[:, 0], cfg.kappa)
+            for b in range(cfg.batch):
+                n, c = int(gpc[b, 0]), int(ocnt2[b])
+                assert int(gcnt[b, 0]) == c
+                r = dict(zip(gpool[b, 0, :n].tolist(), orr[b].tolist()))
+                check_index_set(gidx[b, 0, :c], oidx[b, :c], lambda t: r[t], f"L{l} seq idx {b}")
+                assert set(gidx[b, 0, :c].tolist()) <= set(gpool[b, 0, :n].tolist())
+            oout, olse = pipeline.attend_layer_sets(lay.q, lay.k, lay.v, cu, gidx[:, 0], gcnt[:, 0],
+                                                    "sequence", dec.scale)
+        else:
+            oidx, ocnt2, orr = pipeline.refine_layer_heads(lay.q, lay.k, cu, gpool, gpc, cfg.kappa)
+            G = cfg.G
+            for b in range(cfg.batch):
+                for hq in range(cfg.num_q_heads):
+                    h = hq // G
+                    n, c = int(gpc[b, h]), int(ocnt2[b, hq])
+                    assert int(gcnt[b, hq]) == c
+                    r = dict(zip(gpool[b, h, :n].tolist(), orr[(b, hq)].tolist()))
+                    check_index_set(gidx[b, hq, :c], oidx[b, hq, :c], lambda t: r[t], f"L{l} idx {b},{hq}")
+                    assert set(gidx[b, hq, :c].tolist()) <= set(gpool[b, h, :n].tolist())
+            oout, olse = pipeline.attend_layer_sets(lay.q, lay.k, lay.v, cu, gidx, gcnt, "q_head",
+                                                    dec.scale)
+        assert np.abs(_np(dec.out[l]) - oout).max() <= tol, l
+        assert np.abs(_np(dec.lse[l]) - olse).max() <= 10 * tol, l
