@@ -44,6 +44,7 @@
 
 #include <cstdlib>
 #include <cstring>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -297,6 +298,136 @@ struct ScoreMma {
   }
 };
 
+// Key rows of a bf16 cache, per warp: warp w streams its own 16-row tiles
+// (w, w + kWarps, ...) through its own kWS slots of the ring with cp.async and
+// scores each tile with mma.sync as soon as it lands, so the key phase has no
+// block-wide barrier.  Slots are laid out as the shared ring's stages (16-byte
+// chunks XOR-swizzled by row: conflict-free ldmatrix).  prime() issues the
+// first kWS tiles and leaves the row at npos unwritten; fill_new() copies it
+// from nrow (so prime() reads the cache only).
+template <int D, int GP>
+struct WarpKeys {
+  static constexpr int RB = D * 2;
+  static constexpr int VPR = RB / 16;                // 16-byte chunks per row
+  static constexpr int TB = 16 * RB;                 // tile bytes
+  static constexpr int kWS = kRing / (kWarps * TB);  // slots per warp: 2 (d = 128), 4 (d = 64)
+  static constexpr int CPL = 16 * VPR / 32;          // chunks one lane copies per tile
+  static constexpr int KS = D / 16;
+  static constexpr int NT = (GP + 7) / 8;
+  static_assert(kWS >= 2 && CPL >= 1, "per-warp slots");
+  const __nv_bfloat16* kb;
+  const __nv_bfloat16* nrow;
+  int npos;
+  const int* spos;
+  int m, nt;
+  unsigned char* slots;
+  uint32_t bq[NT][KS][2];
+
+  __device__ __forceinline__ WarpKeys(const __nv_bfloat16* kb_, const __nv_bfloat16* nrow_, int npos_,
+                                      const int* spos_, int m_, unsigned char* ring)
+      : kb(kb_), nrow(nrow_), npos(npos_), spos(spos_), m(m_) {
+    const int warp = threadIdx.x >> 5;
+    const int tiles = (m_ + 15) >> 4;
+    nt = tiles > warp ? (tiles - warp + kWarps - 1) / kWarps : 0;
+    slots = ring + warp * kWS * TB;
+  }
+  // this warp's tile tl (slice tile warp + tl kWarps) into slot tl % kWS
+  __device__ __forceinline__ void issue(int tl, bool defer_new) {
+    const int lane = threadIdx.x & 31;
+    if (tl < nt) {
+      const int r0 = ((threadIdx.x >> 5) + tl * kWarps) * 16;
+      unsigned char* buf = slots + (tl % kWS) * TB;
+#pragma unroll
+      for (int j = 0; j < CPL; ++j) {
+        const int x = lane + 32 * j, rr = x / VPR, c = x % VPR;
+        const int i = r0 + rr;
+        const int pos = i < m ? spos[i] : -1;
+        const bool fresh = nrow && pos == npos;
+        if (fresh && defer_new) continue;
+        const __nv_bfloat16* src = fresh ? nrow + c * 8 : kb + (int64_t)(pos >= 0 ? pos : 0) * D + c * 8;
+        cp_async16(smem_u32(buf + swz<RB>(rr, c)), src, pos >= 0);
+      }
+    }
+    cp_async_commit();  // one group per call (possibly empty): constant wait depth
+  }
+  __device__ __forceinline__ void prime() {
+#pragma unroll
+    for (int tl = 0; tl < kWS; ++tl) issue(tl, true);
+  }
+  __device__ __forceinline__ void fill_new() {
+    if (!nrow) return;
+    const int lane = threadIdx.x & 31;
+    for (int tl = 0; tl < kWS && tl < nt; ++tl) {
+      const int r0 = ((threadIdx.x >> 5) + tl * kWarps) * 16;
+      unsigned char* buf = slots + tl * TB;
+#pragma unroll
+      for (int j = 0; j < CPL; ++j) {
+        const int x = lane + 32 * j, rr = x / VPR, c = x % VPR;
+        const int i = r0 + rr;
+        if (i < m && spos[i] == npos) *reinterpret_cast<uint4*>(buf + swz<RB>(rr, c)) = ld16(nrow + c * 8);
+      }
+    }
+  }
+  __device__ __forceinline__ void load_q(const __nv_bfloat16* q, int G) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const int n = t * 8 + g;
+#pragma unroll
+      for (int s = 0; s < KS; ++s) {
+        if (n < G) {
+          const uint32_t* qr = reinterpret_cast<const uint32_t*>(q + (int64_t)n * D + s * 16);
+          bq[t][s][0] = qr[tig];
+          bq[t][s][1] = qr[4 + tig];
+        } else {
+          bq[t][s][0] = bq[t][s][1] = 0u;
+        }
+      }
+    }
+  }
+  // dots[g * mc + i] = q_g . k_i for the warp's tiles (-inf at a bad position)
+  __device__ __forceinline__ void run(int G, int mc, float* dots) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
+    const int lrow = (lane & 7) + ((lane >> 3) & 1) * 8;
+    for (int tl = 0; tl < nt; ++tl) {
+      cp_async_wait<kWS - 1>();
+      __syncwarp();
+      const unsigned char* buf = slots + (tl % kWS) * TB;
+      float acc[2][NT][4];
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int t = 0; t < NT; ++t) acc[u][t][0] = acc[u][t][1] = acc[u][t][2] = acc[u][t][3] = 0.0f;
+#pragma unroll
+      for (int s = 0; s < KS; ++s) {
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(smem_u32(buf + swz<RB>(lrow, 2 * s + (lane >> 4))), a0, a1, a2, a3);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) mma_bf16(acc[s & 1][t], a0, a1, a2, a3, bq[t][s][0], bq[t][s][1]);
+      }
+      __syncwarp();  // the slot is read: refill it
+      issue(tl + kWS, false);
+      const int r0 = ((threadIdx.x >> 5) + tl * kWarps) * 16;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int i = r0 + g + 8 * half;
+        if (i < m) {
+          const bool ok = spos[i] >= 0;
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            const int col = t * 8 + 2 * tig;
+            const float v0 = acc[0][t][2 * half] + acc[1][t][2 * half];
+            const float v1 = acc[0][t][2 * half + 1] + acc[1][t][2 * half + 1];
+            if (col < G) dots[col * mc + i] = ok ? v0 : -INFINITY;
+            if (col + 1 < G) dots[(col + 1) * mc + i] = ok ? v1 : -INFINITY;
+          }
+        }
+      }
+    }
+    cp_async_wait<0>();
+  }
+};
+
 // CUDA cores (fp32 cache): lane groups of LPR lanes per row, transposed
 // butterfly over the query heads.
 template <typename T, int D, int GP>
@@ -488,8 +619,13 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
     for (int i = tid; i < (rank == 0 ? kHistWords : kH2); i += kThreads) hist[i] = 0u;
   __syncthreads();
   cluster_arrive();  // rank 0's histograms are cleared once every CTA has arrived
+  // bf16: every warp streams its own key tiles; fp32: the shared stage ring
+  constexpr bool kWarpKeys = std::is_same<T, __nv_bfloat16>::value;
   RowStream<T, D> kst(kb, knew, L - 1, spos, nullptr, m, ring);
-  kst.prime(true);  // cache rows at pool positions only
+  WarpKeys<D, GP> wk(reinterpret_cast<const __nv_bfloat16*>(kb),
+                     reinterpret_cast<const __nv_bfloat16*>(knew), L - 1, spos, m, ring);
+  if constexpr (kWarpKeys) wk.prime();  // cache rows at pool positions only
+  else kst.prime(true);
 
   // Up to here the kernel has read the pool and the key cache only, which
   // the previous kernel on the stream does not write when the launch
@@ -505,10 +641,14 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
       reinterpret_cast<uint4*>(const_cast<T*>(vb) + (int64_t)(L - 1) * D)[c] = ld16(vnew + c * (16 / (int)sizeof(T)));
     }
   }
-  kst.fill_new();
+  if constexpr (kWarpKeys) wk.fill_new();
+  else kst.fill_new();
 
   // ---- 1. exact logits of the slice
-  {
+  if constexpr (kWarpKeys) {
+    wk.load_q(reinterpret_cast<const __nv_bfloat16*>(qrow), a.G);
+    wk.run(a.G, a.mc, dots);
+  } else {
     typename ScorePick<T, D, GP>::type sc;
     sc.init(qrow, a.G);
     kst.run([&](int r0, const unsigned char* buf, int nrows) {
@@ -531,7 +671,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
   cluster_wait();
 
   // ---- 2. selection keys; their first digit into the cluster histogram
-  constexpr bool kSplit = ScorePick<T, D, GP>::type::kSplit;  // second half-sums in pw
+  constexpr bool kSplit = !kWarpKeys && ScorePick<T, D, GP>::type::kSplit;  // second half-sums in pw
   const bool sum_group = a.sum_group != 0;  // the group's heads summed, not maxed
   for (int i = tid; i < m; i += kThreads) {
     float best = sum_group ? 0.0f : -INFINITY;
@@ -781,16 +921,18 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
     }
   }
 
-  // ---- 4. selected members of the slice, positions to idx (ascending)
+  // ---- 4. selected members of the slice, positions to idx (ascending).
+  // Warp w owns members [w pw, (w + 1) pw) in slot order; three ballot passes
+  // (keys at P per warp, selected per warp, placement) with two block barriers.
   int nsel = 0;
   {
     const int off = all ? lo : s_mine[0];
     const int take = all ? 0 : s_mine[1];
     int32_t* idx = a.idx + (int64_t)row * a.kappa;
-    int base = 0, eqbase = 0;
-    for (int i0 = 0; i0 < m; i0 += kThreads) {  // CTA-uniform trip count
-      const int i = i0 + tid;
-      bool gt = false, eq = false;
+    const int pw = ((m + kWarps - 1) / kWarps + 31) & ~31;
+    const int w0 = warp * pw;
+    auto flags = [&](int i, bool& gt, bool& eq) {
+      gt = eq = false;
       if (i < m) {
         if (all) {
           gt = true;
@@ -800,41 +942,61 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
           eq = pre == P;
         }
       }
+    };
+    int ecount = 0;
+    for (int c = 0; c < pw; c += 32) {
+      bool gt, eq;
+      flags(w0 + c + lane, gt, eq);
+      ecount += __popc(__ballot_sync(0xffffffffu, eq));
+    }
+    if (lane == 0) s_wa[warp] = ecount;
+    __syncthreads();
+    int ebase = 0;
+    for (int w = 0; w < warp; ++w) ebase += s_wa[w];
+    int scount = 0;  // a key at P is taken while its rank among the keys at P is below take
+    for (int c = 0, er = ebase; c < pw; c += 32) {
+      bool gt, eq;
+      flags(w0 + c + lane, gt, eq);
       const unsigned eb = __ballot_sync(0xffffffffu, eq);
-      if (lane == 0) s_wa[warp] = __popc(eb);
-      __syncthreads();
-      int er = eqbase, et = eqbase;
-      for (int w = 0; w < kWarps; ++w) {
-        if (w < warp) er += s_wa[w];
-        et += s_wa[w];
-      }
-      er += __popc(eb & lt);
-      const bool s = gt || (eq && er < take);
-      const unsigned bal = __ballot_sync(0xffffffffu, s);
-      if (lane == 0) s_wb[warp] = __popc(bal);
-      __syncthreads();
-      int before = base, tot = base;
-      for (int w = 0; w < kWarps; ++w) {
-        if (w < warp) before += s_wb[w];
-        tot += s_wb[w];
-      }
-      if (s) {
-        const int o = before + __popc(bal & lt);
-        const int slot = off + o;
-        if (slot < k) idx[slot] = pool[i];
+      scount += __popc(__ballot_sync(0xffffffffu, gt || (eq && er + __popc(eb & lt) < take)));
+      er += __popc(eb);
+    }
+    if (lane == 0) s_wb[warp] = scount;
+    __syncthreads();
+    int base = 0, o = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      if (w < warp) o += s_wb[w];
+      base += s_wb[w];
+    }
+    for (int c = 0, er = ebase; c < pw; c += 32) {
+      const int i = w0 + c + lane;
+      bool gt, eq;
+      flags(i, gt, eq);
+      const unsigned eb = __ballot_sync(0xffffffffu, eq);
+      const bool sl = gt || (eq && er + __popc(eb & lt) < take);
+      const unsigned bal = __ballot_sync(0xffffffffu, sl);
+      if (sl) {
+        const int oo = o + __popc(bal & lt);
+        const int slot = off + oo;
+        if (slot < k) idx[slot] = spos[i];
         else flag_status(a.status, PRISM_DEV_TOO_LONG);  // unreachable if counts are right
-        sel[o] = i;
+        sel[oo] = i;
       }
-      base = tot;
-      eqbase = et;
-      __syncthreads();
+      o += __popc(bal);
+      er += __popc(eb);
     }
     nsel = min(base, m);
     for (int s = k + rank * kThreads + tid; s < a.kappa; s += CL * kThreads) idx[s] = -1;
     if (rank == 0 && tid == 0) a.cnt[row] = k;
+    __syncthreads();  // sel is complete
   }
 
-  // ---- 5. softmax partial over the selected members of the slice
+  // ---- 5. softmax partial over the selected members of the slice.  The
+  // value rows are requested first (the ring is free: no peer reads it after
+  // the selection's last cluster barrier), so their latency overlaps the
+  // softmax statistics
+  RowStream<T, D> vst(vb, vnew, L - 1, spos, sel, nsel, ring);
+  vst.prime(false);
   float mx[GP];
 #pragma unroll
   for (int g = 0; g < GP; ++g) mx[g] = -INFINITY;
@@ -886,8 +1048,6 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
     for (int e = 0; e < E; ++e) o[g][e] = 0.0f;
   // stream the selected value rows (the weights are read after the first
   // stage barrier of the stream)
-  RowStream<T, D> vst(vb, vnew, L - 1, spos, sel, nsel, ring);
-  vst.prime(false);
   vst.run([&](int j0, const unsigned char* buf, int nrows) {
         for (int r = warp * RPW + sub; r < nrows; r += NG) {
           float f[E];
