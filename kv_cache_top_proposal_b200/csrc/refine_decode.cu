@@ -42,8 +42,6 @@
 // value rows, d * sizeof(T) each.
 #include <cooperative_groups.h>
 
-#include <cstdlib>
-#include <cstring>
 #include <type_traits>
 
 #include "common.cuh"
@@ -66,16 +64,9 @@ constexpr int kBins2 = 1024;  // second and third digits: bits 19..10, 9..0
 constexpr int kH1 = 0;
 constexpr int kH2 = kH1 + kBins1 / 2;
 constexpr int kH3 = kH2 + kBins2 / 2;
-// gathered selection: the summed first-digit slice (at most kBins1 / 4 words,
-// over kH2 and kH3, which it does not use), then the local later-digit bins
-constexpr int kHSlice = kH2;
-constexpr int kHLocal = kH3 + kBins2 / 2;
-constexpr int kHistWords = kHLocal + kBins2 / 2;
+constexpr int kHistWords = kH3 + kBins2 / 2;
 constexpr int kMaxCount = 65535;  // largest pool a 16-bit bin count can hold
 constexpr int kMaxCluster = 16;
-// gathered selection: every thread holds kGatherU x 4 of the row's keys
-constexpr int kGatherU = 8;
-constexpr int kGatherMax = kGatherU * 4 * kThreads;  // 8192 pool members
 
 struct RDArgs {
   const void* q;
@@ -99,7 +90,6 @@ struct RDArgs {
   float* lse;
   int32_t* status;
   int sum_group;  // selection score: sum over the group's query heads instead of the maximum
-  int gather;     // gathered selection (every CTA reads the row's keys), pools up to kGatherMax
 };
 
 // Byte offset of 16-byte chunk `c` of row `r` in a stage: chunks are XOR
@@ -775,97 +765,14 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
       __syncthreads();
     };
     int r = k;
-    // the summed slices: the ring with the cluster rounds below (later
-    // cluster barriers keep it intact while peers read it); a dedicated
-    // region with the gathered selection, which has no further barrier
+    // the summed slices go to the ring: the later cluster barriers keep it
+    // intact while the peers read it
     if (CL == 1) resolve(hist + kH1, kBins1, r);
-    else cluster_digit(hist + kH1, kBins1, r, a.gather ? hist + kHSlice : reinterpret_cast<uint32_t*>(ring));
+    else cluster_digit(hist + kH1, kBins1, r, reinterpret_cast<uint32_t*>(ring));
     P = (uint32_t)s_dig[0];
     shift = 20;
     r -= s_dig[1];
-    if (a.gather) {
-      // Gathered later digits: every CTA reads the whole row's keys (complete
-      // since the first digit's barriers) and resolves the rest of the
-      // prefix, its tie quota and its output offset by itself -- no further
-      // cluster rounds.
-      // Thread tid holds slots slot(j) .. + 3 for j < kGatherU, where the
-      // slot space [0, CL chunk) is walked from this CTA's own slice onward
-      // (rotated by rank), so the CTAs do not all read the same peer at once.
-      const int span = CL * chunk;  // <= kGatherMax (plan)
-      auto slot_of = [&](int j) {
-        const int s0 = 4 * (tid + j * kThreads) + rank * chunk;
-        return s0 >= span ? s0 - span : s0;
-      };
-      uint4 kv[kGatherU];  // all loads in flight at once
-#pragma unroll
-      for (int j = 0; j < kGatherU; ++j) {
-        const int s0 = slot_of(j);
-        kv[j] = make_uint4(0u, 0u, 0u, 0u);
-        if (4 * (tid + j * kThreads) < span && s0 < n) {
-          const int c = s0 / chunk;
-          kv[j] = *reinterpret_cast<const uint4*>(cluster.map_shared_rank(keys, c) + (s0 - c * chunk));
-        }
-      }
-      uint32_t* h2 = hist + kHLocal;
-      // a later 10-bit digit from the row's keys whose prefix is `pre`
-      auto local_digit = [&](int pshift, uint32_t pre, int dshift) {
-        for (int i = tid; i < kBins2 / 2; i += kThreads) h2[i] = 0u;
-        __syncthreads();
-#pragma unroll
-        for (int j = 0; j < kGatherU; ++j) {
-          const int s0 = slot_of(j);
-          const bool in = 4 * (tid + j * kThreads) < span;
-          const uint32_t w4[4] = {kv[j].x, kv[j].y, kv[j].z, kv[j].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (in && s0 + e < n && (w4[e] >> pshift) == pre) hist_push(h2, (w4[e] >> dshift) & 1023u);
-        }
-        __syncthreads();
-        find_digit<kBins2>(h2, r, scratch, s_dig);
-      };
-      if (r < s_dig[2]) {
-        local_digit(20, P, 10);
-        P = (P << 10) | (uint32_t)s_dig[0];
-        shift = 10;
-        r -= s_dig[1];
-        if (r < s_dig[2]) {
-          local_digit(10, P, 0);
-          P = (P << 10) | (uint32_t)s_dig[0];
-          shift = 0;
-          r -= s_dig[1];
-        }
-      }
-      rtie = r;
-      // keys before this CTA's slice above / at P, and at P inside it
-      int gtb = 0, eqb = 0, eqo = 0;
-#pragma unroll
-      for (int j = 0; j < kGatherU; ++j) {
-        const int s0 = slot_of(j);
-        const bool in = 4 * (tid + j * kThreads) < span;
-        const uint32_t w4[4] = {kv[j].x, kv[j].y, kv[j].z, kv[j].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int sl = s0 + e;
-          if (!in || sl >= n) continue;
-          const uint32_t pre = w4[e] >> shift;
-          if (sl < lo) {
-            gtb += pre > P;
-            eqb += pre == P;
-          } else if (sl < hi) {
-            eqo += pre == P;
-          }
-        }
-      }
-      int tot1, tot2;
-      block_excl_scan((gtb << 16) | eqb, scratch, &tot1);  // both counts <= kGatherMax
-      block_excl_scan(eqo, scratch, &tot2);
-      if (tid == 0) {
-        const int gb = tot1 >> 16, eb = tot1 & 0xFFFF;
-        s_mine[0] = gb + min(rtie, eb);
-        s_mine[1] = min(max(rtie - eb, 0), tot2);
-      }
-      __syncthreads();
-    } else if (r < s_dig[2]) {  // part of the bin: the second digit of its (few) keys, in rank 0
+    if (r < s_dig[2]) {  // part of the bin: the second digit of its (few) keys, in rank 0
       for (int i = tid; i < m; i += kThreads) {
         const uint32_t key = keys[i];
         if ((key >> 20) == P) hist_push(h0 + kH2, (key >> 10) & 1023u);
@@ -885,40 +792,38 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
         r -= s_dig[1];
       }
     }
-    if (!a.gather) {
-      rtie = r;
-      // this CTA's counts above and at P, then every CTA's, in rank order
-      int gt = 0, eq = 0;
-      for (int i = tid; i < m; i += kThreads) {
-        const uint32_t pre = keys[i] >> shift;
-        gt += pre > P;
-        eq += pre == P;
-      }
-      int tot;
-      block_excl_scan((gt << 16) | eq, scratch, &tot);  // both counts <= 65535
-      if (tid == 0) {
-        s_cnt[0] = tot >> 16;
-        s_cnt[1] = tot & 0xFFFF;
-      }
-      cluster.sync();  // S4: every CTA's counts are published
-      if (warp == 0) {
-        int g_s = 0, e_s = 0;
-        if (lane < CL) {
-          const int* rc = cluster.map_shared_rank(s_cnt, lane);
-          g_s = rc[0];
-          e_s = rc[1];
-        }
-        const int ebefore = warp_incl_scan(e_s) - e_s;
-        const int take = min(max(rtie - ebefore, 0), e_s);
-        const int nsel_s = g_s + take;
-        const int before = warp_incl_scan(nsel_s) - nsel_s;
-        if (lane == rank) {
-          s_mine[0] = before;
-          s_mine[1] = take;
-        }
-      }
-      __syncthreads();
+    rtie = r;
+    // this CTA's counts above and at P, then every CTA's, in rank order
+    int gt = 0, eq = 0;
+    for (int i = tid; i < m; i += kThreads) {
+      const uint32_t pre = keys[i] >> shift;
+      gt += pre > P;
+      eq += pre == P;
     }
+    int tot;
+    block_excl_scan((gt << 16) | eq, scratch, &tot);  // both counts <= 65535
+    if (tid == 0) {
+      s_cnt[0] = tot >> 16;
+      s_cnt[1] = tot & 0xFFFF;
+    }
+    cluster.sync();  // S4: every CTA's counts are published
+    if (warp == 0) {
+      int g_s = 0, e_s = 0;
+      if (lane < CL) {
+        const int* rc = cluster.map_shared_rank(s_cnt, lane);
+        g_s = rc[0];
+        e_s = rc[1];
+      }
+      const int ebefore = warp_incl_scan(e_s) - e_s;
+      const int take = min(max(rtie - ebefore, 0), e_s);
+      const int nsel_s = g_s + take;
+      const int before = warp_incl_scan(nsel_s) - nsel_s;
+      if (lane == rank) {
+        s_mine[0] = before;
+        s_mine[1] = take;
+      }
+    }
+    __syncthreads();
   }
 
   // ---- 4. selected members of the slice, positions to idx (ascending).
@@ -1207,14 +1112,6 @@ cudaError_t by_group(const Dims& d, const RDArgs& a, int cl, bool ov, cudaStream
 
 }  // namespace
 
-// The later digits take the cluster-wide rounds unless PRISM_RD_SELECT=gather
-// selects the gathered resolution (pools up to kGatherMax; A/B switch of two
-// exact selections with identical results)
-bool gather_off() {
-  const char* e = std::getenv("PRISM_RD_SELECT");
-  return !(e && std::strcmp(e, "gather") == 0);
-}
-
 RefineDecodePlan plan_refine_decode(const Dims& d, int kappa_p) {
   const int rows = d.B * d.Hkv;
   const int GP = padded_group(d.G);
@@ -1238,9 +1135,7 @@ cudaError_t launch_refine_decode(const Dims& d, const RefineDecodePlan& p, const
                                  cudaStream_t st) {
   if (d.B * d.Hkv == 0) return cudaSuccess;
   RDArgs a{q, k, v, k_next, k_new, v_new, d.cu_dev, pool, pool_cnt, kappa_p, kappa, d.Hkv, d.G, d.Hq, d.T, p.mc,
-           softmax_scale * 1.4426950408889634f, idx, cnt, out, lse, status, sum_group ? 1 : 0,
-           (p.cluster * (((kappa_p + p.cluster - 1) / p.cluster + 3) & ~3) <= kGatherMax && !gather_off()) ? 1
-                                                                                             : 0};
+           softmax_scale * 1.4426950408889634f, idx, cnt, out, lse, status, sum_group ? 1 : 0};
   if (d.bf16)
     return d.D == 128 ? by_group<__nv_bfloat16, 128>(d, a, p.cluster, overlap, st)
                       : by_group<__nv_bfloat16, 64>(d, a, p.cluster, overlap, st);

@@ -709,11 +709,11 @@ def test_refine_decode_large_ties(P, kp, kap):
     assert np.abs(_np(out) - oout).max() <= 2e-3
 
 
-GATHER_CASES = [
+SELECT_CASES = [
     # (seqlens, Hq, Hkv, d, kappa_p, kappa, integer keys): the c128k row
-    # shape, a ragged batch with an empty and a short sequence, the largest
-    # gathered pool and the first one past it (cluster rounds on both
-    # paths), and integer keys (many exactly equal scores at the threshold)
+    # shape, a ragged batch with an empty and a short sequence, pools of
+    # 8192 and 8193 members, and integer keys (many exactly equal scores at
+    # the threshold, resolved by the lower position)
     ([131072], 32, 8, 128, 8192, 2048, False),
     ([40000, 9000, 0, 300, 12300], 32, 8, 128, 4096, 1024, False),
     ([30000], 8, 2, 128, 8192, 3000, False),
@@ -723,11 +723,10 @@ GATHER_CASES = [
 ]
 
 
-@pytest.mark.parametrize("case", GATHER_CASES, ids=lambda c: f"{len(c[0])}seq-kp{c[4]}-k{c[5]}-int{int(c[6])}")
-def test_refine_decode_gathered_selection(P, case, monkeypatch):
-    """The gathered selection (every CTA reads the row's keys and resolves
-    the threshold itself) against the cluster-wide digit rounds: the same
-    index sets and bit-identical outputs; and against the oracle."""
+@pytest.mark.parametrize("case", SELECT_CASES, ids=lambda c: f"{len(c[0])}seq-kp{c[4]}-k{c[5]}-int{int(c[6])}")
+def test_refine_decode_selection_cases(P, case):
+    """The fused refined layer's exact top-kappa on the shapes and score
+    distributions above, against the oracle; attention on the GPU's set."""
     seqlens, hq, hkv, d, kp, kap, integer = case
     B = len(seqlens)
     prob = problem(P, seqlens, hq, hkv, d, "bf16")
@@ -747,20 +746,13 @@ def test_refine_decode_gathered_selection(P, case, monkeypatch):
     pool_t, pcnt_t = torch.tensor(pool, device=DEV), torch.tensor(pcnt, device=DEV)
     scale = float(np.float32(1 / math.sqrt(d)))
     ws = ws_for(P, prob, P.OP_REFINE_DECODE, kp, kap)
-    res = []
-    for mode in ("cluster", "gather"):
-        monkeypatch.setenv("PRISM_RD_SELECT", mode)
-        idx = torch.full((B, hkv, kap), -7, dtype=torch.int32, device=DEV)
-        cnt = torch.zeros((B, hkv), dtype=torch.int32, device=DEV)
-        out = torch.full((B, hq, d), 77.0, device=DEV)
-        lse = torch.full((B, hq), 77.0, device=DEV)
-        P.refine_decode(prob, q, k, v, pool_t, pcnt_t, kp, kap, scale, idx, cnt, out, ws, lse=lse)
-        torch.cuda.synchronize()
-        res.append((idx, cnt, out, lse))
+    i1 = torch.full((B, hkv, kap), -7, dtype=torch.int32, device=DEV)
+    c1 = torch.zeros((B, hkv), dtype=torch.int32, device=DEV)
+    o1 = torch.full((B, hq, d), 77.0, device=DEV)
+    l1 = torch.full((B, hq), 77.0, device=DEV)
+    P.refine_decode(prob, q, k, v, pool_t, pcnt_t, kp, kap, scale, i1, c1, o1, ws, lse=l1)
+    torch.cuda.synchronize()
     assert P.get_device_status(ws) == 0
-    (i0, c0, o0, l0), (i1, c1, o1, l1) = res
-    assert torch.equal(i0, i1) and torch.equal(c0, c1)
-    assert torch.equal(o0, o1) and torch.equal(l0, l1)
     oidx, ocnt, oscores = pipeline.refine_layer(q, k, prob.cu_host.tolist(), pool, pcnt, kap)
     gi, gc = _np(i1), _np(c1)
     assert np.array_equal(gc, ocnt)
