@@ -344,17 +344,52 @@ __global__ void __launch_bounds__(kDThreads, GP <= 4 ? 2 : 1) dense_kernel(const
     __syncthreads();  // the stage is in registers: hand it back
     if (tid == 0) issue(i + kDStages);
     float lg[2][GP];
+    if constexpr (LPR == 16 && GP == 4) {
+      // both rows' four head dot products reduced over the 16 lanes of the
+      // group at once, transposed (each exchange halves the values a lane
+      // keeps), then every value broadcast from the lane that holds it
+      float v[8];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      float f[E];
-      Vec16<T>::unpack(kr[u], f);
+      for (int u = 0; u < 2; ++u) {
+        float f[E];
+        Vec16<T>::unpack(kr[u], f);
 #pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        float sdot = 0.0f;
+        for (int g = 0; g < 4; ++g) {
+          float sdot = 0.0f;
 #pragma unroll
-        for (int e = 0; e < E; ++e) sdot = fmaf(qf[g][e], f[e], sdot);
-        sdot = group_sum<LPR>(sdot);
-        lg[u][g] = ok[u] ? sdot * a.scale_log2 : -INFINITY;
+          for (int e = 0; e < E; ++e) sdot = fmaf(qf[g][e], f[e], sdot);
+          v[u * 4 + g] = sdot;
+        }
+      }
+      const bool b8 = li & 8, b4 = li & 4, b2 = li & 2;
+      float w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        w[j] = (b8 ? v[4 + j] : v[j]) + __shfl_xor_sync(0xffffffffu, b8 ? v[j] : v[4 + j], 8);
+      float x[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        x[j] = (b4 ? w[2 + j] : w[j]) + __shfl_xor_sync(0xffffffffu, b4 ? w[j] : w[2 + j], 4);
+      float y = (b2 ? x[1] : x[0]) + __shfl_xor_sync(0xffffffffu, b2 ? x[0] : x[1], 2);
+      y += __shfl_xor_sync(0xffffffffu, y, 1);  // value (li >> 1) & 7: row u = bit 2, head = bits 0-1
+#pragma unroll
+      for (int vi = 0; vi < 8; ++vi) {
+        const float sdot = __shfl_sync(0xffffffffu, y, (lane & 16) + 2 * vi);
+        lg[vi >> 2][vi & 3] = ok[vi >> 2] ? sdot * a.scale_log2 : -INFINITY;
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        float f[E];
+        Vec16<T>::unpack(kr[u], f);
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          float sdot = 0.0f;
+#pragma unroll
+          for (int e = 0; e < E; ++e) sdot = fmaf(qf[g][e], f[e], sdot);
+          sdot = group_sum<LPR>(sdot);
+          lg[u][g] = ok[u] ? sdot * a.scale_log2 : -INFINITY;
+        }
       }
     }
     float vf[2][E];
@@ -362,14 +397,21 @@ __global__ void __launch_bounds__(kDThreads, GP <= 4 ? 2 : 1) dense_kernel(const
     for (int u = 0; u < 2; ++u) Vec16<T>::unpack(vr[u], vf[u]);
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
-      const float mx = fmaxf(m[g], fmaxf(lg[0][g], lg[1][g]));
-      if (mx == -INFINITY) continue;
-      const float alpha = exp2f(m[g] - mx);
-      const float p0 = exp2f(lg[0][g] - mx), p1 = exp2f(lg[1][g] - mx);
-      l[g] = l[g] * alpha + (p0 + p1);
+      // the accumulators are rescaled only when the running maximum grows
+      // (the same value per lane group, so the branch is uniform there)
+      const float mx = fmaxf(lg[0][g], lg[1][g]);
+      if (mx > m[g]) {
+        const float alpha = exp2f(m[g] - mx);  // 0 while nothing was seen
+        l[g] *= alpha;
 #pragma unroll
-      for (int e = 0; e < E; ++e) o[g][e] = fmaf(p1, vf[1][e], fmaf(p0, vf[0][e], o[g][e] * alpha));
-      m[g] = mx;
+        for (int e = 0; e < E; ++e) o[g][e] *= alpha;
+        m[g] = mx;
+      }
+      if (m[g] == -INFINITY) continue;
+      const float p0 = exp2f(lg[0][g] - m[g]), p1 = exp2f(lg[1][g] - m[g]);
+      l[g] += p0 + p1;
+#pragma unroll
+      for (int e = 0; e < E; ++e) o[g][e] = fmaf(p1, vf[1][e], fmaf(p0, vf[0][e], o[g][e]));
     }
   }
 
