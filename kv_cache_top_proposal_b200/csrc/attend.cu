@@ -13,6 +13,11 @@
 //   M = max_s m_s,  out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s,
 //   lse = (M + log2 sum_s 2^(m_s - M) l_s) * ln 2.
 // HBM bound: 2 * d * sizeof(T) bytes per listed row.
+#include <algorithm>
+#include <queue>
+#include <type_traits>
+#include <vector>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -463,6 +468,323 @@ constexpr int dense_smem() {
   return ring > comb ? ring : comb;
 }
 
+// ---- dense pass on tensor cores (bf16 cache, up to 8 query heads per KV head)
+//
+// Stages of kTRows = 128 contiguous K rows and the same V rows arrive by 2D
+// tensor copies with the 128-byte swizzle (16-byte chunk c of row r of a
+// 64-feature box at r * 128 + ((c ^ (r & 7)) << 4)), so eight rows read at
+// one chunk by ldmatrix hit eight bank groups.  Warp w takes rows
+// [16 w, 16 w + 16) of every stage:
+//   S = K_w Q^T      mma m16n8k16: 16 rows x 8 heads, k over d (Q in registers)
+//   per head: online softmax over the 16 rows (log2 domain, the accumulators
+//   rescaled only when the running maximum grows)
+//   O^T += V_w^T P^T mma m16n8k16: 16 features x 8 heads, k over the rows;
+//   V^T by transposing ldmatrix, P^T by movmatrix from S's accumulator
+//   layout, as three bf16 parts whose sum is p to 2^-24 relative
+// bf16 operands make every product exact in fp32; the sums are fp32.  One CTA
+// per SM keeps 192 KB of stages in flight.
+constexpr int kTRows = 128;
+constexpr int kTBox = kTRows * 128;  // one tensor copy: 128 rows x 64 features
+
+template <int D>
+__host__ __device__ constexpr int tc_part() { return kTRows * D * 2; }  // one stage's K (or V) bytes
+template <int D>
+__host__ __device__ constexpr int tc_stages() { return D == 128 ? 3 : 6; }
+template <int D>
+__host__ __device__ constexpr int tc_smem() { return tc_stages<D>() * 2 * tc_part<D>() + 1024; }  // + alignment
+
+__device__ __forceinline__ void t_ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void t_ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ uint32_t t_movtrans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ void t_mma(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t t_bits(__nv_bfloat162 x) { return *reinterpret_cast<uint32_t*>(&x); }
+// rows [y, y + 128) x features [x, x + 64) into a swizzled box; completes on bar
+__device__ __forceinline__ void t_box(unsigned char* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <int D, int GP>
+__global__ void __launch_bounds__(kDThreads, 1)
+    dense_tc_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                    const AttendArgs a) {
+  static_assert(GP <= 8, "eight heads per tile");
+  constexpr int S = tc_stages<D>();
+  constexpr int PB = tc_part<D>();
+  constexpr int BOX = D / 64;  // tensor copies per part
+  constexpr int KS = D / 16;   // k-steps of S = K Q^T, and 16-feature tiles of O^T
+  constexpr int SLOTS = kDWarps;
+  extern __shared__ unsigned char dsm_raw[];
+  __shared__ __align__(8) uint64_t full[S];
+  unsigned char* dsm = dsm_raw + ((1024u - (smem_u32(dsm_raw) & 1023u)) & 1023u);
+
+  const int row = blockIdx.x, split = blockIdx.y;
+  const int b = row / a.Hkv, h = row - b * a.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int t0 = a.cu[b];
+  const int L = a.cu[b + 1] - t0;
+  const int e0 = split * a.per_split;
+  const int e1 = min(L, e0 + a.per_split);
+  const int nst = e1 > e0 ? (e1 - e0 + kTRows - 1) / kTRows : 0;
+  const int64_t y0 = (int64_t)h * a.T + t0 + e0;  // tensor row of the split's first position
+  auto stage = [&](int i) { return dsm + (i % S) * 2 * PB; };
+  auto issue = [&](int i) {  // thread 0
+    if (i < nst) {
+      uint64_t* bar = &full[i % S];
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
+                   "r"(2 * PB)
+                   : "memory");
+      const int y = (int)(y0 + (int64_t)i * kTRows);
+#pragma unroll
+      for (int x = 0; x < BOX; ++x) {
+        t_box(stage(i) + x * kTBox, &tk, x * 64, y, bar);
+        t_box(stage(i) + PB + x * kTBox, &tv, x * 64, y, bar);
+      }
+    }
+  };
+  if (tid == 0) {
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tk)) : "memory");
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tv)) : "memory");
+    for (int i = 0; i < S; ++i) d_mbar_init(&full[i]);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    for (int i = 0; i < S; ++i) issue(i);
+  }
+  // B operand of S = K Q^T: b0 = q_g[16 j + 2 t, + 1], b1 = q_g[16 j + 2 t + 8, + 9]
+  uint32_t qb[KS][2];
+  {
+    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q) +
+                             ((int64_t)b * a.Hq + (int64_t)h * a.G + (g < a.G ? g : 0)) * D + 2 * t;
+#pragma unroll
+    for (int j = 0; j < KS; ++j) {
+      qb[j][0] = g < a.G ? *reinterpret_cast<const uint32_t*>(q + 16 * j) : 0u;
+      qb[j][1] = g < a.G ? *reinterpret_cast<const uint32_t*>(q + 16 * j + 8) : 0u;
+    }
+  }
+  __syncthreads();
+
+  // O^T tile mt: (feature 16 mt + g, heads 2t, 2t+1) and (feature 16 mt + g + 8, same)
+  float acc[KS][4];
+#pragma unroll
+  for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.0f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;  // heads 2t, 2t + 1
+  const int mi = lane >> 3, rr = lane & 7;
+  const int kr = 16 * warp + (mi & 1) * 8 + rr;   // K: matrix mi = (row half mi & 1, chunk half mi >> 1)
+  const int vr = 16 * warp + (mi >> 1) * 8 + rr;  // V: matrix mi = (row half mi >> 1, chunk half mi & 1)
+
+  for (int i = 0; i < nst; ++i) {
+    bool late = false;
+    {
+      uint32_t it = 0;
+      while (!d_mbar_try_wait(&full[i % S], (uint32_t)(i / S) & 1u)) {
+        if (++it == kDWaitLimit) {
+          late = true;
+          break;
+        }
+      }
+    }
+    if (__syncthreads_or(late)) {  // a stage never arrived: report, drain, stop
+      if (tid == 0) {
+        flag_status(a.status, PRISM_DEV_TIMEOUT);
+        for (int j = i; j < nst && j < i + S; ++j) {
+          uint32_t it = 0;
+          while (!d_mbar_try_wait(&full[j % S], (uint32_t)(j / S) & 1u) && ++it < kDWaitLimit) {
+          }
+        }
+      }
+      return;
+    }
+    const uint32_t kb = smem_u32(stage(i)), vb = kb + PB;
+    uint32_t kf[KS][4], vf[KS][4];
+#pragma unroll
+    for (int j = 0; j < KS; ++j) {
+      const int ck = 2 * j + (mi >> 1), cv = 2 * j + (mi & 1);
+      t_ldsm_x4(kb + (ck >> 3) * kTBox + kr * 128 + (((ck & 7) ^ (kr & 7)) << 4), kf[j]);
+      t_ldsm_x4_trans(vb + (cv >> 3) * kTBox + vr * 128 + (((cv & 7) ^ (vr & 7)) << 4), vf[j]);
+    }
+    __syncthreads();  // the stage is in registers: hand it back
+    if (tid == 0) issue(i + S);
+    const int nv = min(kTRows, e1 - (e0 + i * kTRows)) - 16 * warp;  // valid rows of the warp's tile
+    if (nv <= 0) continue;
+    float sv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int j = 0; j < KS; ++j) t_mma(sv, kf[j], qb[j][0], qb[j][1]);
+    const bool ok0 = g < nv, ok1 = g + 8 < nv;
+    const float x0 = ok0 ? sv[0] * a.scale_log2 : -INFINITY;  // row g, head 2t
+    const float x1 = ok0 ? sv[1] * a.scale_log2 : -INFINITY;  // row g, head 2t + 1
+    const float x2 = ok1 ? sv[2] * a.scale_log2 : -INFINITY;  // row g + 8, head 2t
+    const float x3 = ok1 ? sv[3] * a.scale_log2 : -INFINITY;  // row g + 8, head 2t + 1
+    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    if (mx0 > m0) {  // row 0 of the tile is valid, so mx0 is finite
+      const float al = exp2f(m0 - mx0);
+      l0 *= al;
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        acc[mt][0] *= al;
+        acc[mt][2] *= al;
+      }
+      m0 = mx0;
+    }
+    if (mx1 > m1) {
+      const float al = exp2f(m1 - mx1);
+      l1 *= al;
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        acc[mt][1] *= al;
+        acc[mt][3] *= al;
+      }
+      m1 = mx1;
+    }
+    const float p0 = exp2f(x0 - m0), p1 = exp2f(x1 - m1), p2 = exp2f(x2 - m0), p3 = exp2f(x3 - m1);
+    l0 += p0 + p2;
+    l1 += p1 + p3;
+    // P (rows x heads) packed by rows, each 8 x 8 block transposed into the
+    // B operand (k = rows, n = heads): b0 rows 0-7, b1 rows 8-15
+    uint32_t bp[3][2];  // p = part 0 + part 1 + part 2, each bf16: exact to 2^-24 p
+    {
+      float r0 = p0, r1 = p1, r2 = p2, r3 = p3;
+#pragma unroll
+      for (int u = 0; u < 3; ++u) {
+        const __nv_bfloat162 c01 = __floats2bfloat162_rn(r0, r1), c23 = __floats2bfloat162_rn(r2, r3);
+        bp[u][0] = t_movtrans(t_bits(c01));
+        bp[u][1] = t_movtrans(t_bits(c23));
+        const float2 f01 = __bfloat1622float2(c01), f23 = __bfloat1622float2(c23);
+        r0 -= f01.x;  // exact: r and its bf16 rounding share the leading bits
+        r1 -= f01.y;
+        r2 -= f23.x;
+        r3 -= f23.y;
+      }
+    }
+    if (nv < 16) {  // rows past the split carry no weight, and their bytes may be anything
+      const uint32_t k0 = (2 * t < nv ? 0x0000FFFFu : 0u) | (2 * t + 1 < nv ? 0xFFFF0000u : 0u);
+      const uint32_t k1 = (2 * t + 8 < nv ? 0x0000FFFFu : 0u) | (2 * t + 9 < nv ? 0xFFFF0000u : 0u);
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        vf[mt][0] &= k0;
+        vf[mt][1] &= k0;
+        vf[mt][2] &= k1;
+        vf[mt][3] &= k1;
+      }
+    }
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+      for (int u = 0; u < 3; ++u) t_mma(acc[mt], vf[mt], bp[u][0], bp[u][1]);
+  }
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+
+  // combine the warps in warp order (the ring is free now)
+  float* s_o = reinterpret_cast<float*>(dsm);  // [SLOTS][GP][D]
+  float* s_m = s_o + SLOTS * GP * D;           // [SLOTS][GP]
+  float* s_l = s_m + SLOTS * GP;               // [SLOTS][GP]
+  const int ha = 2 * t, hb = 2 * t + 1;
+#pragma unroll
+  for (int mt = 0; mt < KS; ++mt) {
+    if (ha < GP) {
+      s_o[(warp * GP + ha) * D + 16 * mt + g] = acc[mt][0];
+      s_o[(warp * GP + ha) * D + 16 * mt + g + 8] = acc[mt][2];
+    }
+    if (hb < GP) {
+      s_o[(warp * GP + hb) * D + 16 * mt + g] = acc[mt][1];
+      s_o[(warp * GP + hb) * D + 16 * mt + g + 8] = acc[mt][3];
+    }
+  }
+  if (g == 0) {
+    if (ha < GP) {
+      s_m[warp * GP + ha] = m0;
+      s_l[warp * GP + ha] = l0;
+    }
+    if (hb < GP) {
+      s_m[warp * GP + hb] = m1;
+      s_l[warp * GP + hb] = l1;
+    }
+  }
+  __syncthreads();
+  for (int x = tid; x < a.G * D; x += kDThreads) {
+    const int gg = x / D, j = x - gg * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int sl = 0; sl < SLOTS; ++sl) M = fmaxf(M, s_m[sl * GP + gg]);
+    float Ls = 0.0f, O = 0.0f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int sl = 0; sl < SLOTS; ++sl) {
+        const float ms = s_m[sl * GP + gg];
+        const float w = ms == -INFINITY ? 0.0f : exp2f(ms - M);
+        Ls = fmaf(w, s_l[sl * GP + gg], Ls);
+        O = fmaf(w, s_o[(sl * GP + gg) * D + j], O);
+      }
+    }
+    const int64_t pr = ((int64_t)b * a.Hq + (int64_t)h * a.G + gg) * a.splits + split;
+    a.part_o[pr * D + j] = O;
+    if (j == 0) {
+      a.part_ml[pr * 2] = M;
+      a.part_ml[pr * 2 + 1] = Ls;
+    }
+  }
+}
+
+// The tensor-core dense kernel, when the cache can be described by tensor
+// maps (bf16, 16-byte aligned bases, fewer than 2^31 rows); false otherwise.
+template <int D, int GP>
+bool run_dense_tc(const Dims& d, const AttendPlan& p, const AttendArgs& a, cudaStream_t st, cudaError_t* err) {
+  const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode || (reinterpret_cast<uintptr_t>(a.k) & 15) || (reinterpret_cast<uintptr_t>(a.v) & 15))
+    return false;
+  const uint64_t nrows = (uint64_t)d.Hkv * (uint64_t)d.T;
+  if (nrows == 0 || nrows > 0x7fffff00ull) return false;  // row coordinates + 128 fit an int
+  CUtensorMap tk, tv;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)nrows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kTRows};
+  const cuuint32_t estr[2] = {1, 1};
+  for (int x = 0; x < 2; ++x) {
+    if (encode(x ? &tv : &tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x ? a.v : a.k), dims,
+               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  constexpr int smem = tc_smem<D>();
+  auto kd = dense_tc_kernel<D, GP>;
+  cudaError_t e = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) {
+    kd<<<dim3(d.B * d.Hkv, p.splits), kDThreads, smem, st>>>(tk, tv, a);
+    e = cudaGetLastError();
+  }
+  *err = e;
+  return true;
+}
+
 // One CTA of D threads per (sequence, query head): the split weights
 // 2^(m_s - M) are computed in parallel into shared memory, then thread j sums
 // its feature over the splits with independent (pipelined) loads.
@@ -519,7 +841,11 @@ __global__ void __launch_bounds__(D) merge_kernel(int splits, const float* __res
 
 template <typename T, int D, int GP>
 cudaError_t run(const Dims& d, const AttendPlan& p, const AttendArgs& a, cudaStream_t st) {
-  if (!a.idx) {  // dense: the staged kernel
+  if (!a.idx) {  // dense: the tensor-core kernel, else the staged one
+    if constexpr (std::is_same<T, __nv_bfloat16>::value && GP <= 8) {
+      cudaError_t e;
+      if (run_dense_tc<D, GP>(d, p, a, st, &e)) return e;
+    }
     constexpr int smem = dense_smem<T, D, GP>();
     auto kd = dense_kernel<T, D, GP>;
     cudaError_t e = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -552,7 +878,57 @@ cudaError_t by_group(const Dims& d, const AttendPlan& p, const AttendArgs& a, cu
 
 }  // namespace
 
+namespace {
+
+// Makespan, in row units, of the tensor-core dense grid (splits of `per`
+// rows, launched split-major and row-minor, one CTA per SM at a time) under
+// greedy placement: a CTA costs its rows plus a fixed start, an empty one
+// only the start of a CTA that exits.
+int64_t tc_makespan(const Dims& d, int64_t per, int64_t splits) {
+  constexpr int64_t kStart = 256, kEmpty = 32;
+  std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> free_at;
+  for (int i = 0; i < d.num_sms; ++i) free_at.push(0);
+  int64_t end = 0;
+  for (int64_t s = 0; s < splits; ++s)
+    for (int b = 0; b < d.B; ++b) {
+      const int64_t L = d.cu_host ? (int64_t)d.cu_host[b + 1] - d.cu_host[b] : d.max_len;
+      const int64_t w = std::min(L, (s + 1) * per) - s * per;
+      const int64_t c = w > 0 ? w + kStart : kEmpty;
+      for (int h = 0; h < d.Hkv; ++h) {
+        const int64_t t = free_at.top() + c;
+        free_at.pop();
+        free_at.push(t);
+        end = std::max(end, t);
+      }
+    }
+  return end;
+}
+
+}  // namespace
+
 AttendPlan plan_attend(const Dims& d, int64_t max_rows_per_seq, bool dense) {
+  const int64_t maxl = max_rows_per_seq > 0 ? max_rows_per_seq : 1;
+  if (dense && d.bf16 && padded_group(d.G) <= 8 && d.num_sms > 0) {
+    // tensor-core dense: 128-row stages, one CTA per SM.  Split lengths for
+    // 1, 2, 3, 4, 6 or 8 waves of the rows' CTAs; the shortest simulated
+    // makespan wins (equal lengths fill one wave exactly, ragged ones need
+    // shorter splits to spread the long rows)
+    const int64_t rows = std::max<int64_t>(1, (int64_t)d.B * d.Hkv);
+    AttendPlan best{1, (int)(cdiv(maxl, 128) * 128)};
+    if (rows >= 8LL * d.num_sms) return best;  // one CTA per row: many waves already
+    int64_t best_t = -1;
+    for (int w : {1, 2, 3, 4, 6, 8}) {
+      const int64_t s0 = std::max<int64_t>(1, (int64_t)w * d.num_sms / rows);
+      int64_t per = cdiv(cdiv(maxl, s0), 128) * 128;
+      const int64_t splits = cdiv(maxl, per);
+      const int64_t t = tc_makespan(d, per, splits);
+      if (best_t < 0 || t < best_t) {
+        best_t = t;
+        best = AttendPlan{(int)splits, (int)per};
+      }
+    }
+    return best;
+  }
   // rows one CTA covers per iteration: a sparse pass step (bf16, d = 128), or
   // a dense stage (the largest, fp32 d = 64: 64 rows, so every dtype's
   // stage divides it)

@@ -2,6 +2,8 @@
 // the C ABI layer (prism_api.cu) before any of these is called.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -24,6 +26,9 @@ struct Dims {
 // Query-group sizes a kernel is instantiated for; a group of G query heads
 // runs on the smallest instantiation >= G with the extra heads masked.
 inline int padded_group(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : G <= 8 ? 8 : 16; }
+
+// cuTensorMapEncodeTiled from the driver, looked up once (null if missing)
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 cudaError_t launch_append(const Dims& d, const void* k_new, const void* v_new, void* k_cache,
                           void* v_cache, cudaStream_t st);
