@@ -423,7 +423,10 @@ def test_sparse_decode_vs_oracle(P, case):
 
 
 @pytest.mark.parametrize("case", [([1024], 4, 1, 64, "f32"), ([5000, 1031, 0, 300], 8, 2, 128, "bf16"),
-                                  ([20000], 32, 8, 128, "bf16"), ([999], 16, 1, 64, "bf16")],
+                                  ([20000], 32, 8, 128, "bf16"), ([999], 16, 1, 64, "bf16"),
+                                  ([70000, 3, 129, 12345], 16, 2, 128, "bf16"),
+                                  ([4097, 1], 8, 8, 64, "bf16"), ([3000, 200], 6, 3, 128, "bf16"),
+                                  ([2000], 32, 2, 128, "bf16")],
                          ids=lambda c: f"{c[0]}-{c[1]}/{c[2]}-d{c[3]}-{c[4]}")
 def test_dense_decode_vs_oracle(P, case):
     seqlens, hq, hkv, d, dtype = case
@@ -440,6 +443,30 @@ def test_dense_decode_vs_oracle(P, case):
     assert np.abs(_np(out) - oout).max() <= tol
     fin = np.isfinite(olse)
     assert np.abs(_np(lse)[fin] - olse[fin]).max() <= tol * 10
+
+
+def test_dense_decode_ignores_rows_past_the_end(P):
+    """Cache rows past a sequence's end (the next sequence's, and spare rows
+    holding NaN) share the dense pass's 128-row stages with the last valid
+    rows: they carry no weight and their bytes never reach the output."""
+    seqlens, hq, hkv, d = [1000, 777], 8, 2, 128
+    cap = 2000
+    prob = P.Problem(seqlens, hq, hkv, d, P.BF16, device=DEV, capacity=cap)
+    q, k0, v0 = make_case(seqlens, hq, hkv, d, "bf16", seed=12)
+    k = torch.full((hkv, cap, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    v = torch.full((hkv, cap, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    k[:, :1777], v[:, :1777] = k0, v0
+    out = torch.zeros((2, hq, d), device=DEV)
+    lse = torch.zeros((2, hq), device=DEV)
+    scale = float(np.float32(1 / math.sqrt(d)))
+    ws = ws_for(P, prob, P.OP_DENSE_DECODE)
+    P.dense_decode(prob, q, k, v, scale, out, ws, lse=lse)
+    torch.cuda.synchronize()
+    assert P.get_device_status(ws) == 0
+    oout, olse = pipeline.attend_layer(q, k0, v0, [0, 1000, 1777], None, None, scale)
+    assert np.all(np.isfinite(_np(out)))
+    assert np.abs(_np(out) - oout).max() <= atol_for("bf16")
+    assert np.abs(_np(lse) - olse).max() <= atol_for("bf16") * 10
 
 
 def test_full_budget_sparse_equals_dense(P):
@@ -710,31 +737,39 @@ def test_refine_decode_large_ties(P, kp, kap):
 
 
 SELECT_CASES = [
-    # (seqlens, Hq, Hkv, d, kappa_p, kappa, integer keys): the c128k row
-    # shape, a ragged batch with an empty and a short sequence, pools of
-    # 8192 and 8193 members, and integer keys (many exactly equal scores at
-    # the threshold, resolved by the lower position)
-    ([131072], 32, 8, 128, 8192, 2048, False),
-    ([40000, 9000, 0, 300, 12300], 32, 8, 128, 4096, 1024, False),
-    ([30000], 8, 2, 128, 8192, 3000, False),
-    ([30000], 8, 2, 128, 8193, 3000, False),
-    ([20000, 7000], 32, 8, 128, 8192, 2048, True),
-    ([2000], 4, 1, 64, 256, 64, True),
+    # (seqlens, Hq, Hkv, d, kappa_p, kappa, keys): the c128k row shape, a
+    # ragged batch with an empty and a short sequence, pools of 8192 and 8193
+    # members; "int": small integer keys (many exactly equal scores at the
+    # threshold, resolved by the lower position: a few per value in the
+    # small pool, where they are ranked from the exchanged lists, hundreds in
+    # the large one, where the radix digits resolve them); "outlier": one
+    # position in 997 has its key row scaled by 512, so the value range is
+    # wide and the threshold's window bin crowded (the radix fallback)
+    ([131072], 32, 8, 128, 8192, 2048, "normal"),
+    ([40000, 9000, 0, 300, 12300], 32, 8, 128, 4096, 1024, "normal"),
+    ([30000], 8, 2, 128, 8192, 3000, "normal"),
+    ([30000], 8, 2, 128, 8193, 3000, "normal"),
+    ([20000, 7000], 32, 8, 128, 8192, 2048, "int"),
+    ([2000], 4, 1, 64, 256, 64, "int"),
+    ([30000], 8, 2, 128, 8192, 2048, "outlier"),
+    ([3000, 5000], 8, 2, 128, 1024, 256, "outlier"),
 ]
 
 
-@pytest.mark.parametrize("case", SELECT_CASES, ids=lambda c: f"{len(c[0])}seq-kp{c[4]}-k{c[5]}-int{int(c[6])}")
+@pytest.mark.parametrize("case", SELECT_CASES, ids=lambda c: f"{len(c[0])}seq-kp{c[4]}-k{c[5]}-{c[6]}")
 def test_refine_decode_selection_cases(P, case):
     """The fused refined layer's exact top-kappa on the shapes and score
     distributions above, against the oracle; attention on the GPU's set."""
-    seqlens, hq, hkv, d, kp, kap, integer = case
+    seqlens, hq, hkv, d, kp, kap, keys = case
     B = len(seqlens)
     prob = problem(P, seqlens, hq, hkv, d, "bf16")
     q, k, v = make_case(seqlens, hq, hkv, d, "bf16", seed=31)
-    if integer:  # small integer keys and queries: exact, often equal, scores
+    if keys == "int":  # small integer keys and queries: exact, often equal, scores
         g = torch.Generator(device="cpu").manual_seed(32)
         k.copy_(torch.randint(-2, 3, k.shape, generator=g).to(k.dtype).to(DEV))
         q.copy_(torch.randint(-1, 2, q.shape, generator=g).to(q.dtype).to(DEV))
+    elif keys == "outlier":  # exact in bf16: a power of two
+        k[:, ::997] *= 512
     rng = np.random.default_rng(33)
     pool = np.full((B, hkv, kp), -1, np.int32)
     pcnt = np.zeros((B, hkv), np.int32)
