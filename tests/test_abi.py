@@ -169,3 +169,37 @@ def test_propose_topk_and_overlap_reject_bad_arguments(prism_lib):
     assert ov(-1, f, f, 8, f, f, 8, f, None) == P.ERR_INVALID_ARG
     assert ov(4, None, f, 8, f, f, 8, f, None) == P.ERR_INVALID_ARG
     assert ov(0, None, None, 8, None, None, 8, None, None) == P.OK  # nothing to do
+
+
+def _dense_splits(P, seqlens, hq=32, hkv=8, d=128, dtype=1):
+    """Split count of the dense plan, read back from its workspace size:
+    a 256-byte header, then partial o [B][Hq][splits][d] and (m, l)
+    [B][Hq][splits][2] fp32, each padded to 256 bytes."""
+    s, _ = _shape(P, seqlens, hq, hkv, d, dtype)
+    st, n = _ws(P, s, P.OP_DENSE_DECODE)
+    assert st == P.OK
+    per_split = len(seqlens) * hq * (d + 2) * 4
+    splits = (n - 256) // per_split
+    assert 0 <= (n - 256) - splits * per_split < 512  # the two paddings
+    return splits
+
+
+def test_dense_split_plan(prism_lib):
+    """The tensor-core dense kernel runs one CTA per SM (148 planned): equal
+    lengths fill one wave of whole 128-row stages; a ragged batch gets
+    shorter splits than one wave would give its longest row, so the long rows
+    spread over several SMs; fp32 caches keep the staged kernel's two CTAs
+    per SM."""
+    P = prism_lib
+    # c128k: 8 rows, one wave -> floor(148 / 8) = 18 splits of 7296 positions
+    assert _dense_splits(P, [131072]) == 18
+    # four equal rows of 32768 (32 rows): ceil(32768 / splits) rounded to 128
+    sp = _dense_splits(P, [32768] * 4)
+    assert 4 <= sp <= 37
+    # ragged: a long row among short ones is cut into more pieces than the
+    # one-wave plan (148 // 128 = 1 split) would give it
+    rng = np.random.default_rng(5)
+    ragged = [int(x) for x in rng.integers(4096, 65537, 16)]
+    assert _dense_splits(P, ragged) > 1
+    # fp32: two CTAs per SM over 8 rows -> ceil(296 / 8) = 37 splits
+    assert _dense_splits(P, [131072], dtype=0) == 37
