@@ -361,7 +361,11 @@ PRISM_API prism_status prism_refine_decode(const prism_shape* shape, const void*
 
 /*
  * Dense decode attention over every position t < L_b (the comparison path):
- * the same definition as prism_sparse_decode with idx = 0 .. L_b - 1.
+ * the same definition as prism_sparse_decode with idx = 0 .. L_b - 1.  A
+ * bf16 cache with up to 8 query heads per KV head runs on tensor cores,
+ * split along t by a plan made from every sequence's length (host copy of
+ * cu_seqlens): the workspace (prism_workspace_size, PRISM_OP_DENSE_DECODE)
+ * must be sized with the lengths of the call.  q, k and v 16-byte aligned.
  */
 PRISM_API prism_status prism_dense_decode(const prism_shape* shape, const void* q, const void* k,
                                 const void* v, float softmax_scale, float* out, float* lse_opt,
