@@ -536,27 +536,30 @@ def run_prism(args, dist: Dist):
     ms_per_step = secs * 1e3 / args.steps
     value = dist.world * args.steps / secs
 
-    # ---- end to end: pinned host inputs in, outputs out, every step
-    q_h = torch.empty(q_all.shape, dtype=q_all.dtype).pin_memory()
-    q_h.copy_(q_all)
-    kn_h = torch.empty(k_new.shape, dtype=k_new.dtype).pin_memory()
-    kn_h.copy_(k_new)
-    vn_h = torch.empty(v_new.shape, dtype=v_new.dtype).pin_memory()
-    vn_h.copy_(v_new)
-    out_h = torch.empty(dec.out_all.shape, dtype=torch.float32).pin_memory()
+    # ---- end to end: pinned host inputs in, outputs out, every step, through
+    # PrismDecoder.step_host: one copy per proposal group each way, on a copy
+    # stream while the other groups run; one captured graph per step, like
+    # the device-resident step
+    io = dec.host_io(q_all.dtype)
+    for l in range(L):
+        io.q_host[l].copy_(q_all[l])
+        io.k_new_host[l].copy_(k_new[l])
+        io.v_new_host[l].copy_(v_new[l])
+    copy_stream = torch.cuda.Stream()
 
-    def e2e_step():
-        q_all.copy_(q_h, non_blocking=True)
-        k_new.copy_(kn_h, non_blocking=True)
-        v_new.copy_(vn_h, non_blocking=True)
-        g.replay()
-        out_h.copy_(dec.out_all, non_blocking=True)
+    def e2e_body():
+        if args.grow:
+            dec.advance_on_device(1)
+        dec.step_host(io, ks, vs, kqs, scs, copy_stream, quantize_new=True)
+
+    g_e2e = graph_of(e2e_body, stream)
+    e2e_step = g_e2e.replay
 
     e2e_steps = max(10, args.steps // 2)
     e2e_secs = dist.max(timed(e2e_step, e2e_steps, args.warmup))
-    h2d = (q_h.numel() * q_h.element_size() + kn_h.numel() * kn_h.element_size()
-           + vn_h.numel() * vn_h.element_size())
-    d2h = out_h.numel() * out_h.element_size()
+    h2d = sum(t.numel() * t.element_size() for t in io.q_host + io.k_new_host + io.v_new_host)
+    d2h = io.out_host.numel() * io.out_host.element_size()
+    del g_e2e
 
     if args.grow:
         dec.lengths_from_device()  # the dense comparison sizes its splits from the host copy

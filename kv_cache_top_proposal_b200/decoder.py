@@ -186,6 +186,48 @@ class PrismDecoder:
                        v_new=None if v_new is None else v_new[l],
                        overlap=self.fused and not pl and l > 0, stream=stream)
 
+    def host_io(self, dtype=torch.bfloat16) -> "HostIO":
+        """Page-locked host buffers for step_host, with their device twins."""
+        return HostIO(self, dtype)
+
+    def step_host(self, io: "HostIO", ks, vs, kqs, scales, copy_stream, quantize_new: bool = True):
+        """One decode step whose token inputs start, and whose outputs end,
+        in page-locked host memory: the caller writes this token's rows into
+        io.q_host / io.k_new_host / io.v_new_host and reads io.out_host
+        after the step.  The copies move a proposal group (`group` layers)
+        at a time, one copy per group each way, and meet the layers only at
+        group boundaries, where the step has no overlapped launch to lose:
+          - the first group's rows go up on the current stream, the other
+            groups' on copy_stream meanwhile, awaited by the second group;
+          - each group's outputs go down on copy_stream once its last layer
+            ends, while the next group runs.
+        The current stream joins copy_stream at the end, so the whole step can
+        be captured in one CUDA graph."""
+        main = torch.cuda.current_stream()
+        L, gsz = self.num_layers, self.group
+        io.dev_in[0].copy_(io.host_in[0], non_blocking=True)
+        copy_stream.wait_stream(main)
+        up = torch.cuda.Event()
+        if io.groups > 1:
+            with torch.cuda.stream(copy_stream):
+                io.dev_in[1:].copy_(io.host_in[1:], non_blocking=True)
+                up.record(copy_stream)
+        for l in range(L):
+            pl = l % gsz == 0
+            if l == gsz:
+                main.wait_event(up)
+            self.layer(l, io.q_dev[l], ks[l], vs[l], kqs[l] if pl else None, scales[l] if pl else None,
+                       quantize_new=quantize_new, k_new=io.k_new_dev[l], v_new=io.v_new_dev[l],
+                       overlap=self.fused and not pl and l > 0)
+            if (l + 1) % gsz == 0 or l + 1 == L:  # the group's outputs go down
+                done = torch.cuda.Event()
+                done.record(main)
+                copy_stream.wait_event(done)
+                l0 = l - l % gsz
+                with torch.cuda.stream(copy_stream):
+                    io.out_host[l0:l + 1].copy_(self.out_all[l0:l + 1], non_blocking=True)
+        main.wait_stream(copy_stream)
+
     def grow(self, n: int = 1):
         """Decode loop over one growing sequence: the last sequence gets n more
         tokens (the next step appends its token at the new last position).
@@ -251,3 +293,37 @@ class PrismDecoder:
         for w in self.workspaces():
             s |= prism.get_device_status(w)
         return s
+
+
+class HostIO:
+    """Host-side inputs and outputs of PrismDecoder.step_host.  Per proposal
+    group, one contiguous page-locked block holds its layers' q, then k_new,
+    then v_new rows (so one copy moves a group's inputs), mirrored by a
+    device block; q_host[l] ([B][Hq][d]), k_new_host[l] / v_new_host[l]
+    ([B][Hkv][d]) and their *_dev twins are views into them.  out_host
+    ([L][B][Hq][d] fp32, page-locked) receives every layer's output."""
+
+    def __init__(self, dec: PrismDecoder, dtype=torch.bfloat16):
+        L, gsz, B, Hq, Hkv, D = dec.num_layers, dec.group, dec.B, dec.Hq, dec.Hkv, dec.D
+        es = torch.tensor([], dtype=dtype).element_size()
+        nq, nk = B * Hq * D * es, B * Hkv * D * es  # bytes of one layer's q, k_new rows
+        self.groups = (L + gsz - 1) // gsz
+        blk = gsz * (nq + 2 * nk)
+        self.host_in = torch.zeros((self.groups, blk), dtype=torch.uint8).pin_memory()
+        self.dev_in = torch.zeros((self.groups, blk), dtype=torch.uint8, device=dec.dev)
+
+        def views(buf):
+            q, kn, vn = [], [], []
+            for l in range(L):
+                gi, j = divmod(l, gsz)
+                row = buf[gi]
+                q.append(row[j * nq:(j + 1) * nq].view(dtype).view(B, Hq, D))
+                o = gsz * nq + j * nk
+                kn.append(row[o:o + nk].view(dtype).view(B, Hkv, D))
+                o = gsz * (nq + nk) + j * nk
+                vn.append(row[o:o + nk].view(dtype).view(B, Hkv, D))
+            return q, kn, vn
+
+        self.q_host, self.k_new_host, self.v_new_host = views(self.host_in)
+        self.q_dev, self.k_new_dev, self.v_new_dev = views(self.dev_in)
+        self.out_host = torch.zeros((L, B, Hq, D), dtype=torch.float32).pin_memory()

@@ -487,3 +487,55 @@ def test_step_selection_granularity_every_row(prism_lib, name, sets):
                                                     dec.scale)
         assert np.abs(_np(dec.out[l]) - oout).max() <= tol, l
         assert np.abs(_np(dec.lse[l]) - olse).max() <= 10 * tol, l
+
+
+@pytest.mark.parametrize("name", ["c8k", "ragged16"])
+def test_step_host_matches_device_step(prism_lib, name):
+    """PrismDecoder.step_host (the token's rows from page-locked host memory,
+    the outputs back to it, one copy per proposal group each way on a side
+    stream) in one captured graph gives bit for bit the outputs of the
+    device-resident step on the same inputs, over two groups; replayed
+    twice."""
+    P = prism_lib
+    full = workload.config(name)
+    cfg = full.replace(num_layers=full.group * 2)
+    layers = list(workload.generate(cfg, DEV))
+    cu = cfg.cu_seqlens
+    nz = [b for b in range(cfg.batch) if cu[b + 1] > cu[b]]
+    rows = torch.tensor([cu[b + 1] - 1 for b in nz], dtype=torch.long, device=DEV)
+    k_new = torch.stack([lay.k[:, rows].transpose(0, 1).contiguous() for lay in layers])
+    v_new = torch.stack([lay.v[:, rows].transpose(0, 1).contiguous() for lay in layers])
+    q_all = torch.stack([lay.q for lay in layers])
+    ks, vs = [x.k for x in layers], [x.v for x in layers]
+    dec = PrismDecoder(cfg.seqlens, cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim, P.BF16,
+                       cfg.num_layers, cfg.group, cfg.kappa_p, cfg.kappa, device=DEV,
+                       capacity=cfg.total_tokens)
+    kqs, scs = {}, {}
+    for lay in layers:
+        if cfg.is_proposal(lay.index):
+            kqs[lay.index], scs[lay.index] = _prefill_kq(P, dec, cfg, lay)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        dec.step([q_all[l] for l in range(cfg.num_layers)], ks, vs, kqs, scs, quantize_new=True,
+                 k_new=k_new, v_new=v_new)
+    torch.cuda.synchronize()
+    ref = dec.out_all.clone()
+    io = dec.host_io()
+    for l in range(cfg.num_layers):
+        io.q_host[l].copy_(q_all[l])
+        io.k_new_host[l].copy_(k_new[l])
+        io.v_new_host[l].copy_(v_new[l])
+    cs = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        dec.step_host(io, ks, vs, kqs, scs, cs)
+    for rep in range(2):
+        io.out_host.fill_(55.0)
+        dec.out_all.fill_(-3.0)
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        assert dec.device_status() == 0
+        assert torch.equal(io.out_host, ref.cpu()), rep
+    del g, layers, dec
+    torch.cuda.empty_cache()
