@@ -176,6 +176,41 @@ def refine_row(q, K, pool, kappa: int, agg: str = "max"):
     return idx[:m].copy(), r[:n].copy()
 
 
+def refine_scores_mass(q, K, pool, softmax_scale: float) -> np.ndarray:
+    """Group aggregation by softmax mass (the third reading of how the G query
+    heads of a KV head share one set; Prism Attention sec. 4.1 and sec. 6
+    leave it open): a pool member's score is the attention mass the group's
+    heads put on it, each head's softmax taken over the pool,
+        l_g,i = softmax_scale * (q_g . K[pool_i])     the dot product fp32,
+                                                      j ascending (the
+                                                      one-head exact score)
+        r_i   = sum_g exp(l_g,i - max_i' l_g,i') / sum_i' exp(l_g,i' - max_i' l_g,i')
+    in fp64 after the dot products, g ascending.  Returns r (fp64)."""
+    q, K, pool = _f32(q), _f32(K), _i32(pool)
+    G = q.shape[0]
+    n = pool.size
+    r = np.zeros(n, np.float64)
+    if n == 0:
+        return r
+    for g in range(G):
+        dots = refine_scores(q[g:g + 1], K, pool).astype(np.float64)  # exact fp32 dot products
+        lg = float(softmax_scale) * dots
+        e = np.exp(lg - lg.max())
+        r += e / e.sum()
+    return r
+
+
+def refine_row_mass(q, K, pool, kappa: int, softmax_scale: float):
+    """(refined positions ascending int32 [min(kappa, |pool|)], masses fp64):
+    the top min(kappa, |pool|) members by softmax mass, ties to the lower
+    pool slot (the lower position, as the pool is ascending)."""
+    pool = _i32(pool)
+    r = refine_scores_mass(q, K, pool, softmax_scale)
+    order = sorted(range(pool.size), key=lambda i: (-r[i], i))
+    take = sorted(order[:min(kappa, pool.size)])
+    return pool[np.array(take, np.int64)].astype(np.int32) if take else np.zeros(0, np.int32), r
+
+
 def attend(q, K, V, idx, softmax_scale: float):
     """fp64 softmax attention of one query head over rows idx (None = all rows)."""
     q, K, V = _f32(q), _f32(K), _f32(V)

@@ -27,7 +27,7 @@ from typing import Dict, List, Optional
 import numpy as np
 
 from . import (attend, pool_topk, propose_row, propose_row_int2, propose_row_seq, quantize_int2_rows,
-               quantize_rows, refine_row, refine_row_heads, refine_row_seq)
+               quantize_rows, refine_row, refine_row_heads, refine_row_mass, refine_row_seq)
 
 
 def _np(x):
@@ -104,9 +104,11 @@ def propose_layer_int2(q, codes, params, cu, kappa_p: int, rows=None):
     return pool, cnt, scores
 
 
-def refine_layer(q, k, cu, pool, pool_cnt, kappa: int, rows=None, agg: str = "max"):
+def refine_layer(q, k, cu, pool, pool_cnt, kappa: int, rows=None, agg: str = "max",
+                 softmax_scale: Optional[float] = None):
     """idx [B][Hkv][kappa] (-1 padded), cnt [B][Hkv], exact pool scores per row
-    (agg as in propose_layer)."""
+    (agg as in propose_layer, or "mass": the group's softmax mass over the
+    pool at softmax_scale, default 1/sqrt(d))."""
     q = _np(q).astype(np.float32)
     k = _np(k).astype(np.float32)
     pool, pool_cnt = _np(pool), _np(pool_cnt)
@@ -122,7 +124,11 @@ def refine_layer(q, k, cu, pool, pool_cnt, kappa: int, rows=None, agg: str = "ma
             if rows is not None and (b, h) not in rows:
                 continue
             n = int(pool_cnt[b, h])
-            sel, r = refine_row(q[b, h * G:(h + 1) * G], k[h, t0:t1], pool[b, h, :n], kappa, agg)
+            if agg == "mass":
+                sc = float(np.float32(1.0 / math.sqrt(d))) if softmax_scale is None else softmax_scale
+                sel, r = refine_row_mass(q[b, h * G:(h + 1) * G], k[h, t0:t1], pool[b, h, :n], kappa, sc)
+            else:
+                sel, r = refine_row(q[b, h * G:(h + 1) * G], k[h, t0:t1], pool[b, h, :n], kappa, agg)
             idx[b, h, :sel.size] = sel
             cnt[b, h] = sel.size
             scores[(b, h)] = r
