@@ -53,7 +53,7 @@ def parse():
     ap.add_argument("--profile-steps", type=int, default=5)
     ap.add_argument("--keys", default="int8", choices=["int8", "int2"],
                     help="proposal key cache: int8 per token (the headline workload) or INT2 per 32-feature group")
-    ap.add_argument("--group-agg", default="max", choices=["max", "sum"],
+    ap.add_argument("--group-agg", default="max", choices=["max", "sum", "mass"],
                     help="how the query heads of a KV head combine into the selection score")
     ap.add_argument("--proposal-select", default="exact", choices=["exact", "quantized"],
                     help="what a proposal layer attends over: its own pool refined with exact scores "
@@ -266,11 +266,14 @@ def unit_run(cfg, u, keys: str = "int8", agg: str = "max", proposal_select: str 
         if keys == "int2":
             pool, ps = oracle.propose_row_int2(host[lp][0][b], kq[a:e], sc[a:e], cfg.kappa_p)
         else:
-            pool, ps = oracle.propose_row(host[lp][0][b], kq[a:e], sc[a:e], cfg.kappa_p, agg=agg)
+            pool, ps = oracle.propose_row(host[lp][0][b], kq[a:e], sc[a:e], cfg.kappa_p,
+                                          agg="max" if agg == "mass" else agg)
         for l in u["lays"]:
             q, k, v = host[l]
             if l == lp and proposal_select == "quantized":
                 idx = oracle.pool_topk(ps, pool, cfg.kappa)
+            elif agg == "mass":
+                idx, _ = oracle.refine_row_mass(q[b], k[a:e], pool, cfg.kappa, scale)
             else:
                 idx, _ = oracle.refine_row(q[b], k[a:e], pool, cfg.kappa, agg=agg)
             for g in range(G):
@@ -405,7 +408,8 @@ def line_config(cfg, args, seqlens0=None, n_grow=0):
                     f"write between steps outside its event pair; {touched}") if needs_flush(nbytes)
                 else f"inputs larger than L2: {touched}",
                 refined_layers="fused refine+select+sparse-decode (prism_refine_decode)"
-                if args.sets == "kv_head" else "refine and sparse decode (two calls)",
+                if args.sets == "kv_head" and args.group_agg != "mass"
+                else "refine and sparse decode (two calls)",
                 proposal_select=args.proposal_select, selection_sets=args.sets,
                 proposal_keys="int8 per token" if args.keys == "int8"
                 else "INT2 per 32-feature group (fp16 step and zero point)",
@@ -564,7 +568,7 @@ def run_prism(args, dist: Dist):
     if args.grow:
         dec.lengths_from_device()  # the dense comparison sizes its splits from the host copy
 
-    variant = args.sets != "kv_head" or args.proposal_select != "exact"
+    variant = args.sets != "kv_head" or args.proposal_select != "exact" or args.group_agg == "mass"
     if not variant:
         # ---- per-op durations (one graph per op; the queue is filled behind a
         # long memset so every event pair brackets device time only)

@@ -244,6 +244,26 @@ PRISM_API prism_status prism_refine(const prism_shape* shape, const void* q, con
                           void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Refined selection by softmax mass (sec. 4.1 and sec. 6 leave open how the
+ * G query heads of a KV head share one set; this is the third reading next
+ * to the maximum and the sum): for each (sequence, KV head) row and each
+ * pool member i, with l_g,i = softmax_scale * q_g . K[pool_i] (the exact fp32
+ * per-head score),
+ *   r_i = sum_g exp(l_g,i - max_i' l_g,i') / sum_i' exp(l_g,i' - max_i' l_g,i'),
+ * the attention mass the group puts on the member, each head's softmax over
+ * the pool.  idx / cnt as prism_refine: the top min(kappa, n) members by r_i,
+ * ties to the lower pool slot, positions ascending, -1 padded.  The masses
+ * are fp32 (the oracle's fp64), so sets agree with it up to near-ties.
+ * Workspace: PRISM_OP_REFINE with the same kappa_p, kappa.  softmax_scale
+ * finite and > 0 (else PRISM_ERR_INVALID_ARG); other errors as prism_refine.
+ */
+PRISM_API prism_status prism_refine_mass(const prism_shape* shape, const void* q, const void* k,
+                                         const int32_t* pool_idx, const int32_t* pool_cnt,
+                                         int32_t kappa_p, int32_t kappa, float softmax_scale,
+                                         int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes,
+                                         void* stream);
+
+/*
  * Selection granularity (sec. 4.1 shares index sets under GQA without saying
  * at which granularity; sec. 3 analyses attention per head; sec. 2 "Related
  * Work" names a set shared by all heads).  The plain calls use one pool and

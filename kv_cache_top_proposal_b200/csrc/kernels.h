@@ -97,6 +97,10 @@ cudaError_t launch_select(const Dims& d, const SelectArgs& a, int max_row_len, c
 // Exact pool scores r[row][i] = max_g q_g . K[pool_i] (+ per-head dots);
 // row (b, h) reads pool row (b * Hkv + h) / pool_div (pool_div = Hkv: one
 // pool per sequence shared by its KV heads).
+// Softmax mass of every pool member over the G query heads of its row, in
+// place of r (refine.cu); dots [rows][G][pool_stride] from launch_refine_scores.
+cudaError_t launch_refine_mass(const Dims& d, float* r, const float* dots, const int32_t* pool_cnt,
+                               int pool_stride, float softmax_scale, cudaStream_t st);
 cudaError_t launch_refine_scores(const Dims& d, const void* q, const void* k, const int32_t* pool,
                                  const int32_t* pool_cnt, int pool_stride, float* r, float* dots,
                                  int32_t* status, cudaStream_t st, int pool_div = 1);

@@ -419,6 +419,47 @@ prism_status prism_propose_ex(const prism_shape* shape, const void* q, const int
   return cuda_status(launch_select(d1, a, d.max_len, st));
 }
 
+prism_status prism_refine_mass(const prism_shape* shape, const void* q, const void* k,
+                               const int32_t* pool_idx, const int32_t* pool_cnt, int32_t kappa_p,
+                               int32_t kappa, float softmax_scale, int32_t* idx, int32_t* cnt, void* ws,
+                               size_t ws_bytes, void* stream) {
+  Dims d;
+  prism_status s = check_shape(shape, &d);
+  if (s != PRISM_OK) return s;
+  if (!q || !k || !pool_idx || !pool_cnt || !idx || !cnt) return PRISM_ERR_INVALID_ARG;
+  if (kappa_p < 1 || kappa < 1 || kappa > kappa_p) return PRISM_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale) || softmax_scale <= 0.0f) return PRISM_ERR_INVALID_ARG;
+  if (kappa_p > select_capacity_per_row()) return PRISM_ERR_UNSUPPORTED;
+  const Layout L = layout(d, PRISM_OP_REFINE, kappa_p, kappa);
+  if (!ws_ok(ws, ws_bytes, L)) return PRISM_ERR_WORKSPACE;
+  if ((s = set_live_sms(&d)) != PRISM_OK) return s;
+  char* w = static_cast<char*>(ws);
+  int32_t* status = reinterpret_cast<int32_t*>(w);
+  float* r = reinterpret_cast<float*>(w + L.a);
+  float* dots = reinterpret_cast<float*>(w + L.b);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_refine_scores(d, q, k, pool_idx, pool_cnt, kappa_p, r, dots, status, st);
+  if (e != cudaSuccess) return PRISM_ERR_CUDA;
+  if ((e = launch_refine_mass(d, r, dots, pool_cnt, kappa_p, softmax_scale, st)) != cudaSuccess)
+    return PRISM_ERR_CUDA;
+  SelectArgs a{};
+  a.mode = 1;
+  a.Hkv = d.Hkv;
+  a.G = d.G;
+  a.Hq = d.Hq;
+  a.T = d.T;
+  a.cu = d.cu_dev;
+  a.keys = r;
+  a.pool = pool_idx;
+  a.pool_cnt = pool_cnt;
+  a.pool_stride = kappa_p;
+  a.k_req = kappa;
+  a.out = idx;
+  a.out_cnt = cnt;
+  a.status = status;
+  return cuda_status(launch_select(d, a, kappa_p, st));
+}
+
 prism_status prism_refine_ex(const prism_shape* shape, const void* q, const void* k,
                              const int32_t* pool_idx, const int32_t* pool_cnt, int32_t kappa_p,
                              int32_t kappa, int32_t* idx, int32_t* cnt, uint32_t sets, void* ws,

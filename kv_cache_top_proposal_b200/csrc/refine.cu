@@ -167,6 +167,73 @@ __global__ void __launch_bounds__(kThreads) pool_gather_kernel(const float* __re
   }
 }
 
+// Softmax-mass aggregation of a row's pool members (the group's G query
+// heads share one set; each member's score is the attention mass the heads
+// put on it, each head's softmax over the pool):
+//   r_i <- sum_g 2^((d_g,i - M_g) c) / sum_i' 2^((d_g,i' - M_g) c),
+// c = softmax_scale * log2 e, M_g the largest d_g over the row's members.
+// Members flagged by the scoring pass (r_i = -inf) take no part and stay
+// -inf.  One CTA per row; dots [row][G][stride] from the scoring pass.
+template <int GP>
+__global__ void __launch_bounds__(kThreads) mass_kernel(float* __restrict__ r, const float* __restrict__ dots,
+                                                        const int32_t* __restrict__ pool_cnt, int stride,
+                                                        int G, float c) {
+  __shared__ float s_a[kWarps][GP];
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int n = pool_cnt[row];
+  n = n < 0 ? 0 : (n > stride ? stride : n);
+  float* rr = r + (int64_t)row * stride;
+  const float* dr = dots + (int64_t)row * G * stride;
+  // the whole CTA's value of v per head, through the warps
+  auto reduce = [&](float (&v)[GP], bool is_max) {
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float x = __shfl_xor_sync(0xffffffffu, v[g], o);
+        v[g] = is_max ? fmaxf(v[g], x) : v[g] + x;
+      }
+      if (lane == 0) s_a[warp][g] = v[g];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      float t = s_a[0][g];
+#pragma unroll
+      for (int w = 1; w < kWarps; ++w) t = is_max ? fmaxf(t, s_a[w][g]) : t + s_a[w][g];
+      v[g] = t;
+    }
+    __syncthreads();
+  };
+  float m[GP], z[GP];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    m[g] = -INFINITY;
+    z[g] = 0.0f;
+  }
+  for (int i = tid; i < n; i += kThreads)
+    if (rr[i] != -INFINITY)
+#pragma unroll
+      for (int g = 0; g < GP; ++g)
+        if (g < G) m[g] = fmaxf(m[g], dr[(int64_t)g * stride + i]);
+  reduce(m, true);
+  for (int i = tid; i < n; i += kThreads)
+    if (rr[i] != -INFINITY)
+#pragma unroll
+      for (int g = 0; g < GP; ++g)
+        if (g < G) z[g] += exp2f((dr[(int64_t)g * stride + i] - m[g]) * c);
+  reduce(z, false);
+  for (int i = tid; i < n; i += kThreads) {
+    if (rr[i] == -INFINITY) continue;
+    float mass = 0.0f;
+#pragma unroll
+    for (int g = 0; g < GP; ++g)
+      if (g < G) mass += exp2f((dr[(int64_t)g * stride + i] - m[g]) * c) / z[g];
+    rr[i] = mass;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_pool_gather(const Dims& d, const float* scores, const int32_t* pool,
@@ -189,6 +256,25 @@ cudaError_t launch_refine_scores(const Dims& d, const void* q, const void* k, co
   if (d.bf16)
     return d.D == 128 ? by_group<__nv_bfloat16, 128>(d, a, st) : by_group<__nv_bfloat16, 64>(d, a, st);
   return d.D == 128 ? by_group<float, 128>(d, a, st) : by_group<float, 64>(d, a, st);
+}
+
+}  // namespace prism
+
+namespace prism {
+
+cudaError_t launch_refine_mass(const Dims& d, float* r, const float* dots, const int32_t* pool_cnt,
+                               int pool_stride, float softmax_scale, cudaStream_t st) {
+  const int rows = d.B * d.Hkv;
+  if (rows == 0 || pool_stride == 0) return cudaSuccess;
+  const float c = softmax_scale * 1.4426950408889634f;
+  switch (padded_group(d.G)) {
+    case 1: mass_kernel<1><<<rows, kThreads, 0, st>>>(r, dots, pool_cnt, pool_stride, d.G, c); break;
+    case 2: mass_kernel<2><<<rows, kThreads, 0, st>>>(r, dots, pool_cnt, pool_stride, d.G, c); break;
+    case 4: mass_kernel<4><<<rows, kThreads, 0, st>>>(r, dots, pool_cnt, pool_stride, d.G, c); break;
+    case 8: mass_kernel<8><<<rows, kThreads, 0, st>>>(r, dots, pool_cnt, pool_stride, d.G, c); break;
+    default: mass_kernel<16><<<rows, kThreads, 0, st>>>(r, dots, pool_cnt, pool_stride, d.G, c); break;
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace prism

@@ -57,7 +57,9 @@ class PrismDecoder:
         self.sets = sets
         self.sets_code = {"kv_head": prism.SETS_KV_HEAD, "q_head": prism.SETS_Q_HEAD,
                           "sequence": prism.SETS_SEQUENCE}[sets]
-        if sets != "kv_head":
+        # "mass": the refined layers select by the group's softmax mass over
+        # the pool (prism_refine_mass, then the sparse decode: two calls)
+        if sets != "kv_head" or group_agg == "mass":
             fused = False
         ph = 1 if sets == "sequence" else Hkv       # pool rows per sequence
         sh = {"kv_head": Hkv, "q_head": Hq, "sequence": 1}[sets]  # set rows per sequence
@@ -99,9 +101,11 @@ class PrismDecoder:
         self.scorer_appends = (fused and keys == "int8" and dtype == prism.BF16 and head_dim == 128
                                and num_q_heads // num_kv_heads <= 8)
         # how the G query heads of a KV head combine into its selection
-        # score: "max" (the default reading) or "sum" (the variant, carried
-        # by the scorer that takes the new rows and by the fused refined layer)
-        assert group_agg in ("max", "sum")
+        # score: "max" (the default reading), "sum" (the variant, carried by
+        # the scorer that takes the new rows and by the fused refined layer)
+        # or "mass" (refined layers only: the proposal layers keep the max)
+        assert group_agg in ("max", "sum", "mass")
+        self.mass = group_agg == "mass"
         if sets != "kv_head" and (keys != "int8" or group_agg != "max"):
             raise ValueError("the q_head / sequence granularities take int8 keys and the maximum")
         if group_agg == "sum" and not self.scorer_appends:
@@ -169,8 +173,12 @@ class PrismDecoder:
                                 v_new=v_new if fused_append else None, k_prefetch=k_next,
                                 overlap=overlap, sum_group=self.sum_group, stream=stream)
             return
-        prism.refine_ex(p, q, k, self.pool[src], self.pool_cnt[src], self.kappa_p, self.kappa,
-                        self.idx[l], self.cnt[l], self.sets_code, self.ws_ref, stream=stream)
+        if self.mass:
+            prism.refine_mass(p, q, k, self.pool[src], self.pool_cnt[src], self.kappa_p, self.kappa,
+                              self.scale, self.idx[l], self.cnt[l], self.ws_ref, stream=stream)
+        else:
+            prism.refine_ex(p, q, k, self.pool[src], self.pool_cnt[src], self.kappa_p, self.kappa,
+                            self.idx[l], self.cnt[l], self.sets_code, self.ws_ref, stream=stream)
         prism.sparse_decode_ex(p, q, k, v, self.idx[l], self.cnt[l], self.kappa, self.scale,
                                self.sets_code, self.out[l], self.ws_dec, lse=self.lse[l], stream=stream)
 
@@ -277,7 +285,7 @@ class PrismDecoder:
             if proposal and self.proposal_select == "quantized":
                 n += (1 if append and self.fused and scorer_new else 0) + 2 + 2
                 continue
-            n += 1 if self.fused else 2 + 2
+            n += 1 if self.fused else 2 + 2 + (1 if self.mass else 0)
             if self.sets == "sequence":  # the head maxima of the pool scores (and of the proposal's)
                 n += 2 if proposal else 1
         return n

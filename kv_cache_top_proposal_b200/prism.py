@@ -35,7 +35,8 @@ EXPORTS = ("prism_workspace_size", "prism_append_kv", "prism_quantize_k", "prism
            "prism_clear_device_status",
            "prism_get_device_status", "prism_status_str", "prism_sparse_decode_noalloc",
            "prism_quantize_k_int2", "prism_propose_int2", "prism_index_overlap",
-           "prism_propose_topk", "prism_propose_ex", "prism_refine_ex", "prism_sparse_decode_ex")
+           "prism_propose_topk", "prism_propose_ex", "prism_refine_ex", "prism_sparse_decode_ex",
+           "prism_refine_mass")
 
 
 class PrismError(RuntimeError):
@@ -78,6 +79,7 @@ def _load():
         "prism_propose_topk": [sp, P, S, P, P, i32, i32, P, P, P, S, P],
         "prism_propose_ex": [sp, P, P, P, i32, P, P, ctypes.c_uint32, P, S, P],
         "prism_refine_ex": [sp, P, P, P, P, i32, i32, P, P, ctypes.c_uint32, P, S, P],
+        "prism_refine_mass": [sp, P, P, P, P, i32, i32, ctypes.c_float, P, P, P, S, P],
         "prism_sparse_decode_ex": [sp, P, P, P, P, P, i32, ctypes.c_float, ctypes.c_uint32, P, P, P, S,
                                    P],
     }
@@ -312,6 +314,16 @@ def refine_ex(p: Problem, q, k, pool, pool_cnt, kappa_p: int, kappa: int, idx, c
     _check(_lib.prism_refine_ex(p.ref, _ptr(q), _ptr(k), _ptr(pool), _ptr(pool_cnt), kappa_p, kappa,
                                 _ptr(idx), _ptr(cnt), sets, _ptr(ws), _nbytes(ws), _stream(stream)),
            "refine_ex")
+
+
+def refine_mass(p: Problem, q, k, pool, pool_cnt, kappa_p: int, kappa: int, softmax_scale: float, idx,
+                cnt, ws, stream=None):
+    """prism_refine_mass: the refined set by the group's softmax mass over the
+    pool (workspace of OP_REFINE)."""
+    _check(_lib.prism_refine_mass(p.ref, _ptr(q), _ptr(k), _ptr(pool), _ptr(pool_cnt), kappa_p, kappa,
+                                  float(softmax_scale), _ptr(idx), _ptr(cnt), _ptr(ws), _nbytes(ws),
+                                  _stream(stream)),
+           "refine_mass")
 
 
 def sparse_decode_ex(p: Problem, q, k, v, idx, cnt, kappa: int, softmax_scale: float, sets: int, out,

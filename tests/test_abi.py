@@ -103,6 +103,13 @@ def test_calls_validate_before_launch(prism_lib):
     _, nref = _ws(P, s, P.OP_REFINE, 256, 64)
     assert lib.prism_refine(ref, f, f, f, f, 256, 512, f, f, None, ws, nref, None) == P.ERR_INVALID_ARG
     assert lib.prism_refine(ref, f, f, f, f, 256, 0, f, f, None, ws, nref, None) == P.ERR_INVALID_ARG
+    # softmax-mass selection: the same bounds, and a finite positive scale
+    rm = lib.prism_refine_mass
+    assert rm(ref, f, f, f, f, 256, 512, 0.1, f, f, ws, nref, None) == P.ERR_INVALID_ARG
+    assert rm(ref, f, f, f, f, 256, 64, 0.0, f, f, ws, nref, None) == P.ERR_INVALID_ARG
+    assert rm(ref, f, f, f, f, 256, 64, float("inf"), f, f, ws, nref, None) == P.ERR_INVALID_ARG
+    assert rm(ref, None, f, f, f, 256, 64, 0.1, f, f, ws, nref, None) == P.ERR_INVALID_ARG
+    assert rm(ref, f, f, f, f, 256, 64, 0.1, f, f, ws, nref - 1, None) == P.ERR_WORKSPACE
     # non-finite softmax scale
     _, ndec = _ws(P, s, P.OP_SPARSE_DECODE, 0, 64)
     assert lib.prism_sparse_decode(ref, f, f, f, f, f, 64, float("nan"), f, None, ws, ndec,

@@ -379,6 +379,54 @@ def test_refine_vs_oracle(P, case):
 
 # ------------------------------------------------------------------ attention
 
+MASS_CASES = [
+    # (seqlens, Hq, Hkv, d, dtype, kappa_p, kappa): one head (mass order is
+    # score order), groups of 4 / 8 / 16, d = 64, fp32, a ragged batch with
+    # an empty sequence, pools of 8192, kappa = kappa_p
+    ([5000], 4, 4, 128, "bf16", 1024, 256),
+    ([20000, 3000, 0, 777], 32, 8, 128, "bf16", 4096, 1024),
+    ([30000], 16, 2, 128, "bf16", 8192, 2048),
+    ([9000], 16, 1, 64, "bf16", 2048, 300),
+    ([4000, 1500], 8, 2, 64, "f32", 1000, 1000),
+]
+
+
+@pytest.mark.parametrize("case", MASS_CASES, ids=lambda c: f"{len(c[0])}seq-{c[1]}/{c[2]}-d{c[3]}-{c[4]}-kp{c[5]}-k{c[6]}")
+def test_refine_mass_vs_oracle(P, case):
+    """prism_refine_mass against the oracle's softmax-mass selection, every
+    row: counts exact, sets up to near-ties of the fp64 mass, -1 padding."""
+    seqlens, hq, hkv, d, dtype, kp, kap = case
+    B = len(seqlens)
+    prob = problem(P, seqlens, hq, hkv, d, dtype)
+    q, k, v = make_case(seqlens, hq, hkv, d, dtype, seed=41)
+    rng = np.random.default_rng(42)
+    pool = np.full((B, hkv, kp), -1, np.int32)
+    pcnt = np.zeros((B, hkv), np.int32)
+    for b, L in enumerate(seqlens):
+        for h in range(hkv):
+            n = min(kp, L)
+            pool[b, h, :n] = np.sort(rng.choice(L, n, replace=False))
+            pcnt[b, h] = n
+    scale = float(np.float32(1 / math.sqrt(d)))
+    ws = ws_for(P, prob, P.OP_REFINE, kp, kap)
+    idx = torch.full((B, hkv, kap), -7, dtype=torch.int32, device=DEV)
+    cnt = torch.zeros((B, hkv), dtype=torch.int32, device=DEV)
+    P.refine_mass(prob, q, k, torch.tensor(pool, device=DEV), torch.tensor(pcnt, device=DEV), kp, kap,
+                  scale, idx, cnt, ws)
+    torch.cuda.synchronize()
+    assert P.get_device_status(ws) == 0
+    oidx, ocnt, omass = pipeline.refine_layer(q, k, prob.cu_host.tolist(), pool, pcnt, kap, agg="mass",
+                                              softmax_scale=scale)
+    gi, gc = _np(idx), _np(cnt)
+    assert np.array_equal(gc, ocnt)
+    for b in range(B):
+        for h in range(hkv):
+            n, c = int(pcnt[b, h]), int(ocnt[b, h])
+            r = dict(zip(pool[b, h, :n].tolist(), omass[(b, h)].tolist()))
+            check_index_set(gi[b, h, :c], oidx[b, h, :c], lambda t: r[t], f"mass b{b} h{h}")
+            assert np.all(gi[b, h, c:] == -1)
+
+
 ATTEND_CASES = [
     ([1024], 4, 1, 64, "f32", 64),
     ([5000, 1031, 0, 300], 8, 2, 128, "bf16", 256),

@@ -46,7 +46,8 @@ def _check_layer(dec, cfg, l, lay, kq, sc, rows, agg="max"):
     src = l - l % cfg.group
     gpool, gpc = _np(dec.pool[src]), _np(dec.pool_cnt[src])
     if l == src:
-        opool, ocnt, osc = pipeline.propose_layer(lay.q, kq, sc, cu, cfg.kappa_p, rows=rows, agg=agg)
+        pagg = "max" if agg == "mass" else agg  # the mass reading leaves the proposal at the max
+        opool, ocnt, osc = pipeline.propose_layer(lay.q, kq, sc, cu, cfg.kappa_p, rows=rows, agg=pagg)
         for (b, h) in rows:
             n = int(ocnt[b, h])
             assert int(gpc[b, h]) == n
@@ -273,6 +274,32 @@ def test_step_group_sum_c8k_every_row(prism_lib):
         src = l - l % cfg.group
         _invariants(dec, cfg, l)
         _check_layer(dec, cfg, l, lay, kqs[src], scs[src], _all_rows(cfg), agg="sum")
+
+
+@pytest.mark.parametrize("name", ["c8k", "tiny"])
+def test_step_softmax_mass_every_row(prism_lib, name):
+    """A whole step with the softmax-mass selection (the refined layers rank
+    pool members by the group's attention mass, prism_refine_mass, then the
+    sparse decode; the proposal layers keep the maximum): every row of every
+    layer against the oracle's mass mode, sets up to near-ties of the mass,
+    outputs within the tolerance."""
+    P = prism_lib
+    cfg = workload.config(name)
+    layers = list(workload.generate(cfg, DEV))
+    dec = _decoder(P, cfg, group_agg="mass")
+    assert not dec.fused
+    kqs, scs = {}, {}
+    for lay in layers:
+        if cfg.is_proposal(lay.index):
+            kqs[lay.index], scs[lay.index] = _prefill_kq(P, dec, cfg, lay)
+    dec.step([x.q for x in layers], [x.k for x in layers], [x.v for x in layers], kqs, scs)
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    for lay in layers:
+        l = lay.index
+        src = l - l % cfg.group
+        _invariants(dec, cfg, l)
+        _check_layer(dec, cfg, l, lay, kqs[src], scs[src], _all_rows(cfg), agg="mass")
 
 
 def _spoil_last_rows(layers, cu, kqs, scs):
