@@ -408,8 +408,7 @@ def line_config(cfg, args, seqlens0=None, n_grow=0):
                     f"write between steps outside its event pair; {touched}") if needs_flush(nbytes)
                 else f"inputs larger than L2: {touched}",
                 refined_layers="fused refine+select+sparse-decode (prism_refine_decode)"
-                if args.sets == "kv_head" and args.group_agg != "mass"
-                else "refine and sparse decode (two calls)",
+                if args.sets == "kv_head" else "refine and sparse decode (two calls)",
                 proposal_select=args.proposal_select, selection_sets=args.sets,
                 proposal_keys="int8 per token" if args.keys == "int8"
                 else "INT2 per 32-feature group (fp16 step and zero point)",

@@ -366,10 +366,13 @@ PRISM_API prism_status prism_sparse_decode(const prism_shape* shape, const void*
  * former (e.g. the refined layer before this one, on the same pool).
  * PRISM_RD_SUM_GROUP selects the group-sum variant of the exact score:
  * r_i = sum_g sum_j q[g][j] * K[pool_i][j] in place of the maximum over g
- * (the selection and the attention are unchanged).
+ * (the selection and the attention are unchanged).  PRISM_RD_MASS selects
+ * by the group's softmax mass over the pool, as prism_refine_mass at
+ * softmax_scale (not with PRISM_RD_SUM_GROUP: PRISM_ERR_INVALID_ARG).
  */
 #define PRISM_RD_OVERLAP 0x1u
 #define PRISM_RD_SUM_GROUP 0x2u
+#define PRISM_RD_MASS 0x4u
 PRISM_API prism_status prism_refine_decode(const prism_shape* shape, const void* q, void* k,
                                            void* v, const int32_t* pool_idx,
                                            const int32_t* pool_cnt, int32_t kappa_p,

@@ -128,7 +128,7 @@ cudaError_t launch_refine_decode(const Dims& d, const RefineDecodePlan& p, const
                                  const void* v_new, const void* k_next, const int32_t* pool,
                                  const int32_t* pool_cnt, int kappa_p, int kappa,
                                  float softmax_scale, int32_t* idx, int32_t* cnt, float* out,
-                                 float* lse, int32_t* status, bool overlap, bool sum_group,
+                                 float* lse, int32_t* status, bool overlap, int agg,
                                  cudaStream_t st);
 
 // Split-K attention partials over idx rows (idx == nullptr: every position).

@@ -588,7 +588,9 @@ prism_status prism_refine_decode(const prism_shape* shape, const void* q, void* 
   if (!q || !k || !v || !pool_idx || !pool_cnt || !idx || !cnt || !out) return PRISM_ERR_INVALID_ARG;
   if (kappa_p < 1 || kappa < 1 || kappa > kappa_p) return PRISM_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale)) return PRISM_ERR_INVALID_ARG;
-  if (flags & ~(PRISM_RD_OVERLAP | PRISM_RD_SUM_GROUP)) return PRISM_ERR_INVALID_ARG;
+  if (flags & ~(PRISM_RD_OVERLAP | PRISM_RD_SUM_GROUP | PRISM_RD_MASS)) return PRISM_ERR_INVALID_ARG;
+  if ((flags & PRISM_RD_SUM_GROUP) && (flags & PRISM_RD_MASS)) return PRISM_ERR_INVALID_ARG;
+  if ((flags & PRISM_RD_MASS) && !(softmax_scale > 0.0f)) return PRISM_ERR_INVALID_ARG;
   if ((k_new_opt == nullptr) != (v_new_opt == nullptr)) return PRISM_ERR_INVALID_ARG;
   if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v) % 16) return PRISM_ERR_INVALID_ARG;
   if (k_new_opt && (((uintptr_t)k_new_opt | (uintptr_t)v_new_opt | (uintptr_t)k | (uintptr_t)v) % 16))
@@ -601,7 +603,7 @@ prism_status prism_refine_decode(const prism_shape* shape, const void* q, void* 
                                           pool_cnt, kappa_p, kappa, softmax_scale, idx, cnt, out,
                                           lse_opt, static_cast<int32_t*>(ws),
                                           (flags & PRISM_RD_OVERLAP) != 0,
-                                          (flags & PRISM_RD_SUM_GROUP) != 0,
+                                          (flags & PRISM_RD_SUM_GROUP) ? 1 : (flags & PRISM_RD_MASS) ? 2 : 0,
                                           static_cast<cudaStream_t>(stream)));
 }
 

@@ -89,7 +89,7 @@ struct RDArgs {
   float* out;
   float* lse;
   int32_t* status;
-  int sum_group;  // selection score: sum over the group's query heads instead of the maximum
+  int agg;  // selection score over the group's query heads: 0 maximum, 1 sum, 2 softmax mass
 };
 
 // Byte offset of 16-byte chunk `c` of row `r` in a stage: chunks are XOR
@@ -530,13 +530,51 @@ __device__ __forceinline__ void hist_push(uint32_t* hw, uint32_t bin) {
 }
 
 
+// Softmax mass: the cluster's per-head maximum (is_max) or sum of the CTAs'
+// values v[GP]: the CTA reduces its threads' values, stores them into slot
+// `rank` of every CTA's buf, and after one cluster barrier every thread
+// combines the CL slots in rank order into v.  Whole cluster.
+template <int GP>
+__device__ __forceinline__ void mass_exchange(float (&v)[GP], bool is_max, float (&red)[kWarps][GP],
+                                              float (&buf)[kMaxCluster][GP], cg::cluster_group& cluster,
+                                              int CL, int rank) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float x = __shfl_xor_sync(0xffffffffu, v[g], o);
+      v[g] = is_max ? fmaxf(v[g], x) : v[g] + x;
+    }
+    if (lane == 0) red[warp][g] = v[g];
+  }
+  __syncthreads();
+  if (threadIdx.x < GP * CL) {
+    const int g = threadIdx.x % GP, dst = threadIdx.x / GP;
+    float t = red[0][g];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) t = is_max ? fmaxf(t, red[w][g]) : t + red[w][g];
+    cluster.map_shared_rank(&buf[0][0], dst)[rank * GP + g] = t;
+  }
+  cluster.sync();
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    float t = buf[0][g];
+    for (int c = 1; c < CL; ++c) t = is_max ? fmaxf(t, buf[c][g]) : t + buf[c][g];
+    v[g] = t;
+  }
+  __syncthreads();  // red is free again
+}
+
 // the stage ring, which also holds the warps' value partials at the end
 template <typename T, int D, int GP>
 __host__ __device__ constexpr int ring_bytes() {
   return kRing > kWarps * GP * D * 4 ? kRing : kWarps * GP * D * 4;
 }
 
-template <typename T, int D, int GP>
+// MASS: the softmax-mass selection (a separate instance, so that the other
+// selections run none of its code)
+template <typename T, int D, int GP, bool MASS>
 __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs a) {
   constexpr int E = Vec16<T>::E;
   constexpr int LPR = D / E;     // lanes per cache row (value pass)
@@ -564,6 +602,8 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
   __shared__ int s_slice;         // keys in this CTA's slice of the first-digit bins
   __shared__ int s_wa[kWarps], s_wb[kWarps];
   __shared__ float s_red[kWarps][GP];
+  __shared__ float s_mm[kMaxCluster][GP];  // softmax mass: every CTA's per-head maxima
+  __shared__ float s_zz[kMaxCluster][GP];  // and normalizer partials
   __shared__ __align__(16) float part[PART];  // this CTA's partial o, m, l
 
   cg::cluster_group cluster = cg::this_cluster();
@@ -662,8 +702,52 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
 
   // ---- 2. selection keys; their first digit into the cluster histogram
   constexpr bool kSplit = !kWarpKeys && ScorePick<T, D, GP>::type::kSplit;  // second half-sums in pw
-  const bool sum_group = a.sum_group != 0;  // the group's heads summed, not maxed
+  const bool sum_group = a.agg == 1;  // the group's heads summed, not maxed
+  if (MASS && !all) {
+    // softmax mass: each head's maximum and normalizer over the row's pool,
+    // through the cluster (every CTA's partials into every CTA), then the
+    // key of a member is ord(sum_g 2^((l_g - M_g) c) / Z_g)
+    float v[GP];
+#pragma unroll
+    for (int g = 0; g < GP; ++g) v[g] = -INFINITY;
+    for (int i = tid; i < m; i += kThreads)
+#pragma unroll
+      for (int g = 0; g < GP; ++g)
+        if (g < a.G) v[g] = fmaxf(v[g], dots[g * a.mc + i]);
+    mass_exchange<GP>(v, true, s_red, s_mm, cluster, CL, rank);
+    float z[GP];
+#pragma unroll
+    for (int g = 0; g < GP; ++g) z[g] = 0.0f;
+    for (int i = tid; i < m; i += kThreads)
+#pragma unroll
+      for (int g = 0; g < GP; ++g)
+        if (g < a.G && v[g] != -INFINITY) {
+          const float l = dots[g * a.mc + i];
+          if (l != -INFINITY) z[g] += exp2f((l - v[g]) * a.scale_log2);
+        }
+    mass_exchange<GP>(z, false, s_red, s_zz, cluster, CL, rank);
+    for (int i = tid; i < m; i += kThreads) {
+      float mass = 0.0f;
+      bool any = false;
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        if (g < a.G) {
+          const float l = dots[g * a.mc + i];
+          if (l != -INFINITY && z[g] > 0.0f) {
+            mass += exp2f((l - v[g]) * a.scale_log2) / z[g];
+            any = true;
+          }
+        }
+      }
+      keys[i] = ord_key(any ? mass : -INFINITY);
+    }
+    __syncthreads();
+  }
   for (int i = tid; i < m; i += kThreads) {
+    if (MASS && !all) {  // the key is the mass above
+      hist_push(hist + kH1, keys[i] >> 20);
+      continue;
+    }
     float best = sum_group ? 0.0f : -INFINITY;
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
@@ -1073,7 +1157,7 @@ constexpr int kPairBudget = 110 * 1024;
 
 template <typename T, int D, int GP>
 cudaError_t run(const Dims& d, RDArgs a, int cl, bool overlap, cudaStream_t st) {
-  auto kern = refine_decode_kernel<T, D, GP>;
+  auto kern = a.agg == 2 ? refine_decode_kernel<T, D, GP, true> : refine_decode_kernel<T, D, GP, false>;
   const int smem = ring_bytes<T, D, GP>() + kHistWords * 4 + a.mc * per_member_bytes<GP>() +
                    recv_bytes(GP, D);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1131,11 +1215,11 @@ cudaError_t launch_refine_decode(const Dims& d, const RefineDecodePlan& p, const
                                  const void* v_new, const void* k_next, const int32_t* pool,
                                  const int32_t* pool_cnt, int kappa_p, int kappa,
                                  float softmax_scale, int32_t* idx, int32_t* cnt, float* out,
-                                 float* lse, int32_t* status, bool overlap, bool sum_group,
+                                 float* lse, int32_t* status, bool overlap, int agg,
                                  cudaStream_t st) {
   if (d.B * d.Hkv == 0) return cudaSuccess;
   RDArgs a{q, k, v, k_next, k_new, v_new, d.cu_dev, pool, pool_cnt, kappa_p, kappa, d.Hkv, d.G, d.Hq, d.T, p.mc,
-           softmax_scale * 1.4426950408889634f, idx, cnt, out, lse, status, sum_group ? 1 : 0};
+           softmax_scale * 1.4426950408889634f, idx, cnt, out, lse, status, agg};
   if (d.bf16)
     return d.D == 128 ? by_group<__nv_bfloat16, 128>(d, a, p.cluster, overlap, st)
                       : by_group<__nv_bfloat16, 64>(d, a, p.cluster, overlap, st);

@@ -57,9 +57,7 @@ class PrismDecoder:
         self.sets = sets
         self.sets_code = {"kv_head": prism.SETS_KV_HEAD, "q_head": prism.SETS_Q_HEAD,
                           "sequence": prism.SETS_SEQUENCE}[sets]
-        # "mass": the refined layers select by the group's softmax mass over
-        # the pool (prism_refine_mass, then the sparse decode: two calls)
-        if sets != "kv_head" or group_agg == "mass":
+        if sets != "kv_head":
             fused = False
         ph = 1 if sets == "sequence" else Hkv       # pool rows per sequence
         sh = {"kv_head": Hkv, "q_head": Hq, "sequence": 1}[sets]  # set rows per sequence
@@ -103,7 +101,8 @@ class PrismDecoder:
         # how the G query heads of a KV head combine into its selection
         # score: "max" (the default reading), "sum" (the variant, carried by
         # the scorer that takes the new rows and by the fused refined layer)
-        # or "mass" (refined layers only: the proposal layers keep the max)
+        # or "mass" (refined selections only, fused or prism_refine_mass in
+        # the two-call path: the proposal layers keep the max)
         assert group_agg in ("max", "sum", "mass")
         self.mass = group_agg == "mass"
         if sets != "kv_head" and (keys != "int8" or group_agg != "max"):
@@ -171,7 +170,7 @@ class PrismDecoder:
                                 self.ws_rd, lse=self.lse[l],
                                 k_new=k_new if fused_append else None,
                                 v_new=v_new if fused_append else None, k_prefetch=k_next,
-                                overlap=overlap, sum_group=self.sum_group, stream=stream)
+                                overlap=overlap, sum_group=self.sum_group, mass=self.mass, stream=stream)
             return
         if self.mass:
             prism.refine_mass(p, q, k, self.pool[src], self.pool_cnt[src], self.kappa_p, self.kappa,

@@ -25,6 +25,7 @@ DEV_BAD_INDEX, DEV_TOO_LONG, DEV_TIMEOUT = 0x1, 0x2, 0x4
 MAX_SELECT_ROW = 393216
 RD_OVERLAP = 0x1
 RD_SUM_GROUP = 0x2
+RD_MASS = 0x4
 SETS_KV_HEAD, SETS_Q_HEAD, SETS_SEQUENCE = 0, 1, 2
 PROPOSE_SUM_GROUP = 0x1
 WS_HEADER = 256
@@ -243,16 +244,19 @@ def sparse_decode(p: Problem, q, k, v, idx, cnt, kappa: int, softmax_scale: floa
 
 def refine_decode(p: Problem, q, k, v, pool, pool_cnt, kappa_p: int, kappa: int,
                   softmax_scale: float, idx, cnt, out, ws, lse=None, k_new=None, v_new=None,
-                  k_prefetch=None, overlap: bool = False, sum_group: bool = False, stream=None):
+                  k_prefetch=None, overlap: bool = False, sum_group: bool = False, mass: bool = False,
+                  stream=None):
     """Refined layer in one call; k_new / v_new ([B][Hkv][d]) are appended
     at the last position of every sequence first.  overlap: the launch may
     begin before the previous kernel on the stream ends (see PRISM_RD_OVERLAP);
-    sum_group: the exact score sums the group's query heads (PRISM_RD_SUM_GROUP)."""
+    sum_group: the exact score sums the group's query heads (PRISM_RD_SUM_GROUP);
+    mass: the selection ranks by the group's softmax mass (PRISM_RD_MASS)."""
     _check(_lib.prism_refine_decode(p.ref, _ptr(q), _ptr(k), _ptr(v), _ptr(pool), _ptr(pool_cnt),
                                     kappa_p, kappa, float(softmax_scale), _ptr(idx), _ptr(cnt),
                                     _ptr(out), _ptr(lse), _ptr(k_new), _ptr(v_new),
                                     _ptr(k_prefetch),
-                                    (RD_OVERLAP if overlap else 0) | (RD_SUM_GROUP if sum_group else 0),
+                                    (RD_OVERLAP if overlap else 0) | (RD_SUM_GROUP if sum_group else 0)
+                                    | (RD_MASS if mass else 0),
                                     _ptr(ws),
                                     _nbytes(ws), _stream(stream)),
            "refine_decode")

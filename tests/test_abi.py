@@ -120,7 +120,7 @@ def test_calls_validate_before_launch(prism_lib):
     # fused refined layer: unknown flags, a lone new row, misaligned rows
     _, nrd = _ws(P, s, P.OP_REFINE_DECODE, 1024, 256)
     rd = lib.prism_refine_decode
-    assert rd(ref, f, f, f, f, f, 1024, 256, 0.1, f, f, f, None, None, None, None, 4, ws, nrd,
+    assert rd(ref, f, f, f, f, f, 1024, 256, 0.1, f, f, f, None, None, None, None, 8, ws, nrd,
               None) == P.ERR_INVALID_ARG
     assert rd(ref, f, f, f, f, f, 1024, 256, 0.1, f, f, f, None, f, None, None, 0, ws, nrd,
               None) == P.ERR_INVALID_ARG
@@ -128,6 +128,11 @@ def test_calls_validate_before_launch(prism_lib):
     assert rd(ref, bad, f, f, f, f, 1024, 256, 0.1, f, f, f, None, None, None, None, 0, ws, nrd,
               None) == P.ERR_INVALID_ARG
     assert rd(ref, f, f, f, f, f, 1024, 2048, 0.1, f, f, f, None, None, None, None, 0, ws, nrd,
+              None) == P.ERR_INVALID_ARG
+    # the softmax-mass flag: not with the group sum, and a positive scale
+    assert rd(ref, f, f, f, f, f, 1024, 256, 0.1, f, f, f, None, None, None, None, 2 | 4, ws, nrd,
+              None) == P.ERR_INVALID_ARG
+    assert rd(ref, f, f, f, f, f, 1024, 256, -0.1, f, f, f, None, None, None, None, 4, ws, nrd,
               None) == P.ERR_INVALID_ARG
     # proposal with the new key rows: unknown flags, missing rows, unsupported head dim
     pa = lib.prism_propose_append

@@ -276,18 +276,19 @@ def test_step_group_sum_c8k_every_row(prism_lib):
         _check_layer(dec, cfg, l, lay, kqs[src], scs[src], _all_rows(cfg), agg="sum")
 
 
+@pytest.mark.parametrize("fused", [True, False])
 @pytest.mark.parametrize("name", ["c8k", "tiny"])
-def test_step_softmax_mass_every_row(prism_lib, name):
+def test_step_softmax_mass_every_row(prism_lib, name, fused):
     """A whole step with the softmax-mass selection (the refined layers rank
-    pool members by the group's attention mass, prism_refine_mass, then the
-    sparse decode; the proposal layers keep the maximum): every row of every
-    layer against the oracle's mass mode, sets up to near-ties of the mass,
-    outputs within the tolerance."""
+    pool members by the group's attention mass: fused in prism_refine_decode,
+    or prism_refine_mass then the sparse decode; the proposal layers keep the
+    maximum): every row of every layer against the oracle's mass mode, sets
+    up to near-ties of the mass, outputs within the tolerance."""
     P = prism_lib
     cfg = workload.config(name)
     layers = list(workload.generate(cfg, DEV))
-    dec = _decoder(P, cfg, group_agg="mass")
-    assert not dec.fused
+    dec = _decoder(P, cfg, fused=fused, group_agg="mass")
+    assert dec.fused == fused
     kqs, scs = {}, {}
     for lay in layers:
         if cfg.is_proposal(lay.index):
