@@ -15,8 +15,10 @@
 //      ldmatrix fragments -- an fp32 cache takes a CUDA-core path; the logits
 //      stay in shared memory;
 //   2. the selection key of a member is ord(max_g q_g . k) (or of the sum
-//      over g, the group-sum variant); its first 12 bits go into the CTA's
-//      own histogram (two 16-bit counts per word);
+//      over g, the group-sum variant; or, in the MASS instance, of the
+//      group's softmax mass over the pool, after two cluster exchanges of
+//      each head's maximum and normalizer); its first 12 bits go into the
+//      CTA's own histogram (two 16-bit counts per word);
 //   3. CTA c sums slice c of every CTA's histogram (distributed shared
 //      memory reads, no remote atomics), and every CTA finds, from the
 //      slice totals and then the right slice, the bin holding the kappa-th
