@@ -204,21 +204,23 @@ class PrismDecoder:
         after the step.  The copies move a proposal group (`group` layers)
         at a time, one copy per group each way, and meet the layers only at
         group boundaries, where the step has no overlapped launch to lose:
-          - the first group's rows go up on the current stream, the other
-            groups' on copy_stream meanwhile, awaited by the second group;
+          - every group's rows go up on copy_stream, the first group's first;
+            the first layer waits for them, the second group for the rest;
           - each group's outputs go down on copy_stream once its last layer
             ends, while the next group runs.
         The current stream joins copy_stream at the end, so the whole step can
         be captured in one CUDA graph."""
         main = torch.cuda.current_stream()
         L, gsz = self.num_layers, self.group
-        io.dev_in[0].copy_(io.host_in[0], non_blocking=True)
         copy_stream.wait_stream(main)
-        up = torch.cuda.Event()
-        if io.groups > 1:
-            with torch.cuda.stream(copy_stream):
+        up0, up = torch.cuda.Event(), torch.cuda.Event()
+        with torch.cuda.stream(copy_stream):
+            io.dev_in[0].copy_(io.host_in[0], non_blocking=True)
+            up0.record(copy_stream)
+            if io.groups > 1:
                 io.dev_in[1:].copy_(io.host_in[1:], non_blocking=True)
                 up.record(copy_stream)
+        main.wait_event(up0)
         for l in range(L):
             pl = l % gsz == 0
             if l == gsz:
