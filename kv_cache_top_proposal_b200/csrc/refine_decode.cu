@@ -212,84 +212,6 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1
 // dots[g * mc + i] = q_g . k_i for slice member i (-inf for a member whose
 // position is out of range: it ranks last and weighs 0).
 
-// Tensor cores (bf16 cache): warp w takes 16-row tiles w, w + 8, ...; rows
-// are the M dimension, query heads the N dimension (8 per n-tile).  Even and
-// odd k-steps accumulate separately (two short dependency chains).
-template <int D, int GP>
-struct ScoreMma {
-  static constexpr int KS = D / 16;
-  static constexpr int NT = (GP + 7) / 8;
-  uint32_t bq[NT][KS][2];
-
-  __device__ __forceinline__ void init(const __nv_bfloat16* q, int G) {
-    const int lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int n = nt * 8 + g;
-#pragma unroll
-      for (int s = 0; s < KS; ++s) {
-        if (n < G) {
-          const uint32_t* qr = reinterpret_cast<const uint32_t*>(q + (int64_t)n * D + s * 16);
-          bq[nt][s][0] = qr[tig];
-          bq[nt][s][1] = qr[4 + tig];
-        } else {
-          bq[nt][s][0] = bq[nt][s][1] = 0u;
-        }
-      }
-    }
-  }
-
-  // Warp w takes 16-row tiles w % 4, w % 4 + 4, ... and k-steps of half
-  // w / 4 (all eight warps busy on a 64-row stage); the two halves' sums go to
-  // dots and dots2, added by the key pass.
-  static constexpr bool kSplit = true;
-  __device__ __forceinline__ void run(const unsigned char* buf, int r0, int nrows, const int* spos,
-                                      int G, int mc, float* dots, float* dots2) const {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, tig = lane & 3;
-    const int kh = warp >> 2;
-    float* out = kh ? dots2 : dots;
-    const int ntile = (nrows + 15) >> 4;
-    for (int t = warp & 3; t < ntile; t += kWarps / 2) {
-      float acc[2][NT][4];
-#pragma unroll
-      for (int u = 0; u < 2; ++u)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) acc[u][nt][0] = acc[u][nt][1] = acc[u][nt][2] = acc[u][nt][3] = 0.0f;
-      const int lrow = t * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-      for (int s2 = 0; s2 < KS / 2; ++s2) {
-        const int s = kh * (KS / 2) + s2;
-        uint32_t a0, a1, a2, a3;
-        ldmatrix_x4(smem_u32(buf + swz<D * 2>(lrow, 2 * s + (lane >> 4))), a0, a1, a2, a3);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const uint32_t b0 = kh ? bq[nt][KS / 2 + s2][0] : bq[nt][s2][0];
-          const uint32_t b1 = kh ? bq[nt][KS / 2 + s2][1] : bq[nt][s2][1];
-          mma_bf16(acc[s2 & 1][nt], a0, a1, a2, a3, b0, b1);
-        }
-      }
-      // c0,c1: row t*16+g, heads col, col+1; c2,c3: row t*16+g+8
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int r = t * 16 + g + 8 * half;
-        if (r < nrows) {
-          const int i = r0 + r;
-          const bool ok = spos[i] >= 0;
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const int col = nt * 8 + 2 * tig;
-            const float v0 = acc[0][nt][2 * half] + acc[1][nt][2 * half];
-            const float v1 = acc[0][nt][2 * half + 1] + acc[1][nt][2 * half + 1];
-            if (col < G) out[col * mc + i] = ok ? v0 : -INFINITY;
-            if (col + 1 < G) out[(col + 1) * mc + i] = ok ? v1 : -INFINITY;
-          }
-        }
-      }
-    }
-  }
-};
-
 // Key rows of a bf16 cache, per warp: warp w streams its own 16-row tiles
 // (w, w + kWarps, ...) through its own kWS slots of the ring with cp.async and
 // scores each tile with mma.sync as soon as it lands, so the key phase has no
@@ -444,7 +366,6 @@ struct ScoreSimt {
     }
   }
 
-  static constexpr bool kSplit = false;
   __device__ __forceinline__ void run(const unsigned char* buf, int r0, int nrows, const int* spos,
                                       int G, int mc, float* dots, float*) const {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -474,15 +395,6 @@ struct ScoreSimt {
       }
     }
   }
-};
-
-template <typename T, int D, int GP>
-struct ScorePick {
-  using type = ScoreSimt<T, D, GP>;
-};
-template <int D, int GP>
-struct ScorePick<__nv_bfloat16, D, GP> {
-  using type = ScoreMma<D, GP>;
 };
 
 // ---- phase 3: one radix digit from rank 0's histogram ----------------------
@@ -592,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
   int* spos = reinterpret_cast<int*>(hist + kHistWords);              // [mc]
   uint32_t* keys = reinterpret_cast<uint32_t*>(spos + a.mc);          // [mc]
   float* dots = reinterpret_cast<float*>(keys + a.mc);                // [GP][mc]
-  float* pw = dots + GP * a.mc;  // [GP][mc] second half-sums of the logits, then [mc][GP] weights
+  float* pw = dots + GP * a.mc;  // [mc][GP] softmax weights (GP mc floats)
   int* sel = reinterpret_cast<int*>(pw + GP * a.mc);                  // [mc]
   // partials of this CTA's outputs from every CTA: o [CL][per], (m, l) [CL][2 GP]
   float* recv = reinterpret_cast<float*>(sel + a.mc);
@@ -681,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
     wk.load_q(reinterpret_cast<const __nv_bfloat16*>(qrow), a.G);
     wk.run(a.G, a.mc, dots);
   } else {
-    typename ScorePick<T, D, GP>::type sc;
+    ScoreSimt<T, D, GP> sc;
     sc.init(qrow, a.G);
     kst.run([&](int r0, const unsigned char* buf, int nrows) {
       sc.run(buf, r0, nrows, spos, a.G, a.mc, dots, pw);
@@ -703,7 +615,6 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
   cluster_wait();
 
   // ---- 2. selection keys; their first digit into the cluster histogram
-  constexpr bool kSplit = !kWarpKeys && ScorePick<T, D, GP>::type::kSplit;  // second half-sums in pw
   const bool sum_group = a.agg == 1;  // the group's heads summed, not maxed
   if (MASS && !all) {
     // softmax mass: each head's maximum and normalizer over the row's pool,
@@ -755,7 +666,6 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
     for (int g = 0; g < GP; ++g) {
       if (g < a.G) {
         float v = dots[g * a.mc + i];
-        if (kSplit) dots[g * a.mc + i] = v = v + pw[g * a.mc + i];
         best = sum_group ? best + v : fmaxf(best, v);
       }
     }
