@@ -121,6 +121,7 @@ struct RefineDecodePlan {
   int cluster;
   int mc;
   bool ok;
+  bool inplace;  // the softmax weights replace the logits (no separate weight array)
 };
 RefineDecodePlan plan_refine_decode(const Dims& d, int kappa_p);
 cudaError_t launch_refine_decode(const Dims& d, const RefineDecodePlan& p, const void* q,

@@ -487,8 +487,10 @@ __host__ __device__ constexpr int ring_bytes() {
 }
 
 // MASS: the softmax-mass selection (a separate instance, so that the other
-// selections run none of its code)
-template <typename T, int D, int GP, bool MASS>
+// selections run none of its code).  INPL: the selected members' softmax
+// weights replace their logits, with no weight array (fewer shared-memory
+// bytes per member, for clusters with more members per CTA)
+template <typename T, int D, int GP, bool MASS, bool INPL>
 __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs a) {
   constexpr int E = Vec16<T>::E;
   constexpr int LPR = D / E;     // lanes per cache row (value pass)
@@ -504,8 +506,8 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
   int* spos = reinterpret_cast<int*>(hist + kHistWords);              // [mc]
   uint32_t* keys = reinterpret_cast<uint32_t*>(spos + a.mc);          // [mc]
   float* dots = reinterpret_cast<float*>(keys + a.mc);                // [GP][mc]
-  float* pw = dots + GP * a.mc;  // [mc][GP] softmax weights (GP mc floats)
-  int* sel = reinterpret_cast<int*>(pw + GP * a.mc);                  // [mc]
+  float* pw = INPL ? dots : dots + GP * a.mc;  // [mc][GP] softmax weights (unless INPL)
+  int* sel = reinterpret_cast<int*>(dots + (INPL ? 1 : 2) * GP * a.mc);  // [mc]
   // partials of this CTA's outputs from every CTA: o [CL][per], (m, l) [CL][2 GP]
   float* recv = reinterpret_cast<float*>(sel + a.mc);
 
@@ -931,7 +933,11 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
     for (int g = 0; g < GP; ++g) {
       const float l = g < a.G ? dots[g * a.mc + i] : -INFINITY;
       const float p = l == -INFINITY ? 0.0f : exp2f(l * a.scale_log2 - mx[g]);
-      pw[j * GP + g] = p;
+      if constexpr (INPL) {
+        if (g < a.G) dots[g * a.mc + i] = p;  // the member's weight, in place of its logit
+      } else {
+        pw[j * GP + g] = p;
+      }
       lsum[g] += p;
     }
   }
@@ -953,10 +959,10 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
         for (int r = warp * RPW + sub; r < nrows; r += NG) {
           float f[E];
           Vec16<T>::unpack(*reinterpret_cast<const uint4*>(buf + swz<RB>(r, li)), f);
-          const float* p = pw + (j0 + r) * GP;
+          const float* p = INPL ? dots + sel[j0 + r] : pw + (j0 + r) * GP;
 #pragma unroll
           for (int g = 0; g < GP; ++g) {
-            const float pg = p[g];
+            const float pg = INPL ? (g < a.G ? p[g * a.mc] : 0.0f) : p[g];
 #pragma unroll
             for (int e = 0; e < E; ++e) o[g][e] = fmaf(pg, f[e], o[g][e]);
           }
@@ -1050,9 +1056,9 @@ __global__ void __launch_bounds__(kThreads, 2) refine_decode_kernel(const RDArgs
   // every access to this CTA's shared memory by another CTA came before S5
 }
 
-template <int GP>
-constexpr int per_member_bytes() {
-  return (int)(2 * sizeof(int) + sizeof(uint32_t) + 2 * GP * sizeof(float));
+// spos, sel, keys, dots and (unless in place) the weights
+inline int per_member_bytes(int GP, bool inplace) {
+  return (int)(2 * sizeof(int) + sizeof(uint32_t) + (inplace ? 1 : 2) * GP * sizeof(float));
 }
 // stage ring (at least the warps' value partials) and rank 0's histograms
 int fixed_bytes(int D, int GP) {
@@ -1068,9 +1074,12 @@ constexpr int kDynBudget = 227 * 1024 - 8 * 1024;
 constexpr int kPairBudget = 110 * 1024;
 
 template <typename T, int D, int GP>
-cudaError_t run(const Dims& d, RDArgs a, int cl, bool overlap, cudaStream_t st) {
-  auto kern = a.agg == 2 ? refine_decode_kernel<T, D, GP, true> : refine_decode_kernel<T, D, GP, false>;
-  const int smem = ring_bytes<T, D, GP>() + kHistWords * 4 + a.mc * per_member_bytes<GP>() +
+cudaError_t run(const Dims& d, RDArgs a, int cl, bool inplace, bool overlap, cudaStream_t st) {
+  auto kern = a.agg == 2 ? (inplace ? refine_decode_kernel<T, D, GP, true, true>
+                                    : refine_decode_kernel<T, D, GP, true, false>)
+                         : (inplace ? refine_decode_kernel<T, D, GP, false, true>
+                                    : refine_decode_kernel<T, D, GP, false, false>);
+  const int smem = ring_bytes<T, D, GP>() + kHistWords * 4 + a.mc * per_member_bytes(GP, inplace) +
                    recv_bytes(GP, D);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -1109,13 +1118,13 @@ cudaError_t run(const Dims& d, RDArgs a, int cl, bool overlap, cudaStream_t st) 
 }
 
 template <typename T, int D>
-cudaError_t by_group(const Dims& d, const RDArgs& a, int cl, bool ov, cudaStream_t st) {
+cudaError_t by_group(const Dims& d, const RDArgs& a, int cl, bool inpl, bool ov, cudaStream_t st) {
   switch (padded_group(d.G)) {
-    case 1: return run<T, D, 1>(d, a, cl, ov, st);
-    case 2: return run<T, D, 2>(d, a, cl, ov, st);
-    case 4: return run<T, D, 4>(d, a, cl, ov, st);
-    case 8: return run<T, D, 8>(d, a, cl, ov, st);
-    default: return run<T, D, 16>(d, a, cl, ov, st);
+    case 1: return run<T, D, 1>(d, a, cl, inpl, ov, st);
+    case 2: return run<T, D, 2>(d, a, cl, inpl, ov, st);
+    case 4: return run<T, D, 4>(d, a, cl, inpl, ov, st);
+    case 8: return run<T, D, 8>(d, a, cl, inpl, ov, st);
+    default: return run<T, D, 16>(d, a, cl, inpl, ov, st);
   }
 }
 
@@ -1124,15 +1133,35 @@ cudaError_t by_group(const Dims& d, const RDArgs& a, int cl, bool ov, cudaStream
 RefineDecodePlan plan_refine_decode(const Dims& d, int kappa_p) {
   const int rows = d.B * d.Hkv;
   const int GP = padded_group(d.G);
-  const int per = (int)(2 * sizeof(int) + sizeof(uint32_t) + 2 * GP * sizeof(float));
   auto mc_of = [&](int c) { return ((kappa_p + c - 1) / c + 3) & ~3; };
-  auto need = [&](int c) { return fixed_bytes(d.D, GP) + mc_of(c) * per + recv_bytes(GP, d.D); };
-  // enough CTAs to cover every SM twice, then small enough for two per SM
+  auto need = [&](int c, bool inpl) {
+    return fixed_bytes(d.D, GP) + mc_of(c) * per_member_bytes(GP, inpl) + recv_bytes(GP, d.D);
+  };
+  // The largest cluster whose grid still fits one wave of two CTAs per SM:
+  // with more rows, smaller clusters and more pool members per CTA (16-CTA
+  // clusters need their SMs in one GPC, and few are resident at once).  Then
+  // small enough for two CTAs per SM: with a separate weight array if that
+  // fits, else with the weights in place of the logits, else a larger cluster.
   int cl = 1;
-  while (cl < kMaxCluster && (int64_t)rows * cl < 2LL * d.num_sms) cl *= 2;
-  while (cl < kMaxCluster && need(cl) > kPairBudget) cl *= 2;
-  const bool ok = kappa_p <= kMaxCount && need(cl) <= kDynBudget;
-  return RefineDecodePlan{cl, mc_of(cl), ok};
+  while (cl < kMaxCluster && (int64_t)rows * cl * 2 <= 2LL * d.num_sms) cl *= 2;
+  bool inpl = false;
+  for (;;) {
+    if (need(cl, false) <= kPairBudget) {
+      inpl = false;
+      break;
+    }
+    if (need(cl, true) <= kPairBudget) {
+      inpl = true;
+      break;
+    }
+    if (cl >= kMaxCluster) {
+      inpl = need(cl, false) > kDynBudget;
+      break;
+    }
+    cl *= 2;
+  }
+  const bool ok = kappa_p <= kMaxCount && need(cl, inpl) <= kDynBudget;
+  return RefineDecodePlan{cl, mc_of(cl), ok, inpl};
 }
 
 cudaError_t launch_refine_decode(const Dims& d, const RefineDecodePlan& p, const void* q,
@@ -1146,10 +1175,10 @@ cudaError_t launch_refine_decode(const Dims& d, const RefineDecodePlan& p, const
   RDArgs a{q, k, v, k_next, k_new, v_new, d.cu_dev, pool, pool_cnt, kappa_p, kappa, d.Hkv, d.G, d.Hq, d.T, p.mc,
            softmax_scale * 1.4426950408889634f, idx, cnt, out, lse, status, agg};
   if (d.bf16)
-    return d.D == 128 ? by_group<__nv_bfloat16, 128>(d, a, p.cluster, overlap, st)
-                      : by_group<__nv_bfloat16, 64>(d, a, p.cluster, overlap, st);
-  return d.D == 128 ? by_group<float, 128>(d, a, p.cluster, overlap, st)
-                    : by_group<float, 64>(d, a, p.cluster, overlap, st);
+    return d.D == 128 ? by_group<__nv_bfloat16, 128>(d, a, p.cluster, p.inplace, overlap, st)
+                      : by_group<__nv_bfloat16, 64>(d, a, p.cluster, p.inplace, overlap, st);
+  return d.D == 128 ? by_group<float, 128>(d, a, p.cluster, p.inplace, overlap, st)
+                    : by_group<float, 64>(d, a, p.cluster, p.inplace, overlap, st);
 }
 
 }  // namespace prism
