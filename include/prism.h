@@ -105,7 +105,9 @@ typedef enum prism_op {
  * prism_propose, prism_propose_append, prism_refine_decode, prism_refine,
  * prism_sparse_decode) stays valid while the last sequence grows, as long as
  * it stays within 131072 positions when the graph was captured at or below
- * that (the proposal selection then takes the same path).
+ * that (the proposal selection then takes the same path; its cluster size is
+ * planned from the longest length a row can reach, the last row counted up
+ * to total_tokens).
  * prism_dense_decode sizes its split grid from the host copy,
  * which must be current for it.  head_dim is 64 or 128; num_q_heads is a
  * multiple of num_kv_heads with G <= 16; batch <= 4096. */

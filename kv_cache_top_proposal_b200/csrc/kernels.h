@@ -87,7 +87,7 @@ int select_capacity_per_row();  // longest row one cluster can select from
 
 // Proposal-layer selection from the scorer's first-digit histogram (see
 // propose_select.cu); rows up to propose_select_max_row() positions.
-int propose_select_cluster();
+int propose_select_cluster(const Dims& d);
 int propose_select_max_row();
 cudaError_t launch_propose_select(const Dims& d, const float* scores, const uint32_t* hist,
                                   int kappa_p, int32_t* pool, int32_t* pool_cnt, int32_t* status,

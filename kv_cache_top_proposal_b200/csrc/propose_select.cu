@@ -5,7 +5,7 @@
 // "Implementation Details").
 //
 // The scorer has already built, per row, the histogram of the first 12 bits
-// of ord(score).  One cluster of kCL CTAs per row; CTA r owns the contiguous
+// of ord(score).  One cluster of CL CTAs per row; CTA r owns the contiguous
 // slice r of positions and keeps its keys in registers (KPT per thread,
 // coalesced: key u of thread t is slice position u * kThreads + t):
 //   1. every CTA reads the row's histogram and locates the bin holding the
@@ -31,7 +31,7 @@ namespace prism {
 
 namespace {
 
-constexpr int kCL = 16;                       // CTAs per row (a non-portable cluster size)
+constexpr int kMaxCL = 16;                    // largest cluster (non-portable size)
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kKPT = 16;                      // keys per thread
@@ -98,12 +98,14 @@ __device__ __forceinline__ void scan_table(int* tab, int base, int* scratch) {
   __syncthreads();
 }
 
+template <int CL>
 __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArgs a) {
+  static_assert(kBins / CL <= kThreads && CL <= 32, "one slice bin per thread, one rank per lane");
   __shared__ __align__(16) uint32_t hist2[kBins];  // this CTA's digit-2 counts
   __shared__ __align__(16) uint32_t hist3[kBins];  // this CTA's digit-3 counts
   __shared__ int tabE[kKPT * kWarps];  // per (key block, warp): keys at P, then their prefix
   __shared__ int tabK[kKPT * kWarps];  // per (key block, warp): kept keys, then output slots
-  __shared__ uint32_t s_sw[kBins / kCL];  // this CTA's slice of the cluster's digit counts
+  __shared__ uint32_t s_sw[kBins / CL];  // this CTA's slice of the cluster's digit counts
   __shared__ int s_slice;
   __shared__ int scratch[33];
   __shared__ int s_dig[3];
@@ -112,16 +114,19 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
 
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
-  const int row = blockIdx.x / kCL;
+  const int row = blockIdx.x / CL;
   const int b = row / a.Hkv, h = row - b * a.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned lt = (1u << lane) - 1u;
   const int t0 = a.cu[b];
   const int n = a.cu[b + 1] - t0;
-  const int chunk = (n + kCL - 1) / kCL;
+  const int chunk = (n + CL - 1) / CL;
   const int lo = min(n, rank * chunk), hi = min(n, lo + chunk);
   const int m = hi - lo;
   int32_t* out = a.out + (int64_t)row * a.kp;
+  // launched as the scorer's programmatic dependent: the lengths were final
+  // before the scorer started, its scores and histograms are not yet
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
 
   // every branch depends on cluster-wide values only
   if (n <= a.kp || chunk > kMaxSlice) {
@@ -132,7 +137,7 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
       flag_status(a.status, PRISM_DEV_TOO_LONG);
     }
     const int filled = all ? n : 0;
-    for (int i = filled + rank * kThreads + tid; i < a.kp; i += kCL * kThreads) out[i] = -1;
+    for (int i = filled + rank * kThreads + tid; i < a.kp; i += CL * kThreads) out[i] = -1;
     if (rank == 0 && tid == 0) a.out_cnt[row] = filled;
     return;
   }
@@ -175,17 +180,17 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
   int r = k - s_dig[1];
   cluster_wait();
   auto cluster_digit = [&](const uint32_t* hl, int rr) {
-    constexpr int WS = kBins / kCL;  // bins per slice
+    constexpr int WS = kBins / CL;  // bins per slice
     __syncthreads();
     cluster.sync();  // every CTA's histogram is complete
     int part = 0;
     for (int x = tid; x < WS; x += kThreads) {
-      uint32_t v[kCL];  // every CTA's count, all loads in flight at once
+      uint32_t v[CL];  // every CTA's count, all loads in flight at once
 #pragma unroll
-      for (int c = 0; c < kCL; ++c) v[c] = cluster.map_shared_rank(hl, c)[rank * WS + x];
+      for (int c = 0; c < CL; ++c) v[c] = cluster.map_shared_rank(hl, c)[rank * WS + x];
       uint32_t acc = 0u;
 #pragma unroll
-      for (int c = 0; c < kCL; ++c) acc += v[c];
+      for (int c = 0; c < CL; ++c) acc += v[c];
       s_sw[x] = acc;
       part += (int)acc;
     }
@@ -194,10 +199,10 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
     if (tid == 0) s_slice = tot;
     cluster.sync();  // every slice and its total are ready
     if (warp == 0) {
-      const int t = lane < kCL ? *cluster.map_shared_rank(&s_slice, lane) : 0;
+      const int t = lane < CL ? *cluster.map_shared_rank(&s_slice, lane) : 0;
       const int incl = warp_incl_scan(t);  // slices rank in descending bin order
       const int above = __shfl_sync(0xffffffffu, incl, 31) - incl;
-      const unsigned hit = __ballot_sync(0xffffffffu, lane < kCL && above < rr && rr <= above + t);
+      const unsigned hit = __ballot_sync(0xffffffffu, lane < CL && above < rr && rr <= above + t);
       const int src = hit ? __ffs(hit) - 1 : 0;  // exactly one lane when counts are right
       const int above_src = __shfl_sync(0xffffffffu, above, src);
       if (lane == 0) {
@@ -259,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
   cluster.sync();  // every CTA's counts are published
   if (warp == 0) {
     int g_s = 0, e_s = 0;
-    if (lane < kCL) {
+    if (lane < CL) {
       const int* rc = cluster.map_shared_rank(s_cnt, lane);
       g_s = rc[0];
       e_s = rc[1];
@@ -330,8 +335,51 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
 
 }  // namespace
 
-int propose_select_cluster() { return kCL; }
-int propose_select_max_row() { return kCL * kMaxSlice; }
+// Smallest cluster whose CTAs hold the longest row the captured call can
+// meet: the other rows keep their lengths and the last one may grow into the
+// spare rows up to total_tokens.  A shorter row leaves most key registers of
+// its CTAs empty, and every CTA costs about the same whatever its fill, so a
+// cluster sized to the rows cuts the CTAs (and the waves) of a batch of
+// shorter rows.  Past the largest cluster's capacity the largest is used
+// (rows longer than that flag PRISM_DEV_TOO_LONG, as before).
+int propose_select_cluster(const Dims& d) {
+  int64_t bound = 0;
+  for (int b = 0; b < d.B; ++b) {
+    const int64_t L = b + 1 < d.B ? (int64_t)(d.cu_host[b + 1] - d.cu_host[b])
+                                  : d.T - d.cu_host[b];
+    bound = L > bound ? L : bound;
+  }
+  int cl = 4;
+  while (cl < kMaxCL && (int64_t)cl * kMaxSlice < bound) cl *= 2;
+  return cl;
+}
+int propose_select_max_row() { return kMaxCL * kMaxSlice; }
+
+namespace {
+template <int CL>
+cudaError_t launch_ps(const PSArgs& a, int rows, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(rows * CL));
+  cfg.blockDim = dim3(kThreads);
+  if (CL > 8) {
+    cudaError_t e = cudaFuncSetAttribute(propose_select_kernel<CL>,
+                                         cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, propose_select_kernel<CL>, a);
+}
+}  // namespace
 
 cudaError_t launch_propose_select(const Dims& d, const float* scores, const uint32_t* hist,
                                   int kappa_p, int32_t* pool, int32_t* pool_cnt, int32_t* status,
@@ -339,22 +387,11 @@ cudaError_t launch_propose_select(const Dims& d, const float* scores, const uint
   const int rows = d.B * d.Hkv;
   if (rows == 0) return cudaSuccess;
   PSArgs a{scores, hist, d.cu_dev, d.Hkv, d.T, kappa_p, pool, pool_cnt, status};
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(rows * kCL));
-  cfg.blockDim = dim3(kThreads);
-  cudaError_t e =
-      cudaFuncSetAttribute(propose_select_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  if (e != cudaSuccess) return e;
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kCL;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, propose_select_kernel, a);
+  switch (propose_select_cluster(d)) {
+    case 4: return launch_ps<4>(a, rows, st);
+    case 8: return launch_ps<8>(a, rows, st);
+    default: return launch_ps<16>(a, rows, st);
+  }
 }
 
 }  // namespace prism

@@ -296,6 +296,45 @@ def test_propose_query_ranges(P):
             check_index_set(gp[b, h, :n], opool[b, h, :n], lambda t: s[t], f"pool b{b} h{h}")
 
 
+@pytest.mark.parametrize("seqlens,cap,kp", [
+    ([32768, 300], None, 4096),     # 4-CTA clusters, the long row filling all four
+    ([32769, 300], None, 4096),     # one position more: 8-CTA clusters
+    ([65536, 10], None, 8192),      # 8-CTA clusters, full
+    ([1000, 2000], 43000, 700),     # short rows, but the last may grow to 42000: 8
+    ([70000, 4000], None, 6000),    # 16-CTA clusters
+], ids=["cl4-full", "cl8-edge", "cl8-full", "cl8-by-capacity", "cl16"])
+def test_propose_select_cluster_sizes(P, seqlens, cap, kp):
+    """The proposal selection's cluster is the smallest (4, 8 or 16 CTAs of
+    8192 keys) that holds the longest row the call can meet, the last row
+    counted up to the capacity.  Pools match the oracle's on each side of
+    the boundaries; the spare rows past the end hold valid codes that must
+    stay out of the last row's pool."""
+    hq, hkv, d = 8, 2, 128
+    prob = P.Problem(seqlens, hq, hkv, d, P.BF16, device=DEV, capacity=cap)
+    T = prob.total_tokens
+    q, k, _ = make_case(list(seqlens) + ([T - sum(seqlens)] if cap else []), hq, hkv, d,
+                        "bf16", seed=21)
+    kq = torch.zeros((hkv, T, d), dtype=torch.int8, device=DEV)
+    sc = torch.zeros((hkv, T), dtype=torch.float32, device=DEV)
+    P.quantize_k(P.Problem([T], hq, hkv, d, P.BF16, device=DEV), k, kq, sc)
+    q = q[:len(seqlens)].contiguous()
+    pool = torch.full((len(seqlens), hkv, kp), -7, dtype=torch.int32, device=DEV)
+    cnt = torch.full((len(seqlens), hkv), -7, dtype=torch.int32, device=DEV)
+    ws = ws_for(P, prob, P.OP_PROPOSE, kp)
+    P.propose(prob, q, kq, sc, kp, pool, cnt, ws)
+    torch.cuda.synchronize()
+    assert P.get_device_status(ws) == 0
+    opool, ocnt, oscores = pipeline.propose_layer(q, kq, sc, prob.cu_host.tolist(), kp)
+    gp, gc = _np(pool), _np(cnt)
+    assert np.array_equal(gc, ocnt)
+    for b in range(len(seqlens)):
+        for h in range(hkv):
+            s = oscores[(b, h)]
+            n = int(ocnt[b, h])
+            check_index_set(gp[b, h, :n], opool[b, h, :n], lambda t: s[t], f"pool b{b} h{h}")
+            assert np.all(gp[b, h, n:] == -1)
+
+
 @pytest.mark.parametrize("L0,kp", [(3000, 1000), (60000, 8192)], ids=["small", "many-candidates"])
 def test_propose_all_ties_lower_index_wins(P, L0, kp):
     """Equal scores: the lowest positions win.  At 60000 positions every CTA of
