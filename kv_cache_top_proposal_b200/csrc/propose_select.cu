@@ -124,9 +124,6 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
   const int lo = min(n, rank * chunk), hi = min(n, lo + chunk);
   const int m = hi - lo;
   int32_t* out = a.out + (int64_t)row * a.kp;
-  // launched as the scorer's programmatic dependent: the lengths were final
-  // before the scorer started, its scores and histograms are not yet
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");
 
   // every branch depends on cluster-wide values only
   if (n <= a.kp || chunk > kMaxSlice) {
@@ -368,15 +365,13 @@ cudaError_t launch_ps(const PSArgs& a, int rows, cudaStream_t st) {
   }
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CL;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, propose_select_kernel<CL>, a);
 }
 }  // namespace
