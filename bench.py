@@ -203,13 +203,16 @@ class Dist:
             self.pg.destroy_process_group()
 
 
-def traffic_for(op: str):
-    """ncu DRAM bytes per launch recorded for this op's kernels, if the
-    kernel sources are unchanged since the capture."""
+def traffic_for(op: str, workload_name: str, flags: dict):
+    """ncu DRAM bytes per launch recorded for this op's kernels, if this run
+    launches what was captured: the same workload and flags, and kernel
+    sources unchanged since the capture."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         rec = json.load(open(path))[op]
     except Exception:
+        return None
+    if rec.get("workload") != workload_name or rec.get("flags", {}) != flags:
         return None
     h = hashlib.sha256()
     for f in rec.get("sources", []):
@@ -651,7 +654,8 @@ def run_prism(args, dist: Dist):
         achieved = nbytes["refine_decode"] / (instep_us * 1e-6) / 1e9
         roofline = {"bound": "hbm", "kernel": "refine_decode", "achieved": round(achieved, 1),
                     "peak": peak, "peak_source": peak_kind, "unit": "GB/s",
-                    "frac": round(achieved / peak, 4), "traffic": traffic_for("refine_decode"),
+                    "frac": round(achieved / peak, 4), "traffic": traffic_for("refine_decode", cfg.name,
+                                                          {"group_agg": args.group_agg}),
                     "algorithmic_bytes_per_launch": nbytes["refine_decode"],
                     "avg_launch_us": round(instep_us, 3), "launches_per_step": L,
                     "timing": "in step: a graph of the step's refined-layer launches in step order "
