@@ -118,6 +118,15 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
   const int b = row / a.Hkv, h = row - b * a.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned lt = (1u << lane) - 1u;
+  // this thread's bins of the row's first-digit histogram, loaded beside the
+  // lengths: they do not depend on them
+  constexpr int kHPer = kHist / kThreads;
+  uint32_t hc[kHPer];
+  {
+    const uint32_t* gh = a.hist + (int64_t)row * kHist + tid * kHPer;
+#pragma unroll
+    for (int j = 0; j < kHPer; ++j) hc[j] = __ldcg(gh + j);
+  }
   const int t0 = a.cu[b];
   const int n = a.cu[b + 1] - t0;
   const int chunk = (n + CL - 1) / CL;
@@ -146,7 +155,8 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
   __syncthreads();
   cluster_arrive();  // pairs with the wait below (every CTA is running)
 
-  // ---- the slice's keys, kKPT loads in flight per thread
+  // ---- the slice's keys, kKPT loads in flight per thread while the first
+  // digit's bin is found (step 1 below)
   uint32_t key[kKPT];
   {
     const float* kb = a.scores + (int64_t)h * a.T + t0 + lo;
@@ -156,6 +166,7 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
       const int i = u * kThreads + tid;
       v[u] = i < m ? __ldcg(kb + i) : 0.0f;
     }
+    find_digit<kHPer>([&](int bin) { return hc[bin - tid * kHPer]; }, k, scratch, s_dig);
 #pragma unroll
     for (int u = 0; u < kKPT; ++u) key[u] = ord_key(v[u]);
   }
@@ -169,8 +180,6 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
   // memory reads, no remote atomics) and every CTA finds the next bin from
   // the slice totals and the right slice; then the same for the last 10
   // bits.  Finally the CTAs exchange their counts above and at P.
-  const uint32_t* gh = a.hist + (int64_t)row * kHist;
-  find_digit<kHist / kThreads>([&](int bin) { return __ldcg(gh + bin); }, k, scratch, s_dig);
   uint32_t P = (uint32_t)s_dig[0];
   int shift = 20;
   const int c1 = s_dig[2];
@@ -277,6 +286,9 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
     }
   }
   __syncthreads();
+  // this CTA's last read of another CTA's shared memory is done; the wait
+  // at the end keeps every CTA's shared memory alive until all have arrived
+  cluster_arrive();
   const int off = s_mine[0], take = s_mine[1];
   const bool part = take < s_mine[2];  // the slice keeps only some of its keys at P
 
@@ -325,9 +337,7 @@ __global__ void __launch_bounds__(kThreads, 2) propose_select_kernel(const PSArg
     }
   }
   if (rank == 0 && tid == 0) a.out_cnt[row] = k;
-  // no CTA exits while rank 0's shared memory or its counts may still be read
-  cluster_arrive();
-  cluster_wait();
+  cluster_wait();  // no CTA exits while its counts may still be read
 }
 
 }  // namespace
