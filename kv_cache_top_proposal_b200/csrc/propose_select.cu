@@ -5,7 +5,8 @@
 // "Implementation Details").
 //
 // The scorer has already built, per row, the histogram of the first 12 bits
-// of ord(score).  One cluster of CL CTAs per row; CTA r owns the contiguous
+// of ord(score).  One cluster of CL CTAs per row (CL = 4, 8 or 16: see
+// propose_select_cluster); CTA r owns the contiguous
 // slice r of positions and keeps its keys in registers (KPT per thread,
 // coalesced: key u of thread t is slice position u * kThreads + t):
 //   1. every CTA reads the row's histogram and locates the bin holding the
